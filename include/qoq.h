@@ -1,0 +1,222 @@
+/*
+ * qoq.h -- C ABI of libqoq.so, the B200 (sm_100a) QoQ W4A8 linear layer
+ *
+ *     Y = diag(s_x) * (X8 * W8hat^T) * diag(s_c)
+ *
+ * X8 holds per-token INT8 activations, and W8hat is the INT8 weight that
+ * progressive group quantization produces. The steps are:
+ *   - stage 1: per-channel symmetric INT8 in the protective range [-119,119];
+ *   - stage 2: group-wise UINT4 codes q with an integer scale s_g and a zero z.
+ * At run time the kernel expands each code to INT8 as q*s_g - z*s_g. It
+ * multiplies on INT8 tensor cores and accumulates in INT32. The FP16 scales
+ * are applied once, after the K loop.
+ *
+ * Sources, by page title:
+ *   "QServe: Low Bit Width Does Not Guarantee High Throughput", section 4
+ *       "Formalization and procedure": the stage-1 and stage-2 equations, and
+ *       the paragraph after them (multiply by the integer scale first, then
+ *       subtract the precomputed zero compensation).
+ *   "QServe: W4A8KV4 Quantization and System Co-design for Efficient LLM
+ *       Serving" (paper card), Key points: FP16 per-channel scales; the
+ *       protective range; multiply first, subtract afterward.
+ *   "QServe Guide: W4A8KV4 Quantization for LLM Serving":
+ *       - Deep Dive, subsection 1: the per-token activation equation and the
+ *         output rescaling equation;
+ *       - The Architecture, subsection 2: INT8 tensor-core products with
+ *         INT32 accumulation, and scales applied after the products.
+ *
+ * Conventions shared by every call:
+ *   - Pointers marked "device" are CUDA device pointers on the current
+ *     device. The caller allocates and owns every buffer. The library
+ *     allocates no memory.
+ *   - FP16 values cross the ABI as uint16_t bit patterns (IEEE binary16).
+ *   - Matrices are dense row-major with no strides. W and Y follow the
+ *     PyTorch Linear convention: a row of W is an output channel.
+ *   - `stream` is a cudaStream_t passed as void*. NULL means the legacy
+ *     default stream. Every call that launches work is asynchronous on that
+ *     stream.
+ *   - Every call returns a qoq_status. Argument checks run on the host
+ *     before anything is launched. A failed check returns
+ *     QOQ_ERR_INVALID_ARG and launches nothing.
+ *   - Shape limits, checked on every call:
+ *       - M >= 0. M == 0 is a valid empty problem: it returns QOQ_OK and
+ *         launches nothing.
+ *       - N is a multiple of 128, from 128 to 1048576.
+ *       - K is a multiple of 128, from 128 to 65536. The INT32 accumulator
+ *         then cannot overflow: |acc| <= K*128*127 < 2^31.
+ *       - group_size is 128 (g128) or K (per-channel).
+ *       - Pointers are 16-byte aligned.
+ *   - The library needs a B200-class GPU (compute capability 10.0). On any
+ *     other device a call returns QOQ_ERR_UNSUPPORTED.
+ */
+#ifndef QOQ_H
+#define QOQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QOQ_API __attribute__((visibility("default")))
+#else
+#define QOQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QOQ_OK = 0,
+    QOQ_ERR_INVALID_ARG = -1,   /* a shape, pointer or size failed the checks above */
+    QOQ_ERR_UNSUPPORTED = -2,   /* the current device is not compute capability 10.0 */
+    QOQ_ERR_CUDA = -3,          /* a CUDA runtime call or a launch failed */
+    QOQ_ERR_TIMEOUT = -4        /* a kernel's bounded wait ran out (see qoq_device_error) */
+} qoq_status;
+
+/* Short English text for a status code. The string is static. */
+QOQ_API const char *qoq_status_string(int status);
+
+/* ------------------------------------------------------------------------
+ * Packed weight layout: the "Blackwell interleaved UINT4" layout
+ * ------------------------------------------------------------------------
+ * Wp holds one 4-bit code per weight. Bytes are grouped into 8192-byte
+ * chunks, one per (128-channel panel p, 128-wide K block b). Chunks are
+ * ordered p-major:
+ *     chunk(p, b) starts at byte (p * (K/128) + b) * 8192.
+ * A chunk has 4 slabs of 2048 bytes, one per 32-wide K slice j. Inside slab
+ * j, channel r (0..127 within the panel) owns the 16 bytes at j*2048 + r*16.
+ * Those 16 bytes are 4 little-endian 32-bit words. For word w (0..3),
+ * byte i (0..3), with k0 = 128*b + 32*j:
+ *     low nibble  = q[n][k0 + 4*w + i]
+ *     high nibble = q[n][k0 + 16 + 4*w + i]
+ * So one AND of a word with 0x0F0F0F0F gives four consecutive codes in four
+ * byte lanes, and one shift plus one AND gives the next four.
+ *
+ * The group tables are group-major, channel-contiguous, one byte per entry:
+ *     s_g[g*N + n]  the integer group scale (1..16),
+ *     zs[g*N + n]   the zero compensation z*s_g (0..240),
+ * with g = k / group_size. s_c[n] is the FP16 channel scale.
+ */
+
+/* Bytes of Wp for an N x K weight: N*K/2. Returns 0 when N or K is not a
+ * positive multiple of 128. */
+QOQ_API size_t qoq_packed_weight_bytes(int N, int K);
+
+/* Progressive group quantization and packing (the offline step).
+ *
+ * Sources: "QServe: Low Bit Width Does Not Guarantee High Throughput",
+ * section 4, stage-1 and stage-2 equations; FP16 scales per the paper card's
+ * Key points. Choices where the pages are silent:
+ *   - round is half to even;
+ *   - s_c = fp16(max|W_n| / 119), and the stored FP16 value is the one used
+ *     to quantize;
+ *   - per group: mn = min(0, min W8) and mx = max(0, max W8);
+ *     s_g = max(1, ceil((mx - mn)/15)); z = round(-mn/s_g);
+ *     q = clamp(round(W8/s_g) + z, 0, 15).
+ *   - A row whose scale rounds to FP16 zero quantizes to all zeros.
+ *   - W must be finite. Entries with |W| >= 65520*119 make s_c infinite.
+ *
+ *   W      device, float32 [N][K], read only.
+ *   Wp     device, qoq_packed_weight_bytes(N, K) bytes, written in the
+ *          packed layout above.
+ *   s_c    device, uint16_t [N] FP16 bits, written.
+ *   s_g    device, uint8_t [K/group_size][N], written.
+ *   zs     device, uint8_t [K/group_size][N], written.
+ * The result is deterministic and bit-identical on every call.
+ */
+QOQ_API int qoq_pack_weights(const float *W, int N, int K, int group_size,
+                     uint8_t *Wp, uint16_t *s_c, uint8_t *s_g, uint8_t *zs,
+                     void *stream);
+
+/* Per-token symmetric INT8 activation quantization.
+ *
+ * Source: "QServe Guide: W4A8KV4 Quantization for LLM Serving", Deep Dive,
+ * subsection 1, the activation equation. For each row m:
+ *     s_x[m] = fp16(max_k |X[m][k]| / 127)
+ *     X8[m][k] = clamp(round(X[m][k] / s_x[m]), -128, 127)
+ * The division is IEEE FP32 and round is half to even. A row whose scale
+ * rounds to FP16 zero gives all zeros.
+ *
+ *   X      device, uint16_t [M][K] FP16 bits, read only. Must be finite.
+ *   X8     device, int8_t [M][K], written.
+ *   s_x    device, uint16_t [M] FP16 bits, written.
+ * K follows the GEMM limits above (multiple of 128, at most 65536).
+ */
+QOQ_API int qoq_quant_act_per_token(const uint16_t *X, int M, int K,
+                            int8_t *X8, uint16_t *s_x, void *stream);
+
+/* Bytes of scratch workspace qoq_w4a8_gemm needs for this shape.
+ *
+ * The GEMM splits the K loop of some output tiles across SMs so that every
+ * SM streams the same number of weight bytes. The INT32 partial sums of a
+ * split tile meet in this workspace. The sum is exact in any order.
+ * Layout: the first 4096 bytes hold arrival counters (the same region for
+ * every shape); the partial tiles follow. Rules:
+ *   - a fresh workspace must be zero-filled once before its first use;
+ *   - every completed call leaves the counters at zero again, so one
+ *     workspace serves any sequence of shapes on one stream;
+ *   - after a call that returned QOQ_ERR_TIMEOUT from qoq_device_error,
+ *     zero-fill the workspace again.
+ * Returns 0 for an invalid shape. */
+QOQ_API size_t qoq_gemm_workspace_bytes(int M, int N, int K, int group_size);
+
+/* The W4A8 GEMM with its epilogue.
+ *
+ * Sources: "QServe Guide: W4A8KV4 Quantization for LLM Serving", The
+ * Architecture, subsection 2, and Deep Dive, subsection 1, the output
+ * rescaling equation. For every m < M and n < N:
+ *     W8hat[n][k] = q[n][k]*s_g[g][n] - zs[g][n]            (INT8)
+ *     acc[m][n]   = sum_k X8[m][k] * W8hat[n][k]           (INT32, exact)
+ *     Y[m][n]     = fp16( ((float)acc * (float)s_x[m]) * (float)s_c[n] )
+ * The FP32 products are rounded in that order, with no fused multiply-add.
+ *
+ *   X8, s_x      device, from qoq_quant_act_per_token.
+ *   Wp, s_c, s_g, zs
+ *                device, from qoq_pack_weights with the same N, K and
+ *                group_size.
+ *   Y            device, uint16_t [M][N] FP16 bits, written.
+ *   acc_dbg      device int32_t [M][N], or NULL. When given, the raw INT32
+ *                accumulators are written there too (used for parity tests).
+ *   workspace    device, at least qoq_gemm_workspace_bytes(M, N, K,
+ *                group_size) bytes, prepared as described above. Two calls
+ *                that may run at the same time must not share a workspace.
+ *   workspace_bytes  the size of that buffer. A smaller size is rejected.
+ * The kernel's internal waits are bounded. If one runs out, the kernel
+ * stops early and sets a device error flag; qoq_device_error reports it.
+ */
+QOQ_API int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x,
+                  const uint8_t *Wp, const uint16_t *s_c,
+                  const uint8_t *s_g, const uint8_t *zs,
+                  int M, int N, int K, int group_size,
+                  uint16_t *Y, int32_t *acc_dbg,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* Expands the packed codes to the INT8 weights the GEMM multiplies,
+ * W8hat[n][k] = q*s_g - zs. It runs the same device routine as the GEMM's
+ * in-register dequantization. Use it for parity tests and inspection; it is
+ * not on the hot path.
+ *   W8hat  device, int8_t [N][K], written. */
+QOQ_API int qoq_dequant_weights_i8(const uint8_t *Wp, const uint8_t *s_g, const uint8_t *zs,
+                           int N, int K, int group_size, int8_t *W8hat, void *stream);
+
+/* Selects where the GEMM keeps the dequantized weight tile before it feeds
+ * the tensor cores:
+ *   1 (default): tensor memory (TMEM), read by the MMA as its A operand;
+ *   0: shared memory.
+ * The choice applies to later GEMM calls from every thread. Results are
+ * identical either way. Returns QOQ_ERR_INVALID_ARG for other values. */
+QOQ_API int qoq_set_gemm_a_in_tmem(int enable);
+
+/* Synchronizes `stream`, then reads and clears the device error flag of
+ * the current device.
+ *   Returns QOQ_OK when no kernel reported a problem.
+ *   Returns QOQ_ERR_TIMEOUT when a bounded wait in a GEMM ran out. The CUDA
+ *     context stays usable, but the outputs of that call are undefined.
+ *   Returns QOQ_ERR_CUDA when the synchronization itself failed. */
+QOQ_API int qoq_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QOQ_H */

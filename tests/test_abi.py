@@ -1,0 +1,96 @@
+"""The C ABI without a GPU: the library loads, exports exactly what
+include/qoq.h declares, and its host-side checks reject bad arguments
+before touching any device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qoq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w4a8_integer_gemm_b200 import build_lib
+    build_lib.build()
+    import w4a8_integer_gemm_b200 as q
+    return q.lib()
+
+
+def declared():
+    txt = open(HEADER).read()
+    return set(re.findall(r"QOQ_API\s+[\w\s\*]+?\b(qoq_\w+)\s*\(", txt))
+
+
+def test_exports_every_declared_symbol(L):
+    import w4a8_integer_gemm_b200 as q
+    names = declared()
+    assert len(names) == 9
+    for n in names:
+        assert hasattr(L, n), n
+    assert names == set(q.SIGNATURES)
+    # nothing else with C linkage is exported
+    out = os.popen(f"nm -D --defined-only {q.LIB_PATH}").read().split("\n")
+    exported = {l.split()[-1] for l in out if l.strip() and l.split()[-1].startswith("qoq_")}
+    assert exported == names
+
+
+def test_status_strings(L):
+    import w4a8_integer_gemm_b200 as q
+    for s in (0, -1, -2, -3, -4):
+        assert len(q.qoq_status_string(s)) >= 2
+    assert q.qoq_status_string(7) == "unknown status"
+
+
+def test_size_queries(L):
+    import w4a8_integer_gemm_b200 as q
+    assert q.qoq_packed_weight_bytes(14336, 4096) == 14336 * 4096 // 2
+    assert q.qoq_packed_weight_bytes(100, 4096) == 0
+    assert q.qoq_packed_weight_bytes(128, 100) == 0
+    assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 128) > 0
+    assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 64) == 0      # group size not supported
+    assert q.qoq_gemm_workspace_bytes(0, 512, 512, 128) == 0
+    # 4096 bytes of counters, then for each of <= 148 CTAs 2 partial tiles of
+    # BN=16 tokens x 128 channels x int32
+    assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 128) == 4096 + 148 * 2 * 16 * 128 * 4
+    # grid = units when there are fewer units than SMs (4 tiles x 4 K blocks)
+    assert q.qoq_gemm_workspace_bytes(1, 512, 512, 128) == 4096 + 16 * 2 * 16 * 128 * 4
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_invalid_arguments_rejected_on_host(L):
+    A = _fake(0x10000)          # aligned, never dereferenced: checks fail first
+    B = _fake(0x10001)          # misaligned
+    INVALID = -1
+    g = L.qoq_w4a8_gemm
+    ok_args = [A] * 6 + [16, 512, 512, 128, A, None, A, 1 << 30, None]
+
+    def call(**kw):
+        a = list(ok_args)
+        names = ["X8", "s_x", "Wp", "s_c", "s_g", "zs", "M", "N", "K", "G", "Y", "acc", "ws", "wsb", "st"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return g(*a)
+
+    assert call(K=500) == INVALID
+    assert call(K=0) == INVALID
+    assert call(N=500) == INVALID
+    assert call(G=64) == INVALID
+    assert call(M=-1) == INVALID
+    assert call(X8=B) == INVALID
+    assert call(Y=None) == INVALID
+    assert call(ws=None) == INVALID
+    assert call(wsb=16) == INVALID
+    assert call(acc=B) == INVALID
+    assert call(M=0) == 0                        # empty problem: nothing to do
+    assert L.qoq_quant_act_per_token(A, 4, 100, A, A, None) == INVALID
+    assert L.qoq_quant_act_per_token(A, 0, 512, A, A, None) == 0
+    assert L.qoq_pack_weights(A, 512, 512, 100, A, A, A, A, None) == INVALID
+    assert L.qoq_pack_weights(B, 512, 512, 128, A, A, A, A, None) == INVALID
+    assert L.qoq_dequant_weights_i8(A, A, A, 512, 512, 3, A, None) == INVALID
+    assert L.qoq_set_gemm_a_in_tmem(2) == INVALID

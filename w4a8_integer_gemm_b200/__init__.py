@@ -1,1 +1,246 @@
-"""B200-native QoQ W4A8 linear layer: Y = diag(s_x) (X8 W8hat^T) diag(s_c)."""
+"""B200-native QoQ W4A8 linear layer: Y = diag(s_x) (X8 W8hat^T) diag(s_c).
+
+A thin ctypes binding over libqoq.so (include/qoq.h).  Every function here
+has the name of the C entry point it calls and only marshals arguments:
+torch tensors provide device memory and the current CUDA stream, every step
+of the computation runs in the library's sm_100a kernels.  There is no CPU
+fallback: if the shared library is missing or the device is not a B200, the
+calls raise.
+
+    packed = qoq_pack_weights(W_fp32_cuda, group_size)        # offline
+    X8, s_x = qoq_quant_act_per_token(X_fp16_cuda)            # per forward
+    Y = qoq_w4a8_gemm(X8, s_x, packed)                        # per forward
+
+`W4A8Linear` wraps the three for a layer; `w4a8_linear_host` is the end to
+end call a user makes with host tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqoq.so")
+
+QOQ_OK = 0
+QOQ_ERR_INVALID_ARG = -1
+QOQ_ERR_UNSUPPORTED = -2
+QOQ_ERR_CUDA = -3
+QOQ_ERR_TIMEOUT = -4
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+# name -> (restype, argtypes); the exported surface of include/qoq.h
+SIGNATURES = {
+    "qoq_status_string": (ctypes.c_char_p, [_I]),
+    "qoq_packed_weight_bytes": (_SZ, [_I, _I]),
+    "qoq_pack_weights": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "qoq_quant_act_per_token": (_I, [_P, _I, _I, _P, _P, _P]),
+    "qoq_gemm_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "qoq_w4a8_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "qoq_dequant_weights_i8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
+    "qoq_set_gemm_a_in_tmem": (_I, [_I]),
+    "qoq_device_error": (_I, [_P]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class QoQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status} ({qoq_status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libqoq.so.  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"libqoq.so not found at {LIB_PATH}; build it with "
+                    "`python -m w4a8_integer_gemm_b200.build_lib` (there is no CPU fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+        return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(fn: str, status: int):
+    if status != QOQ_OK:
+        raise QoQError(fn, status)
+
+
+def _need(t: torch.Tensor, dtype, name):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+# ------------------------------------------------------------------ ABI ----
+def qoq_status_string(status: int) -> str:
+    return lib().qoq_status_string(int(status)).decode()
+
+
+def qoq_packed_weight_bytes(N: int, K: int) -> int:
+    return int(lib().qoq_packed_weight_bytes(int(N), int(K)))
+
+
+def qoq_gemm_workspace_bytes(M: int, N: int, K: int, group_size: int) -> int:
+    return int(lib().qoq_gemm_workspace_bytes(int(M), int(N), int(K), int(group_size)))
+
+
+def qoq_set_gemm_a_in_tmem(enable: bool) -> None:
+    _check("qoq_set_gemm_a_in_tmem", lib().qoq_set_gemm_a_in_tmem(1 if enable else 0))
+
+
+def qoq_device_error(stream=None) -> int:
+    """QOQ_OK, or QOQ_ERR_TIMEOUT if a GEMM's bounded wait ran out."""
+    return int(lib().qoq_device_error(_stream(stream)))
+
+
+@dataclass
+class PackedWeights:
+    """Output of the offline packer (device tensors, layouts of include/qoq.h)."""
+    Wp: torch.Tensor     # uint8 [N*K/2]  interleaved UINT4 codes
+    s_c: torch.Tensor    # int16 [N]      FP16 bits of the channel scales
+    s_g: torch.Tensor    # uint8 [K/G, N] integer group scales
+    zs: torch.Tensor     # uint8 [K/G, N] zero compensation z*s_g
+    N: int
+    K: int
+    group_size: int
+
+
+def qoq_pack_weights(W: torch.Tensor, group_size: int, out: Optional[PackedWeights] = None,
+                     stream=None) -> PackedWeights:
+    _need(W, torch.float32, "W")
+    N, K = W.shape
+    G = int(group_size)
+    if out is None:
+        dev = W.device
+        nb = qoq_packed_weight_bytes(N, K)
+        ng = K // G if G > 0 and K % G == 0 else 1
+        out = PackedWeights(torch.empty(max(nb, 16), dtype=torch.uint8, device=dev),
+                            torch.empty(N, dtype=torch.int16, device=dev),
+                            torch.empty(ng, N, dtype=torch.uint8, device=dev),
+                            torch.empty(ng, N, dtype=torch.uint8, device=dev), N, K, G)
+    st = lib().qoq_pack_weights(_ptr(W), N, K, G, _ptr(out.Wp), _ptr(out.s_c), _ptr(out.s_g),
+                                _ptr(out.zs), _stream(stream))
+    _check("qoq_pack_weights", st)
+    return out
+
+
+def qoq_quant_act_per_token(X: torch.Tensor, X8: Optional[torch.Tensor] = None,
+                            s_x: Optional[torch.Tensor] = None, stream=None):
+    """X fp16 [M, K] -> (X8 int8 [M, K], s_x int16 [M] FP16 bits)."""
+    _need(X, torch.float16, "X")
+    M, K = X.shape
+    if X8 is None:
+        X8 = torch.empty(M, K, dtype=torch.int8, device=X.device)
+    if s_x is None:
+        s_x = torch.empty(max(M, 8), dtype=torch.int16, device=X.device)
+    st = lib().qoq_quant_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(s_x), _stream(stream))
+    _check("qoq_quant_act_per_token", st)
+    return X8, s_x
+
+
+_ws_cache = {}
+
+
+def gemm_workspace(M: int, N: int, K: int, group_size: int, device) -> torch.Tensor:
+    """A zero-initialised workspace big enough for this shape, cached per
+    device and grown on demand.  The kernels leave its counters at zero, so
+    it is reused across calls on one stream; do not share it between
+    streams that run GEMMs concurrently."""
+    need = qoq_gemm_workspace_bytes(M, N, K, group_size)
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=dev)
+        _ws_cache[key] = ws
+    return ws
+
+
+def qoq_w4a8_gemm(X8: torch.Tensor, s_x: torch.Tensor, packed: PackedWeights,
+                  Y: Optional[torch.Tensor] = None, acc_dbg: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y fp16 [M, N] = fp16(((float)(X8 . W8hat) * s_x) * s_c)."""
+    _need(X8, torch.int8, "X8")
+    M, K = X8.shape
+    if K != packed.K:
+        raise ValueError("K mismatch between X8 and the packed weights")
+    N = packed.N
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float16, device=X8.device)
+    if workspace is None:
+        workspace = gemm_workspace(max(M, 1), N, K, packed.group_size, X8.device)
+    st = lib().qoq_w4a8_gemm(_ptr(X8), _ptr(s_x), _ptr(packed.Wp), _ptr(packed.s_c), _ptr(packed.s_g),
+                             _ptr(packed.zs), M, N, K, packed.group_size, _ptr(Y), _ptr(acc_dbg),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(stream))
+    _check("qoq_w4a8_gemm", st)
+    return Y
+
+
+def qoq_dequant_weights_i8(packed: PackedWeights, out: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(packed.N, packed.K, dtype=torch.int8, device=packed.Wp.device)
+    st = lib().qoq_dequant_weights_i8(_ptr(packed.Wp), _ptr(packed.s_g), _ptr(packed.zs), packed.N,
+                                      packed.K, packed.group_size, _ptr(out), _stream(stream))
+    _check("qoq_dequant_weights_i8", st)
+    return out
+
+
+# ---------------------------------------------------------------- layer ----
+class W4A8Linear:
+    """A linear layer y = x W^T with QoQ W4A8 weights resident on the GPU."""
+
+    def __init__(self, weight_fp32: torch.Tensor, group_size: int = 128):
+        W = weight_fp32.to(device="cuda", dtype=torch.float32).contiguous()
+        self.packed = qoq_pack_weights(W, group_size)
+        self.in_features = W.shape[1]
+        self.out_features = W.shape[0]
+
+    def __call__(self, x_fp16: torch.Tensor, stream=None) -> torch.Tensor:
+        X8, s_x = qoq_quant_act_per_token(x_fp16, stream=stream)
+        return qoq_w4a8_gemm(X8, s_x, self.packed, stream=stream)
+
+
+def w4a8_linear_host(x_host: torch.Tensor, layer: W4A8Linear, y_host: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """End-to-end call from host memory: copy X (fp16, ideally pinned) to the
+    device, quantize it, run the GEMM, copy Y back; returns the host Y."""
+    s = stream or torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        x = x_host.to("cuda", non_blocking=True)
+        y = layer(x, stream=s)
+        if y_host is None:
+            y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        y_host.copy_(y, non_blocking=True)
+    s.synchronize()
+    return y_host

@@ -1,0 +1,152 @@
+// qoq_api.cu -- the extern "C" entry points declared in include/qoq.h:
+// argument validation on the host, then one launch per call.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "../../include/qoq.h"
+#include "qoq_internal.h"
+
+namespace {
+
+std::atomic<int> g_a_in_tmem{1};
+
+constexpr int kMaxK = 65536;
+constexpr int kMaxN = 1 << 20;
+constexpr int kMaxM = 1 << 24;
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool valid_nk(int N, int K)
+{
+    return N >= 128 && N <= kMaxN && N % 128 == 0 && K >= 128 && K <= kMaxK && K % 128 == 0;
+}
+
+bool valid_group(int K, int G)
+{
+    return G == 128 || G == K;
+}
+
+// Compute capability 10.0 check for the current device, cached per device.
+int check_device()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return QOQ_ERR_UNSUPPORTED;
+    int c = cache[dev].load();
+    if (c == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return QOQ_ERR_CUDA;
+        c = (major == 10 && minor == 0) ? 1 : -1;
+        cache[dev].store(c);
+    }
+    return c == 1 ? QOQ_OK : QOQ_ERR_UNSUPPORTED;
+}
+
+int from_cuda(cudaError_t e)
+{
+    return e == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *qoq_status_string(int status)
+{
+    switch (status) {
+    case QOQ_OK: return "ok";
+    case QOQ_ERR_INVALID_ARG: return "invalid argument (shape, alignment, pointer or workspace size)";
+    case QOQ_ERR_UNSUPPORTED: return "unsupported device (needs compute capability 10.0, sm_100a)";
+    case QOQ_ERR_CUDA: return "CUDA runtime or launch error";
+    case QOQ_ERR_TIMEOUT: return "a bounded device wait ran out; outputs of that call are undefined";
+    default: return "unknown status";
+    }
+}
+
+size_t qoq_packed_weight_bytes(int N, int K)
+{
+    if (!valid_nk(N, K)) return 0;
+    return (size_t)N * (size_t)K / 2;
+}
+
+int qoq_pack_weights(const float *W, int N, int K, int group_size, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g,
+                     uint8_t *zs, void *stream)
+{
+    if (!valid_nk(N, K) || !valid_group(K, group_size)) return QOQ_ERR_INVALID_ARG;
+    if (!W || !Wp || !s_c || !s_g || !zs) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) || !aligned16(zs))
+        return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(qoq::launch_pack(W, N, K, group_size, Wp, s_c, s_g, zs, (cudaStream_t)stream));
+}
+
+int qoq_quant_act_per_token(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, void *stream)
+{
+    if (M < 0 || M > kMaxM || K < 128 || K > kMaxK || K % 128 != 0) return QOQ_ERR_INVALID_ARG;
+    if (M == 0) return QOQ_OK;
+    if (!X || !X8 || !s_x || !aligned16(X) || !aligned16(X8) || !aligned16(s_x)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(qoq::launch_act_quant(X, M, K, X8, s_x, (cudaStream_t)stream));
+}
+
+size_t qoq_gemm_workspace_bytes(int M, int N, int K, int group_size)
+{
+    if (M < 1 || M > kMaxM || !valid_nk(N, K) || !valid_group(K, group_size)) return 0;
+    return qoq::gemm_workspace_bytes(M, N, K);
+}
+
+int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
+                  const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int group_size, uint16_t *Y,
+                  int32_t *acc_dbg, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (M < 0 || M > kMaxM || !valid_nk(N, K) || !valid_group(K, group_size)) return QOQ_ERR_INVALID_ARG;
+    if (M == 0) return QOQ_OK;
+    if (!X8 || !s_x || !Wp || !s_c || !s_g || !zs || !Y || !workspace) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(X8) || !aligned16(s_x) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) ||
+        !aligned16(zs) || !aligned16(Y) || !aligned16(workspace) || (acc_dbg && !aligned16(acc_dbg)))
+        return QOQ_ERR_INVALID_ARG;
+    if (workspace_bytes < qoq::gemm_workspace_bytes(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    int tmap_status = 0;
+    cudaError_t e = qoq::launch_gemm(X8, s_x, Wp, s_c, s_g, zs, M, N, K, group_size, Y, acc_dbg, workspace,
+                                     g_a_in_tmem.load() != 0, (cudaStream_t)stream, &tmap_status);
+    if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
+int qoq_dequant_weights_i8(const uint8_t *Wp, const uint8_t *s_g, const uint8_t *zs, int N, int K, int group_size,
+                           int8_t *W8hat, void *stream)
+{
+    if (!valid_nk(N, K) || !valid_group(K, group_size)) return QOQ_ERR_INVALID_ARG;
+    if (!Wp || !s_g || !zs || !W8hat || !aligned16(Wp) || !aligned16(W8hat)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(qoq::launch_dequant(Wp, s_g, zs, N, K, group_size, W8hat, (cudaStream_t)stream));
+}
+
+int qoq_set_gemm_a_in_tmem(int enable)
+{
+    if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;
+    g_a_in_tmem.store(enable);
+    return QOQ_OK;
+}
+
+int qoq_device_error(void *stream)
+{
+    int v = 0;
+    if (qoq::read_and_clear_device_error((cudaStream_t)stream, &v) != cudaSuccess) return QOQ_ERR_CUDA;
+    return v ? QOQ_ERR_TIMEOUT : QOQ_OK;
+}
+
+}  // extern "C"

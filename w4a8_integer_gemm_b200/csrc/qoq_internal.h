@@ -1,0 +1,45 @@
+// qoq_internal.h -- host-side launchers behind the C ABI (C++ linkage, not
+// exported).  Arguments have been validated by the caller (qoq_api.cu).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace qoq {
+
+// Upper bound on the persistent GEMM grid (B200 has 148 SMs); also sizes
+// the split-tile workspace, so the workspace size does not depend on the
+// device a query runs on.
+constexpr int kMaxCtas = 148;
+
+// The split-tile counters (kMaxCtas x 4 int32) occupy this many bytes at the
+// start of every GEMM workspace; the INT32 partial tiles follow.
+constexpr size_t kCounterBytes = 4096;
+static_assert(kMaxCtas * 4 * 4 <= kCounterBytes, "counter region");
+
+cudaError_t launch_pack(const float *W, int N, int K, int G, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g,
+                        uint8_t *zs, cudaStream_t stream);
+
+cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x,
+                             cudaStream_t stream);
+
+cudaError_t launch_dequant(const uint8_t *Wp, const uint8_t *s_g, const uint8_t *zs, int N, int K, int G,
+                           int8_t *W8hat, cudaStream_t stream);
+
+// Tile width along M (tokens) the GEMM uses for a given M.
+int gemm_block_n(int M);
+
+size_t gemm_workspace_bytes(int M, int N, int K);
+
+// Returns cudaSuccess or the launch / tensor-map error.  `tmap_status`
+// receives the driver status of the tensor-map encode (0 on success).
+cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
+                        const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
+                        int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream,
+                        int *tmap_status);
+
+// Device error flag of the current device: read and clear (synchronous).
+cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value);
+
+}  // namespace qoq

@@ -1,0 +1,254 @@
+// qoq_kernels.cu -- the offline weight packer, the per-token activation
+// quantizer and the INT8 weight expansion used for inspection.
+//
+// Sources (by page title):
+//   "QServe: Low Bit Width Does Not Guarantee High Throughput", section 4,
+//       stage-1 equation (per-channel symmetric INT8 in [-119,119]) and
+//       stage-2 equation (group UINT4 with integer scale and zero).
+//   "QServe: W4A8KV4 Quantization and System Co-design for Efficient LLM
+//       Serving" (paper card), Key points: FP16 per-channel scales.
+//   "QServe Guide: W4A8KV4 Quantization for LLM Serving", Deep Dive,
+//       subsection 1: per-token activation equation.
+#include <cuda_fp16.h>
+
+#include "qoq_internal.h"
+#include "qoq_layout.cuh"
+
+namespace qoq {
+namespace {
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h)
+{
+    return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ uint16_t float_to_half_bits(float f)
+{
+    return __half_as_ushort(__float2half_rn(f));
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int warp_min_i(int v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int warp_max_i(int v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Stage 1 for one value: clamp(round(w / sc), -119, 119), IEEE division,
+// round half to even; a zero scale quantizes to zero.
+__device__ __forceinline__ int stage1(float w, float sc)
+{
+    if (sc == 0.0f) return 0;
+    return (int)fminf(fmaxf(rintf(__fdiv_rn(w, sc)), -119.0f), 119.0f);
+}
+
+// Stage 2 code: clamp(round(w8 / s_g) + z, 0, 15).  w8 in [-119,119] and
+// s_g in [1,16]: the FP32 quotient is within 2^-20 of the exact rational,
+// non-tie quotients lie at least 1/32 from a half, and ties are exact, so
+// rintf gives the exact round-half-to-even of the rational.
+__device__ __forceinline__ uint32_t stage2_code(int w8, float sgf, int z)
+{
+    const int v = (int)rintf(__fdiv_rn((float)w8, sgf)) + z;
+    return (uint32_t)min(max(v, 0), 15);
+}
+
+// ------------------------------------------------------------ packer --
+// One warp per output channel n.  Lane l covers k = kc + 4l .. kc + 4l + 3
+// of each 128-wide chunk kc.
+__global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, int N, int K, int G,
+                                                   uint8_t *__restrict__ Wp, uint16_t *__restrict__ s_c,
+                                                   uint8_t *__restrict__ s_g, uint8_t *__restrict__ zs)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = blockIdx.x * 8 + warp;
+    if (n >= N) return;
+    const float *w = W + (size_t)n * K;
+
+    float amax = 0.0f;
+    for (int k = lane * 4; k < K; k += 128) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(w + k));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    amax = warp_max(amax);
+    const uint16_t sch = float_to_half_bits(__fdiv_rn(amax, 119.0f));
+    const float sc = half_bits_to_float(sch);
+    if (lane == 0) s_c[n] = sch;
+
+    const int p = n / kPanelRows, rr = n % kPanelRows;
+    for (int g = 0; g < K / G; ++g) {
+        const int k_lo = g * G, k_hi = k_lo + G;
+        int mn = 0, mx = 0;
+        for (int k = k_lo + lane * 4; k < k_hi; k += 128) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(w + k));
+            const int a0 = stage1(v.x, sc), a1 = stage1(v.y, sc), a2 = stage1(v.z, sc), a3 = stage1(v.w, sc);
+            mn = min(mn, min(min(a0, a1), min(a2, a3)));
+            mx = max(mx, max(max(a0, a1), max(a2, a3)));
+        }
+        mn = warp_min_i(mn);
+        mx = warp_max_i(mx);
+        const int sg = max(1, (mx - mn + 14) / 15);
+        const float sgf = (float)sg;
+        const int z = (int)rintf(__fdiv_rn((float)(-mn), sgf));
+        if (lane == 0) {
+            s_g[(size_t)g * N + n] = (uint8_t)sg;
+            zs[(size_t)g * N + n] = (uint8_t)(z * sg);
+        }
+        for (int kc = k_lo; kc < k_hi; kc += 128) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(w + kc + lane * 4));
+            const uint32_t mine = stage2_code(stage1(v.x, sc), sgf, z) | (stage2_code(stage1(v.y, sc), sgf, z) << 8) |
+                                  (stage2_code(stage1(v.z, sc), sgf, z) << 16) |
+                                  (stage2_code(stage1(v.w, sc), sgf, z) << 24);
+            // lanes l and l+4 of each group of 8 fill the low and high
+            // nibbles of the same packed word
+            const uint32_t partner = __shfl_down_sync(0xffffffffu, mine, 4);
+            if ((lane & 7) < 4) {
+                const int slab = lane >> 3, word = lane & 7;
+                uint8_t *dst = Wp + chunk_offset(p, kc / kBlockK, K) + slab * kSlabBytes + rr * 16 + word * 4;
+                *reinterpret_cast<uint32_t *>(dst) = mine | (partner << 4);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------- activation quant --
+constexpr int kActThreads = 256;
+constexpr int kActCache = 12;  // 16-byte vectors per thread kept in registers (K <= 24576)
+
+__device__ __forceinline__ float absmax8(const uint4 &v)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m = fmaxf(m, fabsf(half_bits_to_float((uint16_t)(w[i] & 0xFFFFu))));
+        m = fmaxf(m, fabsf(half_bits_to_float((uint16_t)(w[i] >> 16))));
+    }
+    return m;
+}
+
+__device__ __forceinline__ int quant_x(float x, float sx)
+{
+    if (sx == 0.0f) return 0;
+    return (int)fminf(fmaxf(rintf(__fdiv_rn(x, sx)), -128.0f), 127.0f);
+}
+
+__device__ __forceinline__ uint2 quant8(const uint4 &v, float sx)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[2] = {0, 0};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = (uint32_t)quant_x(half_bits_to_float((uint16_t)(w[i] & 0xFFFFu)), sx) & 0xFFu;
+        const uint32_t hi = (uint32_t)quant_x(half_bits_to_float((uint16_t)(w[i] >> 16)), sx) & 0xFFu;
+        o[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
+    }
+    return make_uint2(o[0], o[1]);
+}
+
+// One CTA per token row: read the row once (kept in registers up to
+// kActCache vectors per thread), reduce max|x|, then quantize.
+__global__ void __launch_bounds__(kActThreads) act_quant_kernel(const uint16_t *__restrict__ X, int K,
+                                                                 int8_t *__restrict__ X8,
+                                                                 uint16_t *__restrict__ s_x)
+{
+    __shared__ float red[kActThreads / 32];
+    const int m = blockIdx.x;
+    const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)m * K);
+    uint2 *out = reinterpret_cast<uint2 *>(X8 + (size_t)m * K);
+    const int nvec = K / 8;
+    uint4 cache[kActCache];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kActCache; ++i) {
+        const int idx = threadIdx.x + i * kActThreads;
+        if (idx < nvec) {
+            cache[i] = __ldcs(row + idx);
+            amax = fmaxf(amax, absmax8(cache[i]));
+        }
+    }
+    for (int idx = threadIdx.x + kActCache * kActThreads; idx < nvec; idx += kActThreads)
+        amax = fmaxf(amax, absmax8(__ldg(row + idx)));
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < kActThreads / 32 ? red[threadIdx.x] : 0.0f;
+        v = warp_max(v);
+        if (threadIdx.x == 0) red[0] = v;
+    }
+    __syncthreads();
+    amax = red[0];
+    const uint16_t sxh = float_to_half_bits(__fdiv_rn(amax, 127.0f));
+    const float sx = half_bits_to_float(sxh);
+    if (threadIdx.x == 0) s_x[m] = sxh;
+#pragma unroll
+    for (int i = 0; i < kActCache; ++i) {
+        const int idx = threadIdx.x + i * kActThreads;
+        if (idx < nvec) out[idx] = quant8(cache[i], sx);
+    }
+    for (int idx = threadIdx.x + kActCache * kActThreads; idx < nvec; idx += kActThreads)
+        out[idx] = quant8(__ldg(row + idx), sx);
+}
+
+// ------------------------------------------------- INT8 weight expand --
+// One thread per (channel n, 32-wide K slice): the GEMM's dequant routine
+// on one 16-byte row slice, written out as 32 INT8 weights.
+__global__ void dequant_kernel(const uint8_t *__restrict__ Wp, const uint8_t *__restrict__ s_g,
+                               const uint8_t *__restrict__ zs, int N, int K, int G, int8_t *__restrict__ out)
+{
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int slices = K / kSlabK;
+    if (idx >= (size_t)N * slices) return;
+    const int n = (int)(idx / slices);
+    const int k0 = (int)(idx % slices) * kSlabK;
+    const uint4 v = *reinterpret_cast<const uint4 *>(Wp + chunk_offset(n / kPanelRows, k0 / kBlockK, K) +
+                                                     ((k0 % kBlockK) / kSlabK) * kSlabBytes + (n % kPanelRows) * 16);
+    const int g = k0 / G;
+    const uint32_t sg = s_g[(size_t)g * N + n];
+    const uint32_t bias = zero_comp_bias(zs[(size_t)g * N + n]);
+    uint32_t w8[8];
+    dequant_slab(v, sg, bias, w8);
+    uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)n * K + k0);
+    dst[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+    dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const float *W, int N, int K, int G, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g, uint8_t *zs,
+                        cudaStream_t stream)
+{
+    pack_kernel<<<(N + 7) / 8, 256, 0, stream>>>(W, N, K, G, Wp, s_c, s_g, zs);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, cudaStream_t stream)
+{
+    act_quant_kernel<<<M, kActThreads, 0, stream>>>(X, K, X8, s_x);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const uint8_t *Wp, const uint8_t *s_g, const uint8_t *zs, int N, int K, int G,
+                           int8_t *W8hat, cudaStream_t stream)
+{
+    const size_t threads = (size_t)N * (K / kSlabK);
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    dequant_kernel<<<blocks, 256, 0, stream>>>(Wp, s_g, zs, N, K, G, W8hat);
+    return cudaGetLastError();
+}
+
+}  // namespace qoq
