@@ -102,6 +102,14 @@ def max_over_ranks(x: float, dist) -> float:
     return float(t.item())
 
 
+def aggregate(ops_per_rank: float, ms_this_rank: float, world: int, dist):
+    """Whole-job throughput of `world` replicas that each did ops_per_rank
+    operations: the step time is the slowest rank's (max over ranks), the
+    value is all ranks' operations over that time, in TOPS."""
+    ms = max_over_ranks(ms_this_rank, dist)
+    return ms, world * ops_per_rank / (ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- clocks --
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
@@ -244,8 +252,7 @@ def run_ours(args, rank, world, local, dist):
         tot_ms += aq_ms + gm_ms
         g_ms += gm_ms
         g_bytes += byt
-    ms_step = max_over_ranks(tot_ms, dist)
-    value = world * tot_ops / (ms_step * 1e-3) / 1e12
+    ms_step, value = aggregate(tot_ops, tot_ms, world, dist)
 
     # roofline of the dominant kernel (the GEMM), averaged per launch
     n_hbm = sum(1 for p in per if p["bound"] == "hbm")

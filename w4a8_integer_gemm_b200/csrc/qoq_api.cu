@@ -142,6 +142,16 @@ int qoq_set_gemm_a_in_tmem(int enable)
     return QOQ_OK;
 }
 
+#ifdef QOQ_TRACE
+// Trace builds only: a device buffer of [ctas][256] uint64 that later GEMM
+// launches fill with global-timer marks.
+__attribute__((visibility("default"))) int qoq_debug_set_trace(void *buf)
+{
+    qoq::g_trace_buffer = reinterpret_cast<unsigned long long *>(buf);
+    return QOQ_OK;
+}
+#endif
+
 int qoq_device_error(void *stream)
 {
     int v = 0;

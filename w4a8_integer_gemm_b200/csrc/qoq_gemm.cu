@@ -71,8 +71,25 @@ struct GemmArgs {
     int M, N, K, G;
     int m_tiles, ks;        // ks = K / 128 stages per tile
     long long total;        // tiles * ks units
-    unsigned long long timeout_ns;
+    unsigned long long timeout_ns;  // longest any one wait may last
+#ifdef QOQ_TRACE
+    unsigned long long *trace;  // [cta][256] global-timer marks (trace builds only)
+#endif
 };
+
+// Timeline marks for the trace build (compiled out otherwise).
+#ifdef QOQ_TRACE
+// slot 255 holds the CTA's global-timer entry time; the other marks are SM
+// clock cycles since the CTA's entry
+#define QOQ_MARK(idx)                                                                              \
+    do {                                                                                           \
+        if (a.trace) a.trace[(size_t)blockIdx.x * 256 + (idx)] = clock64() - trace_t0;             \
+    } while (0)
+#else
+#define QOQ_MARK(idx) \
+    do {              \
+    } while (0)
+#endif
 
 __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
 {
@@ -87,7 +104,7 @@ struct GemmCfg {
     static constexpr int kStageBytes = ((kXBytes + kWBytes + kTabBytes + 1023) / 1024) * 1024;
     static constexpr int kABytes = A_TMEM ? 0 : 128 * 128;  // dequantized tile in smem
     static constexpr int kBarOff = STAGES * kStageBytes + ASTAGES * kABytes;
-    static constexpr int kNumBars = 2 * STAGES + 2 * ASTAGES + 3;
+    static constexpr int kNumBars = 3 * STAGES + 2 * ASTAGES + 3;
     static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
     // at least ~120 KB so that exactly one CTA (and one TMEM allocation)
     // lives on each SM; +1024 for manual alignment of the dynamic base
@@ -132,6 +149,21 @@ __device__ __forceinline__ uint16_t scale_to_half(int32_t acc, float sx, float s
     return __half_as_ushort(__float2half_rn(y));
 }
 
+// FP16 outputs (and optionally the INT32 accumulators) of 16 consecutive
+// tokens m0.. for channel n; tokens beyond M are skipped.
+__device__ __forceinline__ void store_outputs(const GemmArgs &a, int m0, int n, float sc, const int32_t *acc)
+{
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const int m = m0 + q;
+        if (m < a.M) {
+            const float sx = half_bits_to_float(__ldg(a.s_x + m));
+            a.Y[(size_t)m * a.N + n] = scale_to_half(acc[q], sx, sc);
+            if (a.acc_dbg) a.acc_dbg[(size_t)m * a.N + n] = acc[q];
+        }
+    }
+}
+
 template <int BN, int STAGES, int ASTAGES, bool A_TMEM>
 __global__ void __launch_bounds__(320, 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs a)
@@ -141,11 +173,14 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar0 = sbase + C::kBarOff;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-    auto afull_bar = [&](int t) { return bar0 + 8u * (2 * STAGES + t); };
-    auto aempty_bar = [&](int t) { return bar0 + 8u * (2 * STAGES + ASTAGES + t); };
-    const uint32_t accfull_bar = bar0 + 8u * (2 * STAGES + 2 * ASTAGES);
+    // per ring slot: fullw (weights + tables landed), fullx (X8 tile landed),
+    // empty (dequant warps and the MMA are done with the slot)
+    auto fullw_bar = [&](int s) { return bar0 + 8u * s; };
+    auto fullx_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+    auto afull_bar = [&](int t) { return bar0 + 8u * (3 * STAGES + t); };
+    auto aempty_bar = [&](int t) { return bar0 + 8u * (3 * STAGES + ASTAGES + t); };
+    const uint32_t accfull_bar = bar0 + 8u * (3 * STAGES + 2 * ASTAGES);
     const uint32_t accempty_bar = accfull_bar + 8u;
     const uint32_t mmadone_bar = accfull_bar + 16u;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kNumBars * 8);
@@ -154,9 +189,15 @@ __global__ void __launch_bounds__(320, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+#ifdef QOQ_TRACE
+    const long long trace_t0 = clock64();
+    if (threadIdx.x == 0 && a.trace) a.trace[(size_t)blockIdx.x * 256 + 255] = global_timer_ns();
+#endif
     if (threadIdx.x == 0) {
+        QOQ_MARK(0);
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
+            mbar_init(fullw_bar(s), 1);
+            mbar_init(fullx_bar(s), 1);
             mbar_init(empty_bar(s), 1 + 4);  // MMA commit + 4 dequant warps
         }
         for (int t = 0; t < ASTAGES; ++t) {
@@ -178,7 +219,10 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const uint64_t deadline = global_timer_ns() + a.timeout_ns;
+    if (threadIdx.x == 0) QOQ_MARK(1);
+    int trace_j = 0;  // per-role stage counter for the timeline marks
+    (void)trace_j;
+    const uint64_t deadline = a.timeout_ns;  // budget of any single wait
 
     const long long P = gridDim.x;
     const long long T = a.total;
@@ -189,14 +233,34 @@ __global__ void __launch_bounds__(320, 1)
     // ring slots the producer has filled, and the phase parity of each
     // slot's latest fill (drained on the way out of an aborted CTA)
     uint32_t issued = 0, issued_par = 0;
+    int issued_x_none = 0;  // set when the producer stopped before any X8 load
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            const uint32_t tx = C::kXBytes + C::kWBytes + C::kTabBytes;
             bool ok = true;
+            // The X8 tiles come from the kernel that precedes this one in the
+            // stream (programmatic dependent launch): the weights of the first
+            // STAGES slots stream in before that kernel has finished, the X8
+            // loads of those slots are issued once it has.
+            int n_issued = 0;
+            bool x_ready = false;
+            int pend_kb[STAGES], pend_m[STAGES];
+            auto load_x = [&](int slot, int kb, int m_tile) {
+                mbar_arrive_expect_tx(fullx_bar(slot), C::kXBytes);
+                tma_load_2d(sbase + slot * C::kStageBytes, &tmap_x, kb * kBlockK, m_tile * BN, fullx_bar(slot));
+            };
+            auto release_x = [&]() {
+                grid_dependency_wait();
+                QOQ_MARK(144);
+                x_ready = true;
+                for (int j = 0; j < n_issued; ++j) {
+                    load_x(j, pend_kb[j], pend_m[j]);
+                    if (j < 16) QOQ_MARK(160 + j);
+                }
+            };
             for (long long i = i_begin; i < i_end && ok;) {
                 const long long t = i / ks;
                 const int ks0 = (int)(i - t * ks);
@@ -204,18 +268,30 @@ __global__ void __launch_bounds__(320, 1)
                 const int m_tile = (int)(t % a.m_tiles);
                 const int n_tile = (int)(t / a.m_tiles);
                 for (int kb = ks0; kb < ks1; ++kb) {
+                    if (!x_ready && n_issued == STAGES) release_x();  // every slot waits for X8
+                    if (trace_j < 8) QOQ_MARK(216 + trace_j);
                     if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, deadline)) {
                         ok = false;
                         break;
                     }
                     const uint32_t st = sbase + s * C::kStageBytes;
                     const int g = (kb * kBlockK) / a.G;
-                    mbar_arrive_expect_tx(full_bar(s), tx);
-                    tma_load_2d(st, &tmap_x, kb * kBlockK, m_tile * BN, full_bar(s));
-                    bulk_load(st + C::kXBytes, a.Wp + chunk_offset(n_tile, kb, a.K), C::kWBytes, full_bar(s));
+                    if (trace_j < 16) QOQ_MARK(180 + trace_j);
+                    mbar_arrive_expect_tx(fullw_bar(s), C::kWBytes + C::kTabBytes);
+                    bulk_load(st + C::kXBytes, a.Wp + chunk_offset(n_tile, kb, a.K), C::kWBytes, fullw_bar(s));
+                    if (trace_j < 16) QOQ_MARK(200 + trace_j);
                     const size_t toff = (size_t)g * a.N + (size_t)n_tile * kPanelRows;
-                    bulk_load(st + C::kXBytes + C::kWBytes, a.s_g + toff, 128, full_bar(s));
-                    bulk_load(st + C::kXBytes + C::kWBytes + 128, a.zs + toff, 128, full_bar(s));
+                    bulk_load(st + C::kXBytes + C::kWBytes, a.s_g + toff, 128, fullw_bar(s));
+                    bulk_load(st + C::kXBytes + C::kWBytes + 128, a.zs + toff, 128, fullw_bar(s));
+                    if (trace_j < 32) QOQ_MARK(16 + trace_j);
+                    ++trace_j;
+                    if (x_ready) {
+                        load_x(s, kb, m_tile);
+                    } else {
+                        pend_kb[n_issued] = kb;
+                        pend_m[n_issued] = m_tile;
+                        ++n_issued;
+                    }
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) {
@@ -225,6 +301,8 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 i = t * ks + ks1;
             }
+            if (ok && !x_ready) release_x();
+            if (!x_ready) issued_x_none = 1;
         }
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer --
@@ -240,11 +318,17 @@ __global__ void __launch_bounds__(320, 1)
                 if (!wait_bounded(accempty_bar, accph ^ 1u, abort_flag, deadline)) break;
                 tc_fence_after();
                 for (int kb = ks0; kb < ks1; ++kb) {
-                    if (!wait_bounded(full_bar(s), ph, abort_flag, deadline) ||
-                        !wait_bounded(afull_bar(ta), aph, abort_flag, deadline)) {
+                    if (trace_j < 8) QOQ_MARK(224 + trace_j);
+                    if (!wait_bounded(fullx_bar(s), ph, abort_flag, deadline)) {
                         ok = false;
                         break;
                     }
+                    if (trace_j < 8) QOQ_MARK(232 + trace_j);
+                    if (!wait_bounded(afull_bar(ta), aph, abort_flag, deadline)) {
+                        ok = false;
+                        break;
+                    }
+                    if (trace_j < 8) QOQ_MARK(240 + trace_j);
                     tc_fence_after();
                     const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kStageBytes);
 #pragma unroll
@@ -258,8 +342,11 @@ __global__ void __launch_bounds__(320, 1)
                             mma_i8_ss(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, acc);
                         }
                     }
+                    if (trace_j < 8) QOQ_MARK(248 + trace_j);
                     mma_commit(empty_bar(s));
                     mma_commit(aempty_bar(ta));
+                    if (trace_j < 32) QOQ_MARK(80 + trace_j);
+                    ++trace_j;
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -290,10 +377,11 @@ __global__ void __launch_bounds__(320, 1)
             const int ks0 = (int)(i - t * ks);
             const int ks1 = (int)min((long long)ks, i_end - t * ks);
             for (int kb = ks0; kb < ks1; ++kb) {
-                if (!wait_bounded(full_bar(s), ph, abort_flag, deadline)) {
+                if (!wait_bounded(fullw_bar(s), ph, abort_flag, deadline)) {
                     ok = false;
                     break;
                 }
+                if (warp == 2 && lane == 0 && trace_j < 32) QOQ_MARK(112 + trace_j);
                 const uint8_t *st = smem + s * C::kStageBytes;
                 const uint8_t *sw = st + C::kXBytes;
                 uint4 v[4];
@@ -326,6 +414,8 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(afull_bar(ta));
+                if (warp == 2 && lane == 0 && trace_j < 32) QOQ_MARK(48 + trace_j);
+                ++trace_j;
                 if (++s == STAGES) {
                     s = 0;
                     ph ^= 1u;
@@ -344,6 +434,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
         uint32_t accph = 0;
         const long long first_tile = i_begin / ks;
+        grid_dependency_wait();  // s_x comes from the preceding kernel
         for (long long i = i_begin; i < i_end;) {
             const long long t = i / ks;
             const int ks0 = (int)(i - t * ks);
@@ -352,38 +443,36 @@ __global__ void __launch_bounds__(320, 1)
             const int n_tile = (int)(t / a.m_tiles);
             const int n = n_tile * kPanelRows + r;
             const int m0 = m_tile * BN;
+            const int live = min(BN, a.M - m0);      // token columns that exist
+            const int nchunks = (live + 15) >> 4;     // 16-column chunks holding them
             const bool partial = !(ks0 == 0 && ks1 == ks);
             if (!wait_bounded(accfull_bar, accph, abort_flag, deadline)) break;
+            if (warp == 6 && lane == 0 && trace_j < 4) QOQ_MARK(145 + trace_j);
             tc_fence_after();
             if (!partial) {
                 const float sc = half_bits_to_float(a.s_c[n]);
 #pragma unroll 1
-                for (int cc = 0; cc < BN / 16; ++cc) {
+                for (int cc = 0; cc < nchunks; ++cc) {
                     uint32_t v[16];
                     tmem_ld16(trow + cc * 16, v);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int m = m0 + cc * 16 + q;
-                        if (m < a.M) {
-                            const int32_t acc = (int32_t)v[q];
-                            const float sx = half_bits_to_float(__ldg(a.s_x + m));
-                            a.Y[(size_t)m * a.N + n] = scale_to_half(acc, sx, sc);
-                            if (a.acc_dbg) a.acc_dbg[(size_t)m * a.N + n] = acc;
-                        }
-                    }
+                    store_outputs(a, m0 + cc * 16, n, sc, reinterpret_cast<const int32_t *>(v));
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(accempty_bar);
             } else {
+                // Partial tile: 16 consecutive columns of one channel are 64
+                // contiguous bytes, [chunk][channel][16] per slot.
                 const int slot = (t == first_tile) ? 0 : 1;
-                int32_t *part = a.ws_part + ((size_t)(cta * 2 + slot) * BN) * kPanelRows;
+                int4 *part = reinterpret_cast<int4 *>(a.ws_part + (size_t)(cta * 2 + slot) * BN * kPanelRows);
 #pragma unroll 1
-                for (int cc = 0; cc < BN / 16; ++cc) {
+                for (int cc = 0; cc < nchunks; ++cc) {
                     uint32_t v[16];
                     tmem_ld16(trow + cc * 16, v);
+                    int4 *dst = part + ((size_t)cc * kPanelRows + r) * 4;
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) part[(size_t)(cc * 16 + q) * kPanelRows + r] = (int32_t)v[q];
+                    for (int j = 0; j < 4; ++j)
+                        dst[j] = make_int4((int)v[4 * j], (int)v[4 * j + 1], (int)v[4 * j + 2], (int)v[4 * j + 3]);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -403,22 +492,50 @@ __global__ void __launch_bounds__(320, 1)
                 if (last) {
                     __threadfence();
                     const float sc = half_bits_to_float(a.s_c[n]);
+                    const int nc = (int)(c_hi - c_lo + 1);
 #pragma unroll 1
-                    for (int col = 0; col < BN; ++col) {
-                        const int m = m0 + col;
-                        if (m >= a.M) break;
-                        int32_t acc = 0;
-                        for (long long cc = c_lo; cc <= c_hi; ++cc) {
-                            const int sl = (t == range_begin(cc, P, T) / ks) ? 0 : 1;
-                            acc += __ldcg(a.ws_part + ((size_t)(cc * 2 + sl) * BN + col) * kPanelRows + r);
+                    for (int cc = 0; cc < nchunks; ++cc) {
+                        int32_t sum[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) sum[j] = 0;
+                        // up to 4 contributors per batch: all 16 loads are in
+                        // flight before the first add
+#pragma unroll 1
+                        for (int b = 0; b < nc; b += 4) {
+                            int4 ld[4][4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                if (b + u < nc) {
+                                    const long long c2 = c_lo + b + u;
+                                    const int sl = (t == range_begin(c2, P, T) / ks) ? 0 : 1;
+                                    const int4 *src = reinterpret_cast<const int4 *>(
+                                                          a.ws_part + (size_t)(c2 * 2 + sl) * BN * kPanelRows) +
+                                                      ((size_t)cc * kPanelRows + r) * 4;
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) ld[u][j] = __ldcg(src + j);
+                                } else {
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) ld[u][j] = make_int4(0, 0, 0, 0);
+                                }
+                            }
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    sum[4 * j] += ld[u][j].x;
+                                    sum[4 * j + 1] += ld[u][j].y;
+                                    sum[4 * j + 2] += ld[u][j].z;
+                                    sum[4 * j + 3] += ld[u][j].w;
+                                }
                         }
-                        const float sx = half_bits_to_float(__ldg(a.s_x + m));
-                        a.Y[(size_t)m * a.N + n] = scale_to_half(acc, sx, sc);
-                        if (a.acc_dbg) a.acc_dbg[(size_t)m * a.N + n] = acc;
+                        store_outputs(a, m0 + cc * 16, n, sc, sum);
                     }
                     if (lane == 0) *counter = 0;  // ready for the next call
+                    if (warp == 6 && lane == 0 && trace_j < 4) QOQ_MARK(155 + trace_j);
                 }
             }
+            if (warp == 6 && lane == 0 && trace_j < 4) QOQ_MARK(150 + trace_j);
+            ++trace_j;
             accph ^= 1u;
             i = t * ks + ks1;
         }
@@ -428,11 +545,15 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (threadIdx.x == 0) QOQ_MARK(2);
     if (threadIdx.x == 0 && *abort_flag) {
         atomicExch(&g_dev_error, 1);
         // thread 0 is the producer: let its own copies land before exit
         for (int q = 0; q < STAGES; ++q)
-            if (issued & (1u << q)) drain_wait(full_bar(q), (issued_par >> q) & 1u, 200000000ull);
+            if (issued & (1u << q)) {
+                drain_wait(fullw_bar(q), (issued_par >> q) & 1u, 200000000ull);
+                if (!issued_x_none) drain_wait(fullx_bar(q), (issued_par >> q) & 1u, 200000000ull);
+            }
     }
     if (warp == 0) {
         __syncwarp();
@@ -441,6 +562,10 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ----------------------------------------------------------------- host --
+#ifdef QOQ_TRACE
+extern unsigned long long *g_trace_buffer;
+#endif
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -469,7 +594,22 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     auto kern = w4a8_gemm_kernel<BN, STAGES, ASTAGES, A_TMEM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 320, C::kSmemBytes, stream>>>(tmap, args);
+    // programmatic dependent launch: the GEMM may start (and stream weights)
+    // while the kernel before it in the stream -- normally the activation
+    // quantizer -- is still running; the kernel waits for it before it
+    // touches X8 or s_x.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(320);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tmap, args);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -477,10 +617,12 @@ template <bool A_TMEM>
 cudaError_t dispatch(int BN, const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
 {
     switch (BN) {
-    case 16: return launch_cfg<16, 8, A_TMEM ? 4 : 2, A_TMEM>(tmap, args, grid, stream);
-    case 32: return launch_cfg<32, 8, A_TMEM ? 4 : 2, A_TMEM>(tmap, args, grid, stream);
-    case 64: return launch_cfg<64, 8, A_TMEM ? 4 : 2, A_TMEM>(tmap, args, grid, stream);
-    case 128: return launch_cfg<128, 6, A_TMEM ? 4 : 2, A_TMEM>(tmap, args, grid, stream);
+    // TMEM A ring: as many 32-column slots as fit next to the accumulator
+    // in a power-of-two allocation (256 columns for BN <= 64, else 512)
+    case 16: return launch_cfg<16, A_TMEM ? 16 : 12, A_TMEM ? 7 : 2, A_TMEM>(tmap, args, grid, stream);
+    case 32: return launch_cfg<32, A_TMEM ? 14 : 11, A_TMEM ? 7 : 2, A_TMEM>(tmap, args, grid, stream);
+    case 64: return launch_cfg<64, A_TMEM ? 11 : 9, A_TMEM ? 6 : 2, A_TMEM>(tmap, args, grid, stream);
+    case 128: return launch_cfg<128, A_TMEM ? 7 : 6, A_TMEM ? 7 : 2, A_TMEM>(tmap, args, grid, stream);
     default: return launch_cfg<256, 4, A_TMEM ? 4 : 2, A_TMEM>(tmap, args, grid, stream);
     }
 }
@@ -552,10 +694,17 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     args.m_tiles = (M + BN - 1) / BN;
     args.ks = K / kBlockK;
     args.total = units;
-    args.timeout_ns = 2000000000ull;  // 2 s: far beyond any legitimate wait
+    args.timeout_ns = 2000000000ull;  // 2 s for one wait: far beyond any legitimate one
+#ifdef QOQ_TRACE
+    args.trace = g_trace_buffer;
+#endif
     return a_in_tmem ? dispatch<true>(BN, tmap, args, (int)grid, stream)
                      : dispatch<false>(BN, tmap, args, (int)grid, stream);
 }
+
+#ifdef QOQ_TRACE
+unsigned long long *g_trace_buffer = nullptr;
+#endif
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value)
 {

@@ -39,6 +39,10 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
                         int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream,
                         int *tmap_status);
 
+#ifdef QOQ_TRACE
+extern unsigned long long *g_trace_buffer;
+#endif
+
 // Device error flag of the current device: read and clear (synchronous).
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value);
 

@@ -13,6 +13,7 @@
 
 #include "qoq_internal.h"
 #include "qoq_layout.cuh"
+#include "qoq_ptx.cuh"
 
 namespace qoq {
 namespace {
@@ -166,6 +167,9 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const uint16_t *
                                                                  uint16_t *__restrict__ s_x)
 {
     __shared__ float red[kActThreads / 32];
+    // the GEMM that consumes X8 may launch now and start streaming weights;
+    // it waits for this grid to finish before it reads X8 or s_x
+    grid_launch_dependents();
     const int m = blockIdx.x;
     const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)m * K);
     uint2 *out = reinterpret_cast<uint2 *>(X8 + (size_t)m * K);

@@ -59,23 +59,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up
-// when `*abort` becomes non-zero (another role gave up) or when the global
-// timer passes `deadline_ns`; in the latter case it raises `*abort` itself.
-// Returns true when the phase completed.
+// when `*abort` becomes non-zero (another role gave up) or when this one
+// wait has lasted longer than `budget_ns`; in the latter case it raises
+// `*abort` itself.  Returns true when the phase completed.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
-                                             volatile int *abort, uint64_t deadline_ns)
+                                             volatile int *abort, uint64_t budget_ns)
 {
     if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t start = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0) {
             if (*abort) return false;
-            if (global_timer_ns() > deadline_ns) {
+            if (global_timer_ns() - start > budget_ns) {
                 *abort = 1;
                 return false;
             }
         }
     }
+}
+
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed and their writes are visible ...
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ... and let the grid that depends on this one start launching now.
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ TMA --
