@@ -70,7 +70,9 @@ typedef enum {
     QOQ_ERR_INVALID_ARG = -1,   /* a shape, pointer or size failed the checks above */
     QOQ_ERR_UNSUPPORTED = -2,   /* the current device is not compute capability 10.0 */
     QOQ_ERR_CUDA = -3,          /* a CUDA runtime call or a launch failed */
-    QOQ_ERR_TIMEOUT = -4        /* a kernel's bounded wait ran out (see qoq_device_error) */
+    QOQ_ERR_TIMEOUT = -4,       /* a kernel's bounded wait ran out (see qoq_device_error) */
+    QOQ_ERR_SCRATCH_TOO_SMALL = -5 /* qoq_w4a8_gemm_noalloc: the shape needs more scratch
+                                      than the built-in buffer holds */
 } qoq_status;
 
 /* Short English text for a status code. The string is static. */
@@ -190,6 +192,45 @@ QOQ_API int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x,
                   int M, int N, int K, int group_size,
                   uint16_t *Y, int32_t *acc_dbg,
                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* The same GEMM as qoq_w4a8_gemm, for callers that cannot allocate memory.
+ *
+ * The paper has no counterpart to this call. It exists because some callers
+ * cannot hand qoq_w4a8_gemm a scratch workspace:
+ *   - code inside an inference engine's execute/enqueue step, where
+ *     allocating is forbidden or would synchronize the device (cudaFree
+ *     waits for all outstanding work, and cudaMalloc can too);
+ *   - plug-ins that have no allocator of their own;
+ *   - real-time paths that must never enter the allocator.
+ *
+ * This entry point keeps the GEMM's scratch in a fixed 16 MiB
+ * (QOQ_NOALLOC_SCRATCH_BYTES) buffer in the library's own device image:
+ *   - every GPU that loads the library holds that buffer until the process
+ *     exits;
+ *   - the call itself allocates nothing, through CUDA or any other library;
+ *   - the caller still provides every input and the output Y, with the
+ *     layouts, limits and checks of qoq_w4a8_gemm (there is no acc_dbg).
+ *
+ * Scratch rules:
+ *   - a shape whose qoq_gemm_workspace_bytes exceeds
+ *     QOQ_NOALLOC_SCRATCH_BYTES is rejected with QOQ_ERR_SCRATCH_TOO_SMALL.
+ *     Token counts up to 64 fit for every N and K;
+ *   - every call on a device shares the one buffer, which keeps the last
+ *     call's contents. Each call first clears the part that must start at
+ *     zero (an asynchronous memset on `stream`, not an allocation);
+ *   - two calls whose work can overlap on the GPU (different streams, or
+ *     concurrent graph branches) race on the buffer and give undefined
+ *     results. Serialize them.
+ *
+ * The first call on each device looks up the buffer's device address, with
+ * that device current, and caches it. Make that first call before any
+ * stream capture that should contain this entry point. */
+#define QOQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+QOQ_API int qoq_w4a8_gemm_noalloc(const int8_t *X8, const uint16_t *s_x,
+                                  const uint8_t *Wp, const uint16_t *s_c,
+                                  const uint8_t *s_g, const uint8_t *zs,
+                                  int M, int N, int K, int group_size,
+                                  uint16_t *Y, void *stream);
 
 /* Expands the packed codes to the INT8 weights the GEMM multiplies,
  * W8hat[n][k] = q*s_g - zs. It runs the same device routine as the GEMM's

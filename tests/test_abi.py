@@ -27,7 +27,7 @@ def declared():
 def test_exports_every_declared_symbol(L):
     import w4a8_integer_gemm_b200 as q
     names = declared()
-    assert len(names) == 9
+    assert len(names) == 10
     for n in names:
         assert hasattr(L, n), n
     assert names == set(q.SIGNATURES)
@@ -39,7 +39,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_status_strings(L):
     import w4a8_integer_gemm_b200 as q
-    for s in (0, -1, -2, -3, -4):
+    for s in (0, -1, -2, -3, -4, -5):
         assert len(q.qoq_status_string(s)) >= 2
     assert q.qoq_status_string(7) == "unknown status"
 

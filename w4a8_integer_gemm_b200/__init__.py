@@ -32,6 +32,8 @@ QOQ_ERR_INVALID_ARG = -1
 QOQ_ERR_UNSUPPORTED = -2
 QOQ_ERR_CUDA = -3
 QOQ_ERR_TIMEOUT = -4
+QOQ_ERR_SCRATCH_TOO_SMALL = -5
+QOQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -45,6 +47,7 @@ SIGNATURES = {
     "qoq_quant_act_per_token": (_I, [_P, _I, _I, _P, _P, _P]),
     "qoq_gemm_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "qoq_w4a8_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "qoq_w4a8_gemm_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "qoq_dequant_weights_i8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "qoq_set_gemm_a_in_tmem": (_I, [_I]),
     "qoq_device_error": (_I, [_P]),
@@ -203,6 +206,27 @@ def qoq_w4a8_gemm(X8: torch.Tensor, s_x: torch.Tensor, packed: PackedWeights,
                              _ptr(workspace), workspace.numel() * workspace.element_size(),
                              _stream(stream))
     _check("qoq_w4a8_gemm", st)
+    return Y
+
+
+def qoq_w4a8_gemm_noalloc(X8: torch.Tensor, s_x: torch.Tensor, packed: PackedWeights,
+                          Y: torch.Tensor, stream=None) -> torch.Tensor:
+    """The GEMM with its scratch in the library's built-in buffer.
+
+    For callers that may not allocate while they run the layer (an engine's
+    execute step, a plug-in without an allocator, a real-time path): the
+    caller passes a preallocated Y, and the call itself allocates nothing.
+    Shapes needing more than QOQ_NOALLOC_SCRATCH_BYTES of scratch raise
+    QoQError(QOQ_ERR_SCRATCH_TOO_SMALL); calls that may overlap on the GPU
+    must be serialized, since they share the buffer."""
+    _need(X8, torch.int8, "X8")
+    M, K = X8.shape
+    if K != packed.K:
+        raise ValueError("K mismatch between X8 and the packed weights")
+    st = lib().qoq_w4a8_gemm_noalloc(_ptr(X8), _ptr(s_x), _ptr(packed.Wp), _ptr(packed.s_c),
+                                     _ptr(packed.s_g), _ptr(packed.zs), M, packed.N, K,
+                                     packed.group_size, _ptr(Y), _stream(stream))
+    _check("qoq_w4a8_gemm_noalloc", st)
     return Y
 
 

@@ -67,6 +67,7 @@ const char *qoq_status_string(int status)
     case QOQ_ERR_UNSUPPORTED: return "unsupported device (needs compute capability 10.0, sm_100a)";
     case QOQ_ERR_CUDA: return "CUDA runtime or launch error";
     case QOQ_ERR_TIMEOUT: return "a bounded device wait ran out; outputs of that call are undefined";
+    case QOQ_ERR_SCRATCH_TOO_SMALL: return "shape needs more scratch than the built-in no-alloc buffer holds";
     default: return "unknown status";
     }
 }
