@@ -39,6 +39,7 @@ import torch  # noqa: E402
 from w4a8_integer_gemm_b200 import roofline, workloads as wl  # noqa: E402
 
 FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20
 
 
 def parse():
@@ -52,6 +53,8 @@ def parse():
                     help="restrict the workload to one shape name (for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--a-smem", action="store_true",
+                    help="keep the GEMM's dequantized tile in shared memory instead of TMEM")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample (cpu_baseline / reference arm)")
     return ap.parse_args()
@@ -174,6 +177,7 @@ def run_ours(args, rank, world, local, dist):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     q.lib()
+    q.qoq_set_gemm_a_in_tmem(not args.a_smem)
     peaks = roofline.load_peaks()
     work = select(args)
     stream = torch.cuda.current_stream()
@@ -195,65 +199,125 @@ def run_ours(args, rank, world, local, dist):
     torch.cuda.synchronize()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     n_sh = len(cases)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_sh)]
+    wbytes = sum(c["packed"].Wp.numel() for c in cases)
+    # Each step touches every shape's own packed weights once.  When they
+    # add up to more than 1.5x the L2 (126 MB) the step runs back to back,
+    # as a serving stack would run consecutive layers, and the weights of a
+    # shape are long evicted before the next step comes back to them.
+    # Otherwise L2 is flushed before every shape and each shape is timed
+    # on its own (flush excluded).
+    chained = wbytes > 3 * L2_BYTES // 2
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev = [[E() for _ in range(4)] for _ in range(n_sh)]
+    es = [E(), E(), E(), E()]
 
-    def one_step(record):
+    def one_step():
+        """The hot path of every shape: activation quant, then the GEMM.
+        Returns (step ms, GEMM-only ms summed over shapes)."""
+        if chained:
+            es[0].record(stream)
+            for c in cases:
+                q.qoq_quant_act_per_token(c["X"], c["X8"], c["s_x"], stream=stream)
+                q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
+            es[1].record(stream)
+            torch.cuda.synchronize()
+            return es[0].elapsed_time(es[1])
+        tot = 0.0
         for j, c in enumerate(cases):
             flush.zero_()
-            e = ev[j]
-            e[0].record(stream)
+            ev[j][0].record(stream)
             q.qoq_quant_act_per_token(c["X"], c["X8"], c["s_x"], stream=stream)
-            e[1].record(stream)
             q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
-            e[2].record(stream)
-        if record is not None:
+            ev[j][1].record(stream)
+        torch.cuda.synchronize()
+        for j in range(n_sh):
+            tot += ev[j][0].elapsed_time(ev[j][1])
+        return tot
+
+    def gemm_only():
+        """The GEMM kernel alone, the same way (roofline of the dominant kernel)."""
+        if chained:
+            es[2].record(stream)
+            for c in cases:
+                q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
+            es[3].record(stream)
             torch.cuda.synchronize()
-            for j in range(n_sh):
-                record[j][0] += ev[j][0].elapsed_time(ev[j][1])
-                record[j][1] += ev[j][1].elapsed_time(ev[j][2])
+            return es[2].elapsed_time(es[3])
+        tot = 0.0
+        for j, c in enumerate(cases):
+            flush.zero_()
+            ev[j][2].record(stream)
+            q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
+            ev[j][3].record(stream)
+        torch.cuda.synchronize()
+        for j in range(n_sh):
+            tot += ev[j][2].elapsed_time(ev[j][3])
+        return tot
+
+    def isolated(reps=3):
+        """Per shape, L2 flushed, kernel(s) alone: the per-point breakdown."""
+        out = []
+        for j, c in enumerate(cases):
+            st = gm = 0.0
+            for _ in range(reps):
+                flush.zero_()
+                ev[j][0].record(stream)
+                q.qoq_quant_act_per_token(c["X"], c["X8"], c["s_x"], stream=stream)
+                q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
+                ev[j][1].record(stream)
+                flush.zero_()
+                ev[j][2].record(stream)
+                q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
+                ev[j][3].record(stream)
+                torch.cuda.synchronize()
+                st += ev[j][0].elapsed_time(ev[j][1])
+                gm += ev[j][2].elapsed_time(ev[j][3])
+            out.append((st / reps, gm / reps))
+        return out
 
     for _ in range(max(3, args.warmup)):
-        one_step(None)
+        one_step()
+        gemm_only()
     torch.cuda.synchronize()
     if q.qoq_device_error() != q.QOQ_OK:
         raise RuntimeError("device error during warm-up")
 
-    acc_ms = [[0.0, 0.0] for _ in range(n_sh)]
+    step_ms = []
     with ClockSampler(local) as clk:
         barrier(dist)
         torch.cuda.synchronize()
         t_wall = time.perf_counter()
         for _ in range(args.steps):
-            one_step(acc_ms)
+            step_ms.append(one_step())
         torch.cuda.synchronize()
         barrier(dist)
         wall = time.perf_counter() - t_wall
     clocks = clk.summary()
+    g_ms_total = sum(gemm_only() for _ in range(args.steps)) / args.steps
+    iso = isolated()
     if q.qoq_device_error() != q.QOQ_OK:
         raise RuntimeError("device error in the timed region")
 
-    K_ = args.steps
     per = []
-    tot_ops = tot_ms = g_ms = g_bytes = 0.0
+    tot_ops = g_bytes = 0.0
     for j, c in enumerate(cases):
         s = c["s"]
-        aq_ms, gm_ms = acc_ms[j][0] / K_, acc_ms[j][1] / K_
+        pair_ms, gm_ms = iso[j]
         ops = roofline.ops(s.M, s.N, s.K)
         byt = roofline.algorithmic_bytes(s.M, s.N, s.K, s.G)
         roof = roofline.roofline_ops_per_s(s.M, s.N, s.K, s.G, peaks["int8_tops"] * 1e12, peaks["hbm_gbs"] * 1e9)
         tops = ops / (gm_ms * 1e-3) / 1e12
         per.append({"shape": s.name, "M": s.M, "K": s.K, "N": s.N, "G": s.G,
-                    "gemm_us": round(gm_ms * 1e3, 2), "act_quant_us": round(aq_ms * 1e3, 2),
-                    "gemm_tops": round(tops, 2), "gemm_gbs": round(byt / (gm_ms * 1e-3) / 1e9, 1),
-                    "roofline_tops": round(roof / 1e12, 2), "frac": round(tops * 1e12 / roof, 4),
+                    "isolated_step_us": round(pair_ms * 1e3, 2), "isolated_gemm_us": round(gm_ms * 1e3, 2),
+                    "isolated_gemm_tops": round(tops, 2), "isolated_gemm_gbs": round(byt / (gm_ms * 1e-3) / 1e9, 1),
+                    "roofline_tops": round(roof / 1e12, 2), "isolated_frac": round(tops * 1e12 / roof, 4),
                     "bound": roofline.bound(s.M, s.N, s.K, s.G, peaks["int8_tops"] * 1e12,
                                             peaks["hbm_gbs"] * 1e9)})
         tot_ops += ops
-        tot_ms += aq_ms + gm_ms
-        g_ms += gm_ms
         g_bytes += byt
+    tot_ms = statistics.median(step_ms)
     ms_step, value = aggregate(tot_ops, tot_ms, world, dist)
-
+    g_ms = g_ms_total
     # roofline of the dominant kernel (the GEMM), averaged per launch
     n_hbm = sum(1 for p in per if p["bound"] == "hbm")
     bound = "hbm" if n_hbm * 2 >= len(per) else "tensor"
@@ -310,10 +374,14 @@ def run_ours(args, rank, world, local, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "s8xs8->s32 (u4 weights), fp16 out", "data": "synthetic",
         "config": {"workload": work.name, "shapes": [p["shape"] for p in per],
-                   "l2": "flushed before every shape (256 MB write), flush excluded from timing",
+                   "l2": ("inputs larger than L2: %d MB of distinct packed weights per step, no flush" % (wbytes >> 20))
+                         if chained else "flushed before every shape (256 MB write), flush excluded from timing",
+                   "timing": ("median step of %d; GEMM-only roofline from the same %s runs" %
+                              (args.steps, "back-to-back" if chained else "flushed")),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": rl, "points": per, "clocks": clocks, "e2e": e2e,
         "gpu_launches": 2 * n_sh * args.steps,
+        "a_operand": "smem" if args.a_smem else "tmem",
     }
     return out, cases
 

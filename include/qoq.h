@@ -94,10 +94,13 @@ QOQ_API const char *qoq_status_string(int status);
  * So one AND of a word with 0x0F0F0F0F gives four consecutive codes in four
  * byte lanes, and one shift plus one AND gives the next four.
  *
- * The group tables are group-major, channel-contiguous, one byte per entry:
- *     s_g[g*N + n]  the integer group scale (1..16),
- *     zs[g*N + n]   the zero compensation z*s_g (0..240),
- * with g = k / group_size. s_c[n] is the FP16 channel scale.
+ * The group tables are panel-major, one byte per entry: for channel n in
+ * panel p = n/128 (r = n%128) and group g = k/group_size,
+ *     s_g[(p*(K/group_size) + g)*128 + r]  the integer group scale (1..16),
+ *     zs [(p*(K/group_size) + g)*128 + r]  the zero compensation z*s_g (0..240).
+ * The 128 channels of a panel are contiguous for each group, and the groups
+ * of a panel follow each other, so one bulk copy brings the tables a
+ * pipeline stage needs. s_c[n] is the FP16 channel scale.
  */
 
 /* Bytes of Wp for an N x K weight: N*K/2. Returns 0 when N or K is not a
@@ -122,8 +125,8 @@ QOQ_API size_t qoq_packed_weight_bytes(int N, int K);
  *   Wp     device, qoq_packed_weight_bytes(N, K) bytes, written in the
  *          packed layout above.
  *   s_c    device, uint16_t [N] FP16 bits, written.
- *   s_g    device, uint8_t [K/group_size][N], written.
- *   zs     device, uint8_t [K/group_size][N], written.
+ *   s_g    device, uint8_t [N/128][K/group_size][128], written.
+ *   zs     device, uint8_t [N/128][K/group_size][128], written.
  * The result is deterministic and bit-identical on every call.
  */
 QOQ_API int qoq_pack_weights(const float *W, int N, int K, int group_size,
@@ -214,7 +217,7 @@ QOQ_API int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x,
  * Scratch rules:
  *   - a shape whose qoq_gemm_workspace_bytes exceeds
  *     QOQ_NOALLOC_SCRATCH_BYTES is rejected with QOQ_ERR_SCRATCH_TOO_SMALL.
- *     Token counts up to 64 fit for every N and K;
+ *     Token counts up to 128 fit for every N and K;
  *   - every call on a device shares the one buffer, which keeps the last
  *     call's contents. Each call first clears the part that must start at
  *     zero (an asynchronous memset on `stream`, not an allocation);

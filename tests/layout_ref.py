@@ -13,3 +13,10 @@ def pack_reference(q: np.ndarray) -> np.ndarray:
     t = t.transpose(0, 2, 3, 1, 5, 6, 4)                    # p b j r w i h
     out = (t[..., 0] | (t[..., 1] << 4)).astype(np.uint8)   # p b j r w i
     return np.ascontiguousarray(out).reshape(-1)
+
+
+def tables_reference(t: np.ndarray) -> np.ndarray:
+    """Canonical group table [N][K/G] -> the documented panel-major layout
+    [N/128][K/G][128] (include/qoq.h)."""
+    N, ng = t.shape
+    return np.ascontiguousarray(t.reshape(N // 128, 128, ng).transpose(0, 2, 1))

@@ -15,7 +15,7 @@ import torch
 import oracle
 import w4a8_integer_gemm_b200 as q
 from w4a8_integer_gemm_b200 import workloads as wl
-from layout_ref import pack_reference
+from layout_ref import pack_reference, tables_reference
 
 pytestmark = pytest.mark.gpu
 
@@ -62,6 +62,6 @@ def test_full_size_sampled(name, i):
         _packed_checked.add(key)
         full = oracle.quantize_weights(W.numpy(), s.G)
         assert np.array_equal(packed.s_c.cpu().view(torch.int16).numpy().view(np.uint16), full["s_c"])
-        assert np.array_equal(packed.s_g.cpu().numpy(), full["s_g"].T)
-        assert np.array_equal(packed.zs.cpu().numpy(), full["zs"].T)
+        assert np.array_equal(packed.s_g.cpu().numpy(), tables_reference(full["s_g"]))
+        assert np.array_equal(packed.zs.cpu().numpy(), tables_reference(full["zs"]))
         assert np.array_equal(packed.Wp.cpu().numpy(), pack_reference(full["q"]))

@@ -130,8 +130,8 @@ class PackedWeights:
     """Output of the offline packer (device tensors, layouts of include/qoq.h)."""
     Wp: torch.Tensor     # uint8 [N*K/2]  interleaved UINT4 codes
     s_c: torch.Tensor    # int16 [N]      FP16 bits of the channel scales
-    s_g: torch.Tensor    # uint8 [K/G, N] integer group scales
-    zs: torch.Tensor     # uint8 [K/G, N] zero compensation z*s_g
+    s_g: torch.Tensor    # uint8 [N/128, K/G, 128] integer group scales (panel-major)
+    zs: torch.Tensor     # uint8 [N/128, K/G, 128] zero compensation z*s_g
     N: int
     K: int
     group_size: int
@@ -148,8 +148,8 @@ def qoq_pack_weights(W: torch.Tensor, group_size: int, out: Optional[PackedWeigh
         ng = K // G if G > 0 and K % G == 0 else 1
         out = PackedWeights(torch.empty(max(nb, 16), dtype=torch.uint8, device=dev),
                             torch.empty(N, dtype=torch.int16, device=dev),
-                            torch.empty(ng, N, dtype=torch.uint8, device=dev),
-                            torch.empty(ng, N, dtype=torch.uint8, device=dev), N, K, G)
+                            torch.empty(max(N // 128, 1), ng, 128, dtype=torch.uint8, device=dev),
+                            torch.empty(max(N // 128, 1), ng, 128, dtype=torch.uint8, device=dev), N, K, G)
     st = lib().qoq_pack_weights(_ptr(W), N, K, G, _ptr(out.Wp), _ptr(out.s_c), _ptr(out.s_g),
                                 _ptr(out.zs), _stream(stream))
     _check("qoq_pack_weights", st)

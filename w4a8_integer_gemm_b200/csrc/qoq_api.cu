@@ -103,6 +103,7 @@ int qoq_quant_act_per_token(const uint16_t *X, int M, int K, int8_t *X8, uint16_
 size_t qoq_gemm_workspace_bytes(int M, int N, int K, int group_size)
 {
     if (M < 1 || M > kMaxM || !valid_nk(N, K) || !valid_group(K, group_size)) return 0;
+    if (!qoq::gemm_shape_supported(M, N, K)) return 0;
     return qoq::gemm_workspace_bytes(M, N, K);
 }
 
@@ -116,6 +117,7 @@ int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, cons
     if (!aligned16(X8) || !aligned16(s_x) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) ||
         !aligned16(zs) || !aligned16(Y) || !aligned16(workspace) || (acc_dbg && !aligned16(acc_dbg)))
         return QOQ_ERR_INVALID_ARG;
+    if (!qoq::gemm_shape_supported(M, N, K)) return QOQ_ERR_INVALID_ARG;
     if (workspace_bytes < qoq::gemm_workspace_bytes(M, N, K)) return QOQ_ERR_INVALID_ARG;
     const int dev = check_device();
     if (dev != QOQ_OK) return dev;
@@ -150,6 +152,14 @@ __attribute__((visibility("default"))) int qoq_debug_set_trace(void *buf)
 {
     qoq::g_trace_buffer = reinterpret_cast<unsigned long long *>(buf);
     return QOQ_OK;
+}
+
+// Trace builds only: one thread writes the global timer to *dst.
+__attribute__((visibility("default"))) int qoq_debug_stamp(void *dst, void *stream)
+{
+    return qoq::debug_stamp(reinterpret_cast<unsigned long long *>(dst), (cudaStream_t)stream) == cudaSuccess
+               ? QOQ_OK
+               : QOQ_ERR_CUDA;
 }
 #endif
 

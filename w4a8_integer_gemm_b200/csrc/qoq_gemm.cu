@@ -14,36 +14,44 @@
 // Design (B200-first; the pages' A100/L40S register-fed mma.sync design is
 // prior art only):
 //   * Swap-AB: the 128 output channels of a weight panel are the MMA's M
-//     (A operand), the tokens are its N (B operand, 16..256).  Decode shapes
-//     (M <= 64) therefore waste no tensor-core rows on padding tokens.
+//     (A operand), the tokens are its N (B operand, BN = 16..256).  Decode
+//     shapes (M <= 64) therefore waste no tensor-core rows on padding tokens.
 //   * Persistent grid, one CTA per SM, stream-K schedule: the sequence of
-//     (output tile, 128-wide K block) units is cut into equal contiguous
+//     (output tile, KST-wide K block) units is cut into equal contiguous
 //     ranges, one per CTA, so every SM streams the same number of weight
-//     bytes.  Tiles whose K loop is split across CTAs meet as INT32 partials
-//     in a workspace (exact in any order); the last contributor, found with
-//     a counter per split tile and 32-channel quarter, reduces them and runs
-//     the epilogue.  A split tile is the last tile of the first CTA that
-//     contributes to it, so the counters are indexed by that CTA: a fixed
-//     region at the start of the workspace, whatever the shape, which every
-//     call leaves at zero.
-//   * Warp roles (320 threads):
-//       warp 0      TMA producer: per stage one tiled TMA of the X8 tile
-//                   (128-byte swizzle), one 8 KB bulk copy of the packed
-//                   weight chunk and two 128-byte bulk copies of the group
-//                   tables into a shared-memory ring.
-//       warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 32 each)
-//                   per stage, tcgen05.commit frees ring slots.
+//     bytes.  A tile whose K loop is split across CTAs is finished by its
+//     first contributor (the CTA whose range holds the tile's first unit:
+//     for it the tile is the last one it works on).  Every later
+//     contributor works on the tile first, publishes its INT32 partial
+//     (exact in any order) and bumps a counter; the finisher waits, bounded,
+//     for the count, adds the partials to its own accumulator and runs the
+//     epilogue.  No contributor waits for anything while it still has work,
+//     so the waits cannot form a cycle.
+//   * Warp roles (352 threads):
+//       warp 0      weight producer: per stage one bulk copy of the packed
+//                   weight chunks.
+//       warp 1      MMA issuer (one thread): one barrier wait, KST/32
+//                   tcgen05.mma (K = 32) and one tcgen05.commit per stage.
 //       warps 2-5   dequant: thread r owns output channel r of the panel,
-//                   reads its 64 packed bytes with four 128-bit shared loads,
-//                   expands them to 128 INT8 weights in registers, and
-//                   stores them as the MMA's A operand -- into TMEM with
-//                   tcgen05.st (default), or into shared memory in the
-//                   128-byte-swizzled K-major layout.
+//                   reads its packed bytes with 128-bit shared loads,
+//                   expands them to INT8 in registers, and stores them as
+//                   the MMA's A operand -- into TMEM with tcgen05.st
+//                   (default), or into shared memory in the 128-byte-
+//                   swizzled K-major layout.
 //       warps 6-9   epilogue: tcgen05.ld of the INT32 accumulators, FP32
-//                   scaling, FP16 stores (or INT32 partials for split tiles).
-//   * Every mbarrier wait is bounded by a global-timer deadline; on expiry
-//     the CTA stops, drains its own in-flight copies and MMAs, frees TMEM,
-//     and raises the device error flag that qoq_device_error() reports.
+//                   scaling, FP16 stores; split tiles as above.
+//       warp 10     X8 producer: tiled TMA loads of the activation tiles
+//                   and bulk copies of the group tables.  It alone waits for
+//                   the preceding kernel (programmatic dependent launch), so
+//                   weights stream in while the activation quantizer runs.
+//   * One ring: stage slot s holds the packed weights, tables and X8 tiles
+//     of a K block in shared memory, and A slot s (TMEM or shared memory)
+//     holds its dequantized weights.  When the dequant warps see slot s
+//     filled again, the producers have seen it freed, so the MMA is done
+//     with A slot s too; no separate A-slot barrier is needed.
+//   * Every wait is bounded (per wait, global timer); on expiry the CTA
+//     stops, drains its own in-flight copies and MMAs, frees TMEM, and
+//     raises the device error flag that qoq_device_error() reports.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -67,20 +75,22 @@ struct GemmArgs {
     uint16_t *Y;
     int32_t *acc_dbg;
     int32_t *ws_cnt;   // [kMaxCtas][4] arrival counters, at the start of the workspace
-    int32_t *ws_part;  // [cta][2 slots][BN][128] INT32 partial tiles, after the counters
+    int32_t *ws_part;  // [cta][BN/16][128][16] INT32 partial tile, after the counters
     int M, N, K, G;
-    int m_tiles, ks;        // ks = K / 128 stages per tile
-    long long total;        // tiles * ks units
+    int m_tiles;
+    int ks;            // K / KST units per tile
+    int ngroups;       // K / G
+    int total;         // tiles * ks units
     unsigned long long timeout_ns;  // longest any one wait may last
 #ifdef QOQ_TRACE
-    unsigned long long *trace;  // [cta][256] global-timer marks (trace builds only)
+    unsigned long long *trace;  // [cta][256] clock marks (trace builds only)
 #endif
 };
 
-// Timeline marks for the trace build (compiled out otherwise).
+// Timeline marks for the trace build (compiled out otherwise).  Slot 255
+// holds the CTA's global-timer entry time; the other marks are SM clock
+// cycles since the CTA's entry.
 #ifdef QOQ_TRACE
-// slot 255 holds the CTA's global-timer entry time; the other marks are SM
-// clock cycles since the CTA's entry
 #define QOQ_MARK(idx)                                                                              \
     do {                                                                                           \
         if (a.trace) a.trace[(size_t)blockIdx.x * 256 + (idx)] = clock64() - trace_t0;             \
@@ -96,36 +106,43 @@ __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
     return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
 }
 
-template <int BN, int STAGES, int ASTAGES, bool A_TMEM>
+template <int BN, int KST, int STAGES, bool A_TMEM>
 struct GemmCfg {
-    static constexpr int kXBytes = BN * 128;  // X8 tile: BN tokens x 128 k
-    static constexpr int kWBytes = kChunkBytes;
-    static constexpr int kTabBytes = 256;  // s_g[128] then zs[128]
-    static constexpr int kStageBytes = ((kXBytes + kWBytes + kTabBytes + 1023) / 1024) * 1024;
-    static constexpr int kABytes = A_TMEM ? 0 : 128 * 128;  // dequantized tile in smem
+    static constexpr int ASTAGES = STAGES;               // A slot s belongs to stage slot s
+    static constexpr int kChunks = KST / kBlockK;        // packed 8 KB chunks per stage
+    static constexpr int kXTile = BN * 128;              // one [BN][128 B] swizzled X8 tile
+    static constexpr int kXBytes = kChunks * kXTile;
+    static constexpr int kWBytes = kChunks * kChunkBytes;
+    static constexpr int kTabRegion = 128 * kChunks;     // s_g region, then zs region
+    static constexpr int kStageBytes = ((kXBytes + kWBytes + 2 * kTabRegion + 1023) / 1024) * 1024;
+    static constexpr int kATile = 128 * 128;             // one [128][128 B] swizzled A tile
+    static constexpr int kABytes = A_TMEM ? 0 : kChunks * kATile;
     static constexpr int kBarOff = STAGES * kStageBytes + ASTAGES * kABytes;
-    static constexpr int kNumBars = 3 * STAGES + 2 * ASTAGES + 3;
+    static constexpr int kNumBars = 4 * STAGES + 3;
     static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
     // at least ~120 KB so that exactly one CTA (and one TMEM allocation)
     // lives on each SM; +1024 for manual alignment of the dynamic base
     static constexpr int kSmemBytes = (kUsed > 120 * 1024 ? kUsed : 120 * 1024) + 1024;
-    static constexpr uint32_t kAccCols = BN;
-    static constexpr uint32_t kACol0 = BN;  // first TMEM column of the A ring
-    static constexpr uint32_t kTmemCols = pow2_cols(BN + (A_TMEM ? ASTAGES * 32 : 0));
+    static constexpr uint32_t kACols = KST / 4;          // TMEM columns of one A slot
+    static constexpr uint32_t kACol0 = BN;               // first TMEM column of the A ring
+    static constexpr uint32_t kTmemCols = pow2_cols(BN + (A_TMEM ? ASTAGES * kACols : 0));
+    static constexpr int kSx = (BN + 31) / 32;           // s_x registers per lane
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
-    static_assert(BN + (A_TMEM ? ASTAGES * 32 : 0) <= 512, "TMEM columns");
+    static_assert(KST == 128 || KST == 256, "stage depth");
+    static_assert(BN + (A_TMEM ? ASTAGES * kACols : 0) <= 512, "TMEM columns");
     static_assert(kUsed <= 227 * 1024, "shared memory");
+    static_assert(STAGES <= 32, "ring bookkeeping masks");
 };
 
-// The CTA whose stream-K range contains unit i.
-__device__ __forceinline__ long long cta_of(long long i, long long P, long long T)
+// The CTA whose stream-K range contains unit i (ranges: [c*T/P, (c+1)*T/P)).
+__device__ __forceinline__ int cta_of(int i, int P, int T)
 {
-    return ((i + 1) * P - 1) / T;
+    return (int)((((long long)i + 1) * P - 1) / T);
 }
 
-__device__ __forceinline__ long long range_begin(long long c, long long P, long long T)
+__device__ __forceinline__ int range_begin(int c, int P, int T)
 {
-    return c * T / P;
+    return (int)((long long)c * T / P);
 }
 
 // Waits without the shared abort check; used only to drain in-flight work
@@ -136,6 +153,18 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     while (!mbar_try_wait(bar, parity)) {
         if (global_timer_ns() > end) break;
     }
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(int *p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ float half_bits_to_float(uint16_t h)
@@ -149,38 +178,57 @@ __device__ __forceinline__ uint16_t scale_to_half(int32_t acc, float sx, float s
     return __half_as_ushort(__float2half_rn(y));
 }
 
-// FP16 outputs (and optionally the INT32 accumulators) of 16 consecutive
-// tokens m0.. for channel n; tokens beyond M are skipped.
-__device__ __forceinline__ void store_outputs(const GemmArgs &a, int m0, int n, float sc, const int32_t *acc)
+// FP16 outputs (and optionally the INT32 accumulators) of the 16
+// consecutive tokens m0.. of chunk `cc` for channel n.  The token scales
+// come from the lanes' registers: lane l of sx holds s_x[m0 - 16*(cc&1) + l].
+// A warp's store covers 32 consecutive channels: 64 contiguous bytes.
+__device__ __forceinline__ void store_outputs(const GemmArgs &a, int m0, int cc, int n, float sc, float sx,
+                                              const int32_t *acc)
 {
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
+        const float sxq = __shfl_sync(0xffffffffu, sx, (cc & 1) * 16 + q);
         const int m = m0 + q;
         if (m < a.M) {
-            const float sx = half_bits_to_float(__ldg(a.s_x + m));
-            a.Y[(size_t)m * a.N + n] = scale_to_half(acc[q], sx, sc);
+            a.Y[(size_t)m * a.N + n] = scale_to_half(acc[q], sxq, sc);
             if (a.acc_dbg) a.acc_dbg[(size_t)m * a.N + n] = acc[q];
         }
     }
 }
 
-template <int BN, int STAGES, int ASTAGES, bool A_TMEM>
-__global__ void __launch_bounds__(320, 1)
+// The accumulator columns [c0, c0 + W) of this thread's TMEM lane, W = 16,
+// 32 or 64, in one load.
+template <int W>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *v)
+{
+    if constexpr (W == 64) {
+        tmem_ld64(taddr, v);
+    } else if constexpr (W == 32) {
+        tmem_ld32(taddr, v);
+    } else {
+        uint32_t (&r)[16] = *reinterpret_cast<uint32_t(*)[16]>(v);
+        tmem_ld16(taddr, r);
+    }
+}
+
+template <int BN, int KST, int STAGES, bool A_TMEM>
+__global__ void __launch_bounds__(352, 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs a)
 {
-    using C = GemmCfg<BN, STAGES, ASTAGES, A_TMEM>;
+    using C = GemmCfg<BN, KST, STAGES, A_TMEM>;
+    constexpr int kCh = C::kChunks;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar0 = sbase + C::kBarOff;
-    // per ring slot: fullw (weights + tables landed), fullx (X8 tile landed),
-    // empty (dequant warps and the MMA are done with the slot)
+    // per ring slot: fullw (packed weights landed), fullx (X8 tiles and
+    // group tables landed), afull (dequantized A operand written), empty
+    // (dequant warps and the MMA are done with the slot)
     auto fullw_bar = [&](int s) { return bar0 + 8u * s; };
     auto fullx_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto empty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-    auto afull_bar = [&](int t) { return bar0 + 8u * (3 * STAGES + t); };
-    auto aempty_bar = [&](int t) { return bar0 + 8u * (3 * STAGES + ASTAGES + t); };
-    const uint32_t accfull_bar = bar0 + 8u * (3 * STAGES + 2 * ASTAGES);
+    auto afull_bar = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
+    const uint32_t accfull_bar = bar0 + 8u * (4 * STAGES);
     const uint32_t accempty_bar = accfull_bar + 8u;
     const uint32_t mmadone_bar = accfull_bar + 16u;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kNumBars * 8);
@@ -194,23 +242,22 @@ __global__ void __launch_bounds__(320, 1)
     if (threadIdx.x == 0 && a.trace) a.trace[(size_t)blockIdx.x * 256 + 255] = global_timer_ns();
 #endif
     if (threadIdx.x == 0) {
-        QOQ_MARK(0);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(fullw_bar(s), 1);
             mbar_init(fullx_bar(s), 1);
             mbar_init(empty_bar(s), 1 + 4);  // MMA commit + 4 dequant warps
-        }
-        for (int t = 0; t < ASTAGES; ++t) {
-            mbar_init(afull_bar(t), 4);
-            mbar_init(aempty_bar(t), 1);
+            mbar_init(afull_bar(s), 4);      // 4 dequant warps
         }
         mbar_init(accfull_bar, 1);
         mbar_init(accempty_bar, 4);
         mbar_init(mmadone_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tmap_x);
     }
+    if (threadIdx.x == 320) prefetch_tmap(&tmap_x);
+    // The next kernel in the stream may launch now; whatever it reads from
+    // this GEMM it must read after its own griddepcontrol.wait.
+    grid_launch_dependents();
     if (warp == 0) {
         tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
         tmem_relinquish();
@@ -219,79 +266,59 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    if (threadIdx.x == 0) QOQ_MARK(1);
-    int trace_j = 0;  // per-role stage counter for the timeline marks
-    (void)trace_j;
-    const uint64_t deadline = a.timeout_ns;  // budget of any single wait
+    const uint64_t budget = a.timeout_ns;
+    QOQ_MARK(1);
 
-    const long long P = gridDim.x;
-    const long long T = a.total;
-    const long long cta = blockIdx.x;
-    const long long i_begin = range_begin(cta, P, T);
-    const long long i_end = range_begin(cta + 1, P, T);
+    const int P = gridDim.x;
+    const int T = a.total;
+    const int cta = blockIdx.x;
+    const int i_begin = range_begin(cta, P, T);
+    const int i_end = range_begin(cta + 1, P, T);
     const int ks = a.ks;
-    // ring slots the producer has filled, and the phase parity of each
-    // slot's latest fill (drained on the way out of an aborted CTA)
+    // ring slots a producer has filled, and the phase parity of each slot's
+    // latest fill (drained on the way out of an aborted CTA)
     uint32_t issued = 0, issued_par = 0;
-    int issued_x_none = 0;  // set when the producer stopped before any X8 load
+    int tj = 0;  // trace: per-role unit counter
+    (void)tj;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer --
+    if (warp == 0 || warp == 10) {
+        // --------------------------------------- producers (W and X8) --
         if (lane == 0) {
+            const bool is_w = (warp == 0);
+            if (!is_w) grid_dependency_wait();  // X8 comes from the preceding kernel
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            // The X8 tiles come from the kernel that precedes this one in the
-            // stream (programmatic dependent launch): the weights of the first
-            // STAGES slots stream in before that kernel has finished, the X8
-            // loads of those slots are issued once it has.
-            int n_issued = 0;
-            bool x_ready = false;
-            int pend_kb[STAGES], pend_m[STAGES];
-            auto load_x = [&](int slot, int kb, int m_tile) {
-                mbar_arrive_expect_tx(fullx_bar(slot), C::kXBytes);
-                tma_load_2d(sbase + slot * C::kStageBytes, &tmap_x, kb * kBlockK, m_tile * BN, fullx_bar(slot));
-            };
-            auto release_x = [&]() {
-                grid_dependency_wait();
-                QOQ_MARK(144);
-                x_ready = true;
-                for (int j = 0; j < n_issued; ++j) {
-                    load_x(j, pend_kb[j], pend_m[j]);
-                    if (j < 16) QOQ_MARK(160 + j);
-                }
-            };
-            for (long long i = i_begin; i < i_end && ok;) {
-                const long long t = i / ks;
-                const int ks0 = (int)(i - t * ks);
-                const int ks1 = (int)min((long long)ks, i_end - t * ks);
-                const int m_tile = (int)(t % a.m_tiles);
-                const int n_tile = (int)(t / a.m_tiles);
+            const uint32_t tab = (a.G == kBlockK) ? (uint32_t)C::kTabRegion : 128u;
+            for (int i = i_begin; i < i_end && ok;) {
+                const int t = i / ks;
+                const int ks0 = i - t * ks;
+                const int ks1 = min(ks, i_end - t * ks);
+                const int m_tile = t % a.m_tiles;
+                const int n_tile = t / a.m_tiles;
                 for (int kb = ks0; kb < ks1; ++kb) {
-                    if (!x_ready && n_issued == STAGES) release_x();  // every slot waits for X8
-                    if (trace_j < 8) QOQ_MARK(216 + trace_j);
-                    if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, deadline)) {
+                    if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, budget)) {
                         ok = false;
                         break;
                     }
                     const uint32_t st = sbase + s * C::kStageBytes;
-                    const int g = (kb * kBlockK) / a.G;
-                    if (trace_j < 16) QOQ_MARK(180 + trace_j);
-                    mbar_arrive_expect_tx(fullw_bar(s), C::kWBytes + C::kTabBytes);
-                    bulk_load(st + C::kXBytes, a.Wp + chunk_offset(n_tile, kb, a.K), C::kWBytes, fullw_bar(s));
-                    if (trace_j < 16) QOQ_MARK(200 + trace_j);
-                    const size_t toff = (size_t)g * a.N + (size_t)n_tile * kPanelRows;
-                    bulk_load(st + C::kXBytes + C::kWBytes, a.s_g + toff, 128, fullw_bar(s));
-                    bulk_load(st + C::kXBytes + C::kWBytes + 128, a.zs + toff, 128, fullw_bar(s));
-                    if (trace_j < 32) QOQ_MARK(16 + trace_j);
-                    ++trace_j;
-                    if (x_ready) {
-                        load_x(s, kb, m_tile);
+                    if (is_w) {
+                        mbar_arrive_expect_tx(fullw_bar(s), C::kWBytes);
+                        bulk_load(st + C::kXBytes, a.Wp + chunk_offset(n_tile, kb * kCh, a.K), C::kWBytes,
+                                  fullw_bar(s));
                     } else {
-                        pend_kb[n_issued] = kb;
-                        pend_m[n_issued] = m_tile;
-                        ++n_issued;
+                        mbar_arrive_expect_tx(fullx_bar(s), C::kXBytes + 2 * tab);
+#pragma unroll
+                        for (int c = 0; c < kCh; ++c)
+                            tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN,
+                                        fullx_bar(s));
+                        const int g0 = (kb * KST) / a.G;
+                        const size_t toff = ((size_t)n_tile * a.ngroups + g0) * kPanelRows;
+                        bulk_load(st + C::kXBytes + C::kWBytes, a.s_g + toff, tab, fullx_bar(s));
+                        bulk_load(st + C::kXBytes + C::kWBytes + C::kTabRegion, a.zs + toff, tab, fullx_bar(s));
                     }
+                    if (tj < 32) QOQ_MARK((is_w ? 16 : 48) + tj);
+                    ++tj;
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) {
@@ -301,59 +328,49 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 i = t * ks + ks1;
             }
-            if (ok && !x_ready) release_x();
-            if (!x_ready) issued_x_none = 1;
         }
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer --
         if (lane == 0) {
             const uint32_t idesc = idesc_i8_m128(BN);
-            int s = 0, ta = 0;
-            uint32_t ph = 0, aph = 0, accph = 0;
+            int s = 0;
+            uint32_t ph = 0, accph = 0;
             bool ok = true;
-            for (long long i = i_begin; i < i_end && ok;) {
-                const long long t = i / ks;
-                const int ks0 = (int)(i - t * ks);
-                const int ks1 = (int)min((long long)ks, i_end - t * ks);
-                if (!wait_bounded(accempty_bar, accph ^ 1u, abort_flag, deadline)) break;
+            for (int i = i_begin; i < i_end && ok;) {
+                const int t = i / ks;
+                const int ks0 = i - t * ks;
+                const int ks1 = min(ks, i_end - t * ks);
+                if (!wait_bounded(accempty_bar, accph ^ 1u, abort_flag, budget)) break;
                 tc_fence_after();
                 for (int kb = ks0; kb < ks1; ++kb) {
-                    if (trace_j < 8) QOQ_MARK(224 + trace_j);
-                    if (!wait_bounded(fullx_bar(s), ph, abort_flag, deadline)) {
+                    // the dequant warps arrive on afull only after they have
+                    // seen this slot's X8 tiles land, so one wait covers both
+                    if (!wait_bounded(afull_bar(s), ph, abort_flag, budget)) {
                         ok = false;
                         break;
                     }
-                    if (trace_j < 8) QOQ_MARK(232 + trace_j);
-                    if (!wait_bounded(afull_bar(ta), aph, abort_flag, deadline)) {
-                        ok = false;
-                        break;
-                    }
-                    if (trace_j < 8) QOQ_MARK(240 + trace_j);
                     tc_fence_after();
-                    const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kStageBytes);
+                    if (tj < 32) QOQ_MARK(144 + tj);
+                    const uint32_t st = sbase + s * C::kStageBytes;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
+                    for (int j = 0; j < 4 * kCh; ++j) {
                         const uint32_t acc = (kb > ks0 || j > 0) ? 1u : 0u;
+                        const uint64_t bdesc = smem_desc_sw128(st + (j >> 2) * C::kXTile) + 2 * (j & 3);
                         if constexpr (A_TMEM) {
-                            mma_i8_ts(tmem_base, tmem_base + C::kACol0 + ta * 32 + j * 8, bdesc + 2 * j, idesc, acc);
+                            mma_i8_ts(tmem_base, tmem_base + C::kACol0 + s * C::kACols + j * 8, bdesc, idesc, acc);
                         } else {
                             const uint64_t adesc =
-                                smem_desc_sw128(sbase + STAGES * C::kStageBytes + ta * C::kABytes);
-                            mma_i8_ss(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, acc);
+                                smem_desc_sw128(sbase + STAGES * C::kStageBytes + s * C::kABytes + (j >> 2) * C::kATile) +
+                                2 * (j & 3);
+                            mma_i8_ss(tmem_base, adesc, bdesc, idesc, acc);
                         }
                     }
-                    if (trace_j < 8) QOQ_MARK(248 + trace_j);
                     mma_commit(empty_bar(s));
-                    mma_commit(aempty_bar(ta));
-                    if (trace_j < 32) QOQ_MARK(80 + trace_j);
-                    ++trace_j;
+                    if (tj < 32) QOQ_MARK(176 + tj);
+                    ++tj;
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
-                    }
-                    if (++ta == ASTAGES) {
-                        ta = 0;
-                        aph ^= 1u;
                     }
                 }
                 if (!ok) break;
@@ -361,6 +378,7 @@ __global__ void __launch_bounds__(320, 1)
                 accph ^= 1u;
                 i = t * ks + ks1;
             }
+            QOQ_MARK(3);
             // all MMAs this thread issued have completed once this arrives
             mma_commit(mmadone_bar);
             drain_wait(mmadone_bar, 0, 200000000ull);
@@ -369,60 +387,69 @@ __global__ void __launch_bounds__(320, 1)
         // ------------------------------------------------------ dequant --
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;  // output channel within the panel
-        int s = 0, ta = 0;
-        uint32_t ph = 0, aph = 0;
+        const bool per_group = (a.G == kBlockK);
+        int s = 0;
+        uint32_t ph = 0;
         bool ok = true;
-        for (long long i = i_begin; i < i_end && ok;) {
-            const long long t = i / ks;
-            const int ks0 = (int)(i - t * ks);
-            const int ks1 = (int)min((long long)ks, i_end - t * ks);
-            for (int kb = ks0; kb < ks1; ++kb) {
-                if (!wait_bounded(fullw_bar(s), ph, abort_flag, deadline)) {
+        for (int i = i_begin; i < i_end && ok;) {
+            const int t = i / ks;
+            const int ks1 = min(ks, i_end - t * ks);
+            for (int kb = i - t * ks; kb < ks1; ++kb) {
+                // weights, then X8 tiles + tables; seeing slot s filled again
+                // also means the MMA is done with A slot s
+                if (!wait_bounded(fullw_bar(s), ph, abort_flag, budget) ||
+                    !wait_bounded(fullx_bar(s), ph, abort_flag, budget)) {
                     ok = false;
                     break;
                 }
-                if (warp == 2 && lane == 0 && trace_j < 32) QOQ_MARK(112 + trace_j);
+                if (warp == 2 && lane == 0 && tj < 32) QOQ_MARK(80 + tj);
                 const uint8_t *st = smem + s * C::kStageBytes;
                 const uint8_t *sw = st + C::kXBytes;
-                uint4 v[4];
+                const uint8_t *tg = sw + C::kWBytes;
+                uint4 v[kCh][4];
+                uint32_t sg[kCh], zsv[kCh];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4 *>(sw + j * kSlabBytes + r * 16);
-                const uint32_t sg = st[C::kXBytes + C::kWBytes + r];
-                const uint32_t zsv = st[C::kXBytes + C::kWBytes + 128 + r];
+                for (int c = 0; c < kCh; ++c) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        v[c][j] = *reinterpret_cast<const uint4 *>(sw + c * kChunkBytes + j * kSlabBytes + r * 16);
+                    const int g = per_group ? c : 0;
+                    sg[c] = tg[g * 128 + r];
+                    zsv[c] = tg[C::kTabRegion + g * 128 + r];
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty_bar(s));
-                if (!wait_bounded(aempty_bar(ta), aph ^ 1u, abort_flag, deadline)) {
-                    ok = false;
-                    break;
-                }
                 tc_fence_after();
-                const uint32_t bias = zero_comp_bias(zsv);
-                uint32_t w8[32];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) dequant_slab(v[j], sg, bias, &w8[8 * j]);
+                for (int c = 0; c < kCh; ++c) {
+                    const uint32_t bias = zero_comp_bias(zsv[c]);
+                    uint32_t w8[32];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) dequant_slab(v[c][j], sg[c], bias, &w8[8 * j]);
+                    if constexpr (A_TMEM) {
+                        tmem_st32(tmem_base + ((uint32_t)(quarter * 32) << 16) + C::kACol0 + s * C::kACols + c * 32,
+                                  w8);
+                    } else {
+                        uint8_t *arow = smem + STAGES * C::kStageBytes + s * C::kABytes + c * C::kATile + r * 128;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            *reinterpret_cast<uint4 *>(arow + ((q ^ (r & 7)) << 4)) =
+                                make_uint4(w8[4 * q], w8[4 * q + 1], w8[4 * q + 2], w8[4 * q + 3]);
+                    }
+                }
                 if constexpr (A_TMEM) {
-                    tmem_st32(tmem_base + ((uint32_t)(quarter * 32) << 16) + C::kACol0 + ta * 32, w8);
                     tmem_wait_st();
                     tc_fence_before();
                 } else {
-                    uint8_t *arow = smem + STAGES * C::kStageBytes + ta * C::kABytes + r * 128;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4 *>(arow + ((c ^ (r & 7)) << 4)) =
-                            make_uint4(w8[4 * c], w8[4 * c + 1], w8[4 * c + 2], w8[4 * c + 3]);
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(afull_bar(ta));
-                if (warp == 2 && lane == 0 && trace_j < 32) QOQ_MARK(48 + trace_j);
-                ++trace_j;
+                if (lane == 0) mbar_arrive(afull_bar(s));
+                if (warp == 2 && lane == 0 && tj < 32) QOQ_MARK(112 + tj);
+                ++tj;
                 if (++s == STAGES) {
                     s = 0;
                     ph ^= 1u;
-                }
-                if (++ta == ASTAGES) {
-                    ta = 0;
-                    aph ^= 1u;
                 }
             }
             i = t * ks + ks1;
@@ -433,127 +460,195 @@ __global__ void __launch_bounds__(320, 1)
         const int r = quarter * 32 + lane;
         const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
         uint32_t accph = 0;
-        const long long first_tile = i_begin / ks;
         grid_dependency_wait();  // s_x comes from the preceding kernel
-        for (long long i = i_begin; i < i_end;) {
-            const long long t = i / ks;
-            const int ks0 = (int)(i - t * ks);
-            const int ks1 = (int)min((long long)ks, i_end - t * ks);
-            const int m_tile = (int)(t % a.m_tiles);
-            const int n_tile = (int)(t / a.m_tiles);
+        for (int i = i_begin; i < i_end;) {
+            const int t = i / ks;
+            const int ks0 = i - t * ks;
+            const int ks1 = min(ks, i_end - t * ks);
+            const int m_tile = t % a.m_tiles;
+            const int n_tile = t / a.m_tiles;
             const int n = n_tile * kPanelRows + r;
             const int m0 = m_tile * BN;
-            const int live = min(BN, a.M - m0);      // token columns that exist
-            const int nchunks = (live + 15) >> 4;     // 16-column chunks holding them
+            const int nchunks = (min(BN, a.M - m0) + 15) >> 4;  // 16-token chunks that exist
             const bool partial = !(ks0 == 0 && ks1 == ks);
-            if (!wait_bounded(accfull_bar, accph, abort_flag, deadline)) break;
-            if (warp == 6 && lane == 0 && trace_j < 4) QOQ_MARK(145 + trace_j);
-            tc_fence_after();
-            if (!partial) {
-                const float sc = half_bits_to_float(a.s_c[n]);
-#pragma unroll 1
-                for (int cc = 0; cc < nchunks; ++cc) {
-                    uint32_t v[16];
-                    tmem_ld16(trow + cc * 16, v);
-                    store_outputs(a, m0 + cc * 16, n, sc, reinterpret_cast<const int32_t *>(v));
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(accempty_bar);
-            } else {
-                // Partial tile: 16 consecutive columns of one channel are 64
-                // contiguous bytes, [chunk][channel][16] per slot.
-                const int slot = (t == first_tile) ? 0 : 1;
-                int4 *part = reinterpret_cast<int4 *>(a.ws_part + (size_t)(cta * 2 + slot) * BN * kPanelRows);
-#pragma unroll 1
-                for (int cc = 0; cc < nchunks; ++cc) {
-                    uint32_t v[16];
-                    tmem_ld16(trow + cc * 16, v);
-                    int4 *dst = part + ((size_t)cc * kPanelRows + r) * 4;
+            // token scales of this tile, one per lane per 32 tokens
+            float sx_reg[C::kSx];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dst[j] = make_int4((int)v[4 * j], (int)v[4 * j + 1], (int)v[4 * j + 2], (int)v[4 * j + 3]);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(accempty_bar);
-                // publish this partial, then count arrivals for the quarter
-                __threadfence();
-                __syncwarp();
-                const long long c_lo = cta_of(t * ks, P, T);
-                const long long c_hi = cta_of(t * ks + ks - 1, P, T);
-                int *counter = a.ws_cnt + c_lo * 4 + quarter;
-                int last = 0;
+            for (int q = 0; q < C::kSx; ++q) {
+                const int m = m0 + q * 32 + lane;
+                sx_reg[q] = (q * 32 + lane < BN && m < a.M) ? half_bits_to_float(__ldg(a.s_x + m)) : 0.0f;
+            }
+            const float sc = half_bits_to_float(__ldg(a.s_c + n));
+            const int c_lo = partial ? cta_of(t * ks, P, T) : cta;
+            const bool finisher = partial && c_lo == cta;     // this CTA completes a split tile
+            const int c_hi = finisher ? cta_of(t * ks + ks - 1, P, T) : cta;
+            // A finisher's split tile is the last tile of its range, and the
+            // other contributors published their parts at the start of
+            // theirs: wait for the count and sum their partials now, while
+            // this CTA's own MMAs for the tile are still running.
+            bool ready = true;
+            constexpr bool kPresum = (BN <= 64);
+            constexpr int kGrp = BN < 64 ? BN : 64;  // accumulator columns per TMEM load
+            int32_t pre[kPresum ? BN : 1];
+            if (finisher) {
+                int *counter = a.ws_cnt + cta * 4 + quarter;
                 if (lane == 0) {
-                    const int old = atomicAdd(counter, 1);
-                    last = (old == (int)(c_hi - c_lo));
-                }
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (last) {
-                    __threadfence();
-                    const float sc = half_bits_to_float(a.s_c[n]);
-                    const int nc = (int)(c_hi - c_lo + 1);
-#pragma unroll 1
-                    for (int cc = 0; cc < nchunks; ++cc) {
-                        int32_t sum[16];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) sum[j] = 0;
-                        // up to 4 contributors per batch: all 16 loads are in
-                        // flight before the first add
-#pragma unroll 1
-                        for (int b = 0; b < nc; b += 4) {
-                            int4 ld[4][4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                if (b + u < nc) {
-                                    const long long c2 = c_lo + b + u;
-                                    const int sl = (t == range_begin(c2, P, T) / ks) ? 0 : 1;
-                                    const int4 *src = reinterpret_cast<const int4 *>(
-                                                          a.ws_part + (size_t)(c2 * 2 + sl) * BN * kPanelRows) +
-                                                      ((size_t)cc * kPanelRows + r) * 4;
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) ld[u][j] = __ldcg(src + j);
-                                } else {
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) ld[u][j] = make_int4(0, 0, 0, 0);
-                                }
+                    const int want = c_hi - cta;
+                    if (ld_acquire_gpu(counter) < want) {
+                        const uint64_t start = global_timer_ns();
+                        while (ld_acquire_gpu(counter) < want) {
+                            if (*abort_flag || global_timer_ns() - start > budget) {
+                                *abort_flag = 1;
+                                ready = false;
+                                break;
                             }
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    sum[4 * j] += ld[u][j].x;
-                                    sum[4 * j + 1] += ld[u][j].y;
-                                    sum[4 * j + 2] += ld[u][j].z;
-                                    sum[4 * j + 3] += ld[u][j].w;
-                                }
                         }
-                        store_outputs(a, m0 + cc * 16, n, sc, sum);
                     }
-                    if (lane == 0) *counter = 0;  // ready for the next call
-                    if (warp == 6 && lane == 0 && trace_j < 4) QOQ_MARK(155 + trace_j);
+                    if (ready) *counter = 0;  // ready for the next call
+                }
+                ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
+                __syncwarp();  // the other lanes read the partials after lane 0's acquire
+                if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(224 + tj);
+                if constexpr (kPresum) {
+#pragma unroll
+                    for (int q = 0; q < BN; ++q) pre[q] = 0;
+                    if (ready) {
+#pragma unroll 1
+                        for (int c2 = cta + 1; c2 <= c_hi; ++c2) {
+                            const int4 *src = reinterpret_cast<const int4 *>(a.ws_part + (size_t)c2 * BN * kPanelRows);
+                            int4 ld[BN / 4];
+#pragma unroll
+                            for (int cc = 0; cc < BN / 16; ++cc)
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    ld[cc * 4 + j] = (cc < nchunks) ? __ldcg(src + ((size_t)cc * kPanelRows + r) * 4 + j)
+                                                                    : make_int4(0, 0, 0, 0);
+#pragma unroll
+                            for (int j = 0; j < BN / 4; ++j) {
+                                pre[4 * j] += ld[j].x;
+                                pre[4 * j + 1] += ld[j].y;
+                                pre[4 * j + 2] += ld[j].z;
+                                pre[4 * j + 3] += ld[j].w;
+                            }
+                        }
+                    }
                 }
             }
-            if (warp == 6 && lane == 0 && trace_j < 4) QOQ_MARK(150 + trace_j);
-            ++trace_j;
+            if (!wait_bounded(accfull_bar, accph, abort_flag, budget)) break;
+            if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(208 + tj);
+            tc_fence_after();
+            if (partial && !finisher) {
+                // a later contributor: publish the partial, count it, done
+                int4 *my_part = reinterpret_cast<int4 *>(a.ws_part + (size_t)cta * BN * kPanelRows);
+#pragma unroll 1
+                for (int g0 = 0; g0 < nchunks; g0 += kGrp / 16) {
+                    uint32_t v[kGrp];
+                    tmem_load_cols<kGrp>(trow + g0 * 16, v);
+#pragma unroll
+                    for (int u = 0; u < kGrp / 16; ++u) {
+                        if (g0 + u < nchunks) {
+                            int4 *dst = my_part + ((size_t)(g0 + u) * kPanelRows + r) * 4;
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                dst[j] = make_int4((int)v[16 * u + 4 * j], (int)v[16 * u + 4 * j + 1],
+                                                   (int)v[16 * u + 4 * j + 2], (int)v[16 * u + 4 * j + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(accempty_bar);
+                    red_release_gpu_add(a.ws_cnt + c_lo * 4 + quarter, 1);
+                }
+            } else {
+                // a whole tile, or a split tile this CTA finishes
+                if (ready) {
+#pragma unroll 1
+                    for (int g0 = 0; g0 < nchunks; g0 += kGrp / 16) {
+                    uint32_t vg[kGrp];
+                    tmem_load_cols<kGrp>(trow + g0 * 16, vg);
+                    if (warp == 6 && lane == 0 && tj < 2 && g0 == 0) QOQ_MARK(232 + tj * 8);
+#pragma unroll
+                    for (int u = 0; u < kGrp / 16; ++u) {
+                        const int cc = g0 + u;
+                        if (cc >= nchunks) break;
+                        if (warp == 6 && lane == 0 && tj < 2 && cc < 6) QOQ_MARK(233 + tj * 8 + cc);
+                        int32_t acc[16];
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) acc[q] = (int32_t)vg[16 * u + q];
+                        if constexpr (kPresum) {
+                            if (finisher) {
+#pragma unroll
+                                for (int q = 0; q < 16; ++q) {
+                                    // pre[] is indexed by a runtime chunk: select with unrolled compares
+                                    int32_t add = 0;
+#pragma unroll
+                                    for (int c3 = 0; c3 < BN / 16; ++c3)
+                                        if (c3 == cc) add = pre[c3 * 16 + q];
+                                    acc[q] += add;
+                                }
+                            }
+                        } else if (finisher) {
+                            // partials of the later contributors, 16 loads in flight per batch
+#pragma unroll 1
+                            for (int c2 = cta + 1; c2 <= c_hi; c2 += 4) {
+                                int4 ld[4][4];
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    if (c2 + u <= c_hi) {
+                                        const int4 *src = reinterpret_cast<const int4 *>(
+                                                              a.ws_part + (size_t)(c2 + u) * BN * kPanelRows) +
+                                                          ((size_t)cc * kPanelRows + r) * 4;
+#pragma unroll
+                                        for (int j = 0; j < 4; ++j) ld[u][j] = __ldcg(src + j);
+                                    } else {
+#pragma unroll
+                                        for (int j = 0; j < 4; ++j) ld[u][j] = make_int4(0, 0, 0, 0);
+                                    }
+                                }
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        acc[4 * j] += ld[u][j].x;
+                                        acc[4 * j + 1] += ld[u][j].y;
+                                        acc[4 * j + 2] += ld[u][j].z;
+                                        acc[4 * j + 3] += ld[u][j].w;
+                                    }
+                            }
+                        }
+                        float sxr = sx_reg[0];
+#pragma unroll
+                        for (int q = 1; q < C::kSx; ++q)
+                            if ((cc >> 1) == q) sxr = sx_reg[q];
+                        store_outputs(a, m0 + cc * 16, cc, n, sc, sxr, acc);
+                    }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(accempty_bar);
+            }
+            if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(216 + tj);
+            ++tj;
             accph ^= 1u;
             i = t * ks + ks1;
         }
+        if (warp == 6 && lane == 0) QOQ_MARK(4);
     }
 
     __syncwarp();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (threadIdx.x == 0) QOQ_MARK(2);
-    if (threadIdx.x == 0 && *abort_flag) {
-        atomicExch(&g_dev_error, 1);
-        // thread 0 is the producer: let its own copies land before exit
+    QOQ_MARK(2);
+    if ((threadIdx.x == 0 || threadIdx.x == 320) && *abort_flag) {
+        if (threadIdx.x == 0) atomicExch(&g_dev_error, 1);
+        // the producers: let their own copies land before the CTA exits
         for (int q = 0; q < STAGES; ++q)
-            if (issued & (1u << q)) {
-                drain_wait(fullw_bar(q), (issued_par >> q) & 1u, 200000000ull);
-                if (!issued_x_none) drain_wait(fullx_bar(q), (issued_par >> q) & 1u, 200000000ull);
-            }
+            if (issued & (1u << q))
+                drain_wait(threadIdx.x == 0 ? fullw_bar(q) : fullx_bar(q), (issued_par >> q) & 1u, 200000000ull);
     }
     if (warp == 0) {
         __syncwarp();
@@ -563,7 +658,18 @@ __global__ void __launch_bounds__(320, 1)
 
 // ----------------------------------------------------------------- host --
 #ifdef QOQ_TRACE
-extern unsigned long long *g_trace_buffer;
+unsigned long long *g_trace_buffer = nullptr;
+
+__global__ void stamp_kernel(unsigned long long *dst)
+{
+    *dst = global_timer_ns();
+}
+
+cudaError_t debug_stamp(unsigned long long *dst, cudaStream_t stream)
+{
+    stamp_kernel<<<1, 1, 0, stream>>>(dst);
+    return cudaGetLastError();
+}
 #endif
 
 namespace {
@@ -587,11 +693,11 @@ EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-template <int BN, int STAGES, int ASTAGES, bool A_TMEM>
+template <int BN, int KST, int STAGES, bool A_TMEM>
 cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, STAGES, ASTAGES, A_TMEM>;
-    auto kern = w4a8_gemm_kernel<BN, STAGES, ASTAGES, A_TMEM>;
+    using C = GemmCfg<BN, KST, STAGES, A_TMEM>;
+    auto kern = w4a8_gemm_kernel<BN, KST, STAGES, A_TMEM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: the GEMM may start (and stream weights)
@@ -600,7 +706,7 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     // touches X8 or s_x.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(320);
+    cfg.blockDim = dim3(352);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -613,24 +719,40 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     return cudaGetLastError();
 }
 
+// Ring depth per token-tile width and stage depth: as many stages as fit
+// in shared memory (~227 KB) and, with the A operand in TMEM, as many A
+// slots as fit next to the accumulator in 512 columns.
 template <bool A_TMEM>
-cudaError_t dispatch(int BN, const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
+cudaError_t dispatch(int BN, int KST, const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
 {
+    if (KST == 256) {
+        switch (BN) {
+        case 16: return launch_cfg<16, 256, A_TMEM ? 7 : 4, A_TMEM>(tmap, args, grid, stream);
+        case 32: return launch_cfg<32, 256, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
+        default: return launch_cfg<64, 256, A_TMEM ? 6 : 3, A_TMEM>(tmap, args, grid, stream);
+        }
+    }
     switch (BN) {
-    // TMEM A ring: as many 32-column slots as fit next to the accumulator
-    // in a power-of-two allocation (256 columns for BN <= 64, else 512)
-    case 16: return launch_cfg<16, A_TMEM ? 16 : 12, A_TMEM ? 7 : 2, A_TMEM>(tmap, args, grid, stream);
-    case 32: return launch_cfg<32, A_TMEM ? 14 : 11, A_TMEM ? 7 : 2, A_TMEM>(tmap, args, grid, stream);
-    case 64: return launch_cfg<64, A_TMEM ? 11 : 9, A_TMEM ? 6 : 2, A_TMEM>(tmap, args, grid, stream);
-    case 128: return launch_cfg<128, A_TMEM ? 7 : 6, A_TMEM ? 7 : 2, A_TMEM>(tmap, args, grid, stream);
-    default: return launch_cfg<256, 4, A_TMEM ? 4 : 2, A_TMEM>(tmap, args, grid, stream);
+    case 16: return launch_cfg<16, 128, A_TMEM ? 12 : 7, A_TMEM>(tmap, args, grid, stream);
+    case 32: return launch_cfg<32, 128, A_TMEM ? 12 : 7, A_TMEM>(tmap, args, grid, stream);
+    case 64: return launch_cfg<64, 128, A_TMEM ? 11 : 6, A_TMEM>(tmap, args, grid, stream);
+    case 128: return launch_cfg<128, 128, A_TMEM ? 7 : 5, A_TMEM>(tmap, args, grid, stream);
+    default: return launch_cfg<256, 128, A_TMEM ? 4 : 3, A_TMEM>(tmap, args, grid, stream);
     }
 }
 
-long long gemm_units(int M, int N, int K, int BN)
+// K depth of one pipeline stage: two packed chunks when K allows it and the
+// token tile leaves room for enough stages, else one.
+int gemm_stage_k(int M, int K)
 {
+    return (gemm_block_n(M) <= 64 && K % 256 == 0) ? 256 : 128;
+}
+
+long long gemm_units(int M, int N, int K)
+{
+    const int BN = gemm_block_n(M);
     const long long m_tiles = (M + BN - 1) / BN;
-    return m_tiles * (long long)(N / kPanelRows) * (long long)(K / kBlockK);
+    return m_tiles * (long long)(N / kPanelRows) * (long long)(K / gemm_stage_k(M, K));
 }
 
 }  // namespace
@@ -640,12 +762,16 @@ int gemm_block_n(int M)
     return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
 }
 
+bool gemm_shape_supported(int M, int N, int K)
+{
+    return gemm_units(M, N, K) < (1ll << 31);
+}
+
 size_t gemm_workspace_bytes(int M, int N, int K)
 {
     const int BN = gemm_block_n(M);
-    const long long units = gemm_units(M, N, K, BN);
-    const long long grid = std::min<long long>(kMaxCtas, units);
-    return kCounterBytes + (size_t)grid * 2 * BN * kPanelRows * sizeof(int32_t);
+    const long long grid = std::min<long long>(kMaxCtas, gemm_units(M, N, K));
+    return kCounterBytes + (size_t)grid * BN * kPanelRows * sizeof(int32_t);
 }
 
 cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
@@ -654,6 +780,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
 {
     *tmap_status = 0;
     const int BN = gemm_block_n(M);
+    const int KST = gemm_stage_k(M, K);
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) {
         *tmap_status = -1;
@@ -674,7 +801,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     int dev = 0, sms = kMaxCtas;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long long units = gemm_units(M, N, K, BN);
+    const long long units = gemm_units(M, N, K);
     const long long grid = std::min<long long>(std::min(kMaxCtas, sms), units);
 
     GemmArgs args;
@@ -692,19 +819,16 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     args.K = K;
     args.G = G;
     args.m_tiles = (M + BN - 1) / BN;
-    args.ks = K / kBlockK;
-    args.total = units;
+    args.ks = K / KST;
+    args.ngroups = K / G;
+    args.total = (int)units;
     args.timeout_ns = 2000000000ull;  // 2 s for one wait: far beyond any legitimate one
 #ifdef QOQ_TRACE
     args.trace = g_trace_buffer;
 #endif
-    return a_in_tmem ? dispatch<true>(BN, tmap, args, (int)grid, stream)
-                     : dispatch<false>(BN, tmap, args, (int)grid, stream);
+    return a_in_tmem ? dispatch<true>(BN, KST, tmap, args, (int)grid, stream)
+                     : dispatch<false>(BN, KST, tmap, args, (int)grid, stream);
 }
-
-#ifdef QOQ_TRACE
-unsigned long long *g_trace_buffer = nullptr;
-#endif
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value)
 {

@@ -30,6 +30,10 @@ cudaError_t launch_dequant(const uint8_t *Wp, const uint8_t *s_g, const uint8_t 
 // Tile width along M (tokens) the GEMM uses for a given M.
 int gemm_block_n(int M);
 
+// False when the shape has more work units than the GEMM's 32-bit
+// scheduling arithmetic covers.
+bool gemm_shape_supported(int M, int N, int K);
+
 size_t gemm_workspace_bytes(int M, int N, int K);
 
 // Returns cudaSuccess or the launch / tensor-map error.  `tmap_status`
@@ -41,6 +45,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
 
 #ifdef QOQ_TRACE
 extern unsigned long long *g_trace_buffer;
+cudaError_t debug_stamp(unsigned long long *dst, cudaStream_t stream);
 #endif
 
 // Device error flag of the current device: read and clear (synchronous).

@@ -105,8 +105,9 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
         const float sgf = (float)sg;
         const int z = (int)rintf(__fdiv_rn((float)(-mn), sgf));
         if (lane == 0) {
-            s_g[(size_t)g * N + n] = (uint8_t)sg;
-            zs[(size_t)g * N + n] = (uint8_t)(z * sg);
+            const size_t ti = ((size_t)p * (K / G) + g) * kPanelRows + rr;
+            s_g[ti] = (uint8_t)sg;
+            zs[ti] = (uint8_t)(z * sg);
         }
         for (int kc = k_lo; kc < k_hi; kc += 128) {
             const float4 v = __ldg(reinterpret_cast<const float4 *>(w + kc + lane * 4));
@@ -170,6 +171,10 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const uint16_t *
     // the GEMM that consumes X8 may launch now and start streaming weights;
     // it waits for this grid to finish before it reads X8 or s_x
     grid_launch_dependents();
+    // this grid may itself have launched early (programmatic dependent
+    // launch): X, and the buffers written below, belong to the kernels
+    // before it until they have finished
+    grid_dependency_wait();
     const int m = blockIdx.x;
     const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)m * K);
     uint2 *out = reinterpret_cast<uint2 *>(X8 + (size_t)m * K);
@@ -221,9 +226,9 @@ __global__ void dequant_kernel(const uint8_t *__restrict__ Wp, const uint8_t *__
     const int k0 = (int)(idx % slices) * kSlabK;
     const uint4 v = *reinterpret_cast<const uint4 *>(Wp + chunk_offset(n / kPanelRows, k0 / kBlockK, K) +
                                                      ((k0 % kBlockK) / kSlabK) * kSlabBytes + (n % kPanelRows) * 16);
-    const int g = k0 / G;
-    const uint32_t sg = s_g[(size_t)g * N + n];
-    const uint32_t bias = zero_comp_bias(zs[(size_t)g * N + n]);
+    const size_t ti = ((size_t)(n / kPanelRows) * (K / G) + k0 / G) * kPanelRows + n % kPanelRows;
+    const uint32_t sg = s_g[ti];
+    const uint32_t bias = zero_comp_bias(zs[ti]);
     uint32_t w8[8];
     dequant_slab(v, sg, bias, w8);
     uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)n * K + k0);
@@ -242,7 +247,21 @@ cudaError_t launch_pack(const float *W, int N, int K, int G, uint8_t *Wp, uint16
 
 cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, cudaStream_t stream)
 {
-    act_quant_kernel<<<M, kActThreads, 0, stream>>>(X, K, X8, s_x);
+    // programmatic dependent launch: the CTAs may be scheduled while the
+    // previous kernel (for instance the previous layer's GEMM) finishes;
+    // they wait for it at the top of the kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)M);
+    cfg.blockDim = dim3(kActThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, X, K, X8, s_x);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

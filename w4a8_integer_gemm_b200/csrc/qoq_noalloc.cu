@@ -67,7 +67,9 @@ int qoq_w4a8_gemm_noalloc(const int8_t *X8, const uint16_t *s_x, const uint8_t *
     if (!aligned16(X8) || !aligned16(s_x) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) ||
         !aligned16(zs) || !aligned16(Y))
         return QOQ_ERR_INVALID_ARG;
-    if (qoq_gemm_workspace_bytes(M, N, K, group_size) > kScratchBytes) return QOQ_ERR_SCRATCH_TOO_SMALL;
+    const size_t need = qoq_gemm_workspace_bytes(M, N, K, group_size);
+    if (need == 0) return QOQ_ERR_INVALID_ARG;
+    if (need > kScratchBytes) return QOQ_ERR_SCRATCH_TOO_SMALL;
     int major = 0, minor = 0, dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
