@@ -106,32 +106,36 @@ __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
     return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
 }
 
-template <int BN, int KST, int STAGES, bool A_TMEM>
+template <int BN, int KST, int SW, int SX, bool A_TMEM>
 struct GemmCfg {
-    static constexpr int ASTAGES = STAGES;               // A slot s belongs to stage slot s
-    static constexpr int kChunks = KST / kBlockK;        // packed 8 KB chunks per stage
+    static constexpr int kChunks = KST / kBlockK;        // packed 8 KB chunks per K block
     static constexpr int kXTile = BN * 128;              // one [BN][128 B] swizzled X8 tile
-    static constexpr int kXBytes = kChunks * kXTile;
-    static constexpr int kWBytes = kChunks * kChunkBytes;
-    static constexpr int kTabRegion = 128 * kChunks;     // s_g region, then zs region
-    static constexpr int kStageBytes = ((kXBytes + kWBytes + 2 * kTabRegion + 1023) / 1024) * 1024;
+    static constexpr int kXSlot = kChunks * kXTile;      // X8 tiles of one K block
     static constexpr int kATile = 128 * 128;             // one [128][128 B] swizzled A tile
     static constexpr int kABytes = A_TMEM ? 0 : kChunks * kATile;
-    static constexpr int kBarOff = STAGES * kStageBytes + ASTAGES * kABytes;
-    static constexpr int kNumBars = 4 * STAGES + 3;
+    static constexpr int kWBytes = kChunks * kChunkBytes;
+    static constexpr int kTabRegion = 128 * kChunks;     // s_g region, then zs region
+    static constexpr int kWSlot = kWBytes + 2 * kTabRegion;
+    // shared memory: [X8 ring][A ring (A in shared memory only)][W ring][barriers]
+    static constexpr int kAOff = SX * kXSlot;
+    static constexpr int kWOff = kAOff + SX * kABytes;
+    static constexpr int kStgOff = kWOff + SW * kWSlot;  // per epilogue warp: 16 tokens x 32 channels FP16
+    static constexpr int kBarOff = kStgOff + 4 * 1024;
+    static constexpr int kNumBars = 2 * SW + 3 * SX + 3;
     static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
     // at least ~120 KB so that exactly one CTA (and one TMEM allocation)
     // lives on each SM; +1024 for manual alignment of the dynamic base
     static constexpr int kSmemBytes = (kUsed > 120 * 1024 ? kUsed : 120 * 1024) + 1024;
     static constexpr uint32_t kACols = KST / 4;          // TMEM columns of one A slot
     static constexpr uint32_t kACol0 = BN;               // first TMEM column of the A ring
-    static constexpr uint32_t kTmemCols = pow2_cols(BN + (A_TMEM ? ASTAGES * kACols : 0));
+    static constexpr uint32_t kTmemCols = pow2_cols(BN + (A_TMEM ? SX * kACols : 0));
     static constexpr int kSx = (BN + 31) / 32;           // s_x registers per lane
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
-    static_assert(KST == 128 || KST == 256, "stage depth");
-    static_assert(BN + (A_TMEM ? ASTAGES * kACols : 0) <= 512, "TMEM columns");
+    static_assert(KST == 128 || KST == 256, "K block");
+    static_assert(BN + (A_TMEM ? SX * kACols : 0) <= 512, "TMEM columns");
     static_assert(kUsed <= 227 * 1024, "shared memory");
-    static_assert(STAGES <= 32, "ring bookkeeping masks");
+    static_assert(SW <= 32 && SX <= 32, "ring bookkeeping masks");
+    static_assert(kXSlot % 1024 == 0 && kAOff % 1024 == 0 && kWOff % 1024 == 0, "swizzle atoms");
 };
 
 // The CTA whose stream-K range contains unit i (ranges: [c*T/P, (c+1)*T/P)).
@@ -179,20 +183,33 @@ __device__ __forceinline__ uint16_t scale_to_half(int32_t acc, float sx, float s
 }
 
 // FP16 outputs (and optionally the INT32 accumulators) of the 16
-// consecutive tokens m0.. of chunk `cc` for channel n.  The token scales
-// come from the lanes' registers: lane l of sx holds s_x[m0 - 16*(cc&1) + l].
-// A warp's store covers 32 consecutive channels: 64 contiguous bytes.
-__device__ __forceinline__ void store_outputs(const GemmArgs &a, int m0, int cc, int n, float sc, float sx,
-                                              const int32_t *acc)
+// consecutive tokens m0.. of chunk `cc` for this lane's channel n0 + lane.
+// The token scales come from the lanes' registers: lane l of sx holds
+// s_x[m0 - 16*(cc&1) + l].  The warp stages its 16 x 32 block in its own
+// 1 KB of shared memory ([token][32 channels], 64 bytes per token) and then
+// writes Y with 16-byte stores: in store j, lane l writes token 8*j + l/4,
+// channels 8*(l%4) .. 8*(l%4)+7.
+__device__ __forceinline__ void store_outputs(const GemmArgs &a, uint8_t *stg, int m0, int cc, int n0, int lane,
+                                              float sc, float sx, const int32_t *acc)
 {
+    __syncwarp();  // the previous chunk's reads of the staging block are done
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
         const float sxq = __shfl_sync(0xffffffffu, sx, (cc & 1) * 16 + q);
+        *reinterpret_cast<uint16_t *>(stg + q * 64 + lane * 2) = scale_to_half(acc[q], sxq, sc);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int q = 8 * j + (lane >> 2);
         const int m = m0 + q;
-        if (m < a.M) {
-            a.Y[(size_t)m * a.N + n] = scale_to_half(acc[q], sxq, sc);
-            if (a.acc_dbg) a.acc_dbg[(size_t)m * a.N + n] = acc[q];
-        }
+        const uint4 v = *reinterpret_cast<const uint4 *>(stg + q * 64 + (lane & 3) * 16);
+        if (m < a.M) *reinterpret_cast<uint4 *>(a.Y + (size_t)m * a.N + n0 + (lane & 3) * 8) = v;
+    }
+    if (a.acc_dbg) {
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            if (m0 + q < a.M) a.acc_dbg[(size_t)(m0 + q) * a.N + n0 + lane] = acc[q];
     }
 }
 
@@ -211,24 +228,28 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *v)
     }
 }
 
-template <int BN, int KST, int STAGES, bool A_TMEM>
+template <int BN, int KST, int SW, int SX, bool A_TMEM>
 __global__ void __launch_bounds__(352, 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs a)
 {
-    using C = GemmCfg<BN, KST, STAGES, A_TMEM>;
+    using C = GemmCfg<BN, KST, SW, SX, A_TMEM>;
     constexpr int kCh = C::kChunks;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar0 = sbase + C::kBarOff;
-    // per ring slot: fullw (packed weights landed), fullx (X8 tiles and
-    // group tables landed), afull (dequantized A operand written), empty
-    // (dequant warps and the MMA are done with the slot)
-    auto fullw_bar = [&](int s) { return bar0 + 8u * s; };
-    auto fullx_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-    auto afull_bar = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
-    const uint32_t accfull_bar = bar0 + 8u * (4 * STAGES);
+    // W ring (packed weights + group tables of one K block):
+    //   wfull (bulk copies landed), wempty (the dequant warps have read it)
+    // X8/A ring (X8 tiles in shared memory, dequantized weights in A slot):
+    //   xfull (X8 tiles landed), afull (A slot written; the dequant warps
+    //   arrive only after they have seen xfull, so it covers both),
+    //   xaempty (the MMAs reading the slot have completed)
+    auto wfull_bar = [&](int s) { return bar0 + 8u * s; };
+    auto wempty_bar = [&](int s) { return bar0 + 8u * (SW + s); };
+    auto xfull_bar = [&](int s) { return bar0 + 8u * (2 * SW + s); };
+    auto afull_bar = [&](int s) { return bar0 + 8u * (2 * SW + SX + s); };
+    auto xaempty_bar = [&](int s) { return bar0 + 8u * (2 * SW + 2 * SX + s); };
+    const uint32_t accfull_bar = bar0 + 8u * (2 * SW + 3 * SX);
     const uint32_t accempty_bar = accfull_bar + 8u;
     const uint32_t mmadone_bar = accfull_bar + 16u;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kNumBars * 8);
@@ -236,17 +257,28 @@ __global__ void __launch_bounds__(352, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Scheduling state, computed first: its reads of the kernel parameters
+    // start filling the constant cache while the prologue below runs.
+    const int P = gridDim.x;
+    const int T = a.total;
+    const int cta = blockIdx.x;
+    const int i_begin = range_begin(cta, P, T);
+    const int i_end = range_begin(cta + 1, P, T);
+    const int ks = a.ks;
 
 #ifdef QOQ_TRACE
     const long long trace_t0 = clock64();
     if (threadIdx.x == 0 && a.trace) a.trace[(size_t)blockIdx.x * 256 + 255] = global_timer_ns();
 #endif
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(fullw_bar(s), 1);
-            mbar_init(fullx_bar(s), 1);
-            mbar_init(empty_bar(s), 1 + 4);  // MMA commit + 4 dequant warps
+        for (int s = 0; s < SW; ++s) {
+            mbar_init(wfull_bar(s), 1);
+            mbar_init(wempty_bar(s), 4);     // 4 dequant warps
+        }
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(xfull_bar(s), 1);
             mbar_init(afull_bar(s), 4);      // 4 dequant warps
+            mbar_init(xaempty_bar(s), 1);    // MMA commit
         }
         mbar_init(accfull_bar, 1);
         mbar_init(accempty_bar, 4);
@@ -268,60 +300,74 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t budget = a.timeout_ns;
     QOQ_MARK(1);
-
-    const int P = gridDim.x;
-    const int T = a.total;
-    const int cta = blockIdx.x;
-    const int i_begin = range_begin(cta, P, T);
-    const int i_end = range_begin(cta + 1, P, T);
-    const int ks = a.ks;
     // ring slots a producer has filled, and the phase parity of each slot's
     // latest fill (drained on the way out of an aborted CTA)
     uint32_t issued = 0, issued_par = 0;
     int tj = 0;  // trace: per-role unit counter
     (void)tj;
 
-    if (warp == 0 || warp == 10) {
-        // --------------------------------------- producers (W and X8) --
+    if (warp == 0) {
+        // ---------------------------------------------- weight producer --
         if (lane == 0) {
-            const bool is_w = (warp == 0);
-            if (!is_w) grid_dependency_wait();  // X8 comes from the preceding kernel
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            const uint32_t tab = (a.G == kBlockK) ? (uint32_t)C::kTabRegion : 128u;
+            const bool per_group = (a.G == kBlockK);
+            const uint32_t tab = per_group ? (uint32_t)C::kTabRegion : 128u;
             for (int i = i_begin; i < i_end && ok;) {
                 const int t = i / ks;
-                const int ks0 = i - t * ks;
                 const int ks1 = min(ks, i_end - t * ks);
-                const int m_tile = t % a.m_tiles;
                 const int n_tile = t / a.m_tiles;
-                for (int kb = ks0; kb < ks1; ++kb) {
-                    if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, budget)) {
+                for (int kb = i - t * ks; kb < ks1; ++kb) {
+                    if (!wait_bounded(wempty_bar(s), ph ^ 1u, abort_flag, budget)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t st = sbase + s * C::kStageBytes;
-                    if (is_w) {
-                        mbar_arrive_expect_tx(fullw_bar(s), C::kWBytes);
-                        bulk_load(st + C::kXBytes, a.Wp + chunk_offset(n_tile, kb * kCh, a.K), C::kWBytes,
-                                  fullw_bar(s));
-                    } else {
-                        mbar_arrive_expect_tx(fullx_bar(s), C::kXBytes + 2 * tab);
-#pragma unroll
-                        for (int c = 0; c < kCh; ++c)
-                            tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN,
-                                        fullx_bar(s));
-                        const int g0 = (kb * KST) / a.G;
-                        const size_t toff = ((size_t)n_tile * a.ngroups + g0) * kPanelRows;
-                        bulk_load(st + C::kXBytes + C::kWBytes, a.s_g + toff, tab, fullx_bar(s));
-                        bulk_load(st + C::kXBytes + C::kWBytes + C::kTabRegion, a.zs + toff, tab, fullx_bar(s));
-                    }
-                    if (tj < 32) QOQ_MARK((is_w ? 16 : 48) + tj);
+                    const uint32_t st = sbase + C::kWOff + s * C::kWSlot;
+                    mbar_arrive_expect_tx(wfull_bar(s), C::kWBytes + 2 * tab);
+                    bulk_load(st, a.Wp + chunk_offset(n_tile, kb * kCh, a.K), C::kWBytes, wfull_bar(s));
+                    // group tables of the K block (G = 128: kCh groups; G = K: the one group)
+                    const size_t toff = ((size_t)n_tile * a.ngroups + (per_group ? kb * kCh : 0)) * kPanelRows;
+                    bulk_load(st + C::kWBytes, a.s_g + toff, tab, wfull_bar(s));
+                    bulk_load(st + C::kWBytes + C::kTabRegion, a.zs + toff, tab, wfull_bar(s));
+                    if (tj < 32) QOQ_MARK(16 + tj);
                     ++tj;
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
-                    if (++s == STAGES) {
+                    if (++s == SW) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                i = t * ks + ks1;
+            }
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------- X8 producer --
+        if (lane == 0) {
+            grid_dependency_wait();  // X8 comes from the preceding kernel
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int i = i_begin; i < i_end && ok;) {
+                const int t = i / ks;
+                const int ks1 = min(ks, i_end - t * ks);
+                const int m_tile = t % a.m_tiles;
+                for (int kb = i - t * ks; kb < ks1; ++kb) {
+                    if (!wait_bounded(xaempty_bar(s), ph ^ 1u, abort_flag, budget)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t st = sbase + s * C::kXSlot;
+                    mbar_arrive_expect_tx(xfull_bar(s), C::kXSlot);
+#pragma unroll
+                    for (int c = 0; c < kCh; ++c)
+                        tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN, xfull_bar(s));
+                    if (tj < 32) QOQ_MARK(48 + tj);
+                    ++tj;
+                    issued |= 1u << s;
+                    issued_par = (issued_par & ~(1u << s)) | (ph << s);
+                    if (++s == SX) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -343,15 +389,13 @@ __global__ void __launch_bounds__(352, 1)
                 if (!wait_bounded(accempty_bar, accph ^ 1u, abort_flag, budget)) break;
                 tc_fence_after();
                 for (int kb = ks0; kb < ks1; ++kb) {
-                    // the dequant warps arrive on afull only after they have
-                    // seen this slot's X8 tiles land, so one wait covers both
                     if (!wait_bounded(afull_bar(s), ph, abort_flag, budget)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     if (tj < 32) QOQ_MARK(144 + tj);
-                    const uint32_t st = sbase + s * C::kStageBytes;
+                    const uint32_t st = sbase + s * C::kXSlot;
 #pragma unroll
                     for (int j = 0; j < 4 * kCh; ++j) {
                         const uint32_t acc = (kb > ks0 || j > 0) ? 1u : 0u;
@@ -360,15 +404,14 @@ __global__ void __launch_bounds__(352, 1)
                             mma_i8_ts(tmem_base, tmem_base + C::kACol0 + s * C::kACols + j * 8, bdesc, idesc, acc);
                         } else {
                             const uint64_t adesc =
-                                smem_desc_sw128(sbase + STAGES * C::kStageBytes + s * C::kABytes + (j >> 2) * C::kATile) +
-                                2 * (j & 3);
+                                smem_desc_sw128(sbase + C::kAOff + s * C::kABytes + (j >> 2) * C::kATile) + 2 * (j & 3);
                             mma_i8_ss(tmem_base, adesc, bdesc, idesc, acc);
                         }
                     }
-                    mma_commit(empty_bar(s));
+                    mma_commit(xaempty_bar(s));
                     if (tj < 32) QOQ_MARK(176 + tj);
                     ++tj;
-                    if (++s == STAGES) {
+                    if (++s == SX) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -388,49 +431,57 @@ __global__ void __launch_bounds__(352, 1)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;  // output channel within the panel
         const bool per_group = (a.G == kBlockK);
-        int s = 0;
-        uint32_t ph = 0;
+        int sw = 0, sx = 0;
+        uint32_t pw = 0, px = 0;
         bool ok = true;
         for (int i = i_begin; i < i_end && ok;) {
             const int t = i / ks;
             const int ks1 = min(ks, i_end - t * ks);
             for (int kb = i - t * ks; kb < ks1; ++kb) {
-                // weights, then X8 tiles + tables; seeing slot s filled again
-                // also means the MMA is done with A slot s
-                if (!wait_bounded(fullw_bar(s), ph, abort_flag, budget) ||
-                    !wait_bounded(fullx_bar(s), ph, abort_flag, budget)) {
+                if (!wait_bounded(wfull_bar(sw), pw, abort_flag, budget)) {
                     ok = false;
                     break;
                 }
                 if (warp == 2 && lane == 0 && tj < 32) QOQ_MARK(80 + tj);
-                const uint8_t *st = smem + s * C::kStageBytes;
-                const uint8_t *sw = st + C::kXBytes;
-                const uint8_t *tg = sw + C::kWBytes;
+                const uint8_t *wsl = smem + C::kWOff + sw * C::kWSlot;
+                const uint8_t *tg = wsl + C::kWBytes;
                 uint4 v[kCh][4];
                 uint32_t sg[kCh], zsv[kCh];
 #pragma unroll
                 for (int c = 0; c < kCh; ++c) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        v[c][j] = *reinterpret_cast<const uint4 *>(sw + c * kChunkBytes + j * kSlabBytes + r * 16);
+                        v[c][j] = *reinterpret_cast<const uint4 *>(wsl + c * kChunkBytes + j * kSlabBytes + r * 16);
                     const int g = per_group ? c : 0;
                     sg[c] = tg[g * 128 + r];
                     zsv[c] = tg[C::kTabRegion + g * 128 + r];
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
+                if (lane == 0) mbar_arrive(wempty_bar(sw));  // the weight slot may be refilled now
+                if (++sw == SW) {
+                    sw = 0;
+                    pw ^= 1u;
+                }
+                // A slot sx is free once the MMAs of its previous use have
+                // completed; its X8 tiles must have landed before afull
+                if (!wait_bounded(xaempty_bar(sx), px ^ 1u, abort_flag, budget) ||
+                    !wait_bounded(xfull_bar(sx), px, abort_flag, budget)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < kCh; ++c) {
+                    const uint32_t sgc = sg[c];
                     const uint32_t bias = zero_comp_bias(zsv[c]);
                     uint32_t w8[32];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) dequant_slab(v[c][j], sg[c], bias, &w8[8 * j]);
+                    for (int j = 0; j < 4; ++j) dequant_slab(v[c][j], sgc, bias, &w8[8 * j]);
                     if constexpr (A_TMEM) {
-                        tmem_st32(tmem_base + ((uint32_t)(quarter * 32) << 16) + C::kACol0 + s * C::kACols + c * 32,
+                        tmem_st32(tmem_base + ((uint32_t)(quarter * 32) << 16) + C::kACol0 + sx * C::kACols + c * 32,
                                   w8);
                     } else {
-                        uint8_t *arow = smem + STAGES * C::kStageBytes + s * C::kABytes + c * C::kATile + r * 128;
+                        uint8_t *arow = smem + C::kAOff + sx * C::kABytes + c * C::kATile + r * 128;
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             *reinterpret_cast<uint4 *>(arow + ((q ^ (r & 7)) << 4)) =
@@ -444,12 +495,12 @@ __global__ void __launch_bounds__(352, 1)
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(afull_bar(s));
+                if (lane == 0) mbar_arrive(afull_bar(sx));
                 if (warp == 2 && lane == 0 && tj < 32) QOQ_MARK(112 + tj);
                 ++tj;
-                if (++s == STAGES) {
-                    s = 0;
-                    ph ^= 1u;
+                if (++sx == SX) {
+                    sx = 0;
+                    px ^= 1u;
                 }
             }
             i = t * ks + ks1;
@@ -459,6 +510,7 @@ __global__ void __launch_bounds__(352, 1)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
+        uint8_t *stg = smem + C::kStgOff + quarter * 1024;  // this warp's output staging block
         uint32_t accph = 0;
         grid_dependency_wait();  // s_x comes from the preceding kernel
         for (int i = i_begin; i < i_end;) {
@@ -622,7 +674,7 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
                         for (int q = 1; q < C::kSx; ++q)
                             if ((cc >> 1) == q) sxr = sx_reg[q];
-                        store_outputs(a, m0 + cc * 16, cc, n, sc, sxr, acc);
+                        store_outputs(a, stg, m0 + cc * 16, cc, n - lane, lane, sc, sxr, acc);
                     }
                     }
                 }
@@ -646,9 +698,10 @@ __global__ void __launch_bounds__(352, 1)
     if ((threadIdx.x == 0 || threadIdx.x == 320) && *abort_flag) {
         if (threadIdx.x == 0) atomicExch(&g_dev_error, 1);
         // the producers: let their own copies land before the CTA exits
-        for (int q = 0; q < STAGES; ++q)
+        const int nslots = threadIdx.x == 0 ? SW : SX;
+        for (int q = 0; q < nslots; ++q)
             if (issued & (1u << q))
-                drain_wait(threadIdx.x == 0 ? fullw_bar(q) : fullx_bar(q), (issued_par >> q) & 1u, 200000000ull);
+                drain_wait(threadIdx.x == 0 ? wfull_bar(q) : xfull_bar(q), (issued_par >> q) & 1u, 200000000ull);
     }
     if (warp == 0) {
         __syncwarp();
@@ -693,11 +746,11 @@ EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-template <int BN, int KST, int STAGES, bool A_TMEM>
+template <int BN, int KST, int SW, int SX, bool A_TMEM>
 cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, KST, STAGES, A_TMEM>;
-    auto kern = w4a8_gemm_kernel<BN, KST, STAGES, A_TMEM>;
+    using C = GemmCfg<BN, KST, SW, SX, A_TMEM>;
+    auto kern = w4a8_gemm_kernel<BN, KST, SW, SX, A_TMEM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: the GEMM may start (and stream weights)
@@ -719,25 +772,26 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     return cudaGetLastError();
 }
 
-// Ring depth per token-tile width and stage depth: as many stages as fit
-// in shared memory (~227 KB) and, with the A operand in TMEM, as many A
-// slots as fit next to the accumulator in 512 columns.
+// Ring depths per token-tile width and K block: the X8/A ring as deep as
+// the TMEM next to the accumulator allows (A in TMEM) or shared memory
+// allows (A in shared memory); the weight ring fills the rest of the
+// ~227 KB of shared memory, since it is what streams from HBM.
 template <bool A_TMEM>
 cudaError_t dispatch(int BN, int KST, const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
 {
     if (KST == 256) {
         switch (BN) {
-        case 16: return launch_cfg<16, 256, A_TMEM ? 7 : 4, A_TMEM>(tmap, args, grid, stream);
-        case 32: return launch_cfg<32, 256, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
-        default: return launch_cfg<64, 256, A_TMEM ? 6 : 3, A_TMEM>(tmap, args, grid, stream);
+        case 16: return launch_cfg<16, 256, A_TMEM ? 11 : 6, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
+        case 32: return launch_cfg<32, 256, A_TMEM ? 9 : 6, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
+        default: return launch_cfg<64, 256, A_TMEM ? 7 : 4, A_TMEM ? 6 : 2, A_TMEM>(tmap, args, grid, stream);
         }
     }
     switch (BN) {
-    case 16: return launch_cfg<16, 128, A_TMEM ? 12 : 7, A_TMEM>(tmap, args, grid, stream);
-    case 32: return launch_cfg<32, 128, A_TMEM ? 12 : 7, A_TMEM>(tmap, args, grid, stream);
-    case 64: return launch_cfg<64, 128, A_TMEM ? 11 : 6, A_TMEM>(tmap, args, grid, stream);
-    case 128: return launch_cfg<128, 128, A_TMEM ? 7 : 5, A_TMEM>(tmap, args, grid, stream);
-    default: return launch_cfg<256, 128, A_TMEM ? 4 : 3, A_TMEM>(tmap, args, grid, stream);
+    case 16: return launch_cfg<16, 128, A_TMEM ? 16 : 12, A_TMEM ? 8 : 4, A_TMEM>(tmap, args, grid, stream);
+    case 32: return launch_cfg<32, 128, A_TMEM ? 16 : 12, A_TMEM ? 8 : 4, A_TMEM>(tmap, args, grid, stream);
+    case 64: return launch_cfg<64, 128, A_TMEM ? 16 : 12, A_TMEM ? 8 : 4, A_TMEM>(tmap, args, grid, stream);
+    case 128: return launch_cfg<128, 128, A_TMEM ? 10 : 10, A_TMEM ? 8 : 3, A_TMEM>(tmap, args, grid, stream);
+    default: return launch_cfg<256, 128, A_TMEM ? 6 : 8, A_TMEM ? 5 : 3, A_TMEM>(tmap, args, grid, stream);
     }
 }
 

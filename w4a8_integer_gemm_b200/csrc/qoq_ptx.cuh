@@ -58,23 +58,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the phase of `bar` with the given parity to complete.  Gives up
-// when `*abort` becomes non-zero (another role gave up) or when this one
-// wait has lasted longer than `budget_ns`; in the latter case it raises
-// `*abort` itself.  Returns true when the phase completed.
+// As mbar_try_wait, but the thread sleeps in hardware until the phase
+// completes or about `suspend_ns` have passed, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t suspend_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity to complete.  The
+// waiting thread sleeps in hardware between checks (it is woken when the
+// phase completes), so waiters do not steal issue slots or shared-memory
+// bandwidth from the warps doing the work.  Gives up when `*abort` becomes
+// non-zero (another role gave up) or when this one wait has lasted longer
+// than `budget_ns`; in the latter case it raises `*abort` itself.  Returns
+// true when the phase completed.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile int *abort, uint64_t budget_ns)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t start = global_timer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*abort) return false;
-            if (global_timer_ns() - start > budget_ns) {
-                *abort = 1;
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;  // up to 0.2 ms per sleep
+        if (*abort) return false;
+        if (global_timer_ns() - start > budget_ns) {
+            *abort = 1;
+            return false;
         }
     }
 }
