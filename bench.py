@@ -9,12 +9,16 @@ sizes: M in {1, 8, 32, 64}, K = 4096, N = 14336, per-channel and g128
 weights (8 GEMMs per step).  `--workload sweep|large_batch|qwen|tiny` selects
 the other workloads for ad-hoc measurement.
 
-Timing: L2 (126 MB) is flushed by writing a 256 MB buffer before every
-shape; each shape is bracketed by CUDA events on the launching stream
-(flush excluded); the step time is the sum.  K timed steps follow W
-untimed ones, bracketed by a barrier and a device synchronize; with N > 1
-every rank runs the same workload (replicas, weak scaling) and the time is
-the max over ranks.
+Timing: when the distinct packed weights of a step exceed 1.5x L2
+(126 MB; the decode workload holds 224 MB), the shapes run back to back and
+the step is bracketed by CUDA events on the launching stream: every weight
+byte comes from HBM, because the step has cycled more than L2 since it last
+read the same weights.  Smaller workloads flush L2 (a 256 MB write) before
+every shape instead, bracket each shape with events (flush excluded) and sum.
+K timed steps follow W untimed ones, bracketed by a barrier and a device
+synchronize; with N > 1 every rank runs the same workload (replicas, weak
+scaling) and the time is the max over ranks.  Per shape, an isolated run
+(L2 flushed, the kernels alone) gives the per-point breakdown.
 
 --impl reference times the CPU oracle (plain C, OpenMP) on a bounded sample
 of the same workload instead.
@@ -40,6 +44,19 @@ from w4a8_integer_gemm_b200 import roofline, workloads as wl  # noqa: E402
 
 FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20
+GEMM_SOURCES = ("qoq_gemm.cu", "qoq_layout.cuh", "qoq_ptx.cuh", "qoq_internal.h")
+
+
+def gemm_source_hash() -> str:
+    """Short hash of the GEMM kernel's sources: DRAM traffic recorded under
+    profiles/ is reported only while it matches (the counters describe that
+    kernel and no later one)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "w4a8_integer_gemm_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def parse():
@@ -336,7 +353,9 @@ def run_ours(args, rank, world, local, dist):
     if os.path.exists(prof):
         try:
             t = json.load(open(prof))
-            rl["traffic"] = t.get("dram_bytes_per_gemm_launch")
+            if t.get("kernel_source_hash") == gemm_source_hash():
+                rl["traffic"] = t.get("dram_bytes_per_gemm_launch")
+                rl["traffic_capture"] = t.get("capture")
         except (OSError, ValueError):
             pass
 

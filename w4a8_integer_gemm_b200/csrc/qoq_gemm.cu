@@ -319,6 +319,7 @@ __global__ void __launch_bounds__(352, 1)
                 const int ks1 = min(ks, i_end - t * ks);
                 const int n_tile = t / a.m_tiles;
                 for (int kb = i - t * ks; kb < ks1; ++kb) {
+                    if (tj == 0) QOQ_MARK(5);
                     if (!wait_bounded(wempty_bar(s), ph ^ 1u, abort_flag, budget)) {
                         ok = false;
                         break;
@@ -330,7 +331,7 @@ __global__ void __launch_bounds__(352, 1)
                     const size_t toff = ((size_t)n_tile * a.ngroups + (per_group ? kb * kCh : 0)) * kPanelRows;
                     bulk_load(st + C::kWBytes, a.s_g + toff, tab, wfull_bar(s));
                     bulk_load(st + C::kWBytes + C::kTabRegion, a.zs + toff, tab, wfull_bar(s));
-                    if (tj < 32) QOQ_MARK(16 + tj);
+                    if (tj < 16) QOQ_MARK(16 + tj);
                     ++tj;
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
                     for (int c = 0; c < kCh; ++c)
                         tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN, xfull_bar(s));
-                    if (tj < 32) QOQ_MARK(48 + tj);
+                    if (tj < 16) QOQ_MARK(32 + tj);
                     ++tj;
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(352, 1)
                         break;
                     }
                     tc_fence_after();
-                    if (tj < 32) QOQ_MARK(144 + tj);
+                    if (tj < 16) QOQ_MARK(112 + tj);
                     const uint32_t st = sbase + s * C::kXSlot;
 #pragma unroll
                     for (int j = 0; j < 4 * kCh; ++j) {
@@ -409,7 +410,7 @@ __global__ void __launch_bounds__(352, 1)
                         }
                     }
                     mma_commit(xaempty_bar(s));
-                    if (tj < 32) QOQ_MARK(176 + tj);
+                    if (tj < 16) QOQ_MARK(128 + tj);
                     ++tj;
                     if (++s == SX) {
                         s = 0;
@@ -442,7 +443,7 @@ __global__ void __launch_bounds__(352, 1)
                     ok = false;
                     break;
                 }
-                if (warp == 2 && lane == 0 && tj < 32) QOQ_MARK(80 + tj);
+                if (warp == 2 && lane == 0 && tj < 16) QOQ_MARK(48 + tj);
                 const uint8_t *wsl = smem + C::kWOff + sw * C::kWSlot;
                 const uint8_t *tg = wsl + C::kWBytes;
                 uint4 v[kCh][4];
@@ -458,6 +459,7 @@ __global__ void __launch_bounds__(352, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(wempty_bar(sw));  // the weight slot may be refilled now
+                if (warp == 2 && lane == 0 && tj < 16) QOQ_MARK(64 + tj);
                 if (++sw == SW) {
                     sw = 0;
                     pw ^= 1u;
@@ -470,6 +472,7 @@ __global__ void __launch_bounds__(352, 1)
                     break;
                 }
                 tc_fence_after();
+                if (warp == 2 && lane == 0 && tj < 16) QOQ_MARK(80 + tj);
 #pragma unroll
                 for (int c = 0; c < kCh; ++c) {
                     const uint32_t sgc = sg[c];
@@ -496,7 +499,7 @@ __global__ void __launch_bounds__(352, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(afull_bar(sx));
-                if (warp == 2 && lane == 0 && tj < 32) QOQ_MARK(112 + tj);
+                if (warp == 2 && lane == 0 && tj < 16) QOQ_MARK(96 + tj);
                 ++tj;
                 if (++sx == SX) {
                     sx = 0;
