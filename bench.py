@@ -70,6 +70,8 @@ def parse():
                     help="restrict the workload to one shape name (for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every kernel from Python in the timed steps instead of replaying a CUDA graph")
     ap.add_argument("--a-smem", action="store_true",
                     help="keep the GEMM's dequantized tile in shared memory instead of TMEM")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -228,14 +230,24 @@ def run_ours(args, rank, world, local, dist):
     ev = [[E() for _ in range(4)] for _ in range(n_sh)]
     es = [E(), E(), E(), E()]
 
-    def one_step():
+    def enqueue_step(st, gemm=True, quant=True):
+        for c in cases:
+            if quant:
+                q.qoq_quant_act_per_token(c["X"], c["X8"], c["s_x"], stream=st)
+            if gemm:
+                q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=st)
+
+    graphs = {}
+
+    def one_step(eager=False):
         """The hot path of every shape: activation quant, then the GEMM.
-        Returns (step ms, GEMM-only ms summed over shapes)."""
+        Returns the step's device time in ms."""
         if chained:
             es[0].record(stream)
-            for c in cases:
-                q.qoq_quant_act_per_token(c["X"], c["X8"], c["s_x"], stream=stream)
-                q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
+            if "step" in graphs and not eager:
+                graphs["step"].replay()
+            else:
+                enqueue_step(stream)
             es[1].record(stream)
             torch.cuda.synchronize()
             return es[0].elapsed_time(es[1])
@@ -255,8 +267,10 @@ def run_ours(args, rank, world, local, dist):
         """The GEMM kernel alone, the same way (roofline of the dominant kernel)."""
         if chained:
             es[2].record(stream)
-            for c in cases:
-                q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
+            if "gemm" in graphs:
+                graphs["gemm"].replay()
+            else:
+                enqueue_step(stream, quant=False)
             es[3].record(stream)
             torch.cuda.synchronize()
             return es[2].elapsed_time(es[3])
@@ -298,6 +312,26 @@ def run_ours(args, rank, world, local, dist):
     torch.cuda.synchronize()
     if q.qoq_device_error() != q.QOQ_OK:
         raise RuntimeError("device error during warm-up")
+    # Decode-sized steps are launch-bound when every kernel is launched from
+    # Python; a serving loop replays them as one CUDA graph, and so does the
+    # timed region (the eager step time is reported beside it).
+    eager_ms = None
+    if chained and not args.eager:
+        eager_ms = statistics.median(one_step(eager=True) for _ in range(max(3, args.warmup)))
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(stream)
+        for name, kw in (("step", {}), ("gemm", {"quant": False})):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                enqueue_step(cap, **kw)
+            graphs[name] = g
+        stream.wait_stream(cap)
+        for _ in range(max(3, args.warmup)):
+            one_step()
+            gemm_only()
+        torch.cuda.synchronize()
+        if q.qoq_device_error() != q.QOQ_OK:
+            raise RuntimeError("device error while warming up the CUDA graphs")
 
     step_ms = []
     with ClockSampler(local) as clk:
@@ -397,7 +431,10 @@ def run_ours(args, rank, world, local, dist):
                          if chained else "flushed before every shape (256 MB write), flush excluded from timing",
                    "timing": ("median step of %d; GEMM-only roofline from the same %s runs" %
                               (args.steps, "back-to-back" if chained else "flushed")),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "launch": ("cuda_graph (one graph per step, programmatic dependent launch between kernels)"
+                              if graphs else "eager (every kernel launched from Python)"),
+                   "eager_ms_per_step": None if eager_ms is None else round(eager_ms, 5)},
         "roofline": rl, "points": per, "clocks": clocks, "e2e": e2e,
         "gpu_launches": 2 * n_sh * args.steps,
         "a_operand": "smem" if args.a_smem else "tmem",

@@ -23,8 +23,10 @@
 //     first contributor (the CTA whose range holds the tile's first unit:
 //     for it the tile is the last one it works on).  Every later
 //     contributor works on the tile first, publishes its INT32 partial
-//     (exact in any order) and bumps a counter; the finisher waits, bounded,
-//     for the count, adds the partials to its own accumulator and runs the
+//     (exact in any order) and counts it: every lane adds 1 with release
+//     semantics after its own stores, so the count covers every lane's
+//     bytes.  The finisher's lanes each wait (acquire, bounded) for the
+//     full count, add the partials to their accumulators and run the
 //     epilogue.  No contributor waits for anything while it still has work,
 //     so the waits cannot form a cycle.
 //   * Warp roles (352 threads):
@@ -44,11 +46,14 @@
 //                   and bulk copies of the group tables.  It alone waits for
 //                   the preceding kernel (programmatic dependent launch), so
 //                   weights stream in while the activation quantizer runs.
-//   * One ring: stage slot s holds the packed weights, tables and X8 tiles
-//     of a K block in shared memory, and A slot s (TMEM or shared memory)
-//     holds its dequantized weights.  When the dequant warps see slot s
-//     filled again, the producers have seen it freed, so the MMA is done
-//     with A slot s too; no separate A-slot barrier is needed.
+//   * Rings: a weight ring (packed chunks and tables of a K block, freed
+//     as soon as the dequant warps hold them in registers); an X8/A ring
+//     (slot s holds the X8 tiles of a K block in shared memory and its
+//     dequantized weights in A slot s, TMEM or shared memory; the X8
+//     producer refills slot s only after the MMAs reading it completed, so
+//     a landed X8 slot also means a free A slot); and one or two TMEM
+//     accumulators, so the MMAs of the next tile need not wait for the
+//     epilogue of the last one.
 //   * Every wait is bounded (per wait, global timer); on expiry the CTA
 //     stops, drains its own in-flight copies and MMAs, frees TMEM, and
 //     raises the device error flag that qoq_device_error() reports.
@@ -56,6 +61,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "qoq_internal.h"
@@ -101,6 +107,9 @@ struct GemmArgs {
     } while (0)
 #endif
 
+// Weight stages issued by the setup thread before the CTA-wide barrier.
+constexpr int kPrologueStages = 2;
+
 __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
 {
     return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
@@ -121,14 +130,17 @@ struct GemmCfg {
     static constexpr int kWOff = kAOff + SX * kABytes;
     static constexpr int kStgOff = kWOff + SW * kWSlot;  // per epilogue warp: 16 tokens x 32 channels FP16
     static constexpr int kBarOff = kStgOff + 4 * 1024;
-    static constexpr int kNumBars = 2 * SW + 3 * SX + 3;
+    static constexpr uint32_t kACols = KST / 4;          // TMEM columns of one A slot
+    // two accumulators (the MMAs of the next tile run while the epilogue
+    // drains the last one) wherever TMEM has room for them
+    static constexpr int kAccBufs = (2 * BN + (A_TMEM ? SX * (int)kACols : 0) <= 512) ? 2 : 1;
+    static constexpr int kNumBars = 2 * SW + 3 * SX + 2 * kAccBufs + 1;
     static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
     // at least ~120 KB so that exactly one CTA (and one TMEM allocation)
     // lives on each SM; +1024 for manual alignment of the dynamic base
     static constexpr int kSmemBytes = (kUsed > 120 * 1024 ? kUsed : 120 * 1024) + 1024;
-    static constexpr uint32_t kACols = KST / 4;          // TMEM columns of one A slot
-    static constexpr uint32_t kACol0 = BN;               // first TMEM column of the A ring
-    static constexpr uint32_t kTmemCols = pow2_cols(BN + (A_TMEM ? SX * kACols : 0));
+    static constexpr uint32_t kACol0 = kAccBufs * BN;    // first TMEM column of the A ring
+    static constexpr uint32_t kTmemCols = pow2_cols(kACol0 + (A_TMEM ? SX * kACols : 0));
     static constexpr int kSx = (BN + 31) / 32;           // s_x registers per lane
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
     static_assert(KST == 128 || KST == 256, "K block");
@@ -249,9 +261,11 @@ __global__ void __launch_bounds__(352, 1)
     auto xfull_bar = [&](int s) { return bar0 + 8u * (2 * SW + s); };
     auto afull_bar = [&](int s) { return bar0 + 8u * (2 * SW + SX + s); };
     auto xaempty_bar = [&](int s) { return bar0 + 8u * (2 * SW + 2 * SX + s); };
-    const uint32_t accfull_bar = bar0 + 8u * (2 * SW + 3 * SX);
-    const uint32_t accempty_bar = accfull_bar + 8u;
-    const uint32_t mmadone_bar = accfull_bar + 16u;
+    // accumulator b: accfull (its tile's MMAs are done), accempty (the
+    // epilogue has read it)
+    auto accfull_bar = [&](int b) { return bar0 + 8u * (2 * SW + 3 * SX + b); };
+    auto accempty_bar = [&](int b) { return bar0 + 8u * (2 * SW + 3 * SX + C::kAccBufs + b); };
+    const uint32_t mmadone_bar = bar0 + 8u * (2 * SW + 3 * SX + 2 * C::kAccBufs);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -265,6 +279,32 @@ __global__ void __launch_bounds__(352, 1)
     const int i_begin = range_begin(cta, P, T);
     const int i_end = range_begin(cta + 1, P, T);
     const int ks = a.ks;
+
+    // ring slots a producer has filled, and the phase parity of each slot's
+    // latest fill (drained on the way out of an aborted CTA)
+    uint32_t issued = 0, issued_par = 0;
+    int tj = 0;  // trace: per-role unit counter
+    (void)tj;
+    // The weight copies of unit u (tile u / ks, K block u % ks) into W slot s.
+    const bool per_group = (a.G == kBlockK);
+    auto issue_weights = [&](int u, int s, uint32_t ph) {
+        const int t = u / ks;
+        const int kb = u - t * ks;
+        const int n_tile = t / a.m_tiles;
+        const uint32_t tab = per_group ? (uint32_t)C::kTabRegion : 128u;
+        const uint32_t st = sbase + C::kWOff + s * C::kWSlot;
+        mbar_arrive_expect_tx(wfull_bar(s), C::kWBytes + 2 * tab);
+        bulk_load(st, a.Wp + chunk_offset(n_tile, kb * kCh, a.K), C::kWBytes, wfull_bar(s));
+        // group tables of the K block (G = 128: kCh groups; G = K: the one group)
+        const size_t toff = ((size_t)n_tile * a.ngroups + (per_group ? kb * kCh : 0)) * kPanelRows;
+        bulk_load(st + C::kWBytes, a.s_g + toff, tab, wfull_bar(s));
+        bulk_load(st + C::kWBytes + C::kTabRegion, a.zs + toff, tab, wfull_bar(s));
+        issued |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | (ph << s);
+    };
+    // the first stages go out before anything else (no slot is taken yet);
+    // only a few, since the whole CTA waits for this thread at the barrier
+    const int n_pro = min(min(SW, kPrologueStages), i_end - i_begin);
 
 #ifdef QOQ_TRACE
     const long long trace_t0 = clock64();
@@ -280,17 +320,26 @@ __global__ void __launch_bounds__(352, 1)
             mbar_init(afull_bar(s), 4);      // 4 dequant warps
             mbar_init(xaempty_bar(s), 1);    // MMA commit
         }
-        mbar_init(accfull_bar, 1);
-        mbar_init(accempty_bar, 4);
+        for (int b = 0; b < C::kAccBufs; ++b) {
+            mbar_init(accfull_bar(b), 1);
+            mbar_init(accempty_bar(b), 4);   // 4 epilogue warps
+        }
         mbar_init(mmadone_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
+        // weights stream from here on, while the rest of the CTA sets up
+        for (int j = 0; j < n_pro; ++j) {
+            issue_weights(i_begin + j, j, 0u);
+            if (tj < 16) QOQ_MARK(16 + tj);
+            ++tj;
+        }
     }
     if (threadIdx.x == 320) prefetch_tmap(&tmap_x);
     // The next kernel in the stream may launch now; whatever it reads from
     // this GEMM it must read after its own griddepcontrol.wait.
     grid_launch_dependents();
     if (warp == 0) {
+        __syncwarp();
         tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
@@ -300,47 +349,23 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t budget = a.timeout_ns;
     QOQ_MARK(1);
-    // ring slots a producer has filled, and the phase parity of each slot's
-    // latest fill (drained on the way out of an aborted CTA)
-    uint32_t issued = 0, issued_par = 0;
-    int tj = 0;  // trace: per-role unit counter
-    (void)tj;
 
     if (warp == 0) {
         // ---------------------------------------------- weight producer --
+        // (the first n_pro units were issued before the CTA-wide barrier)
         if (lane == 0) {
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            const bool per_group = (a.G == kBlockK);
-            const uint32_t tab = per_group ? (uint32_t)C::kTabRegion : 128u;
-            for (int i = i_begin; i < i_end && ok;) {
-                const int t = i / ks;
-                const int ks1 = min(ks, i_end - t * ks);
-                const int n_tile = t / a.m_tiles;
-                for (int kb = i - t * ks; kb < ks1; ++kb) {
-                    if (tj == 0) QOQ_MARK(5);
-                    if (!wait_bounded(wempty_bar(s), ph ^ 1u, abort_flag, budget)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t st = sbase + C::kWOff + s * C::kWSlot;
-                    mbar_arrive_expect_tx(wfull_bar(s), C::kWBytes + 2 * tab);
-                    bulk_load(st, a.Wp + chunk_offset(n_tile, kb * kCh, a.K), C::kWBytes, wfull_bar(s));
-                    // group tables of the K block (G = 128: kCh groups; G = K: the one group)
-                    const size_t toff = ((size_t)n_tile * a.ngroups + (per_group ? kb * kCh : 0)) * kPanelRows;
-                    bulk_load(st + C::kWBytes, a.s_g + toff, tab, wfull_bar(s));
-                    bulk_load(st + C::kWBytes + C::kTabRegion, a.zs + toff, tab, wfull_bar(s));
-                    if (tj < 16) QOQ_MARK(16 + tj);
-                    ++tj;
-                    issued |= 1u << s;
-                    issued_par = (issued_par & ~(1u << s)) | (ph << s);
-                    if (++s == SW) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
+            int s = n_pro == SW ? 0 : n_pro;
+            uint32_t ph = (n_pro == SW) ? 1u : 0u;
+            for (int u = i_begin + n_pro; u < i_end; ++u) {
+                if (tj == n_pro) QOQ_MARK(5);
+                if (!wait_bounded(wempty_bar(s), ph ^ 1u, abort_flag, budget)) break;
+                issue_weights(u, s, ph);
+                if (tj < 16) QOQ_MARK(16 + tj);
+                ++tj;
+                if (++s == SW) {
+                    s = 0;
+                    ph ^= 1u;
                 }
-                i = t * ks + ks1;
             }
         }
     } else if (warp == 10) {
@@ -381,14 +406,17 @@ __global__ void __launch_bounds__(352, 1)
         if (lane == 0) {
             const uint32_t idesc = idesc_i8_m128(BN);
             int s = 0;
-            uint32_t ph = 0, accph = 0;
+            uint32_t ph = 0;
+            int ab = 0;          // accumulator of the current tile
+            uint32_t accph = 0;  // its phase parity
             bool ok = true;
             for (int i = i_begin; i < i_end && ok;) {
                 const int t = i / ks;
                 const int ks0 = i - t * ks;
                 const int ks1 = min(ks, i_end - t * ks);
-                if (!wait_bounded(accempty_bar, accph ^ 1u, abort_flag, budget)) break;
+                if (!wait_bounded(accempty_bar(ab), accph ^ 1u, abort_flag, budget)) break;
                 tc_fence_after();
+                const uint32_t dacc = tmem_base + (uint32_t)(ab * BN);
                 for (int kb = ks0; kb < ks1; ++kb) {
                     if (!wait_bounded(afull_bar(s), ph, abort_flag, budget)) {
                         ok = false;
@@ -402,11 +430,11 @@ __global__ void __launch_bounds__(352, 1)
                         const uint32_t acc = (kb > ks0 || j > 0) ? 1u : 0u;
                         const uint64_t bdesc = smem_desc_sw128(st + (j >> 2) * C::kXTile) + 2 * (j & 3);
                         if constexpr (A_TMEM) {
-                            mma_i8_ts(tmem_base, tmem_base + C::kACol0 + s * C::kACols + j * 8, bdesc, idesc, acc);
+                            mma_i8_ts(dacc, tmem_base + C::kACol0 + s * C::kACols + j * 8, bdesc, idesc, acc);
                         } else {
                             const uint64_t adesc =
                                 smem_desc_sw128(sbase + C::kAOff + s * C::kABytes + (j >> 2) * C::kATile) + 2 * (j & 3);
-                            mma_i8_ss(tmem_base, adesc, bdesc, idesc, acc);
+                            mma_i8_ss(dacc, adesc, bdesc, idesc, acc);
                         }
                     }
                     mma_commit(xaempty_bar(s));
@@ -418,8 +446,11 @@ __global__ void __launch_bounds__(352, 1)
                     }
                 }
                 if (!ok) break;
-                mma_commit(accfull_bar);
-                accph ^= 1u;
+                mma_commit(accfull_bar(ab));
+                if (++ab == C::kAccBufs) {
+                    ab = 0;
+                    accph ^= 1u;
+                }
                 i = t * ks + ks1;
             }
             QOQ_MARK(3);
@@ -431,7 +462,6 @@ __global__ void __launch_bounds__(352, 1)
         // ------------------------------------------------------ dequant --
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;  // output channel within the panel
-        const bool per_group = (a.G == kBlockK);
         int sw = 0, sx = 0;
         uint32_t pw = 0, px = 0;
         bool ok = true;
@@ -464,10 +494,11 @@ __global__ void __launch_bounds__(352, 1)
                     sw = 0;
                     pw ^= 1u;
                 }
-                // A slot sx is free once the MMAs of its previous use have
-                // completed; its X8 tiles must have landed before afull
-                if (!wait_bounded(xaempty_bar(sx), px ^ 1u, abort_flag, budget) ||
-                    !wait_bounded(xfull_bar(sx), px, abort_flag, budget)) {
+                // X8 slot sx has landed.  That also means A slot sx is free:
+                // the X8 producer refills slot sx only after the MMAs of its
+                // previous use have completed (xaempty), so those MMAs are
+                // done reading A slot sx by the time xfull completes.
+                if (!wait_bounded(xfull_bar(sx), px, abort_flag, budget)) {
                     ok = false;
                     break;
                 }
@@ -514,7 +545,8 @@ __global__ void __launch_bounds__(352, 1)
         const int r = quarter * 32 + lane;
         const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
         uint8_t *stg = smem + C::kStgOff + quarter * 1024;  // this warp's output staging block
-        uint32_t accph = 0;
+        int ab = 0;          // accumulator of the current tile
+        uint32_t accph = 0;  // its phase parity
         grid_dependency_wait();  // s_x comes from the preceding kernel
         for (int i = i_begin; i < i_end;) {
             const int t = i / ks;
@@ -546,23 +578,24 @@ __global__ void __launch_bounds__(352, 1)
             constexpr int kGrp = BN < 64 ? BN : 64;  // accumulator columns per TMEM load
             int32_t pre[kPresum ? BN : 1];
             if (finisher) {
+                // Every lane of every later contributor counts its own
+                // stores (32 per contributor and quarter); every lane here
+                // acquires the count itself before it reads the partials.
                 int *counter = a.ws_cnt + cta * 4 + quarter;
-                if (lane == 0) {
-                    const int want = c_hi - cta;
-                    if (ld_acquire_gpu(counter) < want) {
-                        const uint64_t start = global_timer_ns();
-                        while (ld_acquire_gpu(counter) < want) {
-                            if (*abort_flag || global_timer_ns() - start > budget) {
-                                *abort_flag = 1;
-                                ready = false;
-                                break;
-                            }
+                const int want = 32 * (c_hi - cta);
+                if (ld_acquire_gpu(counter) < want) {
+                    const uint64_t start = global_timer_ns();
+                    while (ld_acquire_gpu(counter) < want) {
+                        if (*abort_flag || global_timer_ns() - start > budget) {
+                            *abort_flag = 1;
+                            ready = false;
+                            break;
                         }
                     }
-                    if (ready) *counter = 0;  // ready for the next call
                 }
-                ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-                __syncwarp();  // the other lanes read the partials after lane 0's acquire
+                ready = __all_sync(0xffffffffu, ready);
+                __syncwarp();  // every lane has seen the full count
+                if (lane == 0 && ready) *counter = 0;  // ready for the next call
                 if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(224 + tj);
                 if constexpr (kPresum) {
 #pragma unroll
@@ -589,16 +622,27 @@ __global__ void __launch_bounds__(352, 1)
                     }
                 }
             }
-            if (!wait_bounded(accfull_bar, accph, abort_flag, budget)) break;
+            if (!wait_bounded(accfull_bar(ab), accph, abort_flag, budget)) break;
             if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(208 + tj);
             tc_fence_after();
+            const uint32_t tacc = trow + (uint32_t)(ab * BN);
+            // the accumulator goes back to the MMA as soon as its last
+            // columns are in registers
+            bool released = false;
+            auto release_acc = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(accempty_bar(ab));
+                released = true;
+            };
             if (partial && !finisher) {
                 // a later contributor: publish the partial, count it, done
                 int4 *my_part = reinterpret_cast<int4 *>(a.ws_part + (size_t)cta * BN * kPanelRows);
 #pragma unroll 1
                 for (int g0 = 0; g0 < nchunks; g0 += kGrp / 16) {
                     uint32_t v[kGrp];
-                    tmem_load_cols<kGrp>(trow + g0 * 16, v);
+                    tmem_load_cols<kGrp>(tacc + g0 * 16, v);
+                    if (g0 + kGrp / 16 >= nchunks) release_acc();
 #pragma unroll
                     for (int u = 0; u < kGrp / 16; ++u) {
                         if (g0 + u < nchunks) {
@@ -610,19 +654,17 @@ __global__ void __launch_bounds__(352, 1)
                         }
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(accempty_bar);
-                    red_release_gpu_add(a.ws_cnt + c_lo * 4 + quarter, 1);
-                }
+                if (!released) release_acc();
+                // each lane's release covers its own partial stores
+                red_release_gpu_add(a.ws_cnt + c_lo * 4 + quarter, 1);
             } else {
                 // a whole tile, or a split tile this CTA finishes
                 if (ready) {
 #pragma unroll 1
                     for (int g0 = 0; g0 < nchunks; g0 += kGrp / 16) {
                     uint32_t vg[kGrp];
-                    tmem_load_cols<kGrp>(trow + g0 * 16, vg);
+                    tmem_load_cols<kGrp>(tacc + g0 * 16, vg);
+                    if (g0 + kGrp / 16 >= nchunks) release_acc();
                     if (warp == 6 && lane == 0 && tj < 2 && g0 == 0) QOQ_MARK(232 + tj * 8);
 #pragma unroll
                     for (int u = 0; u < kGrp / 16; ++u) {
@@ -681,13 +723,14 @@ __global__ void __launch_bounds__(352, 1)
                     }
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(accempty_bar);
+                if (!released) release_acc();
             }
             if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(216 + tj);
             ++tj;
-            accph ^= 1u;
+            if (++ab == C::kAccBufs) {
+                ab = 0;
+                accph ^= 1u;
+            }
             i = t * ks + ks1;
         }
         if (warp == 6 && lane == 0) QOQ_MARK(4);
@@ -754,8 +797,17 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
 {
     using C = GemmCfg<BN, KST, SW, SX, A_TMEM>;
     auto kern = w4a8_gemm_kernel<BN, KST, SW, SX, A_TMEM>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    // the shared-memory opt-in is per device and per kernel: set it once
+    static std::atomic<unsigned long long> opted_in{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(opted_in.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        opted_in.fetch_or(bit, std::memory_order_acq_rel);
+    }
     // programmatic dependent launch: the GEMM may start (and stream weights)
     // while the kernel before it in the stream -- normally the activation
     // quantizer -- is still running; the kernel waits for it before it
@@ -796,6 +848,20 @@ cudaError_t dispatch(int BN, int KST, const CUtensorMap &tmap, const GemmArgs &a
     case 128: return launch_cfg<128, 128, A_TMEM ? 10 : 10, A_TMEM ? 8 : 3, A_TMEM>(tmap, args, grid, stream);
     default: return launch_cfg<256, 128, A_TMEM ? 6 : 8, A_TMEM ? 5 : 3, A_TMEM>(tmap, args, grid, stream);
     }
+}
+
+// SMs of the current device, looked up once per device.
+int sm_count()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kMaxCtas;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = kMaxCtas;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
 }
 
 // K depth of one pipeline stage: two packed chunks when K allows it and the
@@ -855,9 +921,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
         *tmap_status = (int)r;
         return cudaErrorInvalidValue;
     }
-    int dev = 0, sms = kMaxCtas;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = sm_count();
     const long long units = gemm_units(M, N, K);
     const long long grid = std::min<long long>(std::min(kMaxCtas, sms), units);
 
