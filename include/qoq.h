@@ -81,11 +81,17 @@ QOQ_API const char *qoq_status_string(int status);
 /* ------------------------------------------------------------------------
  * Packed weight layout: the "Blackwell interleaved UINT4" layout
  * ------------------------------------------------------------------------
- * Wp holds one 4-bit code per weight. Bytes are grouped into 8192-byte
- * chunks, one per (128-channel panel p, 128-wide K block b). Chunks are
- * ordered p-major:
- *     chunk(p, b) starts at byte (p * (K/128) + b) * 8192.
- * A chunk has 4 slabs of 2048 bytes, one per 32-wide K slice j. Inside slab
+ * Wp holds one 4-bit code per weight, grouped into chunks, one per
+ * (128-channel panel p, 128-wide K block b). Chunks are ordered p-major, S
+ * bytes apart:
+ *     chunk(p, b) starts at byte (p * (K/128) + b) * S,
+ *     S = 8192 + 256 when group_size == 128, S = 8192 when group_size == K.
+ * The first 8192 bytes of a chunk hold its codes. With group_size == 128
+ * the chunk covers exactly one group, and bytes 8192..8319 hold that
+ * group's s_g for channels r = 0..127 of the panel, bytes 8320..8447 its
+ * zs (the same values as in the s_g and zs arrays below): one copy brings
+ * a stage's codes and tables together.
+ * The codes of a chunk form 4 slabs of 2048 bytes, one per 32-wide K slice j. Inside slab
  * j, channel r (0..127 within the panel) owns the 16 bytes at j*2048 + r*16.
  * Those 16 bytes are 4 little-endian 32-bit words. For word w (0..3),
  * byte i (0..3), with k0 = 128*b + 32*j:
@@ -94,18 +100,19 @@ QOQ_API const char *qoq_status_string(int status);
  * So one AND of a word with 0x0F0F0F0F gives four consecutive codes in four
  * byte lanes, and one shift plus one AND gives the next four.
  *
- * The group tables are panel-major, one byte per entry: for channel n in
- * panel p = n/128 (r = n%128) and group g = k/group_size,
+ * The group tables are also written as arrays, panel-major, one byte per
+ * entry: for channel n in panel p = n/128 (r = n%128) and group
+ * g = k/group_size,
  *     s_g[(p*(K/group_size) + g)*128 + r]  the integer group scale (1..16),
  *     zs [(p*(K/group_size) + g)*128 + r]  the zero compensation z*s_g (0..240).
- * The 128 channels of a panel are contiguous for each group, and the groups
- * of a panel follow each other, so one bulk copy brings the tables a
- * pipeline stage needs. s_c[n] is the FP16 channel scale.
+ * The GEMM reads per-channel tables (group_size == K) from these arrays and
+ * 128-wide groups' tables from the chunks. s_c[n] is the FP16 channel scale.
  */
 
-/* Bytes of Wp for an N x K weight: N*K/2. Returns 0 when N or K is not a
- * positive multiple of 128. */
-QOQ_API size_t qoq_packed_weight_bytes(int N, int K);
+/* Bytes of Wp for an N x K weight: N*K/2, plus N*K/64 for the tables the
+ * chunks carry when group_size == 128. Returns 0 when N or K is not a
+ * positive multiple of 128 or group_size is neither 128 nor K. */
+QOQ_API size_t qoq_packed_weight_bytes(int N, int K, int group_size);
 
 /* Progressive group quantization and packing (the offline step).
  *
@@ -122,7 +129,7 @@ QOQ_API size_t qoq_packed_weight_bytes(int N, int K);
  *   - W must be finite. Entries with |W| >= 65520*119 make s_c infinite.
  *
  *   W      device, float32 [N][K], read only.
- *   Wp     device, qoq_packed_weight_bytes(N, K) bytes, written in the
+ *   Wp     device, qoq_packed_weight_bytes(N, K, group_size) bytes, written in the
  *          packed layout above.
  *   s_c    device, uint16_t [N] FP16 bits, written.
  *   s_g    device, uint8_t [N/128][K/group_size][128], written.

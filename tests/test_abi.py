@@ -46,9 +46,12 @@ def test_status_strings(L):
 
 def test_size_queries(L):
     import w4a8_integer_gemm_b200 as q
-    assert q.qoq_packed_weight_bytes(14336, 4096) == 14336 * 4096 // 2
-    assert q.qoq_packed_weight_bytes(100, 4096) == 0
-    assert q.qoq_packed_weight_bytes(128, 100) == 0
+    # codes, plus the tables the chunks carry for 128-wide groups
+    assert q.qoq_packed_weight_bytes(14336, 4096, 4096) == 14336 * 4096 // 2
+    assert q.qoq_packed_weight_bytes(14336, 4096, 128) == 14336 * 4096 // 2 + 14336 * 4096 // 64
+    assert q.qoq_packed_weight_bytes(100, 4096, 128) == 0
+    assert q.qoq_packed_weight_bytes(128, 100, 100) == 0
+    assert q.qoq_packed_weight_bytes(128, 512, 64) == 0
     assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 128) > 0
     assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 64) == 0      # group size not supported
     assert q.qoq_gemm_workspace_bytes(0, 512, 512, 128) == 0

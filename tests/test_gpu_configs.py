@@ -64,4 +64,4 @@ def test_full_size_sampled(name, i):
         assert np.array_equal(packed.s_c.cpu().view(torch.int16).numpy().view(np.uint16), full["s_c"])
         assert np.array_equal(packed.s_g.cpu().numpy(), tables_reference(full["s_g"]))
         assert np.array_equal(packed.zs.cpu().numpy(), tables_reference(full["zs"]))
-        assert np.array_equal(packed.Wp.cpu().numpy(), pack_reference(full["q"]))
+        assert np.array_equal(packed.Wp.cpu().numpy(), pack_reference(full["q"], s.G, full["s_g"], full["zs"]))

@@ -83,7 +83,7 @@ def test_pack_bit_exact(N, K, G):
     assert np.array_equal(_u16(p.s_c), r["s_c"])
     assert np.array_equal(p.s_g.cpu().numpy(), tables_reference(r["s_g"]))
     assert np.array_equal(p.zs.cpu().numpy(), tables_reference(r["zs"]))
-    assert np.array_equal(p.Wp.cpu().numpy()[: N * K // 2], pack_reference(r["q"]))
+    assert np.array_equal(p.Wp.cpu().numpy(), pack_reference(r["q"], G, r["s_g"], r["zs"]))
 
 
 def test_pack_degenerate_rows():
@@ -97,7 +97,7 @@ def test_pack_degenerate_rows():
     assert np.array_equal(_u16(p.s_c), r["s_c"])
     assert np.array_equal(p.s_g.cpu().numpy(), tables_reference(r["s_g"]))
     assert np.array_equal(p.zs.cpu().numpy(), tables_reference(r["zs"]))
-    assert np.array_equal(p.Wp.cpu().numpy()[: 128 * 128], pack_reference(r["q"]))
+    assert np.array_equal(p.Wp.cpu().numpy(), pack_reference(r["q"], 128, r["s_g"], r["zs"]))
 
 
 @pytest.mark.parametrize("N,K,G", [(512, 512, 128), (256, 1024, 1024)])
@@ -138,7 +138,7 @@ def test_tiny_workload_full_parity():
     s = w.shapes[0]
     packed, X8, s_x, Y, acc = run_layer(X, W, s.G)
     r = oracle.linear(X.numpy(), W.numpy(), s.G)
-    assert np.array_equal(packed.Wp.cpu().numpy(), pack_reference(r["q"]))
+    assert np.array_equal(packed.Wp.cpu().numpy(), pack_reference(r["q"], s.G, r["s_g"], r["zs"]))
     assert np.array_equal(X8.cpu().numpy(), r["X8"])
     assert np.array_equal(acc.cpu().numpy(), r["acc"])
     assert np.array_equal(q.qoq_dequant_weights_i8(packed).cpu().numpy(), r["W8hat"])

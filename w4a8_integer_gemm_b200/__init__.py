@@ -42,7 +42,7 @@ _SZ = ctypes.c_size_t
 # name -> (restype, argtypes); the exported surface of include/qoq.h
 SIGNATURES = {
     "qoq_status_string": (ctypes.c_char_p, [_I]),
-    "qoq_packed_weight_bytes": (_SZ, [_I, _I]),
+    "qoq_packed_weight_bytes": (_SZ, [_I, _I, _I]),
     "qoq_pack_weights": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "qoq_quant_act_per_token": (_I, [_P, _I, _I, _P, _P, _P]),
     "qoq_gemm_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
@@ -108,8 +108,8 @@ def qoq_status_string(status: int) -> str:
     return lib().qoq_status_string(int(status)).decode()
 
 
-def qoq_packed_weight_bytes(N: int, K: int) -> int:
-    return int(lib().qoq_packed_weight_bytes(int(N), int(K)))
+def qoq_packed_weight_bytes(N: int, K: int, group_size: int) -> int:
+    return int(lib().qoq_packed_weight_bytes(int(N), int(K), int(group_size)))
 
 
 def qoq_gemm_workspace_bytes(M: int, N: int, K: int, group_size: int) -> int:
@@ -144,7 +144,7 @@ def qoq_pack_weights(W: torch.Tensor, group_size: int, out: Optional[PackedWeigh
     G = int(group_size)
     if out is None:
         dev = W.device
-        nb = qoq_packed_weight_bytes(N, K)
+        nb = qoq_packed_weight_bytes(N, K, G)
         ng = K // G if G > 0 and K % G == 0 else 1
         out = PackedWeights(torch.empty(max(nb, 16), dtype=torch.uint8, device=dev),
                             torch.empty(N, dtype=torch.int16, device=dev),

@@ -7,6 +7,7 @@
 
 #include "../../include/qoq.h"
 #include "qoq_internal.h"
+#include "qoq_layout.cuh"
 
 namespace {
 
@@ -72,10 +73,10 @@ const char *qoq_status_string(int status)
     }
 }
 
-size_t qoq_packed_weight_bytes(int N, int K)
+size_t qoq_packed_weight_bytes(int N, int K, int group_size)
 {
-    if (!valid_nk(N, K)) return 0;
-    return (size_t)N * (size_t)K / 2;
+    if (!valid_nk(N, K) || !valid_group(K, group_size)) return 0;
+    return (size_t)(N / qoq::kPanelRows) * (size_t)(K / qoq::kBlockK) * (size_t)qoq::chunk_stride(group_size);
 }
 
 int qoq_pack_weights(const float *W, int N, int K, int group_size, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g,

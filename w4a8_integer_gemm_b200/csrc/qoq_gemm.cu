@@ -110,6 +110,16 @@ struct GemmArgs {
 // Weight stages issued by the setup thread before the CTA-wide barrier.
 constexpr int kPrologueStages = 2;
 
+// Warpgroups: producers and MMA issuer (warps 0-3), kDq dequant groups of
+// four warps that take the stages in turn, and the epilogue (the last four
+// warps).  Token tiles up to 64 wide use two dequant groups (512 threads,
+// 128 registers each): there the dequantization, not the MMA, bounds a
+// stage, and one group's barrier waits and TMEM stores overlap the other's
+// arithmetic.  Wider tiles keep one group (384 threads, 168 registers) for
+// their larger epilogue.
+__host__ __device__ constexpr int dequant_groups(int BN) { return BN <= 64 ? 2 : 1; }
+__host__ __device__ constexpr int gemm_threads(int BN) { return 128 * (2 + dequant_groups(BN)); }
+
 __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
 {
     return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
@@ -122,9 +132,9 @@ struct GemmCfg {
     static constexpr int kXSlot = kChunks * kXTile;      // X8 tiles of one K block
     static constexpr int kATile = 128 * 128;             // one [128][128 B] swizzled A tile
     static constexpr int kABytes = A_TMEM ? 0 : kChunks * kATile;
-    static constexpr int kWBytes = kChunks * kChunkBytes;
-    static constexpr int kTabRegion = 128 * kChunks;     // s_g region, then zs region
-    static constexpr int kWSlot = kWBytes + 2 * kTabRegion;
+    // one W slot: the K block's packed chunks, each followed by its group
+    // tables when G = 128 (the layout of the packed buffer itself)
+    static constexpr int kWSlot = kChunks * (kChunkBytes + kChunkTabBytes);
     // shared memory: [X8 ring][A ring (A in shared memory only)][W ring][barriers]
     static constexpr int kAOff = SX * kXSlot;
     static constexpr int kWOff = kAOff + SX * kABytes;
@@ -134,7 +144,7 @@ struct GemmCfg {
     // two accumulators (the MMAs of the next tile run while the epilogue
     // drains the last one) wherever TMEM has room for them
     static constexpr int kAccBufs = (2 * BN + (A_TMEM ? SX * (int)kACols : 0) <= 512) ? 2 : 1;
-    static constexpr int kNumBars = 2 * SW + 3 * SX + 2 * kAccBufs + 1;
+    static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * kAccBufs + 1;
     static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
     // at least ~120 KB so that exactly one CTA (and one TMEM allocation)
     // lives on each SM; +1024 for manual alignment of the dynamic base
@@ -241,31 +251,34 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *v)
 }
 
 template <int BN, int KST, int SW, int SX, bool A_TMEM>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(gemm_threads(BN), 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs a)
 {
     using C = GemmCfg<BN, KST, SW, SX, A_TMEM>;
     constexpr int kCh = C::kChunks;
+    constexpr int kDq = dequant_groups(BN);
+    constexpr int kEpiWarp0 = 4 + 4 * kDq;  // first epilogue warp
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar0 = sbase + C::kBarOff;
     // W ring (packed weights + group tables of one K block):
-    //   wfull (bulk copies landed), wempty (the dequant warps have read it)
+    //   wfull (bulk copy landed), wempty (the dequant warps have read it)
     // X8/A ring (X8 tiles in shared memory, dequantized weights in A slot):
-    //   xfull (X8 tiles landed), afull (A slot written; the dequant warps
-    //   arrive only after they have seen xfull, so it covers both),
-    //   xaempty (the MMAs reading the slot have completed)
+    //   afull (the slot is ready for the MMAs: the 4 dequant warps of the
+    //   stage have written the A slot, and the X8 producer's arrival plus
+    //   its copies' transaction bytes say the X8 tiles have landed),
+    //   xaempty (the MMAs reading the slot have completed: both the X8
+    //   slot and the A slot are free)
     auto wfull_bar = [&](int s) { return bar0 + 8u * s; };
     auto wempty_bar = [&](int s) { return bar0 + 8u * (SW + s); };
-    auto xfull_bar = [&](int s) { return bar0 + 8u * (2 * SW + s); };
-    auto afull_bar = [&](int s) { return bar0 + 8u * (2 * SW + SX + s); };
-    auto xaempty_bar = [&](int s) { return bar0 + 8u * (2 * SW + 2 * SX + s); };
+    auto afull_bar = [&](int s) { return bar0 + 8u * (2 * SW + s); };
+    auto xaempty_bar = [&](int s) { return bar0 + 8u * (2 * SW + SX + s); };
     // accumulator b: accfull (its tile's MMAs are done), accempty (the
     // epilogue has read it)
-    auto accfull_bar = [&](int b) { return bar0 + 8u * (2 * SW + 3 * SX + b); };
-    auto accempty_bar = [&](int b) { return bar0 + 8u * (2 * SW + 3 * SX + C::kAccBufs + b); };
-    const uint32_t mmadone_bar = bar0 + 8u * (2 * SW + 3 * SX + 2 * C::kAccBufs);
+    auto accfull_bar = [&](int b) { return bar0 + 8u * (2 * SW + 2 * SX + b); };
+    auto accempty_bar = [&](int b) { return bar0 + 8u * (2 * SW + 2 * SX + C::kAccBufs + b); };
+    const uint32_t mmadone_bar = bar0 + 8u * (2 * SW + 2 * SX + 2 * C::kAccBufs);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -285,20 +298,19 @@ __global__ void __launch_bounds__(352, 1)
     uint32_t issued = 0, issued_par = 0;
     int tj = 0;  // trace: per-role unit counter
     (void)tj;
-    // The weight copies of unit u (tile u / ks, K block u % ks) into W slot s.
+    // The weight copy of unit u (tile u / ks, K block u % ks) into W slot s:
+    // the kCh chunks of the K block are contiguous in the packed buffer,
+    // with their group tables when G = 128, so one bulk copy brings them.
     const bool per_group = (a.G == kBlockK);
+    const int cstride = chunk_stride(a.G);
     auto issue_weights = [&](int u, int s, uint32_t ph) {
         const int t = u / ks;
         const int kb = u - t * ks;
         const int n_tile = t / a.m_tiles;
-        const uint32_t tab = per_group ? (uint32_t)C::kTabRegion : 128u;
         const uint32_t st = sbase + C::kWOff + s * C::kWSlot;
-        mbar_arrive_expect_tx(wfull_bar(s), C::kWBytes + 2 * tab);
-        bulk_load(st, a.Wp + chunk_offset(n_tile, kb * kCh, a.K), C::kWBytes, wfull_bar(s));
-        // group tables of the K block (G = 128: kCh groups; G = K: the one group)
-        const size_t toff = ((size_t)n_tile * a.ngroups + (per_group ? kb * kCh : 0)) * kPanelRows;
-        bulk_load(st + C::kWBytes, a.s_g + toff, tab, wfull_bar(s));
-        bulk_load(st + C::kWBytes + C::kTabRegion, a.zs + toff, tab, wfull_bar(s));
+        const uint32_t bytes = (uint32_t)(kCh * cstride);
+        mbar_arrive_expect_tx(wfull_bar(s), bytes);
+        bulk_load(st, a.Wp + chunk_offset(n_tile, kb * kCh, a.K, a.G), bytes, wfull_bar(s));
         issued |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
     };
@@ -316,8 +328,7 @@ __global__ void __launch_bounds__(352, 1)
             mbar_init(wempty_bar(s), 4);     // 4 dequant warps
         }
         for (int s = 0; s < SX; ++s) {
-            mbar_init(xfull_bar(s), 1);
-            mbar_init(afull_bar(s), 4);      // 4 dequant warps
+            mbar_init(afull_bar(s), 5);      // 4 dequant warps + the X8 producer
             mbar_init(xaempty_bar(s), 1);    // MMA commit
         }
         for (int b = 0; b < C::kAccBufs; ++b) {
@@ -334,7 +345,7 @@ __global__ void __launch_bounds__(352, 1)
             ++tj;
         }
     }
-    if (threadIdx.x == 320) prefetch_tmap(&tmap_x);
+    if (threadIdx.x == 64) prefetch_tmap(&tmap_x);
     // The next kernel in the stream may launch now; whatever it reads from
     // this GEMM it must read after its own griddepcontrol.wait.
     grid_launch_dependents();
@@ -368,7 +379,7 @@ __global__ void __launch_bounds__(352, 1)
                 }
             }
         }
-    } else if (warp == 10) {
+    } else if (warp == 2) {
         // ------------------------------------------------- X8 producer --
         if (lane == 0) {
             grid_dependency_wait();  // X8 comes from the preceding kernel
@@ -385,10 +396,10 @@ __global__ void __launch_bounds__(352, 1)
                         break;
                     }
                     const uint32_t st = sbase + s * C::kXSlot;
-                    mbar_arrive_expect_tx(xfull_bar(s), C::kXSlot);
+                    mbar_arrive_expect_tx(afull_bar(s), C::kXSlot);
 #pragma unroll
                     for (int c = 0; c < kCh; ++c)
-                        tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN, xfull_bar(s));
+                        tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN, afull_bar(s));
                     if (tj < 16) QOQ_MARK(32 + tj);
                     ++tj;
                     issued |= 1u << s;
@@ -458,52 +469,76 @@ __global__ void __launch_bounds__(352, 1)
             mma_commit(mmadone_bar);
             drain_wait(mmadone_bar, 0, 200000000ull);
         }
-    } else if (warp < 6) {
+    } else if (warp >= 4 && warp < kEpiWarp0) {
         // ------------------------------------------------------ dequant --
+        // With two groups of four warps, group 0 takes the CTA's even
+        // stages and group 1 the odd ones.
+        const int grp = (warp - 4) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;  // output channel within the panel
         int sw = 0, sx = 0;
         uint32_t pw = 0, px = 0;
-        bool ok = true;
-        for (int i = i_begin; i < i_end && ok;) {
-            const int t = i / ks;
-            const int ks1 = min(ks, i_end - t * ks);
-            for (int kb = i - t * ks; kb < ks1; ++kb) {
-                if (!wait_bounded(wfull_bar(sw), pw, abort_flag, budget)) {
-                    ok = false;
-                    break;
+        // per-channel tables (G = K) come from global memory, one byte each
+        // per tile; the next tile's are fetched while this one runs
+        uint32_t pc_sg = 0, pc_zs = 0, nx_sg = 0, nx_zs = 0;
+        int t_cur = -1, t_nx = -1;
+        auto load_tab = [&](int t, uint32_t &sgv, uint32_t &zsv) {
+            const size_t o = (size_t)(t / a.m_tiles) * kPanelRows + r;
+            sgv = __ldg(a.s_g + o);
+            zsv = __ldg(a.zs + o);
+        };
+        if (!per_group && i_begin < i_end) {
+            t_nx = i_begin / ks;
+            load_tab(t_nx, nx_sg, nx_zs);
+        }
+        for (int u = i_begin; u < i_end; ++u) {
+            if ((u - i_begin) % kDq == grp) {
+                if (!per_group) {
+                    const int t = u / ks;
+                    if (t != t_cur) {
+                        if (t == t_nx) {
+                            pc_sg = nx_sg;
+                            pc_zs = nx_zs;
+                        } else {
+                            load_tab(t, pc_sg, pc_zs);
+                        }
+                        t_cur = t;
+                        t_nx = ((t + 1) * ks < i_end) ? t + 1 : -1;
+                        if (t_nx >= 0) load_tab(t_nx, nx_sg, nx_zs);
+                    }
                 }
-                if (warp == 2 && lane == 0 && tj < 16) QOQ_MARK(48 + tj);
+                if (!wait_bounded(wfull_bar(sw), pw, abort_flag, budget)) break;
+                if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(48 + tj);
                 const uint8_t *wsl = smem + C::kWOff + sw * C::kWSlot;
-                const uint8_t *tg = wsl + C::kWBytes;
                 uint4 v[kCh][4];
                 uint32_t sg[kCh], zsv[kCh];
 #pragma unroll
                 for (int c = 0; c < kCh; ++c) {
+                    const uint8_t *chunk = wsl + c * cstride;
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        v[c][j] = *reinterpret_cast<const uint4 *>(wsl + c * kChunkBytes + j * kSlabBytes + r * 16);
-                    const int g = per_group ? c : 0;
-                    sg[c] = tg[g * 128 + r];
-                    zsv[c] = tg[C::kTabRegion + g * 128 + r];
+                        v[c][j] = *reinterpret_cast<const uint4 *>(chunk + j * kSlabBytes + r * 16);
+                    if (per_group) {
+                        sg[c] = chunk[kChunkBytes + r];
+                        zsv[c] = chunk[kChunkBytes + kPanelRows + r];
+                    } else {
+                        sg[c] = pc_sg;
+                        zsv[c] = pc_zs;
+                    }
                 }
+                // The next bulk copy into this slot writes through the async
+                // proxy: order these generic-proxy reads before it, then
+                // release the slot.
+                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(wempty_bar(sw));  // the weight slot may be refilled now
-                if (warp == 2 && lane == 0 && tj < 16) QOQ_MARK(64 + tj);
-                if (++sw == SW) {
-                    sw = 0;
-                    pw ^= 1u;
-                }
-                // X8 slot sx has landed.  That also means A slot sx is free:
-                // the X8 producer refills slot sx only after the MMAs of its
-                // previous use have completed (xaempty), so those MMAs are
-                // done reading A slot sx by the time xfull completes.
-                if (!wait_bounded(xfull_bar(sx), px, abort_flag, budget)) {
-                    ok = false;
-                    break;
-                }
+                if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(64 + tj);
+                // A slot sx is free once the MMAs of its previous use have
+                // completed; the X8 tiles need not have landed (the MMA
+                // issuer waits for those on afull)
+                if (!wait_bounded(xaempty_bar(sx), px ^ 1u, abort_flag, budget)) break;
                 tc_fence_after();
-                if (warp == 2 && lane == 0 && tj < 16) QOQ_MARK(80 + tj);
+                if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(80 + tj);
 #pragma unroll
                 for (int c = 0; c < kCh; ++c) {
                     const uint32_t sgc = sg[c];
@@ -530,16 +565,19 @@ __global__ void __launch_bounds__(352, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(afull_bar(sx));
-                if (warp == 2 && lane == 0 && tj < 16) QOQ_MARK(96 + tj);
+                if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(96 + tj);
                 ++tj;
-                if (++sx == SX) {
-                    sx = 0;
-                    px ^= 1u;
-                }
             }
-            i = t * ks + ks1;
+            if (++sw == SW) {
+                sw = 0;
+                pw ^= 1u;
+            }
+            if (++sx == SX) {
+                sx = 0;
+                px ^= 1u;
+            }
         }
-    } else {
+    } else if (warp >= kEpiWarp0) {
         // ----------------------------------------------------- epilogue --
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
@@ -575,7 +613,9 @@ __global__ void __launch_bounds__(352, 1)
             // this CTA's own MMAs for the tile are still running.
             bool ready = true;
             constexpr bool kPresum = (BN <= 64);
-            constexpr int kGrp = BN < 64 ? BN : 64;  // accumulator columns per TMEM load
+            // accumulator columns per TMEM load (16 where the pre-summed
+            // partials of a 64-wide tile already hold 64 registers)
+            constexpr int kGrp = BN < 64 ? BN : (kPresum ? 16 : 64);
             int32_t pre[kPresum ? BN : 1];
             if (finisher) {
                 // Every lane of every later contributor counts its own
@@ -596,7 +636,7 @@ __global__ void __launch_bounds__(352, 1)
                 ready = __all_sync(0xffffffffu, ready);
                 __syncwarp();  // every lane has seen the full count
                 if (lane == 0 && ready) *counter = 0;  // ready for the next call
-                if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(224 + tj);
+                if (warp == kEpiWarp0 && lane == 0 && tj < 8) QOQ_MARK(224 + tj);
                 if constexpr (kPresum) {
 #pragma unroll
                     for (int q = 0; q < BN; ++q) pre[q] = 0;
@@ -623,7 +663,7 @@ __global__ void __launch_bounds__(352, 1)
                 }
             }
             if (!wait_bounded(accfull_bar(ab), accph, abort_flag, budget)) break;
-            if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(208 + tj);
+            if (warp == kEpiWarp0 && lane == 0 && tj < 8) QOQ_MARK(208 + tj);
             tc_fence_after();
             const uint32_t tacc = trow + (uint32_t)(ab * BN);
             // the accumulator goes back to the MMA as soon as its last
@@ -665,12 +705,12 @@ __global__ void __launch_bounds__(352, 1)
                     uint32_t vg[kGrp];
                     tmem_load_cols<kGrp>(tacc + g0 * 16, vg);
                     if (g0 + kGrp / 16 >= nchunks) release_acc();
-                    if (warp == 6 && lane == 0 && tj < 2 && g0 == 0) QOQ_MARK(232 + tj * 8);
+                    if (warp == kEpiWarp0 && lane == 0 && tj < 2 && g0 == 0) QOQ_MARK(232 + tj * 8);
 #pragma unroll
                     for (int u = 0; u < kGrp / 16; ++u) {
                         const int cc = g0 + u;
                         if (cc >= nchunks) break;
-                        if (warp == 6 && lane == 0 && tj < 2 && cc < 6) QOQ_MARK(233 + tj * 8 + cc);
+                        if (warp == kEpiWarp0 && lane == 0 && tj < 2 && cc < 6) QOQ_MARK(233 + tj * 8 + cc);
                         int32_t acc[16];
 #pragma unroll
                         for (int q = 0; q < 16; ++q) acc[q] = (int32_t)vg[16 * u + q];
@@ -725,7 +765,7 @@ __global__ void __launch_bounds__(352, 1)
                 }
                 if (!released) release_acc();
             }
-            if (warp == 6 && lane == 0 && tj < 8) QOQ_MARK(216 + tj);
+            if (warp == kEpiWarp0 && lane == 0 && tj < 8) QOQ_MARK(216 + tj);
             ++tj;
             if (++ab == C::kAccBufs) {
                 ab = 0;
@@ -733,7 +773,7 @@ __global__ void __launch_bounds__(352, 1)
             }
             i = t * ks + ks1;
         }
-        if (warp == 6 && lane == 0) QOQ_MARK(4);
+        if (warp == kEpiWarp0 && lane == 0) QOQ_MARK(4);
     }
 
     __syncwarp();
@@ -741,13 +781,23 @@ __global__ void __launch_bounds__(352, 1)
     __syncthreads();
     tc_fence_after();
     QOQ_MARK(2);
-    if ((threadIdx.x == 0 || threadIdx.x == 320) && *abort_flag) {
-        if (threadIdx.x == 0) atomicExch(&g_dev_error, 1);
+    if ((threadIdx.x == 0 || threadIdx.x == 64) && *abort_flag) {
         // the producers: let their own copies land before the CTA exits
-        const int nslots = threadIdx.x == 0 ? SW : SX;
-        for (int q = 0; q < nslots; ++q)
-            if (issued & (1u << q))
-                drain_wait(threadIdx.x == 0 ? wfull_bar(q) : xfull_bar(q), (issued_par >> q) & 1u, 200000000ull);
+        if (threadIdx.x == 0) {
+            atomicExch(&g_dev_error, 1);
+            for (int q = 0; q < SW; ++q)
+                if (issued & (1u << q)) drain_wait(wfull_bar(q), (issued_par >> q) & 1u, 200000000ull);
+        } else {
+            // An X8 slot's phase also needs the dequant warps' arrivals,
+            // which an aborted stage may lack: wait briefly for each, then
+            // give any copy still in flight a fixed grace period (a tile
+            // lands within microseconds).
+            for (int q = 0; q < SX; ++q)
+                if (issued & (1u << q)) drain_wait(afull_bar(q), (issued_par >> q) & 1u, 1000000ull);
+            const uint64_t until = global_timer_ns() + 200000ull;
+            while (global_timer_ns() < until) {
+            }
+        }
     }
     if (warp == 0) {
         __syncwarp();
@@ -814,7 +864,7 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     // touches X8 or s_x.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(352);
+    cfg.blockDim = dim3(gemm_threads(BN));
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

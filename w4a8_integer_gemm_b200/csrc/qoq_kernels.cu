@@ -108,6 +108,11 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
             const size_t ti = ((size_t)p * (K / G) + g) * kPanelRows + rr;
             s_g[ti] = (uint8_t)sg;
             zs[ti] = (uint8_t)(z * sg);
+            if (G == kBlockK) {  // the copy inside the group's chunk
+                uint8_t *tab = Wp + chunk_offset(p, g, K, G) + kChunkBytes;
+                tab[rr] = (uint8_t)sg;
+                tab[kPanelRows + rr] = (uint8_t)(z * sg);
+            }
         }
         for (int kc = k_lo; kc < k_hi; kc += 128) {
             const float4 v = __ldg(reinterpret_cast<const float4 *>(w + kc + lane * 4));
@@ -119,7 +124,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
             const uint32_t partner = __shfl_down_sync(0xffffffffu, mine, 4);
             if ((lane & 7) < 4) {
                 const int slab = lane >> 3, word = lane & 7;
-                uint8_t *dst = Wp + chunk_offset(p, kc / kBlockK, K) + slab * kSlabBytes + rr * 16 + word * 4;
+                uint8_t *dst = Wp + chunk_offset(p, kc / kBlockK, K, G) + slab * kSlabBytes + rr * 16 + word * 4;
                 *reinterpret_cast<uint32_t *>(dst) = mine | (partner << 4);
             }
         }
@@ -127,8 +132,11 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
 }
 
 // ---------------------------------------------------- activation quant --
-constexpr int kActThreads = 256;
-constexpr int kActCache = 12;  // 16-byte vectors per thread kept in registers (K <= 24576)
+// A small CTA (128 threads, few registers) so that the quantizer of the
+// next layer fits on an SM beside a running GEMM CTA: it can then start,
+// and trigger the launch of its own GEMM, before the current GEMM ends.
+constexpr int kActThreads = 128;
+constexpr int kActCache = 4;   // 16-byte vectors per thread kept in registers (K <= 4096)
 
 __device__ __forceinline__ float absmax8(const uint4 &v)
 {
@@ -163,7 +171,7 @@ __device__ __forceinline__ uint2 quant8(const uint4 &v, float sx)
 
 // One CTA per token row: read the row once (kept in registers up to
 // kActCache vectors per thread), reduce max|x|, then quantize.
-__global__ void __launch_bounds__(kActThreads) act_quant_kernel(const uint16_t *__restrict__ X, int K,
+__global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16_t *__restrict__ X, int K,
                                                                  int8_t *__restrict__ X8,
                                                                  uint16_t *__restrict__ s_x)
 {
@@ -215,7 +223,9 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const uint16_t *
 
 // ------------------------------------------------- INT8 weight expand --
 // One thread per (channel n, 32-wide K slice): the GEMM's dequant routine
-// on one 16-byte row slice, written out as 32 INT8 weights.
+// on one 16-byte row slice, written out as 32 INT8 weights.  Like the GEMM,
+// it takes 128-wide groups' tables from the chunk and per-channel tables
+// from s_g / zs.
 __global__ void dequant_kernel(const uint8_t *__restrict__ Wp, const uint8_t *__restrict__ s_g,
                                const uint8_t *__restrict__ zs, int N, int K, int G, int8_t *__restrict__ out)
 {
@@ -224,11 +234,19 @@ __global__ void dequant_kernel(const uint8_t *__restrict__ Wp, const uint8_t *__
     if (idx >= (size_t)N * slices) return;
     const int n = (int)(idx / slices);
     const int k0 = (int)(idx % slices) * kSlabK;
-    const uint4 v = *reinterpret_cast<const uint4 *>(Wp + chunk_offset(n / kPanelRows, k0 / kBlockK, K) +
-                                                     ((k0 % kBlockK) / kSlabK) * kSlabBytes + (n % kPanelRows) * 16);
-    const size_t ti = ((size_t)(n / kPanelRows) * (K / G) + k0 / G) * kPanelRows + n % kPanelRows;
-    const uint32_t sg = s_g[ti];
-    const uint32_t bias = zero_comp_bias(zs[ti]);
+    const uint8_t *chunk = Wp + chunk_offset(n / kPanelRows, k0 / kBlockK, K, G);
+    const uint4 v = *reinterpret_cast<const uint4 *>(chunk + ((k0 % kBlockK) / kSlabK) * kSlabBytes +
+                                                     (n % kPanelRows) * 16);
+    uint32_t sg, zsv;
+    if (G == kBlockK) {
+        sg = chunk[kChunkBytes + n % kPanelRows];
+        zsv = chunk[kChunkBytes + kPanelRows + n % kPanelRows];
+    } else {
+        const size_t ti = ((size_t)(n / kPanelRows) * (K / G) + k0 / G) * kPanelRows + n % kPanelRows;
+        sg = s_g[ti];
+        zsv = zs[ti];
+    }
+    const uint32_t bias = zero_comp_bias(zsv);
     uint32_t w8[8];
     dequant_slab(v, sg, bias, w8);
     uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)n * K + k0);

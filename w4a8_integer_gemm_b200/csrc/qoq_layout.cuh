@@ -30,12 +30,21 @@ constexpr int kPanelRows = 128;     // output channels per packed panel (= MMA M
 constexpr int kBlockK = 128;        // K per packed chunk (= one pipeline stage)
 constexpr int kSlabK = 32;          // K per 16-byte row slice (= one MMA K step)
 constexpr int kSlabBytes = 2048;    // 128 rows x 16 bytes
-constexpr int kChunkBytes = 8192;   // 4 slabs
+constexpr int kChunkBytes = 8192;   // 4 slabs of codes
+constexpr int kChunkTabBytes = 256; // G = 128: the chunk's s_g[128], then zs[128]
+
+// Bytes from one chunk to the next: with 128-wide groups every chunk
+// carries its group's tables right after its codes, so one copy brings
+// both; per-channel tables (G = K) are not repeated in the chunks.
+__host__ __device__ __forceinline__ int chunk_stride(int G)
+{
+    return kChunkBytes + (G == kBlockK ? kChunkTabBytes : 0);
+}
 
 // Byte offset of chunk (panel p, K block b) in the packed buffer.
-__host__ __device__ __forceinline__ size_t chunk_offset(int p, int b, int K)
+__host__ __device__ __forceinline__ size_t chunk_offset(int p, int b, int K, int G)
 {
-    return ((size_t)p * (size_t)(K / kBlockK) + (size_t)b) * (size_t)kChunkBytes;
+    return ((size_t)p * (size_t)(K / kBlockK) + (size_t)b) * (size_t)chunk_stride(G);
 }
 
 // The biased zero-compensation constant for a group, replicated in 4 lanes.

@@ -168,8 +168,9 @@ __device__ __forceinline__ void prefetch_tmap(const void *tmap)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
-// Make generic-proxy shared-memory writes visible to the async proxy
-// (tensor-core operand reads).
+// Order this thread's generic-proxy shared-memory accesses before later
+// async-proxy accesses: writes before tensor-core operand reads, and reads
+// before a bulk copy that refills the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
