@@ -203,6 +203,32 @@ QOQ_API int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x,
                   uint16_t *Y, int32_t *acc_dbg,
                   void *workspace, size_t workspace_bytes, void *stream);
 
+/* The whole W4A8 linear layer in one kernel launch: the per-token
+ * quantization of qoq_quant_act_per_token followed by qoq_w4a8_gemm.
+ *
+ * Sources: as for those two calls; the result is bit-identical to calling
+ * them in sequence. The pages describe the two steps as one layer; doing
+ * both in one launch saves the second kernel's launch and its wait for the
+ * first to finish (which is most of a decode-sized layer's time).
+ *
+ *   X        device, uint16_t [M][K] FP16 bits, read only.
+ *   X8, s_x  device, written exactly as qoq_quant_act_per_token writes them
+ *            (int8_t [M][K]; uint16_t [M] FP16 bits, 16-byte aligned).
+ *   Wp, s_c, s_g, zs, Y, workspace, workspace_bytes
+ *            as for qoq_w4a8_gemm (the same workspace rules; this call also
+ *            leaves the workspace's counters at zero).
+ * For M <= 148 the rows are quantized inside the GEMM kernel by the SMs'
+ * otherwise idle epilogue warps (one row per SM), which publish each
+ * finished row with a release operation; the GEMM's loads of X8 and s_x
+ * wait (bounded) until every row is done. Larger M runs the quantizer and
+ * the GEMM as two kernels on the stream. Limits: as for qoq_w4a8_gemm.
+ */
+QOQ_API int qoq_w4a8_linear(const uint16_t *X, int M, int N, int K, int group_size,
+                    const uint8_t *Wp, const uint16_t *s_c,
+                    const uint8_t *s_g, const uint8_t *zs,
+                    int8_t *X8, uint16_t *s_x, uint16_t *Y,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
 /* The same GEMM as qoq_w4a8_gemm, for callers that cannot allocate memory.
  *
  * The paper has no counterpart to this call. It exists because some callers

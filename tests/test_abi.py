@@ -27,7 +27,7 @@ def declared():
 def test_exports_every_declared_symbol(L):
     import w4a8_integer_gemm_b200 as q
     names = declared()
-    assert len(names) == 10
+    assert len(names) == 11
     for n in names:
         assert hasattr(L, n), n
     assert names == set(q.SIGNATURES)
@@ -99,3 +99,20 @@ def test_invalid_arguments_rejected_on_host(L):
     assert L.qoq_pack_weights(B, 512, 512, 128, A, A, A, A, None) == INVALID
     assert L.qoq_dequant_weights_i8(A, A, A, 512, 512, 3, A, None) == INVALID
     assert L.qoq_set_gemm_a_in_tmem(2) == INVALID
+    # the fused layer call: X, M, N, K, G, Wp, s_c, s_g, zs, X8, s_x, Y, ws, wsb, stream
+    f = L.qoq_w4a8_linear
+    fused_ok = [A, 16, 512, 512, 128, A, A, A, A, A, A, A, A, 1 << 30, None]
+
+    def fcall(i, v):
+        a = list(fused_ok)
+        a[i] = v
+        return f(*a)
+
+    assert fcall(0, B) == INVALID                 # misaligned X
+    assert fcall(0, None) == INVALID
+    assert fcall(3, 500) == INVALID               # K
+    assert fcall(4, 64) == INVALID                # group size
+    assert fcall(9, None) == INVALID              # X8
+    assert fcall(10, B) == INVALID                # s_x
+    assert fcall(13, 16) == INVALID               # workspace too small
+    assert fcall(1, 0) == 0                       # M = 0: nothing to do

@@ -48,6 +48,7 @@ SIGNATURES = {
     "qoq_gemm_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "qoq_w4a8_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "qoq_w4a8_gemm_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "qoq_w4a8_linear": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "qoq_dequant_weights_i8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "qoq_set_gemm_a_in_tmem": (_I, [_I]),
     "qoq_device_error": (_I, [_P]),
@@ -209,6 +210,33 @@ def qoq_w4a8_gemm(X8: torch.Tensor, s_x: torch.Tensor, packed: PackedWeights,
     return Y
 
 
+def qoq_w4a8_linear(X: torch.Tensor, packed: PackedWeights, X8: Optional[torch.Tensor] = None,
+                    s_x: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None):
+    """Quantize X (fp16 [M, K]) per token and run the GEMM, in one launch.
+
+    Returns (Y, X8, s_x); bit-identical to qoq_quant_act_per_token followed
+    by qoq_w4a8_gemm."""
+    _need(X, torch.float16, "X")
+    M, K = X.shape
+    if K != packed.K:
+        raise ValueError("K mismatch between X and the packed weights")
+    N = packed.N
+    if X8 is None:
+        X8 = torch.empty(M, K, dtype=torch.int8, device=X.device)
+    if s_x is None:
+        s_x = torch.empty(max(M, 8), dtype=torch.int16, device=X.device)
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float16, device=X.device)
+    if workspace is None:
+        workspace = gemm_workspace(max(M, 1), N, K, packed.group_size, X.device)
+    st = lib().qoq_w4a8_linear(_ptr(X), M, N, K, packed.group_size, _ptr(packed.Wp), _ptr(packed.s_c),
+                               _ptr(packed.s_g), _ptr(packed.zs), _ptr(X8), _ptr(s_x), _ptr(Y), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("qoq_w4a8_linear", st)
+    return Y, X8, s_x
+
+
 def qoq_w4a8_gemm_noalloc(X8: torch.Tensor, s_x: torch.Tensor, packed: PackedWeights,
                           Y: torch.Tensor, stream=None) -> torch.Tensor:
     """The GEMM with its scratch in the library's built-in buffer.
@@ -251,8 +279,9 @@ class W4A8Linear:
         self.out_features = W.shape[0]
 
     def __call__(self, x_fp16: torch.Tensor, stream=None) -> torch.Tensor:
-        X8, s_x = qoq_quant_act_per_token(x_fp16, stream=stream)
-        return qoq_w4a8_gemm(X8, s_x, self.packed, stream=stream)
+        """y = fp16 W4A8 linear of x (fp16 [M, in_features]), one kernel launch."""
+        Y, _, _ = qoq_w4a8_linear(x_fp16, self.packed, stream=stream)
+        return Y
 
 
 def w4a8_linear_host(x_host: torch.Tensor, layer: W4A8Linear, y_host: Optional[torch.Tensor] = None,

@@ -129,6 +129,37 @@ int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, cons
     return from_cuda(e);
 }
 
+int qoq_w4a8_linear(const uint16_t *X, int M, int N, int K, int group_size, const uint8_t *Wp,
+                    const uint16_t *s_c, const uint8_t *s_g, const uint8_t *zs, int8_t *X8, uint16_t *s_x,
+                    uint16_t *Y, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (M < 0 || M > kMaxM || !valid_nk(N, K) || !valid_group(K, group_size) || K > kMaxK)
+        return QOQ_ERR_INVALID_ARG;
+    if (M == 0) return QOQ_OK;
+    if (!X || !X8 || !s_x || !Wp || !s_c || !s_g || !zs || !Y || !workspace) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(X8) || !aligned16(s_x) || !aligned16(Wp) || !aligned16(s_c) ||
+        !aligned16(s_g) || !aligned16(zs) || !aligned16(Y) || !aligned16(workspace))
+        return QOQ_ERR_INVALID_ARG;
+    if (!qoq::gemm_shape_supported(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    if (workspace_bytes < qoq::gemm_workspace_bytes(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    int tmap_status = 0;
+    // Up to one row per SM the GEMM quantizes its own input; a longer chain
+    // of rows per SM costs more than the quantizer's own launch, so larger
+    // batches run the two kernels back to back (same results).
+    const bool in_kernel = M <= qoq::kFusedMaxRows;
+    if (!in_kernel) {
+        const cudaError_t eq = qoq::launch_act_quant(X, M, K, X8, s_x, (cudaStream_t)stream);
+        if (eq != cudaSuccess) return from_cuda(eq);
+    }
+    cudaError_t e = qoq::launch_gemm(X8, s_x, Wp, s_c, s_g, zs, M, N, K, group_size, Y, nullptr, workspace,
+                                     g_a_in_tmem.load() != 0, (cudaStream_t)stream, &tmap_status,
+                                     in_kernel ? X : nullptr);
+    if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
 int qoq_dequant_weights_i8(const uint8_t *Wp, const uint8_t *s_g, const uint8_t *zs, int N, int K, int group_size,
                            int8_t *W8hat, void *stream)
 {

@@ -67,6 +67,7 @@
 #include "qoq_internal.h"
 #include "qoq_layout.cuh"
 #include "qoq_ptx.cuh"
+#include "qoq_quant.cuh"
 
 namespace qoq {
 
@@ -82,6 +83,13 @@ struct GemmArgs {
     int32_t *acc_dbg;
     int32_t *ws_cnt;   // [kMaxCtas][4] arrival counters, at the start of the workspace
     int32_t *ws_part;  // [cta][BN/16][128][16] INT32 partial tile, after the counters
+    // The fused call (X non-null): the kernel first quantizes the FP16 rows
+    // of X into X8 / s_x itself, then reads them as in the plain GEMM.
+    const uint16_t *X;
+    int8_t *X8w;       // = the X8 the tensor map reads
+    uint16_t *s_xw;    // = s_x
+    int32_t *ws_ready; // epilogue threads that have stored their part of a row (128 per row)
+    int32_t *ws_done;  // CTAs finished; the last one resets both counters
     int M, N, K, G;
     int m_tiles;
     int ks;            // K / KST units per tile
@@ -188,14 +196,26 @@ __device__ __forceinline__ int ld_acquire_gpu(const int *p)
     return v;
 }
 
+// Wait (acquire, bounded) until *p >= want; false on timeout or abort, and
+// a timeout raises the CTA's abort flag.
+__device__ __forceinline__ bool wait_count_gpu(const int *p, int want, volatile int *abort, uint64_t budget_ns)
+{
+    if (ld_acquire_gpu(p) >= want) return true;
+    const uint64_t start = global_timer_ns();
+    while (ld_acquire_gpu(p) < want) {
+        if (*abort) return false;
+        if (global_timer_ns() - start > budget_ns) {
+            *abort = 1;
+            return false;
+        }
+        __nanosleep(100);
+    }
+    return true;
+}
+
 __device__ __forceinline__ void red_release_gpu_add(int *p, int v)
 {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ float half_bits_to_float(uint16_t h)
-{
-    return __half2float(__ushort_as_half(h));
 }
 
 __device__ __forceinline__ uint16_t scale_to_half(int32_t acc, float sx, float sc)
@@ -383,9 +403,14 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         // ------------------------------------------------- X8 producer --
         if (lane == 0) {
             grid_dependency_wait();  // X8 comes from the preceding kernel
+            bool ok = true;
+            if (a.X) {
+                // fused call: X8 is written by this grid's epilogue warps
+                ok = wait_count_gpu(a.ws_ready, 128 * a.M, abort_flag, budget);
+                fence_proxy_async_global();
+            }
             int s = 0;
             uint32_t ph = 0;
-            bool ok = true;
             for (int i = i_begin; i < i_end && ok;) {
                 const int t = i / ks;
                 const int ks1 = min(ks, i_end - t * ks);
@@ -585,7 +610,64 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         uint8_t *stg = smem + C::kStgOff + quarter * 1024;  // this warp's output staging block
         int ab = 0;          // accumulator of the current tile
         uint32_t accph = 0;  // its phase parity
-        grid_dependency_wait();  // s_x comes from the preceding kernel
+        grid_dependency_wait();  // s_x (or X) comes from the preceding kernel
+        if (a.X) {
+            // Fused call: the four epilogue warps of each CTA quantize token
+            // rows cta, cta + P, ... together (128 threads per row, the
+            // loads of a row in flight at once), then every lane waits until
+            // all rows are done: any token's X8 tiles and s_x may be needed.
+            const int et = threadIdx.x - kEpiWarp0 * 32;           // 0..127
+            float *rowmax = reinterpret_cast<float *>(smem + C::kStgOff);  // [4], in warp 0's staging block
+            const int nvec = a.K / 8;
+            constexpr int kCache = 4;  // 16-byte vectors per thread held across the two passes (K <= 4096)
+            for (int row = cta; row < a.M; row += P) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(a.X + (size_t)row * a.K);
+                uint4 cache[kCache];
+                float amax = 0.0f;
+#pragma unroll
+                for (int c = 0; c < kCache; ++c) {
+                    const int v = et + c * 128;
+                    cache[c] = v < nvec ? __ldcg(src + v) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int c = 0; c < kCache; ++c) amax = fmaxf(amax, absmax8(cache[c]));
+                for (int v0 = et + kCache * 128; v0 < nvec; v0 += 4 * 128) {
+                    uint4 t[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) t[c] = (v0 + c * 128 < nvec) ? __ldcg(src + v0 + c * 128) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) amax = fmaxf(amax, absmax8(t[c]));
+                }
+                amax = warp_max(amax);
+                if (lane == 0) rowmax[warp - kEpiWarp0] = amax;
+                named_barrier(1, 128);
+                amax = fmaxf(fmaxf(rowmax[0], rowmax[1]), fmaxf(rowmax[2], rowmax[3]));
+                named_barrier(1, 128);  // rowmax is free for the next row
+                const uint16_t sxh = token_scale_bits(amax);
+                const float sxf = half_bits_to_float(sxh);
+                uint2 *dst = reinterpret_cast<uint2 *>(a.X8w + (size_t)row * a.K);
+#pragma unroll
+                for (int c = 0; c < kCache; ++c) {
+                    const int v = et + c * 128;
+                    if (v < nvec) dst[v] = quant8(cache[c], sxf);
+                }
+                for (int v0 = et + kCache * 128; v0 < nvec; v0 += 4 * 128) {
+                    uint4 t[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) t[c] = (v0 + c * 128 < nvec) ? __ldcg(src + v0 + c * 128) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        if (v0 + c * 128 < nvec) dst[v0 + c * 128] = quant8(t[c], sxf);
+                }
+                if (et == 0) a.s_xw[row] = sxh;
+                // the X8 tiles are read back by TMA (the async proxy); each
+                // thread's release covers its own stores
+                fence_proxy_async_global();
+                red_release_gpu_add(a.ws_ready, 1);
+            }
+            // 128 counts per row; on a timeout the flag stops every role
+            wait_count_gpu(a.ws_ready, 128 * a.M, abort_flag, budget);
+        }
         for (int i = i_begin; i < i_end;) {
             const int t = i / ks;
             const int ks0 = i - t * ks;
@@ -601,7 +683,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
 #pragma unroll
             for (int q = 0; q < C::kSx; ++q) {
                 const int m = m0 + q * 32 + lane;
-                sx_reg[q] = (q * 32 + lane < BN && m < a.M) ? half_bits_to_float(__ldg(a.s_x + m)) : 0.0f;
+                sx_reg[q] = (q * 32 + lane < BN && m < a.M) ? half_bits_to_float(__ldcg(a.s_x + m)) : 0.0f;
             }
             const float sc = half_bits_to_float(__ldg(a.s_c + n));
             const int c_lo = partial ? cta_of(t * ks, P, T) : cta;
@@ -705,6 +787,32 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     uint32_t vg[kGrp];
                     tmem_load_cols<kGrp>(tacc + g0 * 16, vg);
                     if (g0 + kGrp / 16 >= nchunks) release_acc();
+                    if constexpr (!kPresum) {
+                        if (finisher) {
+                            // the later contributors' partials of this group
+                            // of chunks, all loads of a contributor in flight
+#pragma unroll 1
+                            for (int c2 = cta + 1; c2 <= c_hi; ++c2) {
+                                const int4 *src =
+                                    reinterpret_cast<const int4 *>(a.ws_part + (size_t)c2 * BN * kPanelRows);
+                                int4 ld[kGrp / 4];
+#pragma unroll
+                                for (int u = 0; u < kGrp / 16; ++u)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j)
+                                        ld[u * 4 + j] = (g0 + u < nchunks)
+                                                            ? __ldcg(src + ((size_t)(g0 + u) * kPanelRows + r) * 4 + j)
+                                                            : make_int4(0, 0, 0, 0);
+#pragma unroll
+                                for (int j = 0; j < kGrp / 4; ++j) {
+                                    vg[4 * j] += (uint32_t)ld[j].x;
+                                    vg[4 * j + 1] += (uint32_t)ld[j].y;
+                                    vg[4 * j + 2] += (uint32_t)ld[j].z;
+                                    vg[4 * j + 3] += (uint32_t)ld[j].w;
+                                }
+                            }
+                        }
+                    }
                     if (warp == kEpiWarp0 && lane == 0 && tj < 2 && g0 == 0) QOQ_MARK(232 + tj * 8);
 #pragma unroll
                     for (int u = 0; u < kGrp / 16; ++u) {
@@ -725,34 +833,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                                         if (c3 == cc) add = pre[c3 * 16 + q];
                                     acc[q] += add;
                                 }
-                            }
-                        } else if (finisher) {
-                            // partials of the later contributors, 16 loads in flight per batch
-#pragma unroll 1
-                            for (int c2 = cta + 1; c2 <= c_hi; c2 += 4) {
-                                int4 ld[4][4];
-#pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    if (c2 + u <= c_hi) {
-                                        const int4 *src = reinterpret_cast<const int4 *>(
-                                                              a.ws_part + (size_t)(c2 + u) * BN * kPanelRows) +
-                                                          ((size_t)cc * kPanelRows + r) * 4;
-#pragma unroll
-                                        for (int j = 0; j < 4; ++j) ld[u][j] = __ldcg(src + j);
-                                    } else {
-#pragma unroll
-                                        for (int j = 0; j < 4; ++j) ld[u][j] = make_int4(0, 0, 0, 0);
-                                    }
-                                }
-#pragma unroll
-                                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) {
-                                        acc[4 * j] += ld[u][j].x;
-                                        acc[4 * j + 1] += ld[u][j].y;
-                                        acc[4 * j + 2] += ld[u][j].z;
-                                        acc[4 * j + 3] += ld[u][j].w;
-                                    }
                             }
                         }
                         float sxr = sx_reg[0];
@@ -781,6 +861,14 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     __syncthreads();
     tc_fence_after();
     QOQ_MARK(2);
+    if (a.X && threadIdx.x == 0) {
+        // every CTA is past its waits on ws_ready: the last one to get here
+        // leaves both counters at zero for the next call
+        if (atomicAdd(a.ws_done, 1) == P - 1) {
+            *a.ws_ready = 0;
+            *a.ws_done = 0;
+        }
+    }
     if ((threadIdx.x == 0 || threadIdx.x == 64) && *abort_flag) {
         // the producers: let their own copies land before the CTA exits
         if (threadIdx.x == 0) {
@@ -949,7 +1037,8 @@ size_t gemm_workspace_bytes(int M, int N, int K)
 
 cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
                         const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
-                        int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream, int *tmap_status)
+                        int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream, int *tmap_status,
+                        const uint16_t *X)
 {
     *tmap_status = 0;
     const int BN = gemm_block_n(M);
@@ -984,6 +1073,11 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     args.Y = Y;
     args.acc_dbg = acc_dbg;
     args.ws_cnt = reinterpret_cast<int32_t *>(workspace);
+    args.X = X;
+    args.X8w = const_cast<int8_t *>(X8);
+    args.s_xw = const_cast<uint16_t *>(s_x);
+    args.ws_ready = args.ws_cnt + kFusedReadyWord;
+    args.ws_done = args.ws_cnt + kFusedDoneWord;
     args.ws_part = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(workspace) + kCounterBytes);
     args.M = M;
     args.N = N;

@@ -36,12 +36,21 @@ bool gemm_shape_supported(int M, int N, int K);
 
 size_t gemm_workspace_bytes(int M, int N, int K);
 
+// Word offsets, in the workspace's counter region, of the two counters of
+// the fused call (after the split-tile counters of up to kMaxCtas CTAs).
+constexpr int kFusedReadyWord = 1000;
+constexpr int kFusedDoneWord = 1001;
+// Largest M for which the fused call quantizes inside the GEMM kernel.
+constexpr int kFusedMaxRows = kMaxCtas;
+
 // Returns cudaSuccess or the launch / tensor-map error.  `tmap_status`
 // receives the driver status of the tensor-map encode (0 on success).
+// With X non-null the kernel first quantizes X into X8 and s_x (the fused
+// call); otherwise it reads them.
 cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
                         const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
                         int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream,
-                        int *tmap_status);
+                        int *tmap_status, const uint16_t *X = nullptr);
 
 #ifdef QOQ_TRACE
 extern unsigned long long *g_trace_buffer;

@@ -14,26 +14,10 @@
 #include "qoq_internal.h"
 #include "qoq_layout.cuh"
 #include "qoq_ptx.cuh"
+#include "qoq_quant.cuh"
 
 namespace qoq {
 namespace {
-
-__device__ __forceinline__ float half_bits_to_float(uint16_t h)
-{
-    return __half2float(__ushort_as_half(h));
-}
-
-__device__ __forceinline__ uint16_t float_to_half_bits(float f)
-{
-    return __half_as_ushort(__float2half_rn(f));
-}
-
-__device__ __forceinline__ float warp_max(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
 
 __device__ __forceinline__ int warp_min_i(int v)
 {
@@ -138,37 +122,6 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
 constexpr int kActThreads = 128;
 constexpr int kActCache = 4;   // 16-byte vectors per thread kept in registers (K <= 4096)
 
-__device__ __forceinline__ float absmax8(const uint4 &v)
-{
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        m = fmaxf(m, fabsf(half_bits_to_float((uint16_t)(w[i] & 0xFFFFu))));
-        m = fmaxf(m, fabsf(half_bits_to_float((uint16_t)(w[i] >> 16))));
-    }
-    return m;
-}
-
-__device__ __forceinline__ int quant_x(float x, float sx)
-{
-    if (sx == 0.0f) return 0;
-    return (int)fminf(fmaxf(rintf(__fdiv_rn(x, sx)), -128.0f), 127.0f);
-}
-
-__device__ __forceinline__ uint2 quant8(const uint4 &v, float sx)
-{
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[2] = {0, 0};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = (uint32_t)quant_x(half_bits_to_float((uint16_t)(w[i] & 0xFFFFu)), sx) & 0xFFu;
-        const uint32_t hi = (uint32_t)quant_x(half_bits_to_float((uint16_t)(w[i] >> 16)), sx) & 0xFFu;
-        o[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
-    }
-    return make_uint2(o[0], o[1]);
-}
-
 // One CTA per token row: read the row once (kept in registers up to
 // kActCache vectors per thread), reduce max|x|, then quantize.
 __global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16_t *__restrict__ X, int K,
@@ -209,7 +162,7 @@ __global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16
     }
     __syncthreads();
     amax = red[0];
-    const uint16_t sxh = float_to_half_bits(__fdiv_rn(amax, 127.0f));
+    const uint16_t sxh = token_scale_bits(amax);
     const float sx = half_bits_to_float(sxh);
     if (threadIdx.x == 0) s_x[m] = sxh;
 #pragma unroll
