@@ -284,6 +284,17 @@ QOQ_API int qoq_dequant_weights_i8(const uint8_t *Wp, const uint8_t *s_g, const 
  * identical either way. Returns QOQ_ERR_INVALID_ARG for other values. */
 QOQ_API int qoq_set_gemm_a_in_tmem(int enable);
 
+/* Selects whether 256-token tiles (M > 128) run on pairs of SMs when the
+ * weight tile is in TMEM and N is a multiple of 256:
+ *   1 (default): two CTAs of a cluster compute a 256-channel tile with one
+ *      M = 256 tensor-core instruction per K step (tcgen05 cta_group::2),
+ *      each holding half of the activation tile, which halves the
+ *      activation traffic per SM;
+ *   0: one CTA per 128-channel tile.
+ * The choice applies to later GEMM calls from every thread. Results are
+ * identical either way. Returns QOQ_ERR_INVALID_ARG for other values. */
+QOQ_API int qoq_set_gemm_cta_pairs(int enable);
+
 /* Synchronizes `stream`, then reads and clears the device error flag of
  * the current device.
  *   Returns QOQ_OK when no kernel reported a problem.

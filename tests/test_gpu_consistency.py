@@ -93,3 +93,33 @@ def test_all_outputs_repeated(M, K, N, G):
         assert torch.equal(Y.view(torch.int16), yref.view(torch.int16)), f"graph replay {run}: outputs differ"
     del g
     assert int(ws[:4096].view(torch.int32).abs().sum()) == 0
+
+
+PAIR_SHAPES = [(200, 1024, 512, 128), (513, 512, 256, 512), (1024, 4096, 4096, 128), (4096, 2048, 1024, 128)]
+
+
+@pytest.mark.parametrize("M,K,N,G", PAIR_SHAPES, ids=[f"M{m}_K{k}_N{n}_G{g}" for m, k, n, g in PAIR_SHAPES])
+def test_cta_pairs_match_single(M, K, N, G):
+    """256-token tiles on CTA pairs (2-SM MMA) give the same bits as on
+    single CTAs, and both equal the exact product."""
+    q.qoq_set_gemm_a_in_tmem(True)
+    dev = torch.device("cuda")
+    X = wl.make_activations(M, K, wl.LLAMA, seed=5300 + M)
+    W = wl.make_weights(N, K, wl.LLAMA, seed=5400 + M)
+    packed = q.qoq_pack_weights(W.to(dev), G)
+    X8, s_x = q.qoq_quant_act_per_token(X.to(dev))
+    ref = _ref_acc(X8, q.qoq_dequant_weights_i8(packed))
+    out = {}
+    try:
+        for pairs in (False, True):
+            q.qoq_set_gemm_cta_pairs(pairs)
+            for run in range(3):
+                acc = torch.full((M, N), -7, dtype=torch.int32, device=dev)
+                Y = q.qoq_w4a8_gemm(X8, s_x, packed, acc_dbg=acc)
+                torch.cuda.synchronize()
+                assert q.qoq_device_error() == q.QOQ_OK
+                assert torch.equal(acc, ref), f"pairs={pairs} run {run}: INT32 mismatch"
+            out[pairs] = Y
+    finally:
+        q.qoq_set_gemm_cta_pairs(True)
+    assert torch.equal(out[True].view(torch.int16), out[False].view(torch.int16))

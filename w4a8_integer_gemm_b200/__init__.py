@@ -51,6 +51,7 @@ SIGNATURES = {
     "qoq_w4a8_linear": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "qoq_dequant_weights_i8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "qoq_set_gemm_a_in_tmem": (_I, [_I]),
+    "qoq_set_gemm_cta_pairs": (_I, [_I]),
     "qoq_device_error": (_I, [_P]),
 }
 
@@ -119,6 +120,10 @@ def qoq_gemm_workspace_bytes(M: int, N: int, K: int, group_size: int) -> int:
 
 def qoq_set_gemm_a_in_tmem(enable: bool) -> None:
     _check("qoq_set_gemm_a_in_tmem", lib().qoq_set_gemm_a_in_tmem(1 if enable else 0))
+
+
+def qoq_set_gemm_cta_pairs(enable: bool) -> None:
+    _check("qoq_set_gemm_cta_pairs", lib().qoq_set_gemm_cta_pairs(1 if enable else 0))
 
 
 def qoq_device_error(stream=None) -> int:

@@ -115,6 +115,10 @@ struct GemmArgs {
     } while (0)
 #endif
 
+// Waits of a CTA pair on barriers that the other CTA completes: default
+// (CTA-scope) acquire, the pattern the tcgen05 fences pair with.
+constexpr bool kClusterScopeWaits = false;
+
 // Weight stages issued by the setup thread before the CTA-wide barrier.
 constexpr int kPrologueStages = 2;
 
@@ -133,10 +137,14 @@ __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
     return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
 }
 
-template <int BN, int KST, int SW, int SX, bool A_TMEM>
+// PAIR: a 2-CTA cluster computes a 256-channel x BN-token tile with one
+// M = 256 MMA per K step (tcgen05 cta_group::2): each CTA dequantizes its
+// own 128-channel panel into its TMEM and holds half of the X8 tile.
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false>
 struct GemmCfg {
     static constexpr int kChunks = KST / kBlockK;        // packed 8 KB chunks per K block
-    static constexpr int kXTile = BN * 128;              // one [BN][128 B] swizzled X8 tile
+    static constexpr int kXRows = PAIR ? BN / 2 : BN;    // token rows of X8 this CTA holds
+    static constexpr int kXTile = kXRows * 128;          // one [rows][128 B] swizzled X8 tile
     static constexpr int kXSlot = kChunks * kXTile;      // X8 tiles of one K block
     static constexpr int kATile = 128 * 128;             // one [128][128 B] swizzled A tile
     static constexpr int kABytes = A_TMEM ? 0 : kChunks * kATile;
@@ -270,11 +278,12 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *v)
     }
 }
 
-template <int BN, int KST, int SW, int SX, bool A_TMEM>
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR>
 __global__ void __launch_bounds__(gemm_threads(BN), 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs a)
 {
-    using C = GemmCfg<BN, KST, SW, SX, A_TMEM>;
+    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR>;
+    static_assert(!PAIR || (A_TMEM && BN == 256), "pairs: 256-token tiles, A in TMEM");
     constexpr int kCh = C::kChunks;
     constexpr int kDq = dequant_groups(BN);
     constexpr int kEpiWarp0 = 4 + 4 * kDq;  // first epilogue warp
@@ -306,12 +315,22 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     const int lane = threadIdx.x & 31;
     // Scheduling state, computed first: its reads of the kernel parameters
     // start filling the constant cache while the prologue below runs.
-    const int P = gridDim.x;
-    const int T = a.total;
+    // Stream-K schedules CTAs, or CTA pairs (PAIR: both CTAs of a cluster
+    // take the same range; `rank` picks the panel and the X8 half).
     const int cta = blockIdx.x;
-    const int i_begin = range_begin(cta, P, T);
-    const int i_end = range_begin(cta + 1, P, T);
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const int P = PAIR ? (int)gridDim.x / 2 : (int)gridDim.x;
+    const int sched = PAIR ? (cta >> 1) : cta;  // index among the scheduled units
+    const int T = a.total;
+    const int i_begin = range_begin(sched, P, T);
+    const int i_end = range_begin(sched + 1, P, T);
     const int ks = a.ks;
+    // the weight panel of tile t held by this CTA
+    auto panel_of = [&](int t) { return PAIR ? 2 * (t / a.m_tiles) + (int)rank : t / a.m_tiles; };
+    // the CTA of scheduled unit c that holds this CTA's panel
+    auto cta_index = [&](int c) { return PAIR ? 2 * c + (int)rank : c; };
+    // the MMA's barriers live in CTA 0 of a pair
+    auto leader = [&](uint32_t bar) { return PAIR ? mapa_shared(bar, 0) : bar; };
 
     // ring slots a producer has filled, and the phase parity of each slot's
     // latest fill (drained on the way out of an aborted CTA)
@@ -326,7 +345,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     auto issue_weights = [&](int u, int s, uint32_t ph) {
         const int t = u / ks;
         const int kb = u - t * ks;
-        const int n_tile = t / a.m_tiles;
+        const int n_tile = panel_of(t);
         const uint32_t st = sbase + C::kWOff + s * C::kWSlot;
         const uint32_t bytes = (uint32_t)(kCh * cstride);
         mbar_arrive_expect_tx(wfull_bar(s), bytes);
@@ -348,12 +367,14 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             mbar_init(wempty_bar(s), 4);     // 4 dequant warps
         }
         for (int s = 0; s < SX; ++s) {
-            mbar_init(afull_bar(s), 5);      // 4 dequant warps + the X8 producer
+            // 4 dequant warps (of each CTA of a pair) + the X8 producer (of
+            // CTA 0 of a pair, whose expected bytes cover both halves)
+            mbar_init(afull_bar(s), PAIR ? 9 : 5);
             mbar_init(xaempty_bar(s), 1);    // MMA commit
         }
         for (int b = 0; b < C::kAccBufs; ++b) {
             mbar_init(accfull_bar(b), 1);
-            mbar_init(accempty_bar(b), 4);   // 4 epilogue warps
+            mbar_init(accempty_bar(b), PAIR ? 8 : 4);   // 4 epilogue warps (of each CTA)
         }
         mbar_init(mmadone_bar, 1);
         *abort_flag = 0;
@@ -371,14 +392,27 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     grid_launch_dependents();
     if (warp == 0) {
         __syncwarp();
-        tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_addr(tmem_slot), C::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    // a pair: both CTAs' barriers are initialized before either arrives remotely
+    if constexpr (PAIR) cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t budget = a.timeout_ns;
+    // waits on barriers that a pair's other CTA may complete acquire at
+    // cluster scope
+    auto wait_x = [&](uint32_t bar, uint32_t parity) {
+        return kClusterScopeWaits && PAIR ? wait_bounded_cluster(bar, parity, abort_flag, budget)
+                                          : wait_bounded(bar, parity, abort_flag, budget);
+    };
     QOQ_MARK(1);
 
     if (warp == 0) {
@@ -416,15 +450,27 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 const int ks1 = min(ks, i_end - t * ks);
                 const int m_tile = t % a.m_tiles;
                 for (int kb = i - t * ks; kb < ks1; ++kb) {
-                    if (!wait_bounded(xaempty_bar(s), ph ^ 1u, abort_flag, budget)) {
+                    if (!wait_x(xaempty_bar(s), ph ^ 1u)) {
                         ok = false;
                         break;
                     }
                     const uint32_t st = sbase + s * C::kXSlot;
-                    mbar_arrive_expect_tx(afull_bar(s), C::kXSlot);
+                    if constexpr (PAIR) {
+                        // each CTA loads its half of the tile's tokens; the
+                        // bytes of both count on CTA 0's barrier
+                        if (rank == 0) mbar_arrive_expect_tx(afull_bar(s), 2 * C::kXSlot);
+                        const uint32_t fb = leader(afull_bar(s));
 #pragma unroll
-                    for (int c = 0; c < kCh; ++c)
-                        tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN, afull_bar(s));
+                        for (int c = 0; c < kCh; ++c)
+                            tma_load_2d_pair(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK,
+                                             m_tile * BN + (int)rank * C::kXRows, fb);
+                    } else {
+                        mbar_arrive_expect_tx(afull_bar(s), C::kXSlot);
+#pragma unroll
+                        for (int c = 0; c < kCh; ++c)
+                            tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN,
+                                        afull_bar(s));
+                    }
                     if (tj < 16) QOQ_MARK(32 + tj);
                     ++tj;
                     issued |= 1u << s;
@@ -439,8 +485,8 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         }
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer --
-        if (lane == 0) {
-            const uint32_t idesc = idesc_i8_m128(BN);
+        if (lane == 0 && (!PAIR || rank == 0)) {  // a pair's MMAs are issued by CTA 0
+            const uint32_t idesc = PAIR ? idesc_i8_m256(BN) : idesc_i8_m128(BN);
             int s = 0;
             uint32_t ph = 0;
             int ab = 0;          // accumulator of the current tile
@@ -450,11 +496,11 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 const int t = i / ks;
                 const int ks0 = i - t * ks;
                 const int ks1 = min(ks, i_end - t * ks);
-                if (!wait_bounded(accempty_bar(ab), accph ^ 1u, abort_flag, budget)) break;
+                if (!wait_x(accempty_bar(ab), accph ^ 1u)) break;
                 tc_fence_after();
                 const uint32_t dacc = tmem_base + (uint32_t)(ab * BN);
                 for (int kb = ks0; kb < ks1; ++kb) {
-                    if (!wait_bounded(afull_bar(s), ph, abort_flag, budget)) {
+                    if (!wait_x(afull_bar(s), ph)) {
                         ok = false;
                         break;
                     }
@@ -465,7 +511,9 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     for (int j = 0; j < 4 * kCh; ++j) {
                         const uint32_t acc = (kb > ks0 || j > 0) ? 1u : 0u;
                         const uint64_t bdesc = smem_desc_sw128(st + (j >> 2) * C::kXTile) + 2 * (j & 3);
-                        if constexpr (A_TMEM) {
+                        if constexpr (PAIR) {
+                            mma_i8_ts_pair(dacc, tmem_base + C::kACol0 + s * C::kACols + j * 8, bdesc, idesc, acc);
+                        } else if constexpr (A_TMEM) {
                             mma_i8_ts(dacc, tmem_base + C::kACol0 + s * C::kACols + j * 8, bdesc, idesc, acc);
                         } else {
                             const uint64_t adesc =
@@ -473,7 +521,11 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                             mma_i8_ss(dacc, adesc, bdesc, idesc, acc);
                         }
                     }
-                    mma_commit(xaempty_bar(s));
+                    if constexpr (PAIR) {
+                        mma_commit_pair(xaempty_bar(s), 0x3);
+                    } else {
+                        mma_commit(xaempty_bar(s));
+                    }
                     if (tj < 16) QOQ_MARK(128 + tj);
                     ++tj;
                     if (++s == SX) {
@@ -482,7 +534,11 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     }
                 }
                 if (!ok) break;
-                mma_commit(accfull_bar(ab));
+                if constexpr (PAIR) {
+                    mma_commit_pair(accfull_bar(ab), 0x3);
+                } else {
+                    mma_commit(accfull_bar(ab));
+                }
                 if (++ab == C::kAccBufs) {
                     ab = 0;
                     accph ^= 1u;
@@ -491,7 +547,11 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             }
             QOQ_MARK(3);
             // all MMAs this thread issued have completed once this arrives
-            mma_commit(mmadone_bar);
+            if constexpr (PAIR) {
+                mma_commit_pair(mmadone_bar, 0x1);
+            } else {
+                mma_commit(mmadone_bar);
+            }
             drain_wait(mmadone_bar, 0, 200000000ull);
         }
     } else if (warp >= 4 && warp < kEpiWarp0) {
@@ -508,7 +568,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         uint32_t pc_sg = 0, pc_zs = 0, nx_sg = 0, nx_zs = 0;
         int t_cur = -1, t_nx = -1;
         auto load_tab = [&](int t, uint32_t &sgv, uint32_t &zsv) {
-            const size_t o = (size_t)(t / a.m_tiles) * kPanelRows + r;
+            const size_t o = (size_t)panel_of(t) * kPanelRows + r;
             sgv = __ldg(a.s_g + o);
             zsv = __ldg(a.zs + o);
         };
@@ -561,7 +621,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 // A slot sx is free once the MMAs of its previous use have
                 // completed; the X8 tiles need not have landed (the MMA
                 // issuer waits for those on afull)
-                if (!wait_bounded(xaempty_bar(sx), px ^ 1u, abort_flag, budget)) break;
+                if (!wait_x(xaempty_bar(sx), px ^ 1u)) break;
                 tc_fence_after();
                 if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(80 + tj);
 #pragma unroll
@@ -589,7 +649,13 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(afull_bar(sx));
+                if (lane == 0) {
+                    if constexpr (PAIR) {
+                        mbar_arrive_cluster(leader(afull_bar(sx)));
+                    } else {
+                        mbar_arrive(afull_bar(sx));
+                    }
+                }
                 if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(96 + tj);
                 ++tj;
             }
@@ -620,7 +686,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             float *rowmax = reinterpret_cast<float *>(smem + C::kStgOff);  // [4], in warp 0's staging block
             const int nvec = a.K / 8;
             constexpr int kCache = 4;  // 16-byte vectors per thread held across the two passes (K <= 4096)
-            for (int row = cta; row < a.M; row += P) {
+            for (int row = cta; row < a.M; row += (int)gridDim.x) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(a.X + (size_t)row * a.K);
                 uint4 cache[kCache];
                 float amax = 0.0f;
@@ -673,7 +739,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             const int ks0 = i - t * ks;
             const int ks1 = min(ks, i_end - t * ks);
             const int m_tile = t % a.m_tiles;
-            const int n_tile = t / a.m_tiles;
+            const int n_tile = panel_of(t);
             const int n = n_tile * kPanelRows + r;
             const int m0 = m_tile * BN;
             const int nchunks = (min(BN, a.M - m0) + 15) >> 4;  // 16-token chunks that exist
@@ -686,9 +752,11 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 sx_reg[q] = (q * 32 + lane < BN && m < a.M) ? half_bits_to_float(__ldcg(a.s_x + m)) : 0.0f;
             }
             const float sc = half_bits_to_float(__ldg(a.s_c + n));
-            const int c_lo = partial ? cta_of(t * ks, P, T) : cta;
-            const bool finisher = partial && c_lo == cta;     // this CTA completes a split tile
-            const int c_hi = finisher ? cta_of(t * ks + ks - 1, P, T) : cta;
+            // (scheduled units: CTAs, or CTA pairs; cta_index maps one to
+            // the CTA that holds this CTA's panel)
+            const int c_lo = partial ? cta_of(t * ks, P, T) : sched;
+            const bool finisher = partial && c_lo == sched;   // this CTA completes a split tile
+            const int c_hi = finisher ? cta_of(t * ks + ks - 1, P, T) : sched;
             // A finisher's split tile is the last tile of its range, and the
             // other contributors published their parts at the start of
             // theirs: wait for the count and sum their partials now, while
@@ -704,7 +772,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 // stores (32 per contributor and quarter); every lane here
                 // acquires the count itself before it reads the partials.
                 int *counter = a.ws_cnt + cta * 4 + quarter;
-                const int want = 32 * (c_hi - cta);
+                const int want = 32 * (c_hi - sched);
                 if (ld_acquire_gpu(counter) < want) {
                     const uint64_t start = global_timer_ns();
                     while (ld_acquire_gpu(counter) < want) {
@@ -724,8 +792,9 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     for (int q = 0; q < BN; ++q) pre[q] = 0;
                     if (ready) {
 #pragma unroll 1
-                        for (int c2 = cta + 1; c2 <= c_hi; ++c2) {
-                            const int4 *src = reinterpret_cast<const int4 *>(a.ws_part + (size_t)c2 * BN * kPanelRows);
+                        for (int c2 = sched + 1; c2 <= c_hi; ++c2) {
+                            const int4 *src =
+                                reinterpret_cast<const int4 *>(a.ws_part + (size_t)cta_index(c2) * BN * kPanelRows);
                             int4 ld[BN / 4];
 #pragma unroll
                             for (int cc = 0; cc < BN / 16; ++cc)
@@ -744,7 +813,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     }
                 }
             }
-            if (!wait_bounded(accfull_bar(ab), accph, abort_flag, budget)) break;
+            if (!wait_x(accfull_bar(ab), accph)) break;
             if (warp == kEpiWarp0 && lane == 0 && tj < 8) QOQ_MARK(208 + tj);
             tc_fence_after();
             const uint32_t tacc = trow + (uint32_t)(ab * BN);
@@ -754,7 +823,13 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             auto release_acc = [&]() {
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(accempty_bar(ab));
+                if (lane == 0) {
+                    if constexpr (PAIR) {
+                        mbar_arrive_cluster(leader(accempty_bar(ab)));
+                    } else {
+                        mbar_arrive(accempty_bar(ab));
+                    }
+                }
                 released = true;
             };
             if (partial && !finisher) {
@@ -778,7 +853,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 }
                 if (!released) release_acc();
                 // each lane's release covers its own partial stores
-                red_release_gpu_add(a.ws_cnt + c_lo * 4 + quarter, 1);
+                red_release_gpu_add(a.ws_cnt + cta_index(c_lo) * 4 + quarter, 1);
             } else {
                 // a whole tile, or a split tile this CTA finishes
                 if (ready) {
@@ -792,9 +867,9 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                             // the later contributors' partials of this group
                             // of chunks, all loads of a contributor in flight
 #pragma unroll 1
-                            for (int c2 = cta + 1; c2 <= c_hi; ++c2) {
-                                const int4 *src =
-                                    reinterpret_cast<const int4 *>(a.ws_part + (size_t)c2 * BN * kPanelRows);
+                            for (int c2 = sched + 1; c2 <= c_hi; ++c2) {
+                                const int4 *src = reinterpret_cast<const int4 *>(
+                                    a.ws_part + (size_t)cta_index(c2) * BN * kPanelRows);
                                 int4 ld[kGrp / 4];
 #pragma unroll
                                 for (int u = 0; u < kGrp / 16; ++u)
@@ -859,12 +934,15 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     __syncwarp();
     tc_fence_before();
     __syncthreads();
+    // a pair: CTA 0's MMAs write both CTAs' TMEM and the CTAs arrive on
+    // each other's barriers; neither leaves before both are done
+    if constexpr (PAIR) cluster_sync_all();
     tc_fence_after();
     QOQ_MARK(2);
     if (a.X && threadIdx.x == 0) {
         // every CTA is past its waits on ws_ready: the last one to get here
         // leaves both counters at zero for the next call
-        if (atomicAdd(a.ws_done, 1) == P - 1) {
+        if (atomicAdd(a.ws_done, 1) == (int)gridDim.x - 1) {
             *a.ws_ready = 0;
             *a.ws_done = 0;
         }
@@ -889,7 +967,11 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     }
     if (warp == 0) {
         __syncwarp();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+        if constexpr (PAIR) {
+            tmem_dealloc_pair(tmem_base, C::kTmemCols);
+        } else {
+            tmem_dealloc(tmem_base, C::kTmemCols);
+        }
     }
 }
 
@@ -930,11 +1012,11 @@ EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-template <int BN, int KST, int SW, int SX, bool A_TMEM>
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false>
 cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, KST, SW, SX, A_TMEM>;
-    auto kern = w4a8_gemm_kernel<BN, KST, SW, SX, A_TMEM>;
+    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR>;
+    auto kern = w4a8_gemm_kernel<BN, KST, SW, SX, A_TMEM, PAIR>;
     // the shared-memory opt-in is per device and per kernel: set it once
     static std::atomic<unsigned long long> opted_in{0};
     int dev = 0;
@@ -955,11 +1037,19 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     cfg.blockDim = dim3(gemm_threads(BN));
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if constexpr (PAIR) {
+        // CTA pairs: clusters of two consecutive CTAs
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = 2;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
     e = cudaLaunchKernelEx(&cfg, kern, tmap, args);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
@@ -970,8 +1060,17 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
 // allows (A in shared memory); the weight ring fills the rest of the
 // ~227 KB of shared memory, since it is what streams from HBM.
 template <bool A_TMEM>
-cudaError_t dispatch(int BN, int KST, const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
+cudaError_t dispatch(int BN, int KST, bool pair, const CUtensorMap &tmap, const GemmArgs &args, int grid,
+                     cudaStream_t stream)
 {
+    if constexpr (A_TMEM) {
+        // 256-token tiles on CTA pairs: half the X8 tile per CTA, so a ring
+        // of 8 stages fits beside 10 weight stages
+        if (pair) {
+            if (KST == 256) return launch_cfg<256, 256, 5, 4, true, true>(tmap, args, grid, stream);
+            return launch_cfg<256, 128, 10, 8, true, true>(tmap, args, grid, stream);
+        }
+    }
     if (KST == 256) {
         switch (BN) {
         case 16: return launch_cfg<16, 256, A_TMEM ? 11 : 6, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
@@ -987,6 +1086,8 @@ cudaError_t dispatch(int BN, int KST, const CUtensorMap &tmap, const GemmArgs &a
     default: return launch_cfg<256, 128, A_TMEM ? 6 : 8, A_TMEM ? 5 : 3, A_TMEM>(tmap, args, grid, stream);
     }
 }
+
+std::atomic<int> g_cta_pairs{1};
 
 // SMs of the current device, looked up once per device.
 int sm_count()
@@ -1018,6 +1119,11 @@ long long gemm_units(int M, int N, int K)
 
 }  // namespace
 
+void set_cta_pairs(bool enable)
+{
+    g_cta_pairs.store(enable ? 1 : 0);
+}
+
 int gemm_block_n(int M)
 {
     return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
@@ -1042,7 +1148,11 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
 {
     *tmap_status = 0;
     const int BN = gemm_block_n(M);
-    const int KST = gemm_stage_k(M, K);
+    // 256-token tiles run on CTA pairs (one M = 256 MMA over two weight
+    // panels, each CTA holding half of the X8 tile) when N allows it, with
+    // 256-wide K stages where K allows them
+    const bool pair = a_in_tmem && g_cta_pairs.load(std::memory_order_relaxed) && BN == 256 && N % 256 == 0;
+    const int KST = (pair && K % 256 == 0) ? 256 : gemm_stage_k(M, K);
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) {
         *tmap_status = -1;
@@ -1051,7 +1161,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     CUtensorMap tmap;
     const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t gstride[1] = {(cuuint64_t)K};
-    const cuuint32_t box[2] = {(cuuint32_t)kBlockK, (cuuint32_t)BN};
+    const cuuint32_t box[2] = {(cuuint32_t)kBlockK, (cuuint32_t)(pair ? BN / 2 : BN)};
     const cuuint32_t estride[2] = {1, 1};
     CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(X8), gdim, gstride, box, estride,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1061,8 +1171,10 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
         return cudaErrorInvalidValue;
     }
     const int sms = sm_count();
-    const long long units = gemm_units(M, N, K);
-    const long long grid = std::min<long long>(std::min(kMaxCtas, sms), units);
+    // stream-K units: (tile, K block) per CTA, or per CTA pair
+    const long long units = pair ? (long long)((M + BN - 1) / BN) * (N / 256) * (K / KST) : gemm_units(M, N, K);
+    const long long grid = pair ? 2 * std::min<long long>(std::min(kMaxCtas, sms) / 2, units)
+                                : std::min<long long>(std::min(kMaxCtas, sms), units);
 
     GemmArgs args;
     args.Wp = Wp;
@@ -1091,8 +1203,8 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
 #ifdef QOQ_TRACE
     args.trace = g_trace_buffer;
 #endif
-    return a_in_tmem ? dispatch<true>(BN, KST, tmap, args, (int)grid, stream)
-                     : dispatch<false>(BN, KST, tmap, args, (int)grid, stream);
+    return a_in_tmem ? dispatch<true>(BN, KST, pair, tmap, args, (int)grid, stream)
+                     : dispatch<false>(BN, KST, false, tmap, args, (int)grid, stream);
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value)

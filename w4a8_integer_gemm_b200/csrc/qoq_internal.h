@@ -36,6 +36,9 @@ bool gemm_shape_supported(int M, int N, int K);
 
 size_t gemm_workspace_bytes(int M, int N, int K);
 
+// Whether 256-token tiles run on CTA pairs (2-SM MMA); default on.
+void set_cta_pairs(bool enable);
+
 // Word offsets, in the workspace's counter region, of the two counters of
 // the fused call (after the split-tile counters of up to kMaxCtas CTAs).
 constexpr int kFusedReadyWord = 1000;
