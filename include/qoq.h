@@ -162,7 +162,7 @@ QOQ_API int qoq_quant_act_per_token(const uint16_t *X, int M, int K,
  * The GEMM splits the K loop of some output tiles across SMs so that every
  * SM streams the same number of weight bytes. The INT32 partial sums of a
  * split tile meet in this workspace. The sum is exact in any order.
- * Layout: the first 4096 bytes hold arrival counters (the same region for
+ * Layout: the first 8192 bytes hold arrival counters (the same region for
  * every shape); the partial tiles follow. Rules:
  *   - a fresh workspace must be zero-filled once before its first use;
  *   - every completed call leaves the counters at zero again, so one

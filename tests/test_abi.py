@@ -55,13 +55,13 @@ def test_size_queries(L):
     assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 128) > 0
     assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 64) == 0      # group size not supported
     assert q.qoq_gemm_workspace_bytes(0, 512, 512, 128) == 0
-    # 4096 bytes of counters, then for each of <= 148 CTAs one partial tile
+    # 8192 bytes of counters, then for each of <= 148 CTAs one partial tile
     # of BN=16 tokens x 128 channels x int32
-    assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 128) == 4096 + 148 * 16 * 128 * 4
+    assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 128) == 8192 + 148 * 16 * 128 * 4
     # grid = units when there are fewer units than SMs (4 tiles x 2 K blocks of 256)
-    assert q.qoq_gemm_workspace_bytes(1, 512, 512, 128) == 4096 + 8 * 16 * 128 * 4
+    assert q.qoq_gemm_workspace_bytes(1, 512, 512, 128) == 8192 + 8 * 16 * 128 * 4
     # 256-token tiles use 128-wide K blocks: 4 m-tiles x 64 n-tiles x 64 blocks -> 148 CTAs
-    assert q.qoq_gemm_workspace_bytes(1024, 8192, 8192, 128) == 4096 + 148 * 256 * 128 * 4
+    assert q.qoq_gemm_workspace_bytes(1024, 8192, 8192, 128) == 8192 + 148 * 256 * 128 * 4
 
 
 def _fake(addr):

@@ -50,7 +50,7 @@ def test_fused_equals_separate(M, K, N, G):
         assert torch.equal(X8, X8r), f"run {run}: X8 differs"
         assert torch.equal(sx[:M], sxr[:M]), f"run {run}: s_x differs"
         assert torch.equal(Y.view(torch.int16), Yr.view(torch.int16)), f"run {run}: Y differs"
-        assert int(ws[:4096].view(torch.int32).abs().sum()) == 0
+        assert int(ws[:8192].view(torch.int32).abs().sum()) == 0
 
     main = torch.cuda.current_stream()
     cap = torch.cuda.Stream()

@@ -63,7 +63,7 @@ def test_graph_replay_matches_eager(M, K, N, G):
             assert torch.equal(b[2].view(torch.int16), e.view(torch.int16)), f"replay {rep} differs"
         # the counters at the head of each workspace are back at zero
         for b in bufs:
-            assert int(b[3][:4096].view(torch.int32).abs().sum()) == 0
+            assert int(b[3][:8192].view(torch.int32).abs().sum()) == 0
     del g
 
     rng = np.random.default_rng(M)

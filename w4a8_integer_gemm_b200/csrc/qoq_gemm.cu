@@ -130,7 +130,14 @@ constexpr int kPrologueStages = 2;
 // arithmetic.  Wider tiles keep one group (384 threads, 168 registers) for
 // their larger epilogue.
 __host__ __device__ constexpr int dequant_groups(int BN) { return BN <= 64 ? 2 : 1; }
-__host__ __device__ constexpr int gemm_threads(int BN) { return 128 * (2 + dequant_groups(BN)); }
+// 256-token tiles drain their accumulator with two epilogue warpgroups (one
+// per 128 tokens): with one accumulator in TMEM the MMAs of the next tile
+// wait for the epilogue, so its length is lost tensor time.
+__host__ __device__ constexpr int epilogue_groups(int BN) { return BN == 256 ? 2 : 1; }
+__host__ __device__ constexpr int gemm_threads(int BN)
+{
+    return 128 * (1 + dequant_groups(BN) + epilogue_groups(BN));
+}
 
 __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
 {
@@ -155,7 +162,7 @@ struct GemmCfg {
     static constexpr int kAOff = SX * kXSlot;
     static constexpr int kWOff = kAOff + SX * kABytes;
     static constexpr int kStgOff = kWOff + SW * kWSlot;  // per epilogue warp: 16 tokens x 32 channels FP16
-    static constexpr int kBarOff = kStgOff + 4 * 1024;
+    static constexpr int kBarOff = kStgOff + 4 * 1024 * epilogue_groups(BN);
     static constexpr uint32_t kACols = KST / 4;          // TMEM columns of one A slot
     // two accumulators (the MMAs of the next tile run while the epilogue
     // drains the last one) wherever TMEM has room for them
@@ -287,6 +294,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     constexpr int kCh = C::kChunks;
     constexpr int kDq = dequant_groups(BN);
     constexpr int kEpiWarp0 = 4 + 4 * kDq;  // first epilogue warp
+    constexpr int kEpi = epilogue_groups(BN);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
@@ -374,7 +382,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         }
         for (int b = 0; b < C::kAccBufs; ++b) {
             mbar_init(accfull_bar(b), 1);
-            mbar_init(accempty_bar(b), PAIR ? 8 : 4);   // 4 epilogue warps (of each CTA)
+            mbar_init(accempty_bar(b), 4 * kEpi * (PAIR ? 2 : 1));   // the epilogue warps (of each CTA)
         }
         mbar_init(mmadone_bar, 1);
         *abort_flag = 0;
@@ -671,13 +679,14 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     } else if (warp >= kEpiWarp0) {
         // ----------------------------------------------------- epilogue --
         const int quarter = warp & 3;
+        const int eg = (warp - kEpiWarp0) >> 2;  // epilogue group: which 16-token chunks it drains
         const int r = quarter * 32 + lane;
         const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
-        uint8_t *stg = smem + C::kStgOff + quarter * 1024;  // this warp's output staging block
+        uint8_t *stg = smem + C::kStgOff + (eg * 4 + quarter) * 1024;  // this warp's output staging block
         int ab = 0;          // accumulator of the current tile
         uint32_t accph = 0;  // its phase parity
         grid_dependency_wait();  // s_x (or X) comes from the preceding kernel
-        if (a.X) {
+        if (a.X && eg == 0) {
             // Fused call: the four epilogue warps of each CTA quantize token
             // rows cta, cta + P, ... together (128 threads per row, the
             // loads of a row in flight at once), then every lane waits until
@@ -686,7 +695,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             float *rowmax = reinterpret_cast<float *>(smem + C::kStgOff);  // [4], in warp 0's staging block
             const int nvec = a.K / 8;
             constexpr int kCache = 4;  // 16-byte vectors per thread held across the two passes (K <= 4096)
-            for (int row = cta; row < a.M; row += (int)gridDim.x) {
+            for (int row = cta; row < a.M; row += (int)gridDim.x) {  // (epilogue group 0)
                 const uint4 *src = reinterpret_cast<const uint4 *>(a.X + (size_t)row * a.K);
                 uint4 cache[kCache];
                 float amax = 0.0f;
@@ -731,6 +740,8 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 fence_proxy_async_global();
                 red_release_gpu_add(a.ws_ready, 1);
             }
+        }
+        if (a.X) {
             // 128 counts per row; on a timeout the flag stops every role
             wait_count_gpu(a.ws_ready, 128 * a.M, abort_flag, budget);
         }
@@ -743,6 +754,9 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             const int n = n_tile * kPanelRows + r;
             const int m0 = m_tile * BN;
             const int nchunks = (min(BN, a.M - m0) + 15) >> 4;  // 16-token chunks that exist
+            // this epilogue group's chunks
+            const int ch_lo = eg * (BN / 16 / kEpi);
+            const int ch_hi = min(nchunks, ch_lo + BN / 16 / kEpi);
             const bool partial = !(ks0 == 0 && ks1 == ks);
             // token scales of this tile, one per lane per 32 tokens
             float sx_reg[C::kSx];
@@ -765,13 +779,13 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             constexpr bool kPresum = (BN <= 64);
             // accumulator columns per TMEM load (16 where the pre-summed
             // partials of a 64-wide tile already hold 64 registers)
-            constexpr int kGrp = BN < 64 ? BN : (kPresum ? 16 : 64);
+            constexpr int kGrp = BN < 64 ? BN : (kPresum ? 16 : (kEpi == 2 ? 32 : 64));
             int32_t pre[kPresum ? BN : 1];
             if (finisher) {
                 // Every lane of every later contributor counts its own
                 // stores (32 per contributor and quarter); every lane here
                 // acquires the count itself before it reads the partials.
-                int *counter = a.ws_cnt + cta * 4 + quarter;
+                int *counter = a.ws_cnt + (cta * kEpi + eg) * 4 + quarter;
                 const int want = 32 * (c_hi - sched);
                 if (ld_acquire_gpu(counter) < want) {
                     const uint64_t start = global_timer_ns();
@@ -836,13 +850,13 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 // a later contributor: publish the partial, count it, done
                 int4 *my_part = reinterpret_cast<int4 *>(a.ws_part + (size_t)cta * BN * kPanelRows);
 #pragma unroll 1
-                for (int g0 = 0; g0 < nchunks; g0 += kGrp / 16) {
+                for (int g0 = ch_lo; g0 < ch_hi; g0 += kGrp / 16) {
                     uint32_t v[kGrp];
                     tmem_load_cols<kGrp>(tacc + g0 * 16, v);
-                    if (g0 + kGrp / 16 >= nchunks) release_acc();
+                    if (g0 + kGrp / 16 >= ch_hi) release_acc();
 #pragma unroll
                     for (int u = 0; u < kGrp / 16; ++u) {
-                        if (g0 + u < nchunks) {
+                        if (g0 + u < ch_hi) {
                             int4 *dst = my_part + ((size_t)(g0 + u) * kPanelRows + r) * 4;
 #pragma unroll
                             for (int j = 0; j < 4; ++j)
@@ -853,15 +867,15 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 }
                 if (!released) release_acc();
                 // each lane's release covers its own partial stores
-                red_release_gpu_add(a.ws_cnt + cta_index(c_lo) * 4 + quarter, 1);
+                red_release_gpu_add(a.ws_cnt + (cta_index(c_lo) * kEpi + eg) * 4 + quarter, 1);
             } else {
                 // a whole tile, or a split tile this CTA finishes
                 if (ready) {
 #pragma unroll 1
-                    for (int g0 = 0; g0 < nchunks; g0 += kGrp / 16) {
+                    for (int g0 = ch_lo; g0 < ch_hi; g0 += kGrp / 16) {
                     uint32_t vg[kGrp];
                     tmem_load_cols<kGrp>(tacc + g0 * 16, vg);
-                    if (g0 + kGrp / 16 >= nchunks) release_acc();
+                    if (g0 + kGrp / 16 >= ch_hi) release_acc();
                     if constexpr (!kPresum) {
                         if (finisher) {
                             // the later contributors' partials of this group
@@ -875,7 +889,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                                 for (int u = 0; u < kGrp / 16; ++u)
 #pragma unroll
                                     for (int j = 0; j < 4; ++j)
-                                        ld[u * 4 + j] = (g0 + u < nchunks)
+                                        ld[u * 4 + j] = (g0 + u < ch_hi)
                                                             ? __ldcg(src + ((size_t)(g0 + u) * kPanelRows + r) * 4 + j)
                                                             : make_int4(0, 0, 0, 0);
 #pragma unroll
@@ -892,7 +906,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
 #pragma unroll
                     for (int u = 0; u < kGrp / 16; ++u) {
                         const int cc = g0 + u;
-                        if (cc >= nchunks) break;
+                        if (cc >= ch_hi) break;
                         if (warp == kEpiWarp0 && lane == 0 && tj < 2 && cc < 6) QOQ_MARK(233 + tj * 8 + cc);
                         int32_t acc[16];
 #pragma unroll

@@ -15,8 +15,9 @@ constexpr int kMaxCtas = 148;
 
 // The split-tile counters (kMaxCtas x 4 int32) occupy this many bytes at the
 // start of every GEMM workspace; the INT32 partial tiles follow.
-constexpr size_t kCounterBytes = 4096;
-static_assert(kMaxCtas * 4 * 4 <= kCounterBytes, "counter region");
+constexpr size_t kCounterBytes = 8192;
+// split-tile counters: kMaxCtas CTAs x 2 epilogue groups x 4 quarters
+static_assert(kMaxCtas * 2 * 4 * 4 <= kCounterBytes - 64, "counter region");
 
 cudaError_t launch_pack(const float *W, int N, int K, int G, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g,
                         uint8_t *zs, cudaStream_t stream);
@@ -41,8 +42,8 @@ void set_cta_pairs(bool enable);
 
 // Word offsets, in the workspace's counter region, of the two counters of
 // the fused call (after the split-tile counters of up to kMaxCtas CTAs).
-constexpr int kFusedReadyWord = 1000;
-constexpr int kFusedDoneWord = 1001;
+constexpr int kFusedReadyWord = 2000;
+constexpr int kFusedDoneWord = 2001;
 // Largest M for which the fused call quantizes inside the GEMM kernel.
 constexpr int kFusedMaxRows = kMaxCtas;
 
