@@ -295,6 +295,16 @@ QOQ_API int qoq_set_gemm_a_in_tmem(int enable);
  * identical either way. Returns QOQ_ERR_INVALID_ARG for other values. */
 QOQ_API int qoq_set_gemm_cta_pairs(int enable);
 
+/* Self-test of the failure path (the pages have no counterpart). Launches
+ * one thread that waits on a barrier phase nothing completes, with the same
+ * bounded wait every GEMM role uses and a budget of timeout_ns (1 us ..
+ * 100 ms) instead of the GEMM's 2 s. When the budget runs out the kernel
+ * raises the device error flag and returns normally: nothing traps, and the
+ * context stays usable. A following qoq_device_error therefore reports
+ * QOQ_ERR_TIMEOUT (and clears the flag). Returns QOQ_ERR_INVALID_ARG for a
+ * budget outside the range. */
+QOQ_API int qoq_selftest_wait_timeout(unsigned long long timeout_ns, void *stream);
+
 /* Synchronizes `stream`, then reads and clears the device error flag of
  * the current device.
  *   Returns QOQ_OK when no kernel reported a problem.

@@ -177,6 +177,14 @@ int qoq_set_gemm_a_in_tmem(int enable)
     return QOQ_OK;
 }
 
+int qoq_selftest_wait_timeout(unsigned long long timeout_ns, void *stream)
+{
+    if (timeout_ns < 1000ull || timeout_ns > 100000000ull) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(qoq::launch_stuck_wait(timeout_ns, (cudaStream_t)stream));
+}
+
 int qoq_set_gemm_cta_pairs(int enable)
 {
     if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;

@@ -989,6 +989,24 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     }
 }
 
+// Self-test of the failure path: one thread waits, bounded, on an mbarrier
+// phase that nothing completes, exactly as the GEMM's roles wait; when the
+// budget runs out it raises the device error flag and returns.
+__global__ void stuck_wait_kernel(unsigned long long budget_ns)
+{
+    __shared__ __align__(8) unsigned long long bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (!wait_bounded(smem_addr(&bar), 0u, &abort_flag, budget_ns)) atomicExch(&g_dev_error, 1);
+    }
+}
+
 // ----------------------------------------------------------------- host --
 #ifdef QOQ_TRACE
 unsigned long long *g_trace_buffer = nullptr;
@@ -1132,6 +1150,12 @@ long long gemm_units(int M, int N, int K)
 }
 
 }  // namespace
+
+cudaError_t launch_stuck_wait(unsigned long long budget_ns, cudaStream_t stream)
+{
+    stuck_wait_kernel<<<1, 32, 0, stream>>>(budget_ns);
+    return cudaGetLastError();
+}
 
 void set_cta_pairs(bool enable)
 {

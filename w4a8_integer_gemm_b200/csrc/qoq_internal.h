@@ -37,6 +37,9 @@ bool gemm_shape_supported(int M, int N, int K);
 
 size_t gemm_workspace_bytes(int M, int N, int K);
 
+// One bounded wait that nothing completes (the failure-path self-test).
+cudaError_t launch_stuck_wait(unsigned long long budget_ns, cudaStream_t stream);
+
 // Whether 256-token tiles run on CTA pairs (2-SM MMA); default on.
 void set_cta_pairs(bool enable);
 
