@@ -29,31 +29,37 @@
 //     full count, add the partials to their accumulators and run the
 //     epilogue.  No contributor waits for anything while it still has work,
 //     so the waits cannot form a cycle.
-//   * Warp roles (352 threads):
-//       warp 0      weight producer: per stage one bulk copy of the packed
-//                   weight chunks.
+//   * Warpgroups (384 or 512 threads):
+//       warp 0      weight producer: per stage one bulk copy of the stage's
+//                   packed chunks with their group tables; also TMEM.
 //       warp 1      MMA issuer (one thread): one barrier wait, KST/32
 //                   tcgen05.mma (K = 32) and one tcgen05.commit per stage.
-//       warps 2-5   dequant: thread r owns output channel r of the panel,
-//                   reads its packed bytes with 128-bit shared loads,
-//                   expands them to INT8 in registers, and stores them as
-//                   the MMA's A operand -- into TMEM with tcgen05.st
-//                   (default), or into shared memory in the 128-byte-
-//                   swizzled K-major layout.
-//       warps 6-9   epilogue: tcgen05.ld of the INT32 accumulators, FP32
-//                   scaling, FP16 stores; split tiles as above.
-//       warp 10     X8 producer: tiled TMA loads of the activation tiles
-//                   and bulk copies of the group tables.  It alone waits for
-//                   the preceding kernel (programmatic dependent launch), so
-//                   weights stream in while the activation quantizer runs.
+//       warp 2      X8 producer: tiled TMA loads of the activation tiles.
+//                   It and the epilogue alone wait for the preceding kernel
+//                   (programmatic dependent launch), so weights stream in
+//                   and are dequantized while that kernel still runs.
+//       dequant     one or two groups of four warps (two for tiles up to 64
+//                   tokens, taking alternate stages): thread r owns output
+//                   channel r of the panel, reads its packed bytes with
+//                   128-bit shared loads, expands them to INT8 in registers
+//                   and stores them as the MMA's A operand -- into TMEM
+//                   with tcgen05.st (default), or into shared memory in the
+//                   128-byte-swizzled K-major layout.
+//       epilogue    one or two groups of four warps (two for 256-token
+//                   tiles, one per 128 tokens): tcgen05.ld of the INT32
+//                   accumulators, FP32 scaling, FP16 stores; split tiles as
+//                   above.  In the fused call they first quantize the rows.
 //   * Rings: a weight ring (packed chunks and tables of a K block, freed
 //     as soon as the dequant warps hold them in registers); an X8/A ring
 //     (slot s holds the X8 tiles of a K block in shared memory and its
-//     dequantized weights in A slot s, TMEM or shared memory; the X8
-//     producer refills slot s only after the MMAs reading it completed, so
-//     a landed X8 slot also means a free A slot); and one or two TMEM
-//     accumulators, so the MMAs of the next tile need not wait for the
-//     epilogue of the last one.
+//     dequantized weights in A slot s; one barrier says both are ready, one
+//     commit frees both); and one or two TMEM accumulators, so the MMAs of
+//     the next tile need not wait for the epilogue of the last one.
+//   * CTA pairs (256-token tiles): a cluster of two CTAs computes a
+//     256-channel tile with one M = 256 MMA per K step (cta_group::2);
+//     each CTA dequantizes its own 128-channel panel into its TMEM and
+//     loads half of the X8 tile, CTA 0 issues the MMAs and multicasts the
+//     commits, and the other CTA's warps arrive on CTA 0's barriers.
 //   * Every wait is bounded (per wait, global timer); on expiry the CTA
 //     stops, drains its own in-flight copies and MMAs, frees TMEM, and
 //     raises the device error flag that qoq_device_error() reports.
@@ -114,10 +120,6 @@ struct GemmArgs {
     do {              \
     } while (0)
 #endif
-
-// Waits of a CTA pair on barriers that the other CTA completes: default
-// (CTA-scope) acquire, the pattern the tcgen05 fences pair with.
-constexpr bool kClusterScopeWaits = false;
 
 // Weight stages issued by the setup thread before the CTA-wide barrier.
 constexpr int kPrologueStages = 2;
@@ -415,12 +417,11 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t budget = a.timeout_ns;
-    // waits on barriers that a pair's other CTA may complete acquire at
-    // cluster scope
-    auto wait_x = [&](uint32_t bar, uint32_t parity) {
-        return kClusterScopeWaits && PAIR ? wait_bounded_cluster(bar, parity, abort_flag, budget)
-                                          : wait_bounded(bar, parity, abort_flag, budget);
-    };
+    // waits on the X8/A ring and the accumulators (in a pair, the phases
+    // may be completed by the other CTA's arrivals or the MMA's multicast
+    // commits; the tcgen05 fences around the waits order the tensor-memory
+    // accesses, as with one CTA)
+    auto wait_x = [&](uint32_t bar, uint32_t parity) { return wait_bounded(bar, parity, abort_flag, budget); };
     QOQ_MARK(1);
 
     if (warp == 0) {

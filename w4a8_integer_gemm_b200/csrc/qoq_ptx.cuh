@@ -95,36 +95,6 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
-// wait_bounded with acquire at cluster scope: for phases that the peer CTA
-// of a pair completes (its arrivals, or its MMA issuer's commits).
-__device__ __forceinline__ bool mbar_try_wait_cluster_sleep(uint32_t bar, uint32_t parity, uint32_t suspend_ns)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(suspend_ns)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile int *abort,
-                                                     uint64_t budget_ns)
-{
-    if (mbar_try_wait_cluster_sleep(bar, parity, 0u)) return true;
-    const uint64_t start = global_timer_ns();
-    for (;;) {
-        if (mbar_try_wait_cluster_sleep(bar, parity, 200000u)) return true;
-        if (*abort) return false;
-        if (global_timer_ns() - start > budget_ns) {
-            *abort = 1;
-            return false;
-        }
-    }
-}
-
 // Programmatic dependent launch: wait until the grids this one depends on
 // have completed and their writes are visible ...
 __device__ __forceinline__ void grid_dependency_wait()
@@ -157,34 +127,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
         : "memory");
-}
-
-// 2-D tiled tensor store shared -> global (bulk-group completion).  Rows and
-// columns of the box beyond the tensor's extent are not written.
-__device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, uint32_t src)
-{
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                     reinterpret_cast<uint64_t>(tmap)),
-                 "r"(x), "r"(y), "r"(src)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit_group()
-{
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until at most N committed bulk groups still read shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_group_read()
-{
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// Wait until every committed bulk group has completed its writes.
-__device__ __forceinline__ void bulk_wait_group_all()
-{
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Named barrier over `count` threads (ids other than 0, which __syncthreads uses).
@@ -298,21 +240,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// mbar_try_wait with acquire at cluster scope (the phase may have been
-// completed by the peer CTA's arrivals).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Both CTAs of the cluster: release, then wait (acquire) for the other.
 __device__ __forceinline__ void cluster_sync_all()
 {
@@ -370,11 +297,6 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask)
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
         "h"(cta_mask)
         : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_ld()
-{
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_st()
