@@ -295,6 +295,19 @@ QOQ_API int qoq_set_gemm_a_in_tmem(int enable);
  * identical either way. Returns QOQ_ERR_INVALID_ARG for other values. */
 QOQ_API int qoq_set_gemm_cta_pairs(int enable);
 
+/* Selects the token-tile width rule for M > 64:
+ *   1 (default): 256 tokens per tile (128 for M <= 128), narrowed to 128 and
+ *      then 64 while the tiles are so few that stream-K would share each
+ *      among four or more CTAs (two or more when K <= 4096); every extra
+ *      CTA on a tile adds one INT32 partial tile that the finishing CTA
+ *      reads back;
+ *   0: the tile covers min(M, 256) tokens rounded up to 128 or 256.
+ * qoq_gemm_workspace_bytes covers both rules, so a workspace stays valid
+ * when this changes. The choice applies to later GEMM calls from every
+ * thread. Results are identical either way. Returns QOQ_ERR_INVALID_ARG
+ * for other values. */
+QOQ_API int qoq_set_gemm_narrow_tiles(int enable);
+
 /* Self-test of the failure path (the pages have no counterpart). Launches
  * one thread that waits on a barrier phase nothing completes, with the same
  * bounded wait every GEMM role uses and a budget of timeout_ns (1 us ..

@@ -95,13 +95,14 @@ def test_all_outputs_repeated(M, K, N, G):
     assert int(ws[:8192].view(torch.int32).abs().sum()) == 0
 
 
-PAIR_SHAPES = [(200, 1024, 512, 128), (513, 512, 256, 512), (1024, 4096, 4096, 128), (4096, 2048, 1024, 128)]
+PAIR_SHAPES = [(200, 1024, 512, 128), (256, 4096, 4096, 128), (513, 512, 256, 512), (1024, 4096, 4096, 128), (4096, 2048, 1024, 128)]
 
 
 @pytest.mark.parametrize("M,K,N,G", PAIR_SHAPES, ids=[f"M{m}_K{k}_N{n}_G{g}" for m, k, n, g in PAIR_SHAPES])
 def test_cta_pairs_match_single(M, K, N, G):
     """256-token tiles on CTA pairs (2-SM MMA) give the same bits as on
-    single CTAs, and both equal the exact product."""
+    single CTAs, and as the narrower tiles the default rule picks for few
+    tiles; all equal the exact product."""
     q.qoq_set_gemm_a_in_tmem(True)
     dev = torch.device("cuda")
     X = wl.make_activations(M, K, wl.LLAMA, seed=5300 + M)
@@ -111,15 +112,18 @@ def test_cta_pairs_match_single(M, K, N, G):
     ref = _ref_acc(X8, q.qoq_dequant_weights_i8(packed))
     out = {}
     try:
-        for pairs in (False, True):
+        for narrow, pairs in ((False, False), (False, True), (True, True)):
+            q.qoq_set_gemm_narrow_tiles(narrow)
             q.qoq_set_gemm_cta_pairs(pairs)
             for run in range(3):
                 acc = torch.full((M, N), -7, dtype=torch.int32, device=dev)
                 Y = q.qoq_w4a8_gemm(X8, s_x, packed, acc_dbg=acc)
                 torch.cuda.synchronize()
                 assert q.qoq_device_error() == q.QOQ_OK
-                assert torch.equal(acc, ref), f"pairs={pairs} run {run}: INT32 mismatch"
-            out[pairs] = Y
+                assert torch.equal(acc, ref), f"narrow={narrow} pairs={pairs} run {run}: INT32 mismatch"
+            out[(narrow, pairs)] = Y
     finally:
         q.qoq_set_gemm_cta_pairs(True)
-    assert torch.equal(out[True].view(torch.int16), out[False].view(torch.int16))
+        q.qoq_set_gemm_narrow_tiles(True)
+    for k in out:
+        assert torch.equal(out[k].view(torch.int16), out[(False, False)].view(torch.int16)), k

@@ -120,12 +120,19 @@ GEMM_CASES = [
 ]
 
 
+@pytest.mark.parametrize("narrow", [True, False], ids=["narrow", "wide"])
 @pytest.mark.parametrize("a_in_tmem", [False, True], ids=["A_smem", "A_tmem"])
 @pytest.mark.parametrize("M,K,N,G", GEMM_CASES)
-def test_gemm_bit_exact(M, K, N, G, a_in_tmem):
+def test_gemm_bit_exact(M, K, N, G, a_in_tmem, narrow):
+    # narrow=False keeps the 128/256-token tiles that the default rule
+    # replaces with 64-token ones at these small N
     X = wl.make_activations(M, K, wl.LLAMA, seed=400 + M)
     W = wl.make_weights(N, K, wl.LLAMA, seed=500 + N + K)
-    _, X8, s_x, Y, acc = run_layer(X, W, G, a_in_tmem)
+    q.qoq_set_gemm_narrow_tiles(narrow)
+    try:
+        _, X8, s_x, Y, acc = run_layer(X, W, G, a_in_tmem)
+    finally:
+        q.qoq_set_gemm_narrow_tiles(True)
     r = oracle.linear(X.numpy(), W.numpy(), G)
     assert np.array_equal(acc.cpu().numpy(), r["acc"])
     assert_half_within_1ulp(_u16(Y), r["Y"])

@@ -52,6 +52,7 @@ SIGNATURES = {
     "qoq_dequant_weights_i8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "qoq_set_gemm_a_in_tmem": (_I, [_I]),
     "qoq_set_gemm_cta_pairs": (_I, [_I]),
+    "qoq_set_gemm_narrow_tiles": (_I, [_I]),
     "qoq_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "qoq_device_error": (_I, [_P]),
 }
@@ -125,6 +126,10 @@ def qoq_set_gemm_a_in_tmem(enable: bool) -> None:
 
 def qoq_set_gemm_cta_pairs(enable: bool) -> None:
     _check("qoq_set_gemm_cta_pairs", lib().qoq_set_gemm_cta_pairs(1 if enable else 0))
+
+
+def qoq_set_gemm_narrow_tiles(enable: bool) -> None:
+    _check("qoq_set_gemm_narrow_tiles", lib().qoq_set_gemm_narrow_tiles(1 if enable else 0))
 
 
 def qoq_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:

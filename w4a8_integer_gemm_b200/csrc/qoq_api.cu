@@ -192,6 +192,13 @@ int qoq_set_gemm_cta_pairs(int enable)
     return QOQ_OK;
 }
 
+int qoq_set_gemm_narrow_tiles(int enable)
+{
+    if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;
+    qoq::set_narrow_tiles(enable != 0);
+    return QOQ_OK;
+}
+
 #ifdef QOQ_TRACE
 // Trace builds only: a device buffer of [ctas][256] uint64 that later GEMM
 // launches fill with global-timer marks.

@@ -88,7 +88,7 @@ struct GemmArgs {
     uint16_t *Y;
     int32_t *acc_dbg;
     int32_t *ws_cnt;   // [kMaxCtas][4] arrival counters, at the start of the workspace
-    int32_t *ws_part;  // [cta][BN/16][128][16] INT32 partial tile, after the counters
+    int32_t *ws_part;  // [cta][BN/16][4][128][4] INT32 partial tile, after the counters
     // The fused call (X non-null): the kernel first quantizes the FP16 rows
     // of X into X8 / s_x itself, then reads them as in the plain GEMM.
     const uint16_t *X;
@@ -815,7 +815,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                             for (int cc = 0; cc < BN / 16; ++cc)
 #pragma unroll
                                 for (int j = 0; j < 4; ++j)
-                                    ld[cc * 4 + j] = (cc < nchunks) ? __ldcg(src + ((size_t)cc * kPanelRows + r) * 4 + j)
+                                    ld[cc * 4 + j] = (cc < nchunks) ? __ldcg(src + (size_t)(cc * 4 + j) * kPanelRows + r)
                                                                     : make_int4(0, 0, 0, 0);
 #pragma unroll
                             for (int j = 0; j < BN / 4; ++j) {
@@ -858,10 +858,10 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
 #pragma unroll
                     for (int u = 0; u < kGrp / 16; ++u) {
                         if (g0 + u < ch_hi) {
-                            int4 *dst = my_part + ((size_t)(g0 + u) * kPanelRows + r) * 4;
+                            int4 *dst = my_part + (size_t)(g0 + u) * 4 * kPanelRows + r;
 #pragma unroll
                             for (int j = 0; j < 4; ++j)
-                                dst[j] = make_int4((int)v[16 * u + 4 * j], (int)v[16 * u + 4 * j + 1],
+                                dst[j * kPanelRows] = make_int4((int)v[16 * u + 4 * j], (int)v[16 * u + 4 * j + 1],
                                                    (int)v[16 * u + 4 * j + 2], (int)v[16 * u + 4 * j + 3]);
                         }
                     }
@@ -891,7 +891,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
 #pragma unroll
                                     for (int j = 0; j < 4; ++j)
                                         ld[u * 4 + j] = (g0 + u < ch_hi)
-                                                            ? __ldcg(src + ((size_t)(g0 + u) * kPanelRows + r) * 4 + j)
+                                                            ? __ldcg(src + (size_t)((g0 + u) * 4 + j) * kPanelRows + r)
                                                             : make_int4(0, 0, 0, 0);
 #pragma unroll
                                 for (int j = 0; j < kGrp / 4; ++j) {
@@ -1121,6 +1121,7 @@ cudaError_t dispatch(int BN, int KST, bool pair, const CUtensorMap &tmap, const 
 }
 
 std::atomic<int> g_cta_pairs{1};
+std::atomic<int> g_narrow_tiles{1};
 
 // SMs of the current device, looked up once per device.
 int sm_count()
@@ -1138,17 +1139,6 @@ int sm_count()
 
 // K depth of one pipeline stage: two packed chunks when K allows it and the
 // token tile leaves room for enough stages, else one.
-int gemm_stage_k(int M, int K)
-{
-    return (gemm_block_n(M) <= 64 && K % 256 == 0) ? 256 : 128;
-}
-
-long long gemm_units(int M, int N, int K)
-{
-    const int BN = gemm_block_n(M);
-    const long long m_tiles = (M + BN - 1) / BN;
-    return m_tiles * (long long)(N / kPanelRows) * (long long)(K / gemm_stage_k(M, K));
-}
 
 }  // namespace
 
@@ -1163,21 +1153,57 @@ void set_cta_pairs(bool enable)
     g_cta_pairs.store(enable ? 1 : 0);
 }
 
-int gemm_block_n(int M)
+void set_narrow_tiles(bool enable)
 {
-    return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    g_narrow_tiles.store(enable ? 1 : 0);
+}
+
+// Token tile width.  Up to 128 tokens one tile covers M.  Beyond that,
+// 256-token tiles unless they are so few that stream-K shares each among
+// many CTAs: every extra CTA on a tile costs a full INT32 partial that the
+// finishing CTA reads back, while a narrower tile costs another pass over
+// the weights.  Narrower tiles are taken (down to 64 tokens) while a tile
+// would be shared by four or more CTAs, or, for a short K (<= 4096, where
+// the partials weigh most against the K loop), by two or more.
+static int block_n_for(int M, int N, int K, bool narrow)
+{
+    int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    if (bn < 128 || !narrow) return bn;
+    for (;;) {
+        const long long tiles = (long long)((M + bn - 1) / bn) * (N / kPanelRows);
+        const bool wide_split = tiles * 4 <= kMaxCtas || (K <= 4096 && tiles * 2 <= kMaxCtas);
+        if (bn == 64 || !wide_split) return bn;
+        bn /= 2;
+    }
+}
+
+static long long units_for(int M, int N, int K, int BN)
+{
+    const int KST = (BN <= 64 && K % 256 == 0) ? 256 : 128;
+    return (long long)((M + BN - 1) / BN) * (N / kPanelRows) * (K / KST);
+}
+
+int gemm_block_n(int M, int N, int K)
+{
+    return block_n_for(M, N, K, g_narrow_tiles.load(std::memory_order_relaxed) != 0);
 }
 
 bool gemm_shape_supported(int M, int N, int K)
 {
-    return gemm_units(M, N, K) < (1ll << 31);
+    // the most units either tile choice can give (the narrowest tile)
+    return units_for(M, N, K, block_n_for(M, N, K, true)) < (1ll << 31);
 }
 
+// Sized for both tile choices (narrowing on or off), so that a workspace
+// stays valid across qoq_set_gemm_narrow_tiles: the widest tile's partial
+// times the most CTAs either choice launches.
 size_t gemm_workspace_bytes(int M, int N, int K)
 {
-    const int BN = gemm_block_n(M);
-    const long long grid = std::min<long long>(kMaxCtas, gemm_units(M, N, K));
-    return kCounterBytes + (size_t)grid * BN * kPanelRows * sizeof(int32_t);
+    const int bn_wide = block_n_for(M, N, K, false);
+    const int bn_narrow = block_n_for(M, N, K, true);
+    const long long units = std::max(units_for(M, N, K, bn_wide), units_for(M, N, K, bn_narrow));
+    const long long grid = std::min<long long>(kMaxCtas, units);
+    return kCounterBytes + (size_t)grid * bn_wide * kPanelRows * sizeof(int32_t);
 }
 
 cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
@@ -1186,12 +1212,12 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
                         const uint16_t *X)
 {
     *tmap_status = 0;
-    const int BN = gemm_block_n(M);
+    const int BN = gemm_block_n(M, N, K);
     // 256-token tiles run on CTA pairs (one M = 256 MMA over two weight
     // panels, each CTA holding half of the X8 tile) when N allows it, with
     // 256-wide K stages where K allows them
     const bool pair = a_in_tmem && g_cta_pairs.load(std::memory_order_relaxed) && BN == 256 && N % 256 == 0;
-    const int KST = (pair && K % 256 == 0) ? 256 : gemm_stage_k(M, K);
+    const int KST = (pair && K % 256 == 0) ? 256 : (BN <= 64 && K % 256 == 0) ? 256 : 128;
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) {
         *tmap_status = -1;
@@ -1211,7 +1237,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     }
     const int sms = sm_count();
     // stream-K units: (tile, K block) per CTA, or per CTA pair
-    const long long units = pair ? (long long)((M + BN - 1) / BN) * (N / 256) * (K / KST) : gemm_units(M, N, K);
+    const long long units = pair ? (long long)((M + BN - 1) / BN) * (N / 256) * (K / KST) : units_for(M, N, K, BN);
     const long long grid = pair ? 2 * std::min<long long>(std::min(kMaxCtas, sms) / 2, units)
                                 : std::min<long long>(std::min(kMaxCtas, sms), units);
 

@@ -29,7 +29,7 @@ cudaError_t launch_dequant(const uint8_t *Wp, const uint8_t *s_g, const uint8_t 
                            int8_t *W8hat, cudaStream_t stream);
 
 // Tile width along M (tokens) the GEMM uses for a given M.
-int gemm_block_n(int M);
+int gemm_block_n(int M, int N, int K);
 
 // False when the shape has more work units than the GEMM's 32-bit
 // scheduling arithmetic covers.
@@ -42,6 +42,10 @@ cudaError_t launch_stuck_wait(unsigned long long budget_ns, cudaStream_t stream)
 
 // Whether 256-token tiles run on CTA pairs (2-SM MMA); default on.
 void set_cta_pairs(bool enable);
+
+// Whether few, widely shared 256/128-token tiles give way to narrower ones;
+// default on.
+void set_narrow_tiles(bool enable);
 
 // Word offsets, in the workspace's counter region, of the two counters of
 // the fused call (after the split-tile counters of up to kMaxCtas CTAs).
