@@ -208,6 +208,12 @@ __attribute__((visibility("default"))) int qoq_debug_set_trace(void *buf)
     return QOQ_OK;
 }
 
+// Trace builds only: the first timed-out wait's site and the barrier layout.
+__attribute__((visibility("default"))) int qoq_debug_timeout_site(unsigned long long *out2)
+{
+    return qoq::debug_timeout_site(out2, out2 + 1) == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
+}
+
 // Trace builds only: one thread writes the global timer to *dst.
 __attribute__((visibility("default"))) int qoq_debug_stamp(void *dst, void *stream)
 {

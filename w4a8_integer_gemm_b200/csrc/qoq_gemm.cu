@@ -78,6 +78,9 @@
 namespace qoq {
 
 __device__ int g_dev_error;  // non-zero after a bounded wait ran out
+#ifdef QOQ_TRACE
+__device__ unsigned long long g_bar_info;  // trace builds: barrier base and ring depths of the last launch
+#endif
 
 struct GemmArgs {
     const uint8_t *Wp;
@@ -94,7 +97,7 @@ struct GemmArgs {
     const uint16_t *X;
     int8_t *X8w;       // = the X8 the tensor map reads
     uint16_t *s_xw;    // = s_x
-    int32_t *ws_ready; // epilogue threads that have stored their part of a row (128 per row)
+    int32_t *ws_ready; // token rows quantized and stored (fused call)
     int32_t *ws_done;  // CTAs finished; the last one resets both counters
     int M, N, K, G;
     int m_tiles;
@@ -169,7 +172,7 @@ struct GemmCfg {
     // two accumulators (the MMAs of the next tile run while the epilogue
     // drains the last one) wherever TMEM has room for them
     static constexpr int kAccBufs = (2 * BN + (A_TMEM ? SX * (int)kACols : 0) <= 512) ? 2 : 1;
-    static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * kAccBufs + 1;
+    static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * kAccBufs + 2;
     static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
     // at least ~120 KB so that exactly one CTA (and one TMEM allocation)
     // lives on each SM; +1024 for manual alignment of the dynamic base
@@ -182,6 +185,13 @@ struct GemmCfg {
     static_assert(BN + (A_TMEM ? SX * kACols : 0) <= 512, "TMEM columns");
     static_assert(kUsed <= 227 * 1024, "shared memory");
     static_assert(SW <= 32 && SX <= 32, "ring bookkeeping masks");
+    // The dequant groups take the K blocks in turn, and a group waits on a
+    // weight slot by phase parity.  That is sound only if the slot's
+    // previous fill was this group's own (already consumed): with a ring
+    // depth that the groups do not divide, the previous fill belongs to the
+    // other group, may still be in flight, and its pending phase then reads
+    // as this fill's completed one.
+    static_assert(SW % dequant_groups(BN) == 0, "each weight slot belongs to one dequant group");
     static_assert(kXSlot % 1024 == 0 && kAOff % 1024 == 0 && kWOff % 1024 == 0, "swizzle atoms");
 };
 
@@ -222,6 +232,7 @@ __device__ __forceinline__ bool wait_count_gpu(const int *p, int want, volatile 
     while (ld_acquire_gpu(p) < want) {
         if (*abort) return false;
         if (global_timer_ns() - start > budget_ns) {
+            QOQ_RECORD_TIMEOUT(0xF00001u);
             *abort = 1;
             return false;
         }
@@ -318,6 +329,10 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     auto accfull_bar = [&](int b) { return bar0 + 8u * (2 * SW + 2 * SX + b); };
     auto accempty_bar = [&](int b) { return bar0 + 8u * (2 * SW + 2 * SX + C::kAccBufs + b); };
     const uint32_t mmadone_bar = bar0 + 8u * (2 * SW + 2 * SX + 2 * C::kAccBufs);
+    // fused call: every token row of X8 and s_x is in memory (the X8
+    // producer, the one thread of the CTA that polls the grid-wide count,
+    // passes it on to the epilogue warps)
+    const uint32_t xready_bar = mmadone_bar + 8u;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -368,6 +383,9 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     const int n_pro = min(min(SW, kPrologueStages), i_end - i_begin);
 
 #ifdef QOQ_TRACE
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+        g_bar_info = (unsigned long long)bar0 | ((unsigned long long)SW << 32) | ((unsigned long long)SX << 40) |
+                     ((unsigned long long)C::kAccBufs << 48);
     const long long trace_t0 = clock64();
     if (threadIdx.x == 0 && a.trace) a.trace[(size_t)blockIdx.x * 256 + 255] = global_timer_ns();
 #endif
@@ -387,6 +405,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             mbar_init(accempty_bar(b), 4 * kEpi * (PAIR ? 2 : 1));   // the epilogue warps (of each CTA)
         }
         mbar_init(mmadone_bar, 1);
+        mbar_init(xready_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
         // weights stream from here on, while the rest of the CTA sets up
@@ -446,11 +465,22 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         // ------------------------------------------------- X8 producer --
         if (lane == 0) {
             grid_dependency_wait();  // X8 comes from the preceding kernel
+            QOQ_MARK(10);
+#ifdef QOQ_TRACE
+            if (a.trace) {  // latency of one plain L2 load at this point
+                QOQ_MARK(144);
+                const int v = __ldcg(reinterpret_cast<const int *>(a.s_x));
+                asm volatile("" ::"r"(v));
+                QOQ_MARK(145);
+            }
+#endif
             bool ok = true;
             if (a.X) {
                 // fused call: X8 is written by this grid's epilogue warps
-                ok = wait_count_gpu(a.ws_ready, 128 * a.M, abort_flag, budget);
+                ok = wait_count_gpu(a.ws_ready, a.M, abort_flag, budget);
+                QOQ_MARK(11);
                 fence_proxy_async_global();
+                if (ok) mbar_arrive(xready_bar);
             }
             int s = 0;
             uint32_t ph = 0;
@@ -481,6 +511,14 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                                         afull_bar(s));
                     }
                     if (tj < 16) QOQ_MARK(32 + tj);
+#ifdef QOQ_TRACE
+                    if (a.trace && tj == 6) {  // and again mid-stream
+                        QOQ_MARK(146);
+                        const int v = __ldcg(reinterpret_cast<const int *>(a.s_x) + 1);
+                        asm volatile("" ::"r"(v));
+                        QOQ_MARK(147);
+                    }
+#endif
                     ++tj;
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -687,6 +725,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         int ab = 0;          // accumulator of the current tile
         uint32_t accph = 0;  // its phase parity
         grid_dependency_wait();  // s_x (or X) comes from the preceding kernel
+        if (threadIdx.x == kEpiWarp0 * 32) QOQ_MARK(6);
         if (a.X && eg == 0) {
             // Fused call: the four epilogue warps of each CTA quantize token
             // rows cta, cta + P, ... together (128 threads per row, the
@@ -715,6 +754,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     for (int c = 0; c < 4; ++c) amax = fmaxf(amax, absmax8(t[c]));
                 }
                 amax = warp_max(amax);
+                if (et == 0 && row == cta) QOQ_MARK(7);
                 if (lane == 0) rowmax[warp - kEpiWarp0] = amax;
                 named_barrier(1, 128);
                 amax = fmaxf(fmaxf(rowmax[0], rowmax[1]), fmaxf(rowmax[2], rowmax[3]));
@@ -736,15 +776,23 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                         if (v0 + c * 128 < nvec) dst[v0 + c * 128] = quant8(t[c], sxf);
                 }
                 if (et == 0) a.s_xw[row] = sxh;
-                // the X8 tiles are read back by TMA (the async proxy); each
-                // thread's release covers its own stores
+                if (et == 0 && row == cta) QOQ_MARK(12);
+                // the X8 tiles are read back by TMA (the async proxy); after
+                // the barrier one release covers the row's stores by all 128
+                // threads (one count per row keeps the polled line quiet)
                 fence_proxy_async_global();
-                red_release_gpu_add(a.ws_ready, 1);
+                if (et == 0 && row == cta) QOQ_MARK(13);
+                named_barrier(1, 128);
+                if (et == 0 && row == cta) QOQ_MARK(14);
+                if (et == 0) red_release_gpu_add(a.ws_ready, 1);
+                if (et == 0 && row == cta) QOQ_MARK(8);
             }
         }
         if (a.X) {
-            // 128 counts per row; on a timeout the flag stops every role
-            wait_count_gpu(a.ws_ready, 128 * a.M, abort_flag, budget);
+            // every row is done once the X8 producer has seen the count; on
+            // a timeout the flag stops every role
+            wait_x(xready_bar, 0u);
+            if (threadIdx.x == kEpiWarp0 * 32) QOQ_MARK(9);
         }
         for (int i = i_begin; i < i_end;) {
             const int t = i / ks;
@@ -792,6 +840,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     const uint64_t start = global_timer_ns();
                     while (ld_acquire_gpu(counter) < want) {
                         if (*abort_flag || global_timer_ns() - start > budget) {
+                            if (!*abort_flag) QOQ_RECORD_TIMEOUT(0xF00002u);
                             *abort_flag = 1;
                             ready = false;
                             break;
@@ -1012,6 +1061,20 @@ __global__ void stuck_wait_kernel(unsigned long long budget_ns)
 #ifdef QOQ_TRACE
 unsigned long long *g_trace_buffer = nullptr;
 
+// Trace builds: the first timed-out wait's site since the last read (0 if
+// none), and the barrier layout of the latest launch; both are cleared.
+cudaError_t debug_timeout_site(unsigned long long *site, unsigned long long *bar_info)
+{
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(site, g_timeout_site, sizeof(*site));
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(bar_info, g_bar_info, sizeof(*bar_info));
+    if (e != cudaSuccess) return e;
+    const unsigned long long zero = 0;
+    return cudaMemcpyToSymbol(g_timeout_site, &zero, sizeof(zero));
+}
+
 __global__ void stamp_kernel(unsigned long long *dst)
 {
     *dst = global_timer_ns();
@@ -1106,9 +1169,9 @@ cudaError_t dispatch(int BN, int KST, bool pair, const CUtensorMap &tmap, const 
     }
     if (KST == 256) {
         switch (BN) {
-        case 16: return launch_cfg<16, 256, A_TMEM ? 11 : 6, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
-        case 32: return launch_cfg<32, 256, A_TMEM ? 9 : 6, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
-        default: return launch_cfg<64, 256, A_TMEM ? 7 : 4, A_TMEM ? 6 : 2, A_TMEM>(tmap, args, grid, stream);
+        case 16: return launch_cfg<16, 256, A_TMEM ? 10 : 6, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
+        case 32: return launch_cfg<32, 256, A_TMEM ? 8 : 6, A_TMEM ? 7 : 3, A_TMEM>(tmap, args, grid, stream);
+        default: return launch_cfg<64, 256, A_TMEM ? 8 : 4, A_TMEM ? 5 : 2, A_TMEM>(tmap, args, grid, stream);
         }
     }
     switch (BN) {
@@ -1238,8 +1301,14 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     const int sms = sm_count();
     // stream-K units: (tile, K block) per CTA, or per CTA pair
     const long long units = pair ? (long long)((M + BN - 1) / BN) * (N / 256) * (K / KST) : units_for(M, N, K, BN);
-    const long long grid = pair ? 2 * std::min<long long>(std::min(kMaxCtas, sms) / 2, units)
-                                : std::min<long long>(std::min(kMaxCtas, sms), units);
+    const long long slots = pair ? std::min(kMaxCtas, sms) / 2 : std::min(kMaxCtas, sms);
+    const long long tiles = units / (K / KST);
+    long long sched_units = std::min(slots, units);
+#ifndef QOQ_DP_MIN_PCT
+#define QOQ_DP_MIN_PCT 70
+#endif
+    if (tiles <= slots && tiles * 100 >= slots * QOQ_DP_MIN_PCT) sched_units = tiles;
+    const long long grid = pair ? 2 * sched_units : sched_units;
 
     GemmArgs args;
     args.Wp = Wp;

@@ -66,6 +66,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
 #ifdef QOQ_TRACE
 extern unsigned long long *g_trace_buffer;
 cudaError_t debug_stamp(unsigned long long *dst, cudaStream_t stream);
+cudaError_t debug_timeout_site(unsigned long long *site, unsigned long long *bar_info);
 #endif
 
 // Device error flag of the current device: read and clear (synchronous).
