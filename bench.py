@@ -231,8 +231,8 @@ def run_ours(args, rank, world, local, dist):
     es = [E(), E(), E(), E()]
 
     def enqueue_step(st, gemm=True, quant=True, fused=True):
-        """Launch the step's kernels on stream st: per shape the fused layer
-        call (one kernel), or the quantizer and the GEMM as two kernels."""
+        """Launch the step's kernels on stream st: per shape the layer call
+        (qoq_w4a8_linear), or the quantizer and the GEMM as separate calls."""
         for c in cases:
             if quant and gemm and fused:
                 q.qoq_w4a8_linear(c["X"], c["packed"], X8=c["X8"], s_x=c["s_x"], Y=c["Y"], workspace=c["ws"],
@@ -266,23 +266,28 @@ def run_ours(args, rank, world, local, dist):
         torch.cuda.synchronize()
         return sum(ev[j][0].elapsed_time(ev[j][1]) for j in range(n_sh))
 
-    def two_kernel_step():
-        """The same step with the quantizer and the GEMM as separate kernels
-        (replayed from a graph when chained), for comparison."""
+    def one_launch_step():
+        """The same step with the layer call as one GEMM launch that
+        quantizes its own rows (replayed from a graph when chained), for
+        comparison."""
         if chained:
             es[0].record(stream)
-            graphs["two_kernel"].replay()
+            graphs["one_launch"].replay()
             es[1].record(stream)
             torch.cuda.synchronize()
             return es[0].elapsed_time(es[1])
         tot = 0.0
-        for j, c in enumerate(cases):
-            flush.zero_()
-            ev[j][0].record(stream)
-            q.qoq_quant_act_per_token(c["X"], c["X8"], c["s_x"], stream=stream)
-            q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
-            ev[j][1].record(stream)
-        torch.cuda.synchronize()
+        q.qoq_set_linear_in_kernel_quant(True)
+        try:
+            for j, c in enumerate(cases):
+                flush.zero_()
+                ev[j][0].record(stream)
+                q.qoq_w4a8_linear(c["X"], c["packed"], X8=c["X8"], s_x=c["s_x"], Y=c["Y"], workspace=c["ws"],
+                                  stream=stream)
+                ev[j][1].record(stream)
+            torch.cuda.synchronize()
+        finally:
+            q.qoq_set_linear_in_kernel_quant(False)
         for j in range(n_sh):
             tot += ev[j][0].elapsed_time(ev[j][1])
         return tot
@@ -344,10 +349,14 @@ def run_ours(args, rank, world, local, dist):
         eager_ms = statistics.median(one_step(eager=True) for _ in range(max(3, args.warmup)))
         cap = torch.cuda.Stream(device=dev)
         cap.wait_stream(stream)
-        for name, kw in (("step", {}), ("gemm", {"quant": False}), ("two_kernel", {"fused": False})):
+        for name, kw in (("step", {}), ("gemm", {"quant": False}), ("one_launch", {})):
             g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap):
-                enqueue_step(cap, **kw)
+            q.qoq_set_linear_in_kernel_quant(name == "one_launch")
+            try:
+                with torch.cuda.graph(g, stream=cap):
+                    enqueue_step(cap, **kw)
+            finally:
+                q.qoq_set_linear_in_kernel_quant(False)
             graphs[name] = g
         stream.wait_stream(cap)
         for _ in range(max(3, args.warmup)):
@@ -369,7 +378,7 @@ def run_ours(args, rank, world, local, dist):
         wall = time.perf_counter() - t_wall
     clocks = clk.summary()
     g_ms_total = sum(gemm_only() for _ in range(args.steps)) / args.steps
-    two_ms = statistics.median(two_kernel_step() for _ in range(args.steps)) if (graphs or not chained) else None
+    one_ms = statistics.median(one_launch_step() for _ in range(args.steps)) if (graphs or not chained) else None
     iso = isolated()
     if q.qoq_device_error() != q.QOQ_OK:
         raise RuntimeError("device error in the timed region")
@@ -460,10 +469,11 @@ def run_ours(args, rank, world, local, dist):
                    "launch": ("cuda_graph (one graph per step, programmatic dependent launch between kernels)"
                               if graphs else "eager (every kernel launched from Python)"),
                    "eager_ms_per_step": None if eager_ms is None else round(eager_ms, 5),
-                   "kernels": "per shape one fused launch (qoq_w4a8_linear: per-token quantization + GEMM)",
-                   "two_kernel_ms_per_step": None if two_ms is None else round(two_ms, 5)},
+                   "kernels": ("per shape qoq_w4a8_linear: the per-token quantizer kernel, then the GEMM kernel "
+                               "(programmatic dependent launch)"),
+                   "one_launch_ms_per_step": None if one_ms is None else round(one_ms, 5)},
         "roofline": rl, "points": per, "clocks": clocks, "e2e": e2e,
-        "gpu_launches": n_sh * args.steps,
+        "gpu_launches": 2 * n_sh * args.steps,
         "a_operand": "smem" if args.a_smem else "tmem",
     }
     return out, cases

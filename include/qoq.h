@@ -203,13 +203,11 @@ QOQ_API int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x,
                   uint16_t *Y, int32_t *acc_dbg,
                   void *workspace, size_t workspace_bytes, void *stream);
 
-/* The whole W4A8 linear layer in one kernel launch: the per-token
- * quantization of qoq_quant_act_per_token followed by qoq_w4a8_gemm.
+/* The whole W4A8 linear layer in one call: the per-token quantization of
+ * qoq_quant_act_per_token followed by qoq_w4a8_gemm.
  *
  * Sources: as for those two calls; the result is bit-identical to calling
- * them in sequence. The pages describe the two steps as one layer; doing
- * both in one launch saves the second kernel's launch and its wait for the
- * first to finish (which is most of a decode-sized layer's time).
+ * them in sequence (the pages describe the two steps as one layer).
  *
  *   X        device, uint16_t [M][K] FP16 bits, read only.
  *   X8, s_x  device, written exactly as qoq_quant_act_per_token writes them
@@ -217,11 +215,13 @@ QOQ_API int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x,
  *   Wp, s_c, s_g, zs, Y, workspace, workspace_bytes
  *            as for qoq_w4a8_gemm (the same workspace rules; this call also
  *            leaves the workspace's counters at zero).
- * For M <= 148 the rows are quantized inside the GEMM kernel by the SMs'
- * otherwise idle epilogue warps (one row per SM), which publish each
- * finished row with a release operation; the GEMM's loads of X8 and s_x
- * wait (bounded) until every row is done. Larger M runs the quantizer and
- * the GEMM as two kernels on the stream. Limits: as for qoq_w4a8_gemm.
+ * By default the call launches the quantizer and the GEMM back to back on
+ * the stream (programmatic dependent launch: the GEMM streams its weights
+ * while the quantizer runs). With qoq_set_linear_in_kernel_quant(1) and
+ * M <= 148 it is one launch instead: the GEMM's epilogue warps quantize the
+ * rows (one row per SM) and publish each finished row with a release
+ * operation, and the GEMM's loads of X8 and s_x wait (bounded) until every
+ * row is done. Limits: as for qoq_w4a8_gemm.
  */
 QOQ_API int qoq_w4a8_linear(const uint16_t *X, int M, int N, int K, int group_size,
                     const uint8_t *Wp, const uint16_t *s_c,
@@ -307,6 +307,16 @@ QOQ_API int qoq_set_gemm_cta_pairs(int enable);
  * thread. Results are identical either way. Returns QOQ_ERR_INVALID_ARG
  * for other values. */
 QOQ_API int qoq_set_gemm_narrow_tiles(int enable);
+
+/* Selects how qoq_w4a8_linear runs for M <= 148:
+ *   0 (default): the quantizer kernel, then the GEMM kernel;
+ *   1: one GEMM launch that quantizes its own rows (see qoq_w4a8_linear).
+ * On B200, chains of decode-sized layers measured 0.5-3.8 us per layer
+ * faster with two kernels: one row per SM, all waited for by every SM,
+ * costs more than the quantizer's own launch. The choice applies to later
+ * calls from every thread. Results are identical either way. Returns
+ * QOQ_ERR_INVALID_ARG for other values. */
+QOQ_API int qoq_set_linear_in_kernel_quant(int enable);
 
 /* Self-test of the failure path (the pages have no counterpart). Launches
  * one thread that waits on a barrier phase nothing completes, with the same

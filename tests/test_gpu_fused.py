@@ -1,8 +1,8 @@
-"""The fused layer call (qoq_w4a8_linear): per-token quantization and the
-GEMM in one kernel launch must give exactly what the two separate calls
-give -- X8, s_x and Y bit for bit -- on every output, over repeated calls
-(the call resets its own counters) and from a CUDA graph; a sample is also
-checked against the oracle."""
+"""The layer call (qoq_w4a8_linear), as two kernels (default) and as one
+GEMM launch that quantizes its own rows: each must give exactly what the
+two separate calls give -- X8, s_x and Y bit for bit -- on every output,
+over repeated calls (the one-launch form resets its own counters) and from
+a CUDA graph; a sample is also checked against the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -26,8 +26,15 @@ SHAPES = [
 ]
 
 
+@pytest.fixture(params=[False, True], ids=["two_kernels", "one_launch"])
+def in_kernel(request):
+    q.qoq_set_linear_in_kernel_quant(request.param)
+    yield request.param
+    q.qoq_set_linear_in_kernel_quant(False)
+
+
 @pytest.mark.parametrize("M,K,N,G", SHAPES, ids=[f"M{m}_K{k}_N{n}_G{g}" for m, k, n, g in SHAPES])
-def test_fused_equals_separate(M, K, N, G):
+def test_fused_equals_separate(M, K, N, G, in_kernel):
     q.qoq_set_gemm_a_in_tmem(True)
     dev = torch.device("cuda")
     X = wl.make_activations(M, K, wl.LLAMA, seed=6100 + M)

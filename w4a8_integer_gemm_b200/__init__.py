@@ -53,6 +53,7 @@ SIGNATURES = {
     "qoq_set_gemm_a_in_tmem": (_I, [_I]),
     "qoq_set_gemm_cta_pairs": (_I, [_I]),
     "qoq_set_gemm_narrow_tiles": (_I, [_I]),
+    "qoq_set_linear_in_kernel_quant": (_I, [_I]),
     "qoq_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "qoq_device_error": (_I, [_P]),
 }
@@ -130,6 +131,10 @@ def qoq_set_gemm_cta_pairs(enable: bool) -> None:
 
 def qoq_set_gemm_narrow_tiles(enable: bool) -> None:
     _check("qoq_set_gemm_narrow_tiles", lib().qoq_set_gemm_narrow_tiles(1 if enable else 0))
+
+
+def qoq_set_linear_in_kernel_quant(enable: bool) -> None:
+    _check("qoq_set_linear_in_kernel_quant", lib().qoq_set_linear_in_kernel_quant(1 if enable else 0))
 
 
 def qoq_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:

@@ -12,6 +12,7 @@
 namespace {
 
 std::atomic<int> g_a_in_tmem{1};
+std::atomic<int> g_linear_in_kernel_quant{0};
 
 constexpr int kMaxK = 65536;
 constexpr int kMaxN = 1 << 20;
@@ -145,10 +146,10 @@ int qoq_w4a8_linear(const uint16_t *X, int M, int N, int K, int group_size, cons
     const int dev = check_device();
     if (dev != QOQ_OK) return dev;
     int tmap_status = 0;
-    // Up to one row per SM the GEMM quantizes its own input; a longer chain
-    // of rows per SM costs more than the quantizer's own launch, so larger
-    // batches run the two kernels back to back (same results).
-    const bool in_kernel = M <= qoq::kFusedMaxRows;
+    // The quantizer and the GEMM as two kernels (default), or, up to one
+    // row per SM and when selected, one GEMM launch that quantizes its own
+    // input (same results).
+    const bool in_kernel = g_linear_in_kernel_quant.load() != 0 && M <= qoq::kFusedMaxRows;
     if (!in_kernel) {
         const cudaError_t eq = qoq::launch_act_quant(X, M, K, X8, s_x, (cudaStream_t)stream);
         if (eq != cudaSuccess) return from_cuda(eq);
@@ -196,6 +197,13 @@ int qoq_set_gemm_narrow_tiles(int enable)
 {
     if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;
     qoq::set_narrow_tiles(enable != 0);
+    return QOQ_OK;
+}
+
+int qoq_set_linear_in_kernel_quant(int enable)
+{
+    if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;
+    g_linear_in_kernel_quant.store(enable);
     return QOQ_OK;
 }
 

@@ -1301,13 +1301,13 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     const int sms = sm_count();
     // stream-K units: (tile, K block) per CTA, or per CTA pair
     const long long units = pair ? (long long)((M + BN - 1) / BN) * (N / 256) * (K / KST) : units_for(M, N, K, BN);
+    // Stream-K over the SMs, except when the tiles alone fill at least 70%
+    // of them: then one whole tile per CTA (or pair), so that no tile is
+    // split and no CTA waits at the end for another's partial sums (the
+    // decode projections: 112 tiles on 148 SMs).
     const long long slots = pair ? std::min(kMaxCtas, sms) / 2 : std::min(kMaxCtas, sms);
     const long long tiles = units / (K / KST);
-    long long sched_units = std::min(slots, units);
-#ifndef QOQ_DP_MIN_PCT
-#define QOQ_DP_MIN_PCT 70
-#endif
-    if (tiles <= slots && tiles * 100 >= slots * QOQ_DP_MIN_PCT) sched_units = tiles;
+    const long long sched_units = (tiles <= slots && tiles * 10 >= slots * 7) ? tiles : std::min(slots, units);
     const long long grid = pair ? 2 * sched_units : sched_units;
 
     GemmArgs args;
