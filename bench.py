@@ -44,18 +44,31 @@ from w4a8_integer_gemm_b200 import roofline, workloads as wl  # noqa: E402
 
 FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20
-GEMM_SOURCES = ("qoq_gemm.cu", "qoq_layout.cuh", "qoq_ptx.cuh", "qoq_internal.h")
+GEMM_SOURCES = ("qoq_gemm.cu", "qoq_layout.cuh", "qoq_ptx.cuh", "qoq_internal.h", "qoq_quant.cuh")
 
 
-def gemm_source_hash() -> str:
-    """Short hash of the GEMM kernel's sources: DRAM traffic recorded under
-    profiles/ is reported only while it matches (the counters describe that
-    kernel and no later one)."""
+def code_only(text: str) -> str:
+    """C/C++ source without its comments and with whitespace collapsed, so
+    that a change of wording alone leaves the code's hash as it was."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def gemm_source_hash(read=None) -> str:
+    """Short hash of the GEMM kernel's code (comments excluded): DRAM traffic
+    recorded under profiles/ is reported only while it matches, since the
+    counters describe that kernel and no later one.  `read(name)` returns a
+    source file's text (default: the working tree)."""
     import hashlib
+    if read is None:
+        def read(f):
+            with open(os.path.join(ROOT, "w4a8_integer_gemm_b200", "csrc", f)) as fh:
+                return fh.read()
     h = hashlib.sha256()
     for f in GEMM_SOURCES:
-        with open(os.path.join(ROOT, "w4a8_integer_gemm_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        h.update(code_only(read(f)).encode())
     return h.hexdigest()[:16]
 
 

@@ -16,10 +16,14 @@
 //   * Swap-AB: the 128 output channels of a weight panel are the MMA's M
 //     (A operand), the tokens are its N (B operand, BN = 16..256).  Decode
 //     shapes (M <= 64) therefore waste no tensor-core rows on padding tokens.
+//     Beyond 64 tokens the tile narrows while tiles would be few and
+//     widely shared (gemm_block_n).
 //   * Persistent grid, one CTA per SM, stream-K schedule: the sequence of
 //     (output tile, KST-wide K block) units is cut into equal contiguous
 //     ranges, one per CTA, so every SM streams the same number of weight
-//     bytes.  A tile whose K loop is split across CTAs is finished by its
+//     bytes.  When the tiles alone fill 70-100% of the SMs each CTA takes
+//     one whole tile instead and nothing is split.  A tile whose K loop is
+//     split across CTAs is finished by its
 //     first contributor (the CTA whose range holds the tile's first unit:
 //     for it the tile is the last one it works on).  Every later
 //     contributor works on the tile first, publishes its INT32 partial
@@ -48,9 +52,11 @@
 //       epilogue    one or two groups of four warps (two for 256-token
 //                   tiles, one per 128 tokens): tcgen05.ld of the INT32
 //                   accumulators, FP32 scaling, FP16 stores; split tiles as
-//                   above.  In the fused call they first quantize the rows.
+//                   above.  In the one-launch layer call they first
+//                   quantize the token rows.
 //   * Rings: a weight ring (packed chunks and tables of a K block, freed
-//     as soon as the dequant warps hold them in registers); an X8/A ring
+//     as soon as the dequant warps hold them in registers; with two dequant
+//     groups each slot belongs to one group); an X8/A ring
 //     (slot s holds the X8 tiles of a K block in shared memory and its
 //     dequantized weights in A slot s; one barrier says both are ready, one
 //     commit frees both); and one or two TMEM accumulators, so the MMAs of
@@ -92,12 +98,12 @@ struct GemmArgs {
     int32_t *acc_dbg;
     int32_t *ws_cnt;   // [kMaxCtas][4] arrival counters, at the start of the workspace
     int32_t *ws_part;  // [cta][BN/16][4][128][4] INT32 partial tile, after the counters
-    // The fused call (X non-null): the kernel first quantizes the FP16 rows
+    // The one-launch layer call (X non-null): the kernel first quantizes the FP16 rows
     // of X into X8 / s_x itself, then reads them as in the plain GEMM.
     const uint16_t *X;
     int8_t *X8w;       // = the X8 the tensor map reads
     uint16_t *s_xw;    // = s_x
-    int32_t *ws_ready; // token rows quantized and stored (fused call)
+    int32_t *ws_ready; // token rows quantized and stored (one-launch layer call)
     int32_t *ws_done;  // CTAs finished; the last one resets both counters
     int M, N, K, G;
     int m_tiles;
@@ -329,7 +335,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     auto accfull_bar = [&](int b) { return bar0 + 8u * (2 * SW + 2 * SX + b); };
     auto accempty_bar = [&](int b) { return bar0 + 8u * (2 * SW + 2 * SX + C::kAccBufs + b); };
     const uint32_t mmadone_bar = bar0 + 8u * (2 * SW + 2 * SX + 2 * C::kAccBufs);
-    // fused call: every token row of X8 and s_x is in memory (the X8
+    // one-launch layer call: every token row of X8 and s_x is in memory (the X8
     // producer, the one thread of the CTA that polls the grid-wide count,
     // passes it on to the epilogue warps)
     const uint32_t xready_bar = mmadone_bar + 8u;
@@ -476,7 +482,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
 #endif
             bool ok = true;
             if (a.X) {
-                // fused call: X8 is written by this grid's epilogue warps
+                // one-launch layer call: X8 is written by this grid's epilogue warps
                 ok = wait_count_gpu(a.ws_ready, a.M, abort_flag, budget);
                 QOQ_MARK(11);
                 fence_proxy_async_global();

@@ -48,15 +48,15 @@ void set_cta_pairs(bool enable);
 void set_narrow_tiles(bool enable);
 
 // Word offsets, in the workspace's counter region, of the two counters of
-// the fused call (after the split-tile counters of up to kMaxCtas CTAs).
+// the one-launch layer call (after the split-tile counters of up to kMaxCtas CTAs).
 constexpr int kFusedReadyWord = 2000;
 constexpr int kFusedDoneWord = 2001;
-// Largest M for which the fused call quantizes inside the GEMM kernel.
+// Largest M for which the layer call can quantize inside the GEMM kernel.
 constexpr int kFusedMaxRows = kMaxCtas;
 
 // Returns cudaSuccess or the launch / tensor-map error.  `tmap_status`
 // receives the driver status of the tensor-map encode (0 on success).
-// With X non-null the kernel first quantizes X into X8 and s_x (the fused
+// With X non-null the kernel first quantizes X into X8 and s_x (the one-launch
 // call); otherwise it reads them.
 cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
                         const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
