@@ -234,7 +234,9 @@ def qoq_w4a8_gemm(X8: torch.Tensor, s_x: torch.Tensor, packed: PackedWeights,
 def qoq_w4a8_linear(X: torch.Tensor, packed: PackedWeights, X8: Optional[torch.Tensor] = None,
                     s_x: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
                     workspace: Optional[torch.Tensor] = None, stream=None):
-    """Quantize X (fp16 [M, K]) per token and run the GEMM, in one launch.
+    """Quantize X (fp16 [M, K]) per token and run the GEMM: the quantizer
+    and GEMM kernels back to back, or one launch after
+    qoq_set_linear_in_kernel_quant(True) (M <= 148).
 
     Returns (Y, X8, s_x); bit-identical to qoq_quant_act_per_token followed
     by qoq_w4a8_gemm."""
@@ -300,7 +302,7 @@ class W4A8Linear:
         self.out_features = W.shape[0]
 
     def __call__(self, x_fp16: torch.Tensor, stream=None) -> torch.Tensor:
-        """y = fp16 W4A8 linear of x (fp16 [M, in_features]), one kernel launch."""
+        """y = fp16 W4A8 linear of x (fp16 [M, in_features]) through the layer call."""
         Y, _, _ = qoq_w4a8_linear(x_fp16, self.packed, stream=stream)
         return Y
 
