@@ -62,6 +62,18 @@ def test_size_queries(L):
     assert q.qoq_gemm_workspace_bytes(1, 512, 512, 128) == 8192 + 8 * 16 * 128 * 4
     # 256-token tiles use 128-wide K blocks: 4 m-tiles x 64 n-tiles x 64 blocks -> 148 CTAs
     assert q.qoq_gemm_workspace_bytes(1024, 8192, 8192, 128) == 8192 + 148 * 256 * 128 * 4
+    # Few tiles: the default rule narrows M = 256, N = K = 4096 to 64-token tiles, but the
+    # workspace also covers the 256-token tiles of the other rule (148 CTAs either way).
+    assert q.qoq_gemm_workspace_bytes(256, 4096, 4096, 128) == 8192 + 148 * 256 * 128 * 4
+    # M = 200, N = 512, K = 1024: 64-token tiles give 4 x 4 tiles x 4 K blocks of 256 = 64
+    # units, 256-token tiles 4 tiles x 8 K blocks of 128 = 32: 64 CTAs, 256-token slots.
+    assert q.qoq_gemm_workspace_bytes(200, 512, 1024, 128) == 8192 + 64 * 256 * 128 * 4
+    # and the size does not depend on the switch
+    sizes = []
+    for narrow in (False, True):
+        q.qoq_set_gemm_narrow_tiles(narrow)
+        sizes.append(q.qoq_gemm_workspace_bytes(200, 512, 1024, 128))
+    assert sizes[0] == sizes[1]
 
 
 def _fake(addr):
