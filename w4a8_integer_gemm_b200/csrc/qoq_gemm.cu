@@ -192,11 +192,12 @@ struct GemmCfg {
     static_assert(kUsed <= 227 * 1024, "shared memory");
     static_assert(SW <= 32 && SX <= 32, "ring bookkeeping masks");
     // The dequant groups take the K blocks in turn, and a group waits on a
-    // weight slot by phase parity.  That is sound only if the slot's
-    // previous fill was this group's own (already consumed): with a ring
-    // depth that the groups do not divide, the previous fill belongs to the
-    // other group, may still be in flight, and its pending phase then reads
-    // as this fill's completed one.
+    // weight slot by phase parity.  With a ring depth that the groups do not
+    // divide, the slot's previous fill belongs to the other group and may
+    // still be in flight; its pending phase then reads as this fill's
+    // completed one (unless SW >= SX + 2, when the group's own previous A-slot
+    // wait already proves that fill consumed).  The kernel keeps the simpler
+    // sufficient rule: each weight slot belongs to one group.
     static_assert(SW % dequant_groups(BN) == 0, "each weight slot belongs to one dequant group");
     static_assert(kXSlot % 1024 == 0 && kAOff % 1024 == 0 && kWOff % 1024 == 0, "swizzle atoms");
 };
