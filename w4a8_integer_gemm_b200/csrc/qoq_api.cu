@@ -1,5 +1,6 @@
 // qoq_api.cu -- the extern "C" entry points declared in include/qoq.h:
-// argument validation on the host, then one launch per call.
+// argument validation on the host, then the call's launches (one per call,
+// two for the layer call in its default form).
 #include <cuda_runtime.h>
 
 #include <atomic>
