@@ -493,17 +493,20 @@ def run_ours(args, rank, world, local, dist):
 
 
 # ------------------------------------------------------------ CPU oracle --
-def oracle_sample(work, budget_s):
-    """Time the oracle's act quant + INT32 GEMM + epilogue on every shape of
-    the workload, restricted to a channel sample sized for `budget_s` CPU
-    seconds in total; returns (TOPS, threads, description)."""
+def oracle_sample(work, budget_s, indices=None):
+    """Time the oracle's act quant + INT32 GEMM + epilogue on the shapes of
+    the workload (all, or those at `indices`), restricted to a channel
+    sample sized for `budget_s` CPU seconds in total; returns (TOPS, threads,
+    description)."""
     import oracle
 
-    n_sh = len(work.shapes)
+    idx = list(range(len(work.shapes))) if indices is None else list(indices)
+    n_sh = len(idx)
     per_shape = budget_s / n_sh
     tot_ops = tot_s = 0.0
     descr = []
-    for i, s in enumerate(work.shapes):
+    for i in idx:
+        s = work.shapes[i]
         X, W = wl.make_case(work, i)
         Xn = X.numpy()
         rows = min(s.M, 256)
@@ -528,6 +531,21 @@ def oracle_sample(work, budget_s):
         tot_s += dt
         descr.append(f"{s.name}: {rows} tokens x {n_s} of {s.N} channels")
     return tot_ops / tot_s / 1e12, oracle.num_threads(), "; ".join(descr)
+
+
+def oracle_single_core(work, budget_s):
+    """The same oracle timing on one host core, for the workload's smallest
+    shape (by operations)."""
+    import oracle
+
+    i = min(range(len(work.shapes)), key=lambda j: work.shapes[j].M * work.shapes[j].N * work.shapes[j].K)
+    before = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        v, threads, descr = oracle_sample(work, budget_s, indices=[i])
+    finally:
+        oracle.set_num_threads(before)
+    return {"value": round(v, 6), "unit": "TOPS", "cores": threads, "sample": descr}
 
 
 def run_reference(args, rank, world, local, dist):
@@ -575,7 +593,8 @@ def main():
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             v, threads, descr = oracle_sample(select(args), args.cpu_seconds)
             out["cpu_baseline"] = {"value": round(v, 6), "unit": "TOPS", "cores": threads, "kind": "oracle",
-                                   "sample": descr}
+                                   "sample": descr,
+                                   "single_core": oracle_single_core(select(args), min(5.0, args.cpu_seconds))}
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -86,6 +86,8 @@ def _load():
         lib.oracle_epilogue.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = None
         _lib = lib
         return lib
 
@@ -98,6 +100,12 @@ def _ptr(a: np.ndarray):
 def num_threads() -> int:
     """OpenMP threads the oracle's parallel loops use."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Sets the OpenMP threads of later calls from this thread (timing only:
+    the results do not depend on it)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 # ---------------------------------------------------------------- fp16 ----

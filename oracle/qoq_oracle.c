@@ -280,3 +280,14 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Sets that number (n >= 1) for later calls from this thread; timing only,
+ * the results do not depend on it. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -44,3 +44,32 @@ def test_a_code_change_changes_the_hash():
 
 def test_code_only_strips_both_comment_forms():
     assert bench.code_only("int a; // x\n/* y\n z */ int  b;") == "int a; int b;"
+
+
+def test_single_core_oracle_leg_restores_threads():
+    import oracle
+    from w4a8_integer_gemm_b200 import workloads as wl
+
+    oracle.build()
+    before = oracle.num_threads()
+    r = bench.oracle_single_core(wl.WORKLOADS["tiny"], 0.2)
+    assert r["cores"] == 1
+    assert r["value"] > 0
+    assert r["sample"].startswith("tiny: 16 tokens")
+    assert oracle.num_threads() == before
+
+
+def test_oracle_results_do_not_depend_on_threads():
+    import numpy as np
+    import oracle
+    from w4a8_integer_gemm_b200 import workloads as wl
+
+    X, W = wl.make_case(wl.WORKLOADS["tiny"], 0)
+    before = oracle.num_threads()
+    try:
+        oracle.set_num_threads(1)
+        r1 = oracle.linear(X.numpy(), W.numpy(), 128)
+    finally:
+        oracle.set_num_threads(before)
+    rn = oracle.linear(X.numpy(), W.numpy(), 128)
+    assert np.array_equal(r1["acc"], rn["acc"]) and np.array_equal(r1["Y"], rn["Y"])
