@@ -48,12 +48,27 @@ GEMM_SOURCES = ("qoq_gemm.cu", "qoq_layout.cuh", "qoq_ptx.cuh", "qoq_internal.h"
 
 
 def code_only(text: str) -> str:
-    """C/C++ source without its comments and with whitespace collapsed, so
-    that a change of wording alone leaves the code's hash as it was."""
+    """C/C++ source as the library build compiles it, for hashing: without
+    comments, without the trace build's `#ifdef QOQ_TRACE` branches (their
+    `#else` branches stay), and with whitespace collapsed.  A change of
+    wording or of trace-only code leaves the hash as it was."""
     import re
     text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
     text = re.sub(r"//[^\n]*", " ", text)
-    return " ".join(text.split())
+    kept, stack = [], []  # stack: per open #if, whether we are in its trace-only branch
+    for line in text.splitlines():
+        d = line.strip()
+        if d.startswith("#if"):
+            stack.append(d.split()[:2] == ["#ifdef", "QOQ_TRACE"])
+        elif d.startswith("#else") or d.startswith("#elif"):
+            if stack:
+                stack[-1] = False
+        elif d.startswith("#endif"):
+            if stack:
+                stack.pop()
+        elif not any(stack):
+            kept.append(line)  # conditional directives themselves are not kept
+    return " ".join(" ".join(kept).split())
 
 
 def gemm_source_hash(read=None) -> str:

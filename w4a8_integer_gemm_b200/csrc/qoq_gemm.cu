@@ -473,14 +473,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         if (lane == 0) {
             grid_dependency_wait();  // X8 comes from the preceding kernel
             QOQ_MARK(10);
-#ifdef QOQ_TRACE
-            if (a.trace) {  // latency of one plain L2 load at this point
-                QOQ_MARK(144);
-                const int v = __ldcg(reinterpret_cast<const int *>(a.s_x));
-                asm volatile("" ::"r"(v));
-                QOQ_MARK(145);
-            }
-#endif
             bool ok = true;
             if (a.X) {
                 // one-launch layer call: X8 is written by this grid's epilogue warps
@@ -518,14 +510,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                                         afull_bar(s));
                     }
                     if (tj < 16) QOQ_MARK(32 + tj);
-#ifdef QOQ_TRACE
-                    if (a.trace && tj == 6) {  // and again mid-stream
-                        QOQ_MARK(146);
-                        const int v = __ldcg(reinterpret_cast<const int *>(a.s_x) + 1);
-                        asm volatile("" ::"r"(v));
-                        QOQ_MARK(147);
-                    }
-#endif
                     ++tj;
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
