@@ -169,6 +169,8 @@ QOQ_API int qoq_quant_act_per_token(const uint16_t *X, int M, int K,
  *     workspace serves any sequence of shapes on one stream;
  *   - after a call that returned QOQ_ERR_TIMEOUT from qoq_device_error,
  *     zero-fill the workspace again.
+ * The size covers both token-tile rules of qoq_set_gemm_narrow_tiles, so a
+ * workspace stays valid when that setting changes.
  * Returns 0 for an invalid shape. */
 QOQ_API size_t qoq_gemm_workspace_bytes(int M, int N, int K, int group_size);
 
