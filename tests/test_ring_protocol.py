@@ -59,7 +59,10 @@ class Barrier:
             self.pending = self.count
 
 
-def run_rings(SW, SX, D, units, seed, steps=200000):
+def run_rings(SW, SX, D, units, seed, steps=200000, ks=None, acc_bufs=2, epi=1, accempty_count=None):
+    """ks: units per output tile (default: one tile); acc_bufs: TMEM
+    accumulators; epi: epilogue groups, each draining every tile;
+    accempty_count: the accempty arrival count (default: epi)."""
     rng = random.Random(seed)
     wfull = [Barrier(1) for _ in range(SW)]
     wempty = [Barrier(D and 1) for _ in range(SW)]
@@ -67,6 +70,13 @@ def run_rings(SW, SX, D, units, seed, steps=200000):
     xaempty = [Barrier(1) for _ in range(SX)]  # the MMA's commit
     wslot = [None] * SW                        # unit whose weights a slot holds
     xslot = [None] * SX                        # unit whose X8 tile an X8 slot holds
+    # accumulators: the MMA waits for accempty before a tile and commits
+    # accfull after its last unit; every epilogue group drains every tile
+    ks = ks or units
+    ntiles = (units + ks - 1) // ks
+    accfull = [Barrier(1) for _ in range(acc_bufs)]
+    accempty = [Barrier(accempty_count or epi) for _ in range(acc_bufs)]
+    acc = [None] * acc_bufs                    # [tile, units accumulated, epilogue groups that read it]
     aslot = [None] * SX                        # unit whose dequantized weights an A slot holds
     inflight = []                              # [due time, sequence, action]
     clock = [0, 0]                             # now, sequence numbers
@@ -125,11 +135,25 @@ def run_rings(SW, SX, D, units, seed, steps=200000):
 
     def mma():
         for u in range(units):
+            t = u // ks
+            b, jt = t % acc_bufs, t // acc_bufs
+            if u % ks == 0:
+                while not accempty[b].passes((jt & 1) ^ 1):
+                    yield
+                assert acc[b] is None or acc[b][2] == epi, f"tile {t} overwrites accumulator {b} before it was drained"
+                acc[b] = [t, 0, 0]
             a, j = u % SX, u // SX
             while not afull[a].passes(j & 1):
                 yield
             assert aslot[a] == u and xslot[a] == u, f"MMA of unit {u} read A {aslot[a]} and X8 {xslot[a]}"
+            acc[b][1] += 1
             yield
+            if u % ks == ks - 1 or u == units - 1:
+                def acc_commit(b=b):
+                    accfull[b].arrive()
+                due = max(last_commit[0] + 1, clock[0] + rng.randint(1, 20))
+                last_commit[0] = due
+                later(acc_commit, due - clock[0])
 
             def commit(a=a):
                 aslot[a] = None
@@ -141,7 +165,19 @@ def run_rings(SW, SX, D, units, seed, steps=200000):
             last_commit[0] = due
             later(commit, due - clock[0])
 
-    roles = [w_producer(), x_producer(), mma()] + [dequant(g) for g in range(D)]
+    def epilogue(g):
+        for t in range(ntiles):
+            b, jt = t % acc_bufs, t // acc_bufs
+            while not accfull[b].passes(jt & 1):
+                yield
+            expect = min(ks, units - t * ks)
+            assert acc[b] is not None and acc[b][0] == t and acc[b][1] == expect, \
+                f"epilogue group {g} read accumulator {b} as tile {t}: {acc[b]}"
+            yield
+            acc[b][2] += 1
+            accempty[b].arrive()
+
+    roles = [w_producer(), x_producer(), mma()] + [dequant(g) for g in range(D)] + [epilogue(g) for g in range(epi)]
     live = list(roles)
     for _ in range(steps):
         if not live and not inflight:
@@ -179,6 +215,47 @@ def dispatched_configs():
         for tmem in (True, False):
             out.add((bn, pick(args[2], tmem), pick(args[3], tmem), 2 if bn <= 64 else 1))
     return sorted(out)
+
+
+def accumulator_configs():
+    """(BN, KST, SX, A in TMEM, accumulator buffers, epilogue groups) of every
+    dispatched configuration, with the kernel's rules for the last two (two
+    accumulators where TMEM holds them beside the A ring; two epilogue
+    groups for 256-token tiles)."""
+    src = open(GEMM_SRC).read()
+    assert "kAccBufs = (2 * BN + (A_TMEM ? SX * (int)kACols : 0) <= 512) ? 2 : 1;" in src, \
+        "the kernel's accumulator-count rule changed: update this model"
+    assert "epilogue_groups(int BN) { return BN == 256 ? 2 : 1; }" in src
+    body = src[src.index("cudaError_t dispatch(int BN, int KST, bool pair"):]
+    body = body[:body.index("\n}\n")]
+    out = set()
+    for m in re.finditer(r"launch_cfg<([^>]*)>", body):
+        args = [x.strip() for x in m.group(1).split(",")]
+        bn, kst = int(args[0]), int(args[1])
+        flag = args[4]
+        for tmem in ((True, False) if flag == "A_TMEM" else (flag == "true",)):
+            t = re.match(r"A_TMEM \? (\d+) : (\d+)", args[3])
+            sx = int(t.group(1) if tmem else t.group(2)) if t else int(args[3])
+            bufs = 2 if 2 * bn + (sx * (kst // 4) if tmem else 0) <= 512 else 1
+            out.add((bn, kst, sx, tmem, bufs, 2 if bn == 256 else 1))
+    return sorted(out)
+
+
+@pytest.mark.parametrize("cfg", accumulator_configs(), ids=lambda c: "BN%d_KST%d_SX%d_tmem%d_acc%d_epi%d" % c)
+def test_accumulator_handoff(cfg):
+    bn, kst, SX, tmem, bufs, epi = cfg
+    D = 2 if bn <= 64 else 1
+    for seed in range(20):
+        for ks in (1, 3, 4):
+            run_rings(2 * SX, SX, D, units=4 * ks + 3, seed=seed, ks=ks, acc_bufs=bufs, epi=epi)
+
+
+def test_the_model_catches_an_accumulator_released_by_one_of_two_groups():
+    # accempty expecting one arrival where two epilogue groups drain each tile:
+    # a tile overwrites an undrained accumulator, or the ring deadlocks
+    with pytest.raises(AssertionError, match="accumulator|did not finish"):
+        for seed in range(200):
+            run_rings(4, 2, 1, units=20, seed=seed, ks=2, acc_bufs=1, epi=2, accempty_count=1)
 
 
 def test_dispatch_table_parsed():
