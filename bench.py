@@ -4,21 +4,27 @@ One step = one pass of the whole hot path -- per-token activation
 quantization, then the W4A8 GEMM with its epilogue -- over every shape of the
 workload, with weights packed offline (untimed) and resident in HBM.
 
-The default workload is the Llama-3-8B MLP up-projection at decode batch
-sizes: M in {1, 8, 32, 64}, K = 4096, N = 14336, per-channel and g128
-weights (8 GEMMs per step).  `--workload sweep|large_batch|qwen|tiny` selects
-the other workloads for ad-hoc measurement.
+The default workload is the batch-size sweep the metric is quoted on:
+M = 1, 2, 4, ..., 8192 tokens on K = N = 8192 with g128 weights (14 GEMMs
+per step, 485 MB of distinct packed weights).  `--workload
+decode|large_batch|qwen|tiny` selects the other workloads for ad-hoc
+measurement.
 
 Timing: when the distinct packed weights of a step exceed 1.5x L2
-(126 MB; the decode workload holds 224 MB), the shapes run back to back and
-the step is bracketed by CUDA events on the launching stream: every weight
-byte comes from HBM, because the step has cycled more than L2 since it last
-read the same weights.  Smaller workloads flush L2 (a 256 MB write) before
-every shape instead, bracket each shape with events (flush excluded) and sum.
+(126 MB), the shapes run back to back, replayed from one CUDA graph, and the
+step is bracketed by CUDA events on the launching stream: every weight byte
+comes from HBM, because the step has cycled more than L2 since it last read
+the same weights.  Smaller workloads flush L2 (a 256 MB write) before every
+shape instead, bracket each shape with events (flush excluded) and sum.
 K timed steps follow W untimed ones, bracketed by a barrier and a device
 synchronize; with N > 1 every rank runs the same workload (replicas, weak
-scaling) and the time is the max over ranks.  Per shape, an isolated run
-(L2 flushed, the kernels alone) gives the per-point breakdown.
+scaling) and the time is the max over ranks.
+
+The roofline of the dominant kernel (the GEMM) is reported per regime: the
+HBM-bound shapes and the tensor-bound shapes each run as their own chain of
+GEMM launches (again one graph, weights from HBM), and `achieved` is their
+algorithmic bytes (or operations) over that chain's time.  Per shape, an
+isolated run (L2 flushed, the kernels alone) gives the per-point breakdown.
 
 --impl reference times the CPU oracle (plain C, OpenMP) on a bounded sample
 of the same workload instead.
@@ -48,27 +54,12 @@ GEMM_SOURCES = ("qoq_gemm.cu", "qoq_layout.cuh", "qoq_ptx.cuh", "qoq_internal.h"
 
 
 def code_only(text: str) -> str:
-    """C/C++ source as the library build compiles it, for hashing: without
-    comments, without the trace build's `#ifdef QOQ_TRACE` branches (their
-    `#else` branches stay), and with whitespace collapsed.  A change of
-    wording or of trace-only code leaves the hash as it was."""
+    """C/C++ source without comments and with whitespace collapsed, for
+    hashing: a change of wording leaves the hash as it was."""
     import re
     text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
     text = re.sub(r"//[^\n]*", " ", text)
-    kept, stack = [], []  # stack: per open #if, whether we are in its trace-only branch
-    for line in text.splitlines():
-        d = line.strip()
-        if d.startswith("#if"):
-            stack.append(d.split()[:2] == ["#ifdef", "QOQ_TRACE"])
-        elif d.startswith("#else") or d.startswith("#elif"):
-            if stack:
-                stack[-1] = False
-        elif d.startswith("#endif"):
-            if stack:
-                stack.pop()
-        elif not any(stack):
-            kept.append(line)  # conditional directives themselves are not kept
-    return " ".join(" ".join(kept).split())
+    return " ".join(text.split())
 
 
 def gemm_source_hash(read=None) -> str:
@@ -90,10 +81,10 @@ def gemm_source_hash(read=None) -> str:
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="sweep", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--only", default=None,
                     help="restrict the workload to one shape name (for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -178,7 +169,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except OSError:
@@ -218,6 +209,55 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- our arm --
+def load_traffic(workload_name: str, path: str = None):
+    """The ncu DRAM-traffic record of this workload's GEMM, if its kernel
+    source hash still matches the current code: {capture shape name:
+    {...}} or {} (the counters describe that kernel and no later one)."""
+    prof = path or os.path.join(ROOT, "profiles", f"traffic_{workload_name}.json")
+    try:
+        with open(prof) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    if t.get("kernel_source_hash") != gemm_source_hash():
+        return {}
+    return t.get("captures", {})
+
+
+def regime_roofline(bound, shapes, ms, peaks, traffic):
+    """Roofline record of the GEMM over a chain of shapes of one regime
+    (all HBM-bound or all tensor-bound), timed back to back: `ms` is the
+    chain's time.  `traffic` comes from one ncu capture of a representative
+    shape of the regime, with that shape's algorithmic bytes beside it."""
+    n = len(shapes)
+    byt = sum(roofline.algorithmic_bytes(x.M, x.N, x.K, x.G) for x in shapes)
+    ops = sum(roofline.ops(x.M, x.N, x.K) for x in shapes)
+    if bound == "hbm":
+        achieved = byt / (ms * 1e-3) / 1e9
+        rl = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+              "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+              "peak_source": peaks["source"] + " (HBM copy)"}
+    else:
+        achieved = ops / (ms * 1e-3) / 1e12
+        rl = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peaks["int8_tops"], 1),
+              "unit": "TOPS", "frac": round(achieved / peaks["int8_tops"], 4), "traffic": None,
+              "peak_source": peaks["source"] + " (2 x bf16 cuBLAS burst)",
+              "frac_of_sustained_peak": round(achieved / peaks["int8_tops_sustained"], 4)}
+    rl.update({"kernel": "w4a8_gemm_kernel", "launches": n, "chain_us": round(ms * 1e3, 2),
+               "us_per_launch": round(ms * 1e3 / n, 3), "shapes": [x.name for x in shapes],
+               "algorithmic_bytes_per_launch": int(byt / n), "ops_per_launch": int(ops / n)})
+    rep = [k for k in traffic if k in {x.name for x in shapes}]
+    if rep:
+        t = traffic[rep[0]]
+        rl["traffic"] = t["dram_bytes"]
+        rl["traffic_shape"] = rep[0]
+        rl["traffic_algorithmic_bytes"] = t["algorithmic_bytes"]
+        rl["traffic_capture"] = t.get("capture")
+        if t.get("tensor_pipe_pct") is not None:
+            rl["ncu_tensor_pipe_pct"] = t["tensor_pipe_pct"]
+    return rl
+
+
 def run_ours(args, rank, world, local, dist):
     import w4a8_integer_gemm_b200 as q
 
@@ -226,6 +266,7 @@ def run_ours(args, rank, world, local, dist):
     q.lib()
     q.qoq_set_gemm_a_in_tmem(not args.a_smem)
     peaks = roofline.load_peaks()
+    P8, BW = peaks["int8_tops"] * 1e12, peaks["hbm_gbs"] * 1e9
     work = select(args)
     stream = torch.cuda.current_stream()
 
@@ -241,7 +282,8 @@ def run_ours(args, rank, world, local, dist):
         ws = torch.zeros(q.qoq_gemm_workspace_bytes(s.M, s.N, s.K, s.G), dtype=torch.uint8, device=dev)
         Xh = X.pin_memory()
         Yh = torch.empty(s.M, s.N, dtype=torch.float16, pin_memory=True)
-        cases.append(dict(s=s, packed=packed, X=Xd, X8=X8, s_x=s_x, Y=Y, ws=ws, Xh=Xh, Yh=Yh))
+        cases.append(dict(s=s, packed=packed, X=Xd, X8=X8, s_x=s_x, Y=Y, ws=ws, Xh=Xh, Yh=Yh,
+                          bound=roofline.bound(s.M, s.N, s.K, s.G, P8, BW)))
         del W
     torch.cuda.synchronize()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -254,92 +296,51 @@ def run_ours(args, rank, world, local, dist):
     # Otherwise L2 is flushed before every shape and each shape is timed
     # on its own (flush excluded).
     chained = wbytes > 3 * L2_BYTES // 2
+    # the GEMM's regimes, each chained on its own when its weights alone
+    # exceed the L2 the same way
+    regimes = {}
+    for b in ("hbm", "tensor"):
+        sub = [c for c in cases if c["bound"] == b]
+        if sub:
+            regimes[b] = sub
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     ev = [[E() for _ in range(4)] for _ in range(n_sh)]
-    es = [E(), E(), E(), E()]
+    es = [E(), E()]
 
-    def enqueue_step(st, gemm=True, quant=True, fused=True):
-        """Launch the step's kernels on stream st: per shape the layer call
-        (qoq_w4a8_linear), or the quantizer and the GEMM as separate calls."""
-        for c in cases:
-            if quant and gemm and fused:
+    def enqueue(st, subset, layer=True):
+        """Launch on stream st, per shape of `subset`, the layer call
+        (qoq_w4a8_linear: the quantizer kernel, then the GEMM kernel), or
+        the GEMM kernel alone."""
+        for c in subset:
+            if layer:
                 q.qoq_w4a8_linear(c["X"], c["packed"], X8=c["X8"], s_x=c["s_x"], Y=c["Y"], workspace=c["ws"],
                                   stream=st)
-                continue
-            if quant:
-                q.qoq_quant_act_per_token(c["X"], c["X8"], c["s_x"], stream=st)
-            if gemm:
+            else:
                 q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=st)
 
     graphs = {}
 
-    def one_step(eager=False):
-        """The hot path of every shape: activation quant, then the GEMM.
-        Returns the step's device time in ms."""
+    def timed(name, subset, layer=True, eager=False):
+        """Device time in ms of one pass over `subset`: back to back from a
+        graph when chained, else per shape after an L2 flush (summed)."""
         if chained:
             es[0].record(stream)
-            if "step" in graphs and not eager:
-                graphs["step"].replay()
+            if name in graphs and not eager:
+                graphs[name].replay()
             else:
-                enqueue_step(stream)
+                enqueue(stream, subset, layer)
             es[1].record(stream)
             torch.cuda.synchronize()
             return es[0].elapsed_time(es[1])
-        for j, c in enumerate(cases):
+        tot = 0.0
+        for c in subset:
+            j = cases.index(c)
             flush.zero_()
             ev[j][0].record(stream)
-            q.qoq_w4a8_linear(c["X"], c["packed"], X8=c["X8"], s_x=c["s_x"], Y=c["Y"], workspace=c["ws"],
-                              stream=stream)
+            enqueue(stream, [c], layer)
             ev[j][1].record(stream)
-        torch.cuda.synchronize()
-        return sum(ev[j][0].elapsed_time(ev[j][1]) for j in range(n_sh))
-
-    def one_launch_step():
-        """The same step with the layer call as one GEMM launch that
-        quantizes its own rows (replayed from a graph when chained), for
-        comparison."""
-        if chained:
-            es[0].record(stream)
-            graphs["one_launch"].replay()
-            es[1].record(stream)
             torch.cuda.synchronize()
-            return es[0].elapsed_time(es[1])
-        tot = 0.0
-        q.qoq_set_linear_in_kernel_quant(True)
-        try:
-            for j, c in enumerate(cases):
-                flush.zero_()
-                ev[j][0].record(stream)
-                q.qoq_w4a8_linear(c["X"], c["packed"], X8=c["X8"], s_x=c["s_x"], Y=c["Y"], workspace=c["ws"],
-                                  stream=stream)
-                ev[j][1].record(stream)
-            torch.cuda.synchronize()
-        finally:
-            q.qoq_set_linear_in_kernel_quant(False)
-        for j in range(n_sh):
             tot += ev[j][0].elapsed_time(ev[j][1])
-        return tot
-
-    def gemm_only():
-        """The GEMM kernel alone, the same way (roofline of the dominant kernel)."""
-        if chained:
-            es[2].record(stream)
-            if "gemm" in graphs:
-                graphs["gemm"].replay()
-            else:
-                enqueue_step(stream, quant=False)
-            es[3].record(stream)
-            torch.cuda.synchronize()
-            return es[2].elapsed_time(es[3])
-        tot = 0.0
-        for j, c in enumerate(cases):
-            flush.zero_()
-            ev[j][2].record(stream)
-            q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
-            ev[j][3].record(stream)
-        torch.cuda.synchronize()
-        for j in range(n_sh):
-            tot += ev[j][2].elapsed_time(ev[j][3])
         return tot
 
     def isolated(reps=3):
@@ -350,12 +351,11 @@ def run_ours(args, rank, world, local, dist):
             for _ in range(reps):
                 flush.zero_()
                 ev[j][0].record(stream)
-                q.qoq_w4a8_linear(c["X"], c["packed"], X8=c["X8"], s_x=c["s_x"], Y=c["Y"], workspace=c["ws"],
-                                  stream=stream)
+                enqueue(stream, [c], True)
                 ev[j][1].record(stream)
                 flush.zero_()
                 ev[j][2].record(stream)
-                q.qoq_w4a8_gemm(c["X8"], c["s_x"], c["packed"], Y=c["Y"], workspace=c["ws"], stream=stream)
+                enqueue(stream, [c], False)
                 ev[j][3].record(stream)
                 torch.cuda.synchronize()
                 st += ev[j][0].elapsed_time(ev[j][1])
@@ -363,33 +363,31 @@ def run_ours(args, rank, world, local, dist):
             out.append((st / reps, gm / reps))
         return out
 
+    chains = {"step": (cases, True)}
+    for b, sub in regimes.items():
+        chains["gemm_" + b] = (sub, False)
     for _ in range(max(3, args.warmup)):
-        one_step()
-        gemm_only()
+        for name, (sub, layer) in chains.items():
+            timed(name, sub, layer)
     torch.cuda.synchronize()
     if q.qoq_device_error() != q.QOQ_OK:
         raise RuntimeError("device error during warm-up")
-    # Decode-sized steps are launch-bound when every kernel is launched from
-    # Python; a serving loop replays them as one CUDA graph, and so does the
-    # timed region (the eager step time is reported beside it).
+    # A serving loop replays a step's launches as one CUDA graph, and so does
+    # the timed region (the eager step time is reported beside it).
     eager_ms = None
     if chained and not args.eager:
-        eager_ms = statistics.median(one_step(eager=True) for _ in range(max(3, args.warmup)))
+        eager_ms = statistics.median(timed("step", cases, True, eager=True) for _ in range(max(3, args.warmup)))
         cap = torch.cuda.Stream(device=dev)
         cap.wait_stream(stream)
-        for name, kw in (("step", {}), ("gemm", {"quant": False}), ("one_launch", {})):
+        for name, (sub, layer) in chains.items():
             g = torch.cuda.CUDAGraph()
-            q.qoq_set_linear_in_kernel_quant(name == "one_launch")
-            try:
-                with torch.cuda.graph(g, stream=cap):
-                    enqueue_step(cap, **kw)
-            finally:
-                q.qoq_set_linear_in_kernel_quant(False)
+            with torch.cuda.graph(g, stream=cap):
+                enqueue(cap, sub, layer)
             graphs[name] = g
         stream.wait_stream(cap)
         for _ in range(max(3, args.warmup)):
-            one_step()
-            gemm_only()
+            for name, (sub, layer) in chains.items():
+                timed(name, sub, layer)
         torch.cuda.synchronize()
         if q.qoq_device_error() != q.QOQ_OK:
             raise RuntimeError("device error while warming up the CUDA graphs")
@@ -400,60 +398,40 @@ def run_ours(args, rank, world, local, dist):
         torch.cuda.synchronize()
         t_wall = time.perf_counter()
         for _ in range(args.steps):
-            step_ms.append(one_step())
+            step_ms.append(timed("step", cases, True))
         torch.cuda.synchronize()
         barrier(dist)
         wall = time.perf_counter() - t_wall
     clocks = clk.summary()
-    g_ms_total = sum(gemm_only() for _ in range(args.steps)) / args.steps
-    one_ms = statistics.median(one_launch_step() for _ in range(args.steps)) if (graphs or not chained) else None
+    chain_ms = {b: statistics.median(timed("gemm_" + b, sub, False) for _ in range(args.steps))
+                for b, sub in regimes.items()}
     iso = isolated()
     if q.qoq_device_error() != q.QOQ_OK:
         raise RuntimeError("device error in the timed region")
 
     per = []
-    tot_ops = g_bytes = 0.0
+    tot_ops = 0.0
     for j, c in enumerate(cases):
         s = c["s"]
         pair_ms, gm_ms = iso[j]
         ops = roofline.ops(s.M, s.N, s.K)
         byt = roofline.algorithmic_bytes(s.M, s.N, s.K, s.G)
-        roof = roofline.roofline_ops_per_s(s.M, s.N, s.K, s.G, peaks["int8_tops"] * 1e12, peaks["hbm_gbs"] * 1e9)
+        roof = roofline.roofline_ops_per_s(s.M, s.N, s.K, s.G, P8, BW)
         tops = ops / (gm_ms * 1e-3) / 1e12
-        per.append({"shape": s.name, "M": s.M, "K": s.K, "N": s.N, "G": s.G,
+        per.append({"shape": s.name, "M": s.M, "K": s.K, "N": s.N, "G": s.G, "bound": c["bound"],
                     "isolated_step_us": round(pair_ms * 1e3, 2), "isolated_gemm_us": round(gm_ms * 1e3, 2),
                     "isolated_gemm_tops": round(tops, 2), "isolated_gemm_gbs": round(byt / (gm_ms * 1e-3) / 1e9, 1),
-                    "roofline_tops": round(roof / 1e12, 2), "isolated_frac": round(tops * 1e12 / roof, 4),
-                    "bound": roofline.bound(s.M, s.N, s.K, s.G, peaks["int8_tops"] * 1e12,
-                                            peaks["hbm_gbs"] * 1e9)})
+                    "roofline_tops": round(roof / 1e12, 2), "isolated_frac": round(tops * 1e12 / roof, 4)})
         tot_ops += ops
-        g_bytes += byt
     tot_ms = statistics.median(step_ms)
     ms_step, value = aggregate(tot_ops, tot_ms, world, dist)
-    g_ms = g_ms_total
-    # roofline of the dominant kernel (the GEMM), averaged per launch
-    n_hbm = sum(1 for p in per if p["bound"] == "hbm")
-    bound = "hbm" if n_hbm * 2 >= len(per) else "tensor"
-    if bound == "hbm":
-        achieved = g_bytes / (g_ms * 1e-3) / 1e9
-        rl = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-              "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
-    else:
-        achieved = sum(roofline.ops(p["M"], p["N"], p["K"]) for p in per) / (g_ms * 1e-3) / 1e12
-        rl = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peaks["int8_tops"], 1),
-              "unit": "TOPS", "frac": round(achieved / peaks["int8_tops"], 4), "traffic": None}
-    rl["peak_source"] = peaks["source"] + (" (HBM copy)" if bound == "hbm" else " (bf16 cuBLAS x2, burst)")
-    rl["kernel"] = "w4a8_gemm_kernel"
-    rl["algorithmic_bytes_per_launch"] = int(g_bytes / n_sh)
-    prof = os.path.join(ROOT, "profiles", f"traffic_{args.workload}.json")
-    if os.path.exists(prof):
-        try:
-            t = json.load(open(prof))
-            if t.get("kernel_source_hash") == gemm_source_hash():
-                rl["traffic"] = t.get("dram_bytes_per_gemm_launch")
-                rl["traffic_capture"] = t.get("capture")
-        except (OSError, ValueError):
-            pass
+    traffic = load_traffic(args.workload)
+    by_bound = {b: regime_roofline(b, [c["s"] for c in sub], chain_ms[b], peaks, traffic)
+                for b, sub in regimes.items()}
+    # the dominant kernel's regime: where the GEMM spends most of the step
+    dom = max(by_bound, key=lambda b: by_bound[b]["chain_us"])
+    rl = dict(by_bound[dom])
+    rl["by_bound"] = by_bound
 
     # end to end through the public API from pinned host memory
     e2e = None
@@ -467,19 +445,21 @@ def run_ours(args, rank, world, local, dist):
         h2d = sum(c["Xh"].numel() * 2 for c in cases)
         d2h = sum(c["Yh"].numel() * 2 for c in cases)
         tot = 0.0
-        for it in range(args.warmup + args.steps):
+        for it in range(max(3, args.warmup) + args.steps):
             for j, c in enumerate(cases):
                 flush.zero_()
                 e2e_ev[j][0].record(stream)
                 q.w4a8_linear_host(c["Xh"], layer_like[j], y_host=c["Yh"], stream=stream)
                 e2e_ev[j][1].record(stream)
             torch.cuda.synchronize()
-            if it >= args.warmup:
+            if it >= max(3, args.warmup):
                 tot += sum(e2e_ev[j][0].elapsed_time(e2e_ev[j][1]) for j in range(n_sh))
         e2e_ms = max_over_ranks(tot / args.steps, dist)
         e2e = {"value": round(world * tot_ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": round(e2e_ms, 4)}
+               "ms_per_step": round(e2e_ms, 4),
+               "call": "w4a8_linear_host per shape: X pinned host -> device, layer call, Y -> pinned host, "
+                       "stream synchronize"}
 
     out = {
         "metric": "W4A8 GEMM TOPS (act-quant + GEMM) and % of roofline vs batch M",
@@ -491,15 +471,14 @@ def run_ours(args, rank, world, local, dist):
         "config": {"workload": work.name, "shapes": [p["shape"] for p in per],
                    "l2": ("inputs larger than L2: %d MB of distinct packed weights per step, no flush" % (wbytes >> 20))
                          if chained else "flushed before every shape (256 MB write), flush excluded from timing",
-                   "timing": ("median step of %d; GEMM-only roofline from the same %s runs" %
+                   "timing": ("median step of %d; GEMM roofline per regime from chains of the same %s runs" %
                               (args.steps, "back-to-back" if chained else "flushed")),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": ("cuda_graph (one graph per step, programmatic dependent launch between kernels)"
                               if graphs else "eager (every kernel launched from Python)"),
                    "eager_ms_per_step": None if eager_ms is None else round(eager_ms, 5),
                    "kernels": ("per shape qoq_w4a8_linear: the per-token quantizer kernel, then the GEMM kernel "
-                               "(programmatic dependent launch)"),
-                   "one_launch_ms_per_step": None if one_ms is None else round(one_ms, 5)},
+                               "(programmatic dependent launch)")},
         "roofline": rl, "points": per, "clocks": clocks, "e2e": e2e,
         "gpu_launches": 2 * n_sh * args.steps,
         "a_operand": "smem" if args.a_smem else "tmem",

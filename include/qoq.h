@@ -134,11 +134,17 @@ QOQ_API size_t qoq_packed_weight_bytes(int N, int K, int group_size);
  *   s_c    device, uint16_t [N] FP16 bits, written.
  *   s_g    device, uint8_t [N/128][K/group_size][128], written.
  *   zs     device, uint8_t [N/128][K/group_size][128], written.
+ *   z_dbg  device, uint8_t [N][K/group_size], or NULL. When given, the zero
+ *          points z (0..15) are written there, channel-major (inspection and
+ *          parity tests; the GEMM needs only zs).
+ *   q_dbg  device, uint8_t [N][K], or NULL (16-byte aligned when given).
+ *          When given, the canonical codes q (0..15) are written there, one
+ *          per byte, in the natural [n][k] order (inspection and parity).
  * The result is deterministic and bit-identical on every call.
  */
 QOQ_API int qoq_pack_weights(const float *W, int N, int K, int group_size,
                      uint8_t *Wp, uint16_t *s_c, uint8_t *s_g, uint8_t *zs,
-                     void *stream);
+                     uint8_t *z_dbg, uint8_t *q_dbg, void *stream);
 
 /* Per-token symmetric INT8 activation quantization.
  *
@@ -152,10 +158,16 @@ QOQ_API int qoq_pack_weights(const float *W, int N, int K, int group_size,
  *   X      device, uint16_t [M][K] FP16 bits, read only. Must be finite.
  *   X8     device, int8_t [M][K], written.
  *   s_x    device, uint16_t [M] FP16 bits, written.
+ *   rowsum device, int32_t [M], or NULL (4-byte aligned when given). When
+ *          given, rowsum[m] = sum_k X8[m][k] is written there. It is the term
+ *          a zero point multiplies when the zero compensation is applied after
+ *          the products instead of before them; qoq_w4a8_gemm subtracts z*s_g
+ *          from the weights before the products (multiply first, subtract
+ *          afterward), so it takes no rowsum.
  * K follows the GEMM limits above (multiple of 128, at most 65536).
  */
 QOQ_API int qoq_quant_act_per_token(const uint16_t *X, int M, int K,
-                            int8_t *X8, uint16_t *s_x, void *stream);
+                            int8_t *X8, uint16_t *s_x, int32_t *rowsum, void *stream);
 
 /* Bytes of scratch workspace qoq_w4a8_gemm needs for this shape.
  *

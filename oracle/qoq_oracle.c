@@ -28,7 +28,7 @@
  *           "High-Throughput Native INT8 Tensor Core GEMMs": INT32
  *           accumulation, scales applied once after the inner product.
  *
- * Readings of points the pages leave open (each is also listed in the design doc):
+ * Readings of points the pages leave open:
  *   - "round" is round-half-to-even (IEEE rint in the default mode).
  *   - s_c and s_x are stored as FP16 (round to nearest even) and the stored,
  *     rounded value is the one used to quantize.

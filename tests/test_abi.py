@@ -105,10 +105,12 @@ def test_invalid_arguments_rejected_on_host(L):
     assert call(wsb=16) == INVALID
     assert call(acc=B) == INVALID
     assert call(M=0) == 0                        # empty problem: nothing to do
-    assert L.qoq_quant_act_per_token(A, 4, 100, A, A, None) == INVALID
-    assert L.qoq_quant_act_per_token(A, 0, 512, A, A, None) == 0
-    assert L.qoq_pack_weights(A, 512, 512, 100, A, A, A, A, None) == INVALID
-    assert L.qoq_pack_weights(B, 512, 512, 128, A, A, A, A, None) == INVALID
+    assert L.qoq_quant_act_per_token(A, 4, 100, A, A, None, None) == INVALID
+    assert L.qoq_quant_act_per_token(A, 0, 512, A, A, None, None) == 0
+    assert L.qoq_quant_act_per_token(A, 4, 512, A, A, _fake(0x10002), None) == INVALID   # rowsum misaligned
+    assert L.qoq_pack_weights(A, 512, 512, 100, A, A, A, A, None, None, None) == INVALID
+    assert L.qoq_pack_weights(B, 512, 512, 128, A, A, A, A, None, None, None) == INVALID
+    assert L.qoq_pack_weights(A, 512, 512, 128, A, A, A, A, None, B, None) == INVALID     # q_dbg misaligned
     assert L.qoq_dequant_weights_i8(A, A, A, 512, 512, 3, A, None) == INVALID
     assert L.qoq_set_gemm_a_in_tmem(2) == INVALID
     assert L.qoq_set_gemm_cta_pairs(2) == INVALID
@@ -133,3 +135,37 @@ def test_invalid_arguments_rejected_on_host(L):
     assert fcall(10, B) == INVALID                # s_x
     assert fcall(13, 16) == INVALID               # workspace too small
     assert fcall(1, 0) == 0                       # M = 0: nothing to do
+
+
+def test_noalloc_scratch_bound_and_checks(L):
+    """The no-alloc entry point: its built-in buffer holds the scratch of
+    every shape up to 128 tokens (the header's promise), and it applies the
+    same host-side checks as qoq_w4a8_gemm before touching any device."""
+    import w4a8_integer_gemm_b200 as q
+    for N in (128, 4096, 1 << 20):
+        for K in (128, 4096, 65536):
+            for G in (128, K):
+                for M in (1, 16, 64, 65, 128):
+                    assert 0 < q.qoq_gemm_workspace_bytes(M, N, K, G) <= q.QOQ_NOALLOC_SCRATCH_BYTES, (M, N, K, G)
+    A = _fake(0x10000)
+    B = _fake(0x10001)
+    INVALID = -1
+    f = L.qoq_w4a8_gemm_noalloc
+    ok = [A] * 6 + [16, 512, 512, 128, A, None]
+
+    def call(i, v):
+        a = list(ok)
+        a[i] = v
+        return f(*a)
+
+    for i in range(6):
+        assert call(i, None) == INVALID          # each input pointer null
+        assert call(i, B) == INVALID             # each input pointer misaligned
+    assert call(10, None) == INVALID             # Y
+    assert call(10, B) == INVALID
+    assert call(9, 64) == INVALID                # group size neither 128 nor K
+    assert call(9, 256) == INVALID
+    assert call(8, 500) == INVALID               # K
+    assert call(7, 500) == INVALID               # N
+    assert call(6, -1) == INVALID                # M
+    assert call(6, 0) == 0                       # empty problem

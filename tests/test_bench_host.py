@@ -46,15 +46,6 @@ def test_code_only_strips_both_comment_forms():
     assert bench.code_only("int a; // x\n/* y\n z */ int  b;") == "int a; int b;"
 
 
-def test_trace_only_code_leaves_the_hash_but_its_else_branch_does_not():
-    src = "int a;\n#ifdef QOQ_TRACE\nint t;\n#else\nint p;\n#endif\nint b;"
-    assert bench.code_only(src) == "int a; int p; int b;"
-    assert bench.code_only(src.replace("int t;", "int t2; int t3;")) == bench.code_only(src)
-    assert bench.code_only(src.replace("int p;", "int p2;")) != bench.code_only(src)
-    # other conditionals keep both branches
-    assert bench.code_only("#ifndef X\n#define X 1\n#endif\nint d;") == "#define X 1 int d;"
-
-
 def test_single_core_oracle_leg_restores_threads():
     import oracle
     from w4a8_integer_gemm_b200 import workloads as wl

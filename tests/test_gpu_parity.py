@@ -62,6 +62,17 @@ def test_act_quant_bit_exact(M, K):
     assert np.array_equal(_u16(s_x)[:M], rs)
 
 
+@pytest.mark.parametrize("M,K", [(1, 128), (16, 512), (33, 4096), (5, 24576)])
+def test_act_quant_rowsum_exact(M, K):
+    """The optional rowsum output equals the sum of the oracle's INT8 row."""
+    X = wl.make_activations(M, K, wl.LLAMA, seed=150 + M)
+    rowsum = torch.full((M,), 12345, dtype=torch.int32, device="cuda")
+    X8, s_x = q.qoq_quant_act_per_token(X.cuda(), rowsum=rowsum)
+    rX8, rs = oracle.quant_act(X.numpy())
+    assert np.array_equal(X8.cpu().numpy(), rX8)
+    assert np.array_equal(rowsum.cpu().numpy(), rX8.astype(np.int64).sum(axis=1))
+
+
 def test_act_quant_degenerate_rows():
     X = torch.zeros(4, 256, dtype=torch.float16)
     X[1, :] = 6e-8
@@ -83,6 +94,20 @@ def test_pack_bit_exact(N, K, G):
     assert np.array_equal(_u16(p.s_c), r["s_c"])
     assert np.array_equal(p.s_g.cpu().numpy(), tables_reference(r["s_g"]))
     assert np.array_equal(p.zs.cpu().numpy(), tables_reference(r["zs"]))
+    assert np.array_equal(p.Wp.cpu().numpy(), pack_reference(r["q"], G, r["s_g"], r["zs"]))
+
+
+@pytest.mark.parametrize("N,K,G", [(128, 128, 128), (384, 4096, 128), (256, 1024, 1024)])
+def test_pack_debug_outputs_exact(N, K, G):
+    """The optional canonical codes and zero points equal the oracle's."""
+    W = wl.make_weights(N, K, wl.LLAMA, seed=250 + N + K)
+    z_dbg = torch.full((N, K // G), 99, dtype=torch.uint8, device="cuda")
+    q_dbg = torch.full((N, K), 99, dtype=torch.uint8, device="cuda")
+    p = q.qoq_pack_weights(W.cuda(), G, z_dbg=z_dbg, q_dbg=q_dbg)
+    r = oracle.quantize_weights(W.numpy(), G)
+    assert np.array_equal(q_dbg.cpu().numpy(), r["q"])
+    assert np.array_equal(z_dbg.cpu().numpy(), r["z"])
+    # the tables written beside them are unchanged by the extra outputs
     assert np.array_equal(p.Wp.cpu().numpy(), pack_reference(r["q"], G, r["s_g"], r["zs"]))
 
 

@@ -43,8 +43,8 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "qoq_status_string": (ctypes.c_char_p, [_I]),
     "qoq_packed_weight_bytes": (_SZ, [_I, _I, _I]),
-    "qoq_pack_weights": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P]),
-    "qoq_quant_act_per_token": (_I, [_P, _I, _I, _P, _P, _P]),
+    "qoq_pack_weights": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "qoq_quant_act_per_token": (_I, [_P, _I, _I, _P, _P, _P, _P]),
     "qoq_gemm_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "qoq_w4a8_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "qoq_w4a8_gemm_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
@@ -160,8 +160,16 @@ class PackedWeights:
 
 
 def qoq_pack_weights(W: torch.Tensor, group_size: int, out: Optional[PackedWeights] = None,
-                     stream=None) -> PackedWeights:
+                     stream=None, z_dbg: Optional[torch.Tensor] = None,
+                     q_dbg: Optional[torch.Tensor] = None) -> PackedWeights:
+    """W fp32 [N, K] -> packed weights.  z_dbg (uint8 [N, K/G]) and q_dbg
+    (uint8 [N, K]), when given, receive the zero points and the canonical
+    codes for inspection."""
     _need(W, torch.float32, "W")
+    if z_dbg is not None:
+        _need(z_dbg, torch.uint8, "z_dbg")
+    if q_dbg is not None:
+        _need(q_dbg, torch.uint8, "q_dbg")
     N, K = W.shape
     G = int(group_size)
     if out is None:
@@ -173,21 +181,25 @@ def qoq_pack_weights(W: torch.Tensor, group_size: int, out: Optional[PackedWeigh
                             torch.empty(max(N // 128, 1), ng, 128, dtype=torch.uint8, device=dev),
                             torch.empty(max(N // 128, 1), ng, 128, dtype=torch.uint8, device=dev), N, K, G)
     st = lib().qoq_pack_weights(_ptr(W), N, K, G, _ptr(out.Wp), _ptr(out.s_c), _ptr(out.s_g),
-                                _ptr(out.zs), _stream(stream))
+                                _ptr(out.zs), _ptr(z_dbg), _ptr(q_dbg), _stream(stream))
     _check("qoq_pack_weights", st)
     return out
 
 
 def qoq_quant_act_per_token(X: torch.Tensor, X8: Optional[torch.Tensor] = None,
-                            s_x: Optional[torch.Tensor] = None, stream=None):
-    """X fp16 [M, K] -> (X8 int8 [M, K], s_x int16 [M] FP16 bits)."""
+                            s_x: Optional[torch.Tensor] = None, stream=None,
+                            rowsum: Optional[torch.Tensor] = None):
+    """X fp16 [M, K] -> (X8 int8 [M, K], s_x int16 [M] FP16 bits).  rowsum
+    (int32 [M]), when given, receives sum_k X8[m, k]."""
     _need(X, torch.float16, "X")
+    if rowsum is not None:
+        _need(rowsum, torch.int32, "rowsum")
     M, K = X.shape
     if X8 is None:
         X8 = torch.empty(M, K, dtype=torch.int8, device=X.device)
     if s_x is None:
         s_x = torch.empty(max(M, 8), dtype=torch.int16, device=X.device)
-    st = lib().qoq_quant_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(s_x), _stream(stream))
+    st = lib().qoq_quant_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(s_x), _ptr(rowsum), _stream(stream))
     _check("qoq_quant_act_per_token", st)
     return X8, s_x
 

@@ -19,6 +19,15 @@ constexpr int kMaxK = 65536;
 constexpr int kMaxN = 1 << 20;
 constexpr int kMaxM = 1 << 24;
 
+int from_cuda(cudaError_t e)
+{
+    return e == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
+}
+
+}  // namespace
+
+namespace qoq {
+
 bool aligned16(const void *p)
 {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
@@ -32,6 +41,11 @@ bool valid_nk(int N, int K)
 bool valid_group(int K, int G)
 {
     return G == 128 || G == K;
+}
+
+bool gemm_a_in_tmem()
+{
+    return g_a_in_tmem.load() != 0;
 }
 
 // Compute capability 10.0 check for the current device, cached per device.
@@ -53,12 +67,12 @@ int check_device()
     return c == 1 ? QOQ_OK : QOQ_ERR_UNSUPPORTED;
 }
 
-int from_cuda(cudaError_t e)
-{
-    return e == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
-}
+}  // namespace qoq
 
-}  // namespace
+using qoq::aligned16;
+using qoq::check_device;
+using qoq::valid_group;
+using qoq::valid_nk;
 
 extern "C" {
 
@@ -82,25 +96,30 @@ size_t qoq_packed_weight_bytes(int N, int K, int group_size)
 }
 
 int qoq_pack_weights(const float *W, int N, int K, int group_size, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g,
-                     uint8_t *zs, void *stream)
+                     uint8_t *zs, uint8_t *z_dbg, uint8_t *q_dbg, void *stream)
 {
     if (!valid_nk(N, K) || !valid_group(K, group_size)) return QOQ_ERR_INVALID_ARG;
     if (!W || !Wp || !s_c || !s_g || !zs) return QOQ_ERR_INVALID_ARG;
-    if (!aligned16(W) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) || !aligned16(zs))
+    if (!aligned16(W) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) || !aligned16(zs) ||
+        (q_dbg && !aligned16(q_dbg)))
         return QOQ_ERR_INVALID_ARG;
     const int dev = check_device();
     if (dev != QOQ_OK) return dev;
-    return from_cuda(qoq::launch_pack(W, N, K, group_size, Wp, s_c, s_g, zs, (cudaStream_t)stream));
+    return from_cuda(
+        qoq::launch_pack(W, N, K, group_size, Wp, s_c, s_g, zs, z_dbg, q_dbg, (cudaStream_t)stream));
 }
 
-int qoq_quant_act_per_token(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, void *stream)
+int qoq_quant_act_per_token(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, int32_t *rowsum,
+                            void *stream)
 {
     if (M < 0 || M > kMaxM || K < 128 || K > kMaxK || K % 128 != 0) return QOQ_ERR_INVALID_ARG;
     if (M == 0) return QOQ_OK;
-    if (!X || !X8 || !s_x || !aligned16(X) || !aligned16(X8) || !aligned16(s_x)) return QOQ_ERR_INVALID_ARG;
+    if (!X || !X8 || !s_x || !aligned16(X) || !aligned16(X8) || !aligned16(s_x) ||
+        (rowsum && (reinterpret_cast<uintptr_t>(rowsum) & 3u)))
+        return QOQ_ERR_INVALID_ARG;
     const int dev = check_device();
     if (dev != QOQ_OK) return dev;
-    return from_cuda(qoq::launch_act_quant(X, M, K, X8, s_x, (cudaStream_t)stream));
+    return from_cuda(qoq::launch_act_quant(X, M, K, X8, s_x, rowsum, (cudaStream_t)stream));
 }
 
 size_t qoq_gemm_workspace_bytes(int M, int N, int K, int group_size)
@@ -126,7 +145,7 @@ int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, cons
     if (dev != QOQ_OK) return dev;
     int tmap_status = 0;
     cudaError_t e = qoq::launch_gemm(X8, s_x, Wp, s_c, s_g, zs, M, N, K, group_size, Y, acc_dbg, workspace,
-                                     g_a_in_tmem.load() != 0, (cudaStream_t)stream, &tmap_status);
+                                     qoq::gemm_a_in_tmem(), (cudaStream_t)stream, &tmap_status);
     if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
     return from_cuda(e);
 }
@@ -152,11 +171,11 @@ int qoq_w4a8_linear(const uint16_t *X, int M, int N, int K, int group_size, cons
     // input (same results).
     const bool in_kernel = g_linear_in_kernel_quant.load() != 0 && M <= qoq::kFusedMaxRows;
     if (!in_kernel) {
-        const cudaError_t eq = qoq::launch_act_quant(X, M, K, X8, s_x, (cudaStream_t)stream);
+        const cudaError_t eq = qoq::launch_act_quant(X, M, K, X8, s_x, nullptr, (cudaStream_t)stream);
         if (eq != cudaSuccess) return from_cuda(eq);
     }
     cudaError_t e = qoq::launch_gemm(X8, s_x, Wp, s_c, s_g, zs, M, N, K, group_size, Y, nullptr, workspace,
-                                     g_a_in_tmem.load() != 0, (cudaStream_t)stream, &tmap_status,
+                                     qoq::gemm_a_in_tmem(), (cudaStream_t)stream, &tmap_status,
                                      in_kernel ? X : nullptr);
     if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
     return from_cuda(e);
@@ -208,29 +227,6 @@ int qoq_set_linear_in_kernel_quant(int enable)
     return QOQ_OK;
 }
 
-#ifdef QOQ_TRACE
-// Trace builds only: a device buffer of [ctas][256] uint64 that later GEMM
-// launches fill with global-timer marks.
-__attribute__((visibility("default"))) int qoq_debug_set_trace(void *buf)
-{
-    qoq::g_trace_buffer = reinterpret_cast<unsigned long long *>(buf);
-    return QOQ_OK;
-}
-
-// Trace builds only: the first timed-out wait's site and the barrier layout.
-__attribute__((visibility("default"))) int qoq_debug_timeout_site(unsigned long long *out2)
-{
-    return qoq::debug_timeout_site(out2, out2 + 1) == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
-}
-
-// Trace builds only: one thread writes the global timer to *dst.
-__attribute__((visibility("default"))) int qoq_debug_stamp(void *dst, void *stream)
-{
-    return qoq::debug_stamp(reinterpret_cast<unsigned long long *>(dst), (cudaStream_t)stream) == cudaSuccess
-               ? QOQ_OK
-               : QOQ_ERR_CUDA;
-}
-#endif
 
 int qoq_device_error(void *stream)
 {

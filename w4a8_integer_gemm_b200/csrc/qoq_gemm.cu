@@ -84,9 +84,6 @@
 namespace qoq {
 
 __device__ int g_dev_error;  // non-zero after a bounded wait ran out
-#ifdef QOQ_TRACE
-__device__ unsigned long long g_bar_info;  // trace builds: barrier base and ring depths of the last launch
-#endif
 
 struct GemmArgs {
     const uint8_t *Wp;
@@ -111,24 +108,7 @@ struct GemmArgs {
     int ngroups;       // K / G
     int total;         // tiles * ks units
     unsigned long long timeout_ns;  // longest any one wait may last
-#ifdef QOQ_TRACE
-    unsigned long long *trace;  // [cta][256] clock marks (trace builds only)
-#endif
 };
-
-// Timeline marks for the trace build (compiled out otherwise).  Slot 255
-// holds the CTA's global-timer entry time; the other marks are SM clock
-// cycles since the CTA's entry.
-#ifdef QOQ_TRACE
-#define QOQ_MARK(idx)                                                                              \
-    do {                                                                                           \
-        if (a.trace) a.trace[(size_t)blockIdx.x * 256 + (idx)] = clock64() - trace_t0;             \
-    } while (0)
-#else
-#define QOQ_MARK(idx) \
-    do {              \
-    } while (0)
-#endif
 
 // Weight stages issued by the setup thread before the CTA-wide barrier.
 constexpr int kPrologueStages = 2;
@@ -239,7 +219,6 @@ __device__ __forceinline__ bool wait_count_gpu(const int *p, int want, volatile 
     while (ld_acquire_gpu(p) < want) {
         if (*abort) return false;
         if (global_timer_ns() - start > budget_ns) {
-            QOQ_RECORD_TIMEOUT(0xF00001u);
             *abort = 1;
             return false;
         }
@@ -367,8 +346,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     // ring slots a producer has filled, and the phase parity of each slot's
     // latest fill (drained on the way out of an aborted CTA)
     uint32_t issued = 0, issued_par = 0;
-    int tj = 0;  // trace: per-role unit counter
-    (void)tj;
     // The weight copy of unit u (tile u / ks, K block u % ks) into W slot s:
     // the kCh chunks of the K block are contiguous in the packed buffer,
     // with their group tables when G = 128, so one bulk copy brings them.
@@ -389,13 +366,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     // only a few, since the whole CTA waits for this thread at the barrier
     const int n_pro = min(min(SW, kPrologueStages), i_end - i_begin);
 
-#ifdef QOQ_TRACE
-    if (blockIdx.x == 0 && threadIdx.x == 0)
-        g_bar_info = (unsigned long long)bar0 | ((unsigned long long)SW << 32) | ((unsigned long long)SX << 40) |
-                     ((unsigned long long)C::kAccBufs << 48);
-    const long long trace_t0 = clock64();
-    if (threadIdx.x == 0 && a.trace) a.trace[(size_t)blockIdx.x * 256 + 255] = global_timer_ns();
-#endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < SW; ++s) {
             mbar_init(wfull_bar(s), 1);
@@ -418,8 +388,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         // weights stream from here on, while the rest of the CTA sets up
         for (int j = 0; j < n_pro; ++j) {
             issue_weights(i_begin + j, j, 0u);
-            if (tj < 16) QOQ_MARK(16 + tj);
-            ++tj;
         }
     }
     if (threadIdx.x == 64) prefetch_tmap(&tmap_x);
@@ -448,7 +416,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     // commits; the tcgen05 fences around the waits order the tensor-memory
     // accesses, as with one CTA)
     auto wait_x = [&](uint32_t bar, uint32_t parity) { return wait_bounded(bar, parity, abort_flag, budget); };
-    QOQ_MARK(1);
 
     if (warp == 0) {
         // ---------------------------------------------- weight producer --
@@ -457,11 +424,8 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             int s = n_pro == SW ? 0 : n_pro;
             uint32_t ph = (n_pro == SW) ? 1u : 0u;
             for (int u = i_begin + n_pro; u < i_end; ++u) {
-                if (tj == n_pro) QOQ_MARK(5);
                 if (!wait_bounded(wempty_bar(s), ph ^ 1u, abort_flag, budget)) break;
                 issue_weights(u, s, ph);
-                if (tj < 16) QOQ_MARK(16 + tj);
-                ++tj;
                 if (++s == SW) {
                     s = 0;
                     ph ^= 1u;
@@ -472,12 +436,10 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         // ------------------------------------------------- X8 producer --
         if (lane == 0) {
             grid_dependency_wait();  // X8 comes from the preceding kernel
-            QOQ_MARK(10);
             bool ok = true;
             if (a.X) {
                 // one-launch layer call: X8 is written by this grid's epilogue warps
                 ok = wait_count_gpu(a.ws_ready, a.M, abort_flag, budget);
-                QOQ_MARK(11);
                 fence_proxy_async_global();
                 if (ok) mbar_arrive(xready_bar);
             }
@@ -509,8 +471,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                             tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN,
                                         afull_bar(s));
                     }
-                    if (tj < 16) QOQ_MARK(32 + tj);
-                    ++tj;
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
                     if (++s == SX) {
@@ -543,7 +503,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                         break;
                     }
                     tc_fence_after();
-                    if (tj < 16) QOQ_MARK(112 + tj);
                     const uint32_t st = sbase + s * C::kXSlot;
 #pragma unroll
                     for (int j = 0; j < 4 * kCh; ++j) {
@@ -564,8 +523,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     } else {
                         mma_commit(xaempty_bar(s));
                     }
-                    if (tj < 16) QOQ_MARK(128 + tj);
-                    ++tj;
                     if (++s == SX) {
                         s = 0;
                         ph ^= 1u;
@@ -583,7 +540,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 }
                 i = t * ks + ks1;
             }
-            QOQ_MARK(3);
             // all MMAs this thread issued have completed once this arrives
             if constexpr (PAIR) {
                 mma_commit_pair(mmadone_bar, 0x1);
@@ -631,7 +587,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     }
                 }
                 if (!wait_bounded(wfull_bar(sw), pw, abort_flag, budget)) break;
-                if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(48 + tj);
                 const uint8_t *wsl = smem + C::kWOff + sw * C::kWSlot;
                 uint4 v[kCh][4];
                 uint32_t sg[kCh], zsv[kCh];
@@ -655,13 +610,11 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(wempty_bar(sw));  // the weight slot may be refilled now
-                if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(64 + tj);
                 // A slot sx is free once the MMAs of its previous use have
                 // completed; the X8 tiles need not have landed (the MMA
                 // issuer waits for those on afull)
                 if (!wait_x(xaempty_bar(sx), px ^ 1u)) break;
                 tc_fence_after();
-                if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(80 + tj);
 #pragma unroll
                 for (int c = 0; c < kCh; ++c) {
                     const uint32_t sgc = sg[c];
@@ -694,8 +647,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                         mbar_arrive(afull_bar(sx));
                     }
                 }
-                if (warp == 4 && lane == 0 && tj < 16) QOQ_MARK(96 + tj);
-                ++tj;
             }
             if (++sw == SW) {
                 sw = 0;
@@ -716,7 +667,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
         int ab = 0;          // accumulator of the current tile
         uint32_t accph = 0;  // its phase parity
         grid_dependency_wait();  // s_x (or X) comes from the preceding kernel
-        if (threadIdx.x == kEpiWarp0 * 32) QOQ_MARK(6);
         if (a.X && eg == 0) {
             // Fused call: the four epilogue warps of each CTA quantize token
             // rows cta, cta + P, ... together (128 threads per row, the
@@ -745,7 +695,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     for (int c = 0; c < 4; ++c) amax = fmaxf(amax, absmax8(t[c]));
                 }
                 amax = warp_max(amax);
-                if (et == 0 && row == cta) QOQ_MARK(7);
                 if (lane == 0) rowmax[warp - kEpiWarp0] = amax;
                 named_barrier(1, 128);
                 amax = fmaxf(fmaxf(rowmax[0], rowmax[1]), fmaxf(rowmax[2], rowmax[3]));
@@ -767,23 +716,18 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                         if (v0 + c * 128 < nvec) dst[v0 + c * 128] = quant8(t[c], sxf);
                 }
                 if (et == 0) a.s_xw[row] = sxh;
-                if (et == 0 && row == cta) QOQ_MARK(12);
                 // the X8 tiles are read back by TMA (the async proxy); after
                 // the barrier one release covers the row's stores by all 128
                 // threads (one count per row keeps the polled line quiet)
                 fence_proxy_async_global();
-                if (et == 0 && row == cta) QOQ_MARK(13);
                 named_barrier(1, 128);
-                if (et == 0 && row == cta) QOQ_MARK(14);
                 if (et == 0) red_release_gpu_add(a.ws_ready, 1);
-                if (et == 0 && row == cta) QOQ_MARK(8);
             }
         }
         if (a.X) {
             // every row is done once the X8 producer has seen the count; on
             // a timeout the flag stops every role
             wait_x(xready_bar, 0u);
-            if (threadIdx.x == kEpiWarp0 * 32) QOQ_MARK(9);
         }
         for (int i = i_begin; i < i_end;) {
             const int t = i / ks;
@@ -831,7 +775,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                     const uint64_t start = global_timer_ns();
                     while (ld_acquire_gpu(counter) < want) {
                         if (*abort_flag || global_timer_ns() - start > budget) {
-                            if (!*abort_flag) QOQ_RECORD_TIMEOUT(0xF00002u);
                             *abort_flag = 1;
                             ready = false;
                             break;
@@ -841,7 +784,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 ready = __all_sync(0xffffffffu, ready);
                 __syncwarp();  // every lane has seen the full count
                 if (lane == 0 && ready) *counter = 0;  // ready for the next call
-                if (warp == kEpiWarp0 && lane == 0 && tj < 8) QOQ_MARK(224 + tj);
                 if constexpr (kPresum) {
 #pragma unroll
                     for (int q = 0; q < BN; ++q) pre[q] = 0;
@@ -869,7 +811,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 }
             }
             if (!wait_x(accfull_bar(ab), accph)) break;
-            if (warp == kEpiWarp0 && lane == 0 && tj < 8) QOQ_MARK(208 + tj);
             tc_fence_after();
             const uint32_t tacc = trow + (uint32_t)(ab * BN);
             // the accumulator goes back to the MMA as soon as its last
@@ -943,12 +884,10 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                             }
                         }
                     }
-                    if (warp == kEpiWarp0 && lane == 0 && tj < 2 && g0 == 0) QOQ_MARK(232 + tj * 8);
 #pragma unroll
                     for (int u = 0; u < kGrp / 16; ++u) {
                         const int cc = g0 + u;
                         if (cc >= ch_hi) break;
-                        if (warp == kEpiWarp0 && lane == 0 && tj < 2 && cc < 6) QOQ_MARK(233 + tj * 8 + cc);
                         int32_t acc[16];
 #pragma unroll
                         for (int q = 0; q < 16; ++q) acc[q] = (int32_t)vg[16 * u + q];
@@ -975,15 +914,12 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
                 }
                 if (!released) release_acc();
             }
-            if (warp == kEpiWarp0 && lane == 0 && tj < 8) QOQ_MARK(216 + tj);
-            ++tj;
             if (++ab == C::kAccBufs) {
                 ab = 0;
                 accph ^= 1u;
             }
             i = t * ks + ks1;
         }
-        if (warp == kEpiWarp0 && lane == 0) QOQ_MARK(4);
     }
 
     __syncwarp();
@@ -993,7 +929,6 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
     // each other's barriers; neither leaves before both are done
     if constexpr (PAIR) cluster_sync_all();
     tc_fence_after();
-    QOQ_MARK(2);
     if (a.X && threadIdx.x == 0) {
         // every CTA is past its waits on ws_ready: the last one to get here
         // leaves both counters at zero for the next call
@@ -1049,34 +984,6 @@ __global__ void stuck_wait_kernel(unsigned long long budget_ns)
 }
 
 // ----------------------------------------------------------------- host --
-#ifdef QOQ_TRACE
-unsigned long long *g_trace_buffer = nullptr;
-
-// Trace builds: the first timed-out wait's site since the last read (0 if
-// none), and the barrier layout of the latest launch; both are cleared.
-cudaError_t debug_timeout_site(unsigned long long *site, unsigned long long *bar_info)
-{
-    cudaError_t e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbol(site, g_timeout_site, sizeof(*site));
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbol(bar_info, g_bar_info, sizeof(*bar_info));
-    if (e != cudaSuccess) return e;
-    const unsigned long long zero = 0;
-    return cudaMemcpyToSymbol(g_timeout_site, &zero, sizeof(zero));
-}
-
-__global__ void stamp_kernel(unsigned long long *dst)
-{
-    *dst = global_timer_ns();
-}
-
-cudaError_t debug_stamp(unsigned long long *dst, cudaStream_t stream)
-{
-    stamp_kernel<<<1, 1, 0, stream>>>(dst);
-    return cudaGetLastError();
-}
-#endif
 
 namespace {
 
@@ -1325,9 +1232,6 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     args.ngroups = K / G;
     args.total = (int)units;
     args.timeout_ns = 2000000000ull;  // 2 s for one wait: far beyond any legitimate one
-#ifdef QOQ_TRACE
-    args.trace = g_trace_buffer;
-#endif
     return a_in_tmem ? dispatch<true>(BN, KST, pair, tmap, args, (int)grid, stream)
                      : dispatch<false>(BN, KST, false, tmap, args, (int)grid, stream);
 }

@@ -19,10 +19,12 @@ constexpr size_t kCounterBytes = 8192;
 // split-tile counters: kMaxCtas CTAs x 2 epilogue groups x 4 quarters
 static_assert(kMaxCtas * 2 * 4 * 4 <= kCounterBytes - 64, "counter region");
 
+// z_dbg and q_dbg may be null (optional inspection outputs).
 cudaError_t launch_pack(const float *W, int N, int K, int G, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g,
-                        uint8_t *zs, cudaStream_t stream);
+                        uint8_t *zs, uint8_t *z_dbg, uint8_t *q_dbg, cudaStream_t stream);
 
-cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x,
+// rowsum may be null.
+cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, int32_t *rowsum,
                              cudaStream_t stream);
 
 cudaError_t launch_dequant(const uint8_t *Wp, const uint8_t *s_g, const uint8_t *zs, int N, int K, int G,
@@ -63,13 +65,17 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
                         int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream,
                         int *tmap_status, const uint16_t *X = nullptr);
 
-#ifdef QOQ_TRACE
-extern unsigned long long *g_trace_buffer;
-cudaError_t debug_stamp(unsigned long long *dst, cudaStream_t stream);
-cudaError_t debug_timeout_site(unsigned long long *site, unsigned long long *bar_info);
-#endif
 
 // Device error flag of the current device: read and clear (synchronous).
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value);
+
+// The argument checks every GEMM entry point shares (qoq_api.cu).
+bool valid_nk(int N, int K);
+bool valid_group(int K, int G);
+bool aligned16(const void *p);
+// Where the GEMM keeps its dequantized tile (qoq_set_gemm_a_in_tmem).
+bool gemm_a_in_tmem();
+// QOQ_OK when the current device is compute capability 10.0 (cached per device).
+int check_device();
 
 }  // namespace qoq

@@ -54,9 +54,12 @@ __device__ __forceinline__ uint32_t stage2_code(int w8, float sgf, int z)
 // ------------------------------------------------------------ packer --
 // One warp per output channel n.  Lane l covers k = kc + 4l .. kc + 4l + 3
 // of each 128-wide chunk kc.
+// Optional outputs for inspection: z_dbg [N][K/G] the zero points, q_dbg
+// [N][K] the canonical codes, one per byte.
 __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, int N, int K, int G,
                                                    uint8_t *__restrict__ Wp, uint16_t *__restrict__ s_c,
-                                                   uint8_t *__restrict__ s_g, uint8_t *__restrict__ zs)
+                                                   uint8_t *__restrict__ s_g, uint8_t *__restrict__ zs,
+                                                   uint8_t *__restrict__ z_dbg, uint8_t *__restrict__ q_dbg)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = blockIdx.x * 8 + warp;
@@ -92,6 +95,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
             const size_t ti = ((size_t)p * (K / G) + g) * kPanelRows + rr;
             s_g[ti] = (uint8_t)sg;
             zs[ti] = (uint8_t)(z * sg);
+            if (z_dbg) z_dbg[(size_t)n * (K / G) + g] = (uint8_t)z;
             if (G == kBlockK) {  // the copy inside the group's chunk
                 uint8_t *tab = Wp + chunk_offset(p, g, K, G) + kChunkBytes;
                 tab[rr] = (uint8_t)sg;
@@ -103,6 +107,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
             const uint32_t mine = stage2_code(stage1(v.x, sc), sgf, z) | (stage2_code(stage1(v.y, sc), sgf, z) << 8) |
                                   (stage2_code(stage1(v.z, sc), sgf, z) << 16) |
                                   (stage2_code(stage1(v.w, sc), sgf, z) << 24);
+            if (q_dbg) *reinterpret_cast<uint32_t *>(q_dbg + (size_t)n * K + kc + lane * 4) = mine;
             // lanes l and l+4 of each group of 8 fill the low and high
             // nibbles of the same packed word
             const uint32_t partner = __shfl_down_sync(0xffffffffu, mine, 4);
@@ -124,11 +129,14 @@ constexpr int kActCache = 4;   // 16-byte vectors per thread kept in registers (
 
 // One CTA per token row: read the row once (kept in registers up to
 // kActCache vectors per thread), reduce max|x|, then quantize.
+// With rowsum non-null it also writes rowsum[m] = sum_k X8[m][k] (INT32).
 __global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16_t *__restrict__ X, int K,
                                                                  int8_t *__restrict__ X8,
-                                                                 uint16_t *__restrict__ s_x)
+                                                                 uint16_t *__restrict__ s_x,
+                                                                 int32_t *__restrict__ rowsum)
 {
     __shared__ float red[kActThreads / 32];
+    __shared__ int rsum[kActThreads / 32];
     // the GEMM that consumes X8 may launch now and start streaming weights;
     // it waits for this grid to finish before it reads X8 or s_x
     grid_launch_dependents();
@@ -165,13 +173,33 @@ __global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16
     const uint16_t sxh = token_scale_bits(amax);
     const float sx = half_bits_to_float(sxh);
     if (threadIdx.x == 0) s_x[m] = sxh;
+    int sum = 0;  // sum of this thread's INT8 codes (rowsum only)
 #pragma unroll
     for (int i = 0; i < kActCache; ++i) {
         const int idx = threadIdx.x + i * kActThreads;
-        if (idx < nvec) out[idx] = quant8(cache[i], sx);
+        if (idx < nvec) {
+            const uint2 v = quant8(cache[i], sx);
+            out[idx] = v;
+            if (rowsum) sum = __dp4a((int)v.y, 0x01010101, __dp4a((int)v.x, 0x01010101, sum));
+        }
     }
-    for (int idx = threadIdx.x + kActCache * kActThreads; idx < nvec; idx += kActThreads)
-        out[idx] = quant8(__ldg(row + idx), sx);
+    for (int idx = threadIdx.x + kActCache * kActThreads; idx < nvec; idx += kActThreads) {
+        const uint2 v = quant8(__ldg(row + idx), sx);
+        out[idx] = v;
+        if (rowsum) sum = __dp4a((int)v.y, 0x01010101, __dp4a((int)v.x, 0x01010101, sum));
+    }
+    if (rowsum) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if ((threadIdx.x & 31) == 0) rsum[threadIdx.x >> 5] = sum;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int t = 0;
+#pragma unroll
+            for (int w = 0; w < kActThreads / 32; ++w) t += rsum[w];
+            rowsum[m] = t;
+        }
+    }
 }
 
 // ------------------------------------------------- INT8 weight expand --
@@ -210,13 +238,14 @@ __global__ void dequant_kernel(const uint8_t *__restrict__ Wp, const uint8_t *__
 }  // namespace
 
 cudaError_t launch_pack(const float *W, int N, int K, int G, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g, uint8_t *zs,
-                        cudaStream_t stream)
+                        uint8_t *z_dbg, uint8_t *q_dbg, cudaStream_t stream)
 {
-    pack_kernel<<<(N + 7) / 8, 256, 0, stream>>>(W, N, K, G, Wp, s_c, s_g, zs);
+    pack_kernel<<<(N + 7) / 8, 256, 0, stream>>>(W, N, K, G, Wp, s_c, s_g, zs, z_dbg, q_dbg);
     return cudaGetLastError();
 }
 
-cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, cudaStream_t stream)
+cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, int32_t *rowsum,
+                             cudaStream_t stream)
 {
     // programmatic dependent launch: the CTAs may be scheduled while the
     // previous kernel (for instance the previous layer's GEMM) finishes;
@@ -231,7 +260,7 @@ cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, X, K, X8, s_x);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, X, K, X8, s_x, rowsum);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

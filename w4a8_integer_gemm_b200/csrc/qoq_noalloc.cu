@@ -45,11 +45,6 @@ int scratch_address(void **out)
     return QOQ_OK;
 }
 
-bool aligned16(const void *p)
-{
-    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
-}
-
 }  // namespace
 
 extern "C" {
@@ -58,24 +53,19 @@ int qoq_w4a8_gemm_noalloc(const int8_t *X8, const uint16_t *s_x, const uint8_t *
                           const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int group_size,
                           uint16_t *Y, void *stream)
 {
-    // the same shape and pointer checks as qoq_w4a8_gemm
-    if (M < 0 || M > (1 << 24) || N < 128 || N > (1 << 20) || N % 128 || K < 128 || K > 65536 || K % 128 ||
-        (group_size != 128 && group_size != K))
+    // the same shape and pointer checks as qoq_w4a8_gemm (shared code)
+    if (M < 0 || M > (1 << 24) || !qoq::valid_nk(N, K) || !qoq::valid_group(K, group_size))
         return QOQ_ERR_INVALID_ARG;
     if (M == 0) return QOQ_OK;
     if (!X8 || !s_x || !Wp || !s_c || !s_g || !zs || !Y) return QOQ_ERR_INVALID_ARG;
-    if (!aligned16(X8) || !aligned16(s_x) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) ||
-        !aligned16(zs) || !aligned16(Y))
+    if (!qoq::aligned16(X8) || !qoq::aligned16(s_x) || !qoq::aligned16(Wp) || !qoq::aligned16(s_c) ||
+        !qoq::aligned16(s_g) || !qoq::aligned16(zs) || !qoq::aligned16(Y))
         return QOQ_ERR_INVALID_ARG;
     const size_t need = qoq_gemm_workspace_bytes(M, N, K, group_size);
     if (need == 0) return QOQ_ERR_INVALID_ARG;
     if (need > kScratchBytes) return QOQ_ERR_SCRATCH_TOO_SMALL;
-    int major = 0, minor = 0, dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-        return QOQ_ERR_CUDA;
-    if (major != 10 || minor != 0) return QOQ_ERR_UNSUPPORTED;
+    const int dev = qoq::check_device();
+    if (dev != QOQ_OK) return dev;
 
     void *scratch = nullptr;
     const int st = scratch_address(&scratch);
@@ -87,7 +77,7 @@ int qoq_w4a8_gemm_noalloc(const int8_t *X8, const uint16_t *s_x, const uint8_t *
     if (cudaMemsetAsync(scratch, 0, qoq::kCounterBytes, s) != cudaSuccess) return QOQ_ERR_CUDA;
     int tmap_status = 0;
     const cudaError_t e = qoq::launch_gemm(X8, s_x, Wp, s_c, s_g, zs, M, N, K, group_size, Y, nullptr, scratch,
-                                           true, s, &tmap_status);
+                                           qoq::gemm_a_in_tmem(), s, &tmap_status);
     if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
     return e == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
 }

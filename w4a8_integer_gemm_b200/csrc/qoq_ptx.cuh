@@ -80,23 +80,6 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // non-zero (another role gave up) or when this one wait has lasted longer
 // than `budget_ns`; in the latter case it raises `*abort` itself.  Returns
 // true when the phase completed.
-#ifdef QOQ_TRACE
-// Trace builds: the first wait of a launch sequence to time out records
-// where it was (CTA, thread, and the barrier's shared address or a tag).
-static __device__ unsigned long long g_timeout_site;
-__device__ __forceinline__ void record_timeout(uint32_t tag)
-{
-    const unsigned long long site = (1ull << 63) | ((unsigned long long)blockIdx.x << 40) |
-                                    ((unsigned long long)threadIdx.x << 24) | (tag & 0xFFFFFFu);
-    atomicCAS(&g_timeout_site, 0ull, site);
-}
-#define QOQ_RECORD_TIMEOUT(tag) record_timeout(tag)
-#else
-#define QOQ_RECORD_TIMEOUT(tag) \
-    do {                         \
-    } while (0)
-#endif
-
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile int *abort, uint64_t budget_ns)
 {
@@ -106,7 +89,6 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
         if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;  // up to 0.2 ms per sleep
         if (*abort) return false;
         if (global_timer_ns() - start > budget_ns) {
-            QOQ_RECORD_TIMEOUT(bar);
             *abort = 1;
             return false;
         }
