@@ -84,6 +84,12 @@ def _load():
         lib.oracle_gemm_i32.restype = None
         lib.oracle_epilogue.argtypes = [_P, _P, _P, _I64, _I64, _P]
         lib.oracle_epilogue.restype = None
+        lib.oracle_double_to_half_rn.argtypes = [ctypes.c_double]
+        lib.oracle_double_to_half_rn.restype = ctypes.c_uint16
+        lib.oracle_epilogue_residual.argtypes = [_P, _P, _P, _I64, _I64, _P, _P]
+        lib.oracle_epilogue_residual.restype = None
+        lib.oracle_epilogue_silu_mul.argtypes = [_P, _P, _P, _I64, _I64, _P]
+        lib.oracle_epilogue_silu_mul.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -222,6 +228,39 @@ def epilogue(acc: np.ndarray, s_x: np.ndarray, s_c: np.ndarray) -> np.ndarray:
     Y = np.zeros((M, N), np.uint16)
     _load().oracle_epilogue(_ptr(acc), _ptr(s_x), _ptr(s_c), M, N, _ptr(Y))
     return Y
+
+
+def double_to_half_bits(x: float) -> int:
+    return int(_load().oracle_double_to_half_rn(float(x)))
+
+
+def epilogue_residual(acc: np.ndarray, s_x: np.ndarray, s_c: np.ndarray, R: np.ndarray) -> np.ndarray:
+    """Y = fp16_rn((float)y + (float)R), y the layer's FP16 output -> uint16 bits [M][N]."""
+    acc = np.ascontiguousarray(acc, np.int32)
+    s_x = np.ascontiguousarray(s_x, np.uint16)
+    s_c = np.ascontiguousarray(s_c, np.uint16)
+    R = np.ascontiguousarray(R)
+    if R.dtype == np.float16:
+        R = R.view(np.uint16)
+    R = np.ascontiguousarray(R, np.uint16)
+    M, N = acc.shape
+    Y = np.zeros((M, N), np.uint16)
+    _load().oracle_epilogue_residual(_ptr(acc), _ptr(s_x), _ptr(s_c), M, N, _ptr(R), _ptr(Y))
+    return Y
+
+
+def epilogue_silu_mul(acc: np.ndarray, s_x: np.ndarray, s_c: np.ndarray) -> np.ndarray:
+    """Out[m][j] = fp16_rn(silu(g) * u) with g, u the FP16 outputs of gate column j
+    and up column I + j (acc has 2I columns) -> uint16 bits [M][I]."""
+    acc = np.ascontiguousarray(acc, np.int32)
+    s_x = np.ascontiguousarray(s_x, np.uint16)
+    s_c = np.ascontiguousarray(s_c, np.uint16)
+    M, N2 = acc.shape
+    if N2 % 2:
+        raise ValueError("the gate/up pair needs an even number of columns")
+    Out = np.zeros((M, N2 // 2), np.uint16)
+    _load().oracle_epilogue_silu_mul(_ptr(acc), _ptr(s_x), _ptr(s_c), M, N2, _ptr(Out))
+    return Out
 
 
 # ------------------------------------------------------------ chains ----

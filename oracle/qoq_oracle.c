@@ -271,6 +271,75 @@ void oracle_epilogue(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* binary64 -> binary16, round to nearest, ties to even, from the format     */
+/* definition (11 significant bits; subnormals in units of 2^-24).            */
+/* ------------------------------------------------------------------------ */
+uint16_t oracle_double_to_half_rn(double d)
+{
+    uint16_t sign = signbit(d) ? 0x8000u : 0u;
+    double a = fabs(d);
+    if (isnan(d)) return (uint16_t)(sign | 0x7e00u);
+    if (a >= 65520.0) return (uint16_t)(sign | 0x7c00u);       /* rounds to inf */
+    if (a < 6.103515625e-05) {                                  /* below 2^-14: subnormal */
+        double units = nearbyint(a * 16777216.0);               /* exact scaling, RN-even */
+        return (uint16_t)(sign | (uint16_t)units);              /* 1024 -> min normal */
+    }
+    int ex = 0;
+    (void)frexp(a, &ex);                                        /* a = f * 2^ex, f in [0.5, 1) */
+    double q = nearbyint(ldexp(a, 11 - ex));                    /* 11 significant bits */
+    if (q >= 2048.0) { q = 1024.0; ex += 1; }
+    return (uint16_t)(sign | (uint16_t)(((ex + 14) << 10) | ((int)q - 1024)));
+}
+
+/* ------------------------------------------------------------------------ */
+/* Output-side fusion (the steps after the layer; the pages name the layer's */
+/* epilogue, [GUIDE] "The Architecture" subsection 2, but not what follows). */
+/* Readings: the fused result equals the unfused sequence.                    */
+/*                                                                            */
+/* Residual add: the layer's FP16 output y (as oracle_epilogue), then        */
+/*   Y[m][n] = fp16_rn( (float)y + (float)R[m][n] )   (an FP16 add).          */
+/* ------------------------------------------------------------------------ */
+void oracle_epilogue_residual(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_c,
+                              int64_t M, int64_t N, const uint16_t *R, uint16_t *Y)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        float sx = oracle_half_to_float(s_x[m]);
+        for (int64_t n = 0; n < N; ++n) {
+            float sc = oracle_half_to_float(s_c[n]);
+            float t = (float)acc[m * N + n] * sx;
+            uint16_t y = oracle_float_to_half_rn(t * sc);
+            float sum = oracle_half_to_float(y) + oracle_half_to_float(R[m * N + n]);
+            Y[m * N + n] = oracle_float_to_half_rn(sum);
+        }
+    }
+}
+
+/* SiLU-gated product of a gate/up pair (the MLP activation that follows a   */
+/* fused gate/up projection).  acc has N2 = 2*I columns in their natural     */
+/* order: gate channel j at column j, up channel j at column I + j.  With    */
+/* g and u the layer's FP16 outputs of those two columns,                    */
+/*   Out[m][j] = fp16_rn( g / (1 + exp(-g)) * u )   evaluated in binary64.  */
+/* ------------------------------------------------------------------------ */
+void oracle_epilogue_silu_mul(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_c,
+                              int64_t M, int64_t N2, uint16_t *Out)
+{
+    int64_t I = N2 / 2;
+    for (int64_t m = 0; m < M; ++m) {
+        float sx = oracle_half_to_float(s_x[m]);
+        for (int64_t j = 0; j < I; ++j) {
+            float tg = (float)acc[m * N2 + j] * sx;
+            float tu = (float)acc[m * N2 + I + j] * sx;
+            uint16_t g = oracle_float_to_half_rn(tg * oracle_half_to_float(s_c[j]));
+            uint16_t u = oracle_float_to_half_rn(tu * oracle_half_to_float(s_c[I + j]));
+            double gd = (double)oracle_half_to_float(g);
+            double ud = (double)oracle_half_to_float(u);
+            double silu = gd / (1.0 + exp(-gd));
+            Out[m * I + j] = oracle_double_to_half_rn(silu * ud);
+        }
+    }
+}
+
 /* Number of OpenMP threads the parallel loops above use. */
 int oracle_num_threads(void)
 {
