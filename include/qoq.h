@@ -146,6 +146,23 @@ QOQ_API int qoq_pack_weights(const float *W, int N, int K, int group_size,
                      uint8_t *Wp, uint16_t *s_c, uint8_t *s_g, uint8_t *zs,
                      uint8_t *z_dbg, uint8_t *q_dbg, void *stream);
 
+/* Packs a gate/up projection pair for the SiLU-gated epilogue of
+ * qoq_w4a8_gemm_fused (the pages have no counterpart: it is the layout the
+ * fused MLP activation needs, not part of the method).
+ *
+ *   W      device, float32 [N][K]: rows 0..N/2-1 are the gate projection's
+ *          output channels, rows N/2..N-1 the up projection's (the order of
+ *          a fused gate/up weight). N is a multiple of 128.
+ * The quantization is exactly qoq_pack_weights' (per output channel, so the
+ * row order does not change any value). Only the placement differs: packed
+ * panel p (rows 128p..128p+127 of Wp, s_c, s_g and zs) holds gate channels
+ * 64p..64p+63 followed by up channels 64p..64p+63, so that one tile of the
+ * GEMM holds both halves of 64 outputs. Outputs, sizes and limits as for
+ * qoq_pack_weights (there are no debug outputs). */
+QOQ_API int qoq_pack_weights_gate_up(const float *W, int N, int K, int group_size,
+                             uint8_t *Wp, uint16_t *s_c, uint8_t *s_g, uint8_t *zs,
+                             void *stream);
+
 /* Per-token symmetric INT8 activation quantization.
  *
  * Source: "QServe Guide: W4A8KV4 Quantization for LLM Serving", Deep Dive,
@@ -216,6 +233,80 @@ QOQ_API int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x,
                   int M, int N, int K, int group_size,
                   uint16_t *Y, int32_t *acc_dbg,
                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Output-side fusion in the GEMM's epilogue (the pages stop at the layer's
+ * FP16 output, "QServe Guide: W4A8KV4 Quantization for LLM Serving", The
+ * Architecture, subsection 2; these are the operations that follow it in a
+ * transformer block, done on the layer's FP16 values before they leave the
+ * SM). The layer's own output y[m][n] is rounded exactly as qoq_w4a8_gemm
+ * rounds it; then:
+ *   QOQ_EPILOGUE_NONE      Y = y (the same as qoq_w4a8_gemm).
+ *   QOQ_EPILOGUE_RESIDUAL  Y[m][n] = fp16((float)y[m][n] + (float)R[m][n]):
+ *                          a residual add, the same bits as an FP16 add after
+ *                          the layer.
+ *   QOQ_EPILOGUE_SILU_MUL  Wp, s_c, s_g, zs from qoq_pack_weights_gate_up;
+ *                          with g = y of gate channel j and u = y of up
+ *                          channel j, Y[m][j] = fp16(silu(g) * u) for
+ *                          j < N/2, silu(g) = g / (1 + exp(-g)) in FP32 with
+ *                          IEEE division. Y is [M][N/2].
+ */
+typedef enum {
+    QOQ_EPILOGUE_NONE = 0,
+    QOQ_EPILOGUE_RESIDUAL = 1,
+    QOQ_EPILOGUE_SILU_MUL = 2
+} qoq_epilogue_kind;
+
+/* The GEMM of qoq_w4a8_gemm with an output-side fusion.
+ *   epilogue   a qoq_epilogue_kind; other values give QOQ_ERR_INVALID_ARG.
+ *   residual   device, uint16_t [M][N] FP16 bits, read; required (16-byte
+ *              aligned) for QOQ_EPILOGUE_RESIDUAL, ignored otherwise. It may
+ *              be the same buffer as Y (each element is read before it is
+ *              written, by the same thread).
+ *   Y          device, uint16_t FP16 bits, written: [M][N], or [M][N/2] for
+ *              QOQ_EPILOGUE_SILU_MUL.
+ * Every other argument, limit and workspace rule as for qoq_w4a8_gemm (no
+ * acc_dbg). */
+QOQ_API int qoq_w4a8_gemm_fused(const int8_t *X8, const uint16_t *s_x,
+                        const uint8_t *Wp, const uint16_t *s_c,
+                        const uint8_t *s_g, const uint8_t *zs,
+                        int M, int N, int K, int group_size, int epilogue,
+                        const uint16_t *residual, uint16_t *Y,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* The INT32 inner products alone: acc[m][n] = sum_k X8[m][k] * W8hat[n][k]
+ * for m < M, n < N, over this call's K (the GEMM of qoq_w4a8_gemm without
+ * its output scaling).
+ *
+ * Source: "QServe Guide: W4A8KV4 Quantization for LLM Serving", The
+ * Architecture, subsection 2 (INT8 x INT8 products accumulated in INT32).
+ * It is the per-GPU step of a row-parallel (K-split) layer: each GPU holds a
+ * K slice of the weights (a multiple of the group size), computes these
+ * partial sums, the GPUs add them (an INT32 sum is exact in any order), and
+ * qoq_epilogue_i32 applies the scales once.
+ *   X8, ldx          device, int8_t: row m of this GPU's K slice starts at
+ *                    X8 + m*ldx (ldx >= K, a multiple of 16), so a slice of
+ *                    a full [M][K_total] activation matrix is passed without
+ *                    a copy (X8 = base + k0, ldx = K_total).
+ *   Wp, s_g, zs      device, the packed slice (see the K-split helpers of the
+ *                    Python binding for slicing a packed weight).
+ *   acc              device, int32_t [M][N], written.
+ *   workspace, workspace_bytes  as for qoq_w4a8_gemm.
+ * Limits as for qoq_w4a8_gemm. */
+QOQ_API int qoq_w4a8_gemm_i32(const int8_t *X8, int ldx, const uint8_t *Wp, const uint8_t *s_g,
+                      const uint8_t *zs, int M, int N, int K, int group_size, int32_t *acc,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* The output rescaling on INT32 sums computed elsewhere:
+ *     Y[m][n] = fp16( ((float)acc[m][n] * (float)s_x[m]) * (float)s_c[n] )
+ * rounded exactly as qoq_w4a8_gemm's epilogue.
+ * Source: "QServe Guide: W4A8KV4 Quantization for LLM Serving", Deep Dive,
+ * subsection 1, the output rescaling equation.
+ *   acc    device, int32_t [M][N] (for a K-split layer: the summed partials).
+ *   s_x    device, uint16_t [M] FP16 bits; s_c device, uint16_t [N] FP16 bits.
+ *   Y      device, uint16_t [M][N] FP16 bits, written.
+ * N is a multiple of 128 (at most 1048576); M >= 0 (0 launches nothing). */
+QOQ_API int qoq_epilogue_i32(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_c,
+                     int M, int N, uint16_t *Y, void *stream);
 
 /* The whole W4A8 linear layer in one call: the per-token quantization of
  * qoq_quant_act_per_token followed by qoq_w4a8_gemm.
@@ -308,6 +399,16 @@ QOQ_API int qoq_set_gemm_a_in_tmem(int enable);
  * The choice applies to later GEMM calls from every thread. Results are
  * identical either way. Returns QOQ_ERR_INVALID_ARG for other values. */
 QOQ_API int qoq_set_gemm_cta_pairs(int enable);
+
+/* Selects the CTA size for token tiles up to 64 (decode):
+ *   1: half-SM CTAs (at most half of an SM's registers, shared memory and
+ *      tensor memory, 128-wide K stages), so that the CTA of the next GEMM
+ *      on the stream can be resident beside the current one and stream and
+ *      dequantize its weights while the current one finishes;
+ *   0 (default): one CTA per SM with deeper rings and 256-wide K stages.
+ * The choice applies to later GEMM calls from every thread. Results are
+ * identical either way. Returns QOQ_ERR_INVALID_ARG for other values. */
+QOQ_API int qoq_set_gemm_half_ctas(int enable);
 
 /* Selects the token-tile width rule for M > 64:
  *   1 (default): 256 tokens per tile (128 for M <= 128), narrowed to 128 and

@@ -27,7 +27,7 @@ def declared():
 def test_exports_every_declared_symbol(L):
     import w4a8_integer_gemm_b200 as q
     names = declared()
-    assert len(names) == 15
+    assert len(names) == 20
     for n in names:
         assert hasattr(L, n), n
     assert names == set(q.SIGNATURES)
@@ -58,16 +58,17 @@ def test_size_queries(L):
     # 8192 bytes of counters, then for each of <= 148 CTAs one partial tile
     # of BN=16 tokens x 128 channels x int32
     assert q.qoq_gemm_workspace_bytes(1, 14336, 4096, 128) == 8192 + 148 * 16 * 128 * 4
-    # grid = units when there are fewer units than SMs (4 tiles x 2 K blocks of 256)
-    assert q.qoq_gemm_workspace_bytes(1, 512, 512, 128) == 8192 + 8 * 16 * 128 * 4
+    # grid = units when there are fewer units than SMs (4 tiles x 4 K blocks of 128,
+    # the narrowest stage any configuration uses)
+    assert q.qoq_gemm_workspace_bytes(1, 512, 512, 128) == 8192 + 16 * 16 * 128 * 4
     # 256-token tiles use 128-wide K blocks: 4 m-tiles x 64 n-tiles x 64 blocks -> 148 CTAs
     assert q.qoq_gemm_workspace_bytes(1024, 8192, 8192, 128) == 8192 + 148 * 256 * 128 * 4
     # Few tiles: the default rule narrows M = 256, N = K = 4096 to 64-token tiles, but the
     # workspace also covers the 256-token tiles of the other rule (148 CTAs either way).
     assert q.qoq_gemm_workspace_bytes(256, 4096, 4096, 128) == 8192 + 148 * 256 * 128 * 4
-    # M = 200, N = 512, K = 1024: 64-token tiles give 4 x 4 tiles x 4 K blocks of 256 = 64
-    # units, 256-token tiles 4 tiles x 8 K blocks of 128 = 32: 64 CTAs, 256-token slots.
-    assert q.qoq_gemm_workspace_bytes(200, 512, 1024, 128) == 8192 + 64 * 256 * 128 * 4
+    # M = 200, N = 512, K = 1024: 64-token tiles give 4 x 4 tiles x 8 K blocks of 128 = 128
+    # units, 256-token tiles 4 tiles x 8 K blocks = 32: 128 CTAs, 256-token slots.
+    assert q.qoq_gemm_workspace_bytes(200, 512, 1024, 128) == 8192 + 128 * 256 * 128 * 4
     # and the size does not depend on the switch
     sizes = []
     for narrow in (False, True):
@@ -115,6 +116,7 @@ def test_invalid_arguments_rejected_on_host(L):
     assert L.qoq_set_gemm_a_in_tmem(2) == INVALID
     assert L.qoq_set_gemm_cta_pairs(2) == INVALID
     assert L.qoq_set_gemm_narrow_tiles(-1) == INVALID
+    assert L.qoq_set_gemm_half_ctas(3) == INVALID
     assert L.qoq_set_linear_in_kernel_quant(2) == INVALID
     assert L.qoq_selftest_wait_timeout(ctypes.c_ulonglong(10), None) == INVALID          # budget too short
     assert L.qoq_selftest_wait_timeout(ctypes.c_ulonglong(10 ** 12), None) == INVALID    # too long

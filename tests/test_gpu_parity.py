@@ -163,6 +163,36 @@ def test_gemm_bit_exact(M, K, N, G, a_in_tmem, narrow):
     assert_half_within_1ulp(_u16(Y), r["Y"])
 
 
+HALF_CASES = [c for c in GEMM_CASES if c[0] <= 64] + [(1, 4096, 1024, 128), (64, 4096, 2048, 4096),
+                                                   (40, 8192, 1024, 128), (3, 24576, 256, 128)]
+
+
+@pytest.mark.parametrize("M,K,N,G", HALF_CASES)
+def test_gemm_bit_exact_half_ctas(M, K, N, G):
+    """Token tiles up to 64 in half-SM CTAs (two per SM): INT32 exact."""
+    X = wl.make_activations(M, K, wl.LLAMA, seed=410 + M)
+    W = wl.make_weights(N, K, wl.LLAMA, seed=510 + N + K)
+    q.qoq_set_gemm_half_ctas(True)
+    try:
+        _, X8, s_x, Y, acc = run_layer(X, W, G, True)
+        # several launches in a row on the stream: CTAs of consecutive GEMMs
+        # share SMs
+        packed = q.qoq_pack_weights(W.cuda(), G)
+        outs = []
+        for _ in range(6):
+            a2 = torch.zeros_like(acc)
+            outs.append((q.qoq_w4a8_gemm(X8, s_x, packed, acc_dbg=a2), a2))
+        torch.cuda.synchronize()
+        assert q.qoq_device_error() == q.QOQ_OK
+    finally:
+        q.qoq_set_gemm_half_ctas(False)
+    r = oracle.linear(X.numpy(), W.numpy(), G)
+    assert np.array_equal(acc.cpu().numpy(), r["acc"])
+    assert_half_within_1ulp(_u16(Y), r["Y"])
+    for Yi, ai in outs:
+        assert torch.equal(ai, acc) and torch.equal(Yi.view(torch.int16), Y.view(torch.int16))
+
+
 def test_tiny_workload_full_parity():
     """16 x 512 x 512, g128, the tiny workload's distribution and seeds."""
     w = wl.WORKLOADS["tiny"]

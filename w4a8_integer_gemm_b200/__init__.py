@@ -34,6 +34,9 @@ QOQ_ERR_CUDA = -3
 QOQ_ERR_TIMEOUT = -4
 QOQ_ERR_SCRATCH_TOO_SMALL = -5
 QOQ_NOALLOC_SCRATCH_BYTES = 16 << 20
+QOQ_EPILOGUE_NONE = 0
+QOQ_EPILOGUE_RESIDUAL = 1
+QOQ_EPILOGUE_SILU_MUL = 2
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -44,15 +47,20 @@ SIGNATURES = {
     "qoq_status_string": (ctypes.c_char_p, [_I]),
     "qoq_packed_weight_bytes": (_SZ, [_I, _I, _I]),
     "qoq_pack_weights": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "qoq_pack_weights_gate_up": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "qoq_quant_act_per_token": (_I, [_P, _I, _I, _P, _P, _P, _P]),
     "qoq_gemm_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "qoq_w4a8_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "qoq_w4a8_gemm_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "qoq_w4a8_gemm_fused": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "qoq_w4a8_gemm_i32": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
+    "qoq_epilogue_i32": (_I, [_P, _P, _P, _I, _I, _P, _P]),
     "qoq_w4a8_linear": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "qoq_dequant_weights_i8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "qoq_set_gemm_a_in_tmem": (_I, [_I]),
     "qoq_set_gemm_cta_pairs": (_I, [_I]),
     "qoq_set_gemm_narrow_tiles": (_I, [_I]),
+    "qoq_set_gemm_half_ctas": (_I, [_I]),
     "qoq_set_linear_in_kernel_quant": (_I, [_I]),
     "qoq_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "qoq_device_error": (_I, [_P]),
@@ -133,6 +141,10 @@ def qoq_set_gemm_narrow_tiles(enable: bool) -> None:
     _check("qoq_set_gemm_narrow_tiles", lib().qoq_set_gemm_narrow_tiles(1 if enable else 0))
 
 
+def qoq_set_gemm_half_ctas(enable: bool) -> None:
+    _check("qoq_set_gemm_half_ctas", lib().qoq_set_gemm_half_ctas(1 if enable else 0))
+
+
 def qoq_set_linear_in_kernel_quant(enable: bool) -> None:
     _check("qoq_set_linear_in_kernel_quant", lib().qoq_set_linear_in_kernel_quant(1 if enable else 0))
 
@@ -157,6 +169,7 @@ class PackedWeights:
     N: int
     K: int
     group_size: int
+    gate_up: bool = False   # packed by qoq_pack_weights_gate_up (64 gate + 64 up channels per panel)
 
 
 def qoq_pack_weights(W: torch.Tensor, group_size: int, out: Optional[PackedWeights] = None,
@@ -183,6 +196,26 @@ def qoq_pack_weights(W: torch.Tensor, group_size: int, out: Optional[PackedWeigh
     st = lib().qoq_pack_weights(_ptr(W), N, K, G, _ptr(out.Wp), _ptr(out.s_c), _ptr(out.s_g),
                                 _ptr(out.zs), _ptr(z_dbg), _ptr(q_dbg), _stream(stream))
     _check("qoq_pack_weights", st)
+    return out
+
+
+def qoq_pack_weights_gate_up(W: torch.Tensor, group_size: int, stream=None) -> PackedWeights:
+    """W fp32 [N, K] = [gate rows; up rows] -> packed weights whose panels
+    hold 64 gate channels and the 64 matching up channels, for the SiLU-gated
+    epilogue of qoq_w4a8_gemm_fused."""
+    _need(W, torch.float32, "W")
+    N, K = W.shape
+    G = int(group_size)
+    dev = W.device
+    nb = qoq_packed_weight_bytes(N, K, G)
+    ng = K // G if G > 0 and K % G == 0 else 1
+    out = PackedWeights(torch.empty(max(nb, 16), dtype=torch.uint8, device=dev),
+                        torch.empty(N, dtype=torch.int16, device=dev),
+                        torch.empty(max(N // 128, 1), ng, 128, dtype=torch.uint8, device=dev),
+                        torch.empty(max(N // 128, 1), ng, 128, dtype=torch.uint8, device=dev), N, K, G, True)
+    st = lib().qoq_pack_weights_gate_up(_ptr(W), N, K, G, _ptr(out.Wp), _ptr(out.s_c), _ptr(out.s_g),
+                                        _ptr(out.zs), _stream(stream))
+    _check("qoq_pack_weights_gate_up", st)
     return out
 
 
@@ -240,6 +273,69 @@ def qoq_w4a8_gemm(X8: torch.Tensor, s_x: torch.Tensor, packed: PackedWeights,
                              _ptr(workspace), workspace.numel() * workspace.element_size(),
                              _stream(stream))
     _check("qoq_w4a8_gemm", st)
+    return Y
+
+
+def qoq_w4a8_gemm_fused(X8: torch.Tensor, s_x: torch.Tensor, packed: PackedWeights, epilogue: int,
+                        residual: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The GEMM with an output-side fusion: QOQ_EPILOGUE_RESIDUAL gives
+    fp16(y + residual) ([M, N]); QOQ_EPILOGUE_SILU_MUL (weights from
+    qoq_pack_weights_gate_up) gives fp16(silu(gate) * up) ([M, N/2])."""
+    _need(X8, torch.int8, "X8")
+    M, K = X8.shape
+    if K != packed.K:
+        raise ValueError("K mismatch between X8 and the packed weights")
+    N = packed.N
+    if epilogue == QOQ_EPILOGUE_SILU_MUL and not packed.gate_up:
+        raise ValueError("the SiLU-gated epilogue needs weights from qoq_pack_weights_gate_up")
+    if residual is not None:
+        _need(residual, torch.float16, "residual")
+    ncol = N // 2 if epilogue == QOQ_EPILOGUE_SILU_MUL else N
+    if Y is None:
+        Y = torch.empty(M, ncol, dtype=torch.float16, device=X8.device)
+    if workspace is None:
+        workspace = gemm_workspace(max(M, 1), N, K, packed.group_size, X8.device)
+    st = lib().qoq_w4a8_gemm_fused(_ptr(X8), _ptr(s_x), _ptr(packed.Wp), _ptr(packed.s_c), _ptr(packed.s_g),
+                                   _ptr(packed.zs), M, N, K, packed.group_size, int(epilogue), _ptr(residual),
+                                   _ptr(Y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream(stream))
+    _check("qoq_w4a8_gemm_fused", st)
+    return Y
+
+
+def qoq_w4a8_gemm_i32(X8: torch.Tensor, packed: PackedWeights, acc: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """acc int32 [M, N] = X8 . W8hat^T over this call's K (no scales).  X8
+    may be a column slice of a wider int8 matrix (row stride passed on)."""
+    if not (X8.is_cuda and X8.dtype == torch.int8 and X8.stride(1) == 1):
+        raise ValueError("X8 must be a CUDA int8 tensor with unit column stride")
+    M, K = X8.shape
+    ldx = X8.stride(0) if M > 1 else K
+    if K != packed.K:
+        raise ValueError("K mismatch between X8 and the packed weights")
+    N = packed.N
+    if acc is None:
+        acc = torch.empty(M, N, dtype=torch.int32, device=X8.device)
+    _need(acc, torch.int32, "acc")
+    if workspace is None:
+        workspace = gemm_workspace(max(M, 1), N, K, packed.group_size, X8.device)
+    st = lib().qoq_w4a8_gemm_i32(_ptr(X8), int(ldx), _ptr(packed.Wp), _ptr(packed.s_g), _ptr(packed.zs), M, N, K,
+                                 packed.group_size, _ptr(acc), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("qoq_w4a8_gemm_i32", st)
+    return acc
+
+
+def qoq_epilogue_i32(acc: torch.Tensor, s_x: torch.Tensor, s_c: torch.Tensor, Y: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Y fp16 [M, N] = fp16(((float)acc * s_x) * s_c)."""
+    _need(acc, torch.int32, "acc")
+    M, N = acc.shape
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float16, device=acc.device)
+    st = lib().qoq_epilogue_i32(_ptr(acc), _ptr(s_x), _ptr(s_c), M, N, _ptr(Y), _stream(stream))
+    _check("qoq_epilogue_i32", st)
     return Y
 
 

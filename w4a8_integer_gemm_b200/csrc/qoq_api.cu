@@ -10,6 +10,10 @@
 #include "qoq_internal.h"
 #include "qoq_layout.cuh"
 
+static_assert(QOQ_EPILOGUE_NONE == qoq::kEpiPlain && QOQ_EPILOGUE_RESIDUAL == qoq::kEpiResidual &&
+                  QOQ_EPILOGUE_SILU_MUL == qoq::kEpiSiluMul,
+              "epilogue kinds");
+
 namespace {
 
 std::atomic<int> g_a_in_tmem{1};
@@ -109,6 +113,19 @@ int qoq_pack_weights(const float *W, int N, int K, int group_size, uint8_t *Wp, 
         qoq::launch_pack(W, N, K, group_size, Wp, s_c, s_g, zs, z_dbg, q_dbg, (cudaStream_t)stream));
 }
 
+int qoq_pack_weights_gate_up(const float *W, int N, int K, int group_size, uint8_t *Wp, uint16_t *s_c,
+                             uint8_t *s_g, uint8_t *zs, void *stream)
+{
+    if (!valid_nk(N, K) || !valid_group(K, group_size)) return QOQ_ERR_INVALID_ARG;
+    if (!W || !Wp || !s_c || !s_g || !zs) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) || !aligned16(zs))
+        return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(qoq::launch_pack(W, N, K, group_size, Wp, s_c, s_g, zs, nullptr, nullptr,
+                                      (cudaStream_t)stream, true));
+}
+
 int qoq_quant_act_per_token(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, int32_t *rowsum,
                             void *stream)
 {
@@ -148,6 +165,68 @@ int qoq_w4a8_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, cons
                                      qoq::gemm_a_in_tmem(), (cudaStream_t)stream, &tmap_status);
     if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
     return from_cuda(e);
+}
+
+int qoq_w4a8_gemm_fused(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
+                        const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int group_size, int epilogue,
+                        const uint16_t *residual, uint16_t *Y, void *workspace, size_t workspace_bytes,
+                        void *stream)
+{
+    if (M < 0 || M > kMaxM || !valid_nk(N, K) || !valid_group(K, group_size)) return QOQ_ERR_INVALID_ARG;
+    if (epilogue != QOQ_EPILOGUE_NONE && epilogue != QOQ_EPILOGUE_RESIDUAL && epilogue != QOQ_EPILOGUE_SILU_MUL)
+        return QOQ_ERR_INVALID_ARG;
+    if (M == 0) return QOQ_OK;
+    if (!X8 || !s_x || !Wp || !s_c || !s_g || !zs || !Y || !workspace) return QOQ_ERR_INVALID_ARG;
+    if (epilogue == QOQ_EPILOGUE_RESIDUAL && (!residual || !aligned16(residual))) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(X8) || !aligned16(s_x) || !aligned16(Wp) || !aligned16(s_c) || !aligned16(s_g) ||
+        !aligned16(zs) || !aligned16(Y) || !aligned16(workspace))
+        return QOQ_ERR_INVALID_ARG;
+    if (!qoq::gemm_shape_supported(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    if (workspace_bytes < qoq::gemm_workspace_bytes(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    int tmap_status = 0;
+    cudaError_t e = qoq::launch_gemm(X8, s_x, Wp, s_c, s_g, zs, M, N, K, group_size, Y, nullptr, workspace,
+                                     qoq::gemm_a_in_tmem(), (cudaStream_t)stream, &tmap_status, nullptr, epilogue,
+                                     epilogue == QOQ_EPILOGUE_RESIDUAL ? residual : nullptr);
+    if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
+int qoq_w4a8_gemm_i32(const int8_t *X8, int ldx, const uint8_t *Wp, const uint8_t *s_g, const uint8_t *zs, int M,
+                      int N, int K, int group_size, int32_t *acc, void *workspace, size_t workspace_bytes,
+                      void *stream)
+{
+    if (M < 0 || M > kMaxM || !valid_nk(N, K) || !valid_group(K, group_size)) return QOQ_ERR_INVALID_ARG;
+    if (ldx < K || ldx % 16 != 0) return QOQ_ERR_INVALID_ARG;
+    if (M == 0) return QOQ_OK;
+    if (!X8 || !Wp || !s_g || !zs || !acc || !workspace) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(X8) || !aligned16(Wp) || !aligned16(s_g) || !aligned16(zs) || !aligned16(acc) ||
+        !aligned16(workspace))
+        return QOQ_ERR_INVALID_ARG;
+    if (!qoq::gemm_shape_supported(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    if (workspace_bytes < qoq::gemm_workspace_bytes(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    int tmap_status = 0;
+    // no scales are read and no FP16 output is written: acc receives the sums
+    cudaError_t e = qoq::launch_gemm(X8, nullptr, Wp, nullptr, s_g, zs, M, N, K, group_size, nullptr, acc,
+                                     workspace, qoq::gemm_a_in_tmem(), (cudaStream_t)stream, &tmap_status, nullptr,
+                                     qoq::kEpiI32, nullptr, ldx);
+    if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
+int qoq_epilogue_i32(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_c, int M, int N, uint16_t *Y,
+                     void *stream)
+{
+    if (M < 0 || M > kMaxM || N < 128 || N > kMaxN || N % 128 != 0) return QOQ_ERR_INVALID_ARG;
+    if (M == 0) return QOQ_OK;
+    if (!acc || !s_x || !s_c || !Y || !aligned16(acc) || !aligned16(s_c) || !aligned16(Y))
+        return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(qoq::launch_epilogue_i32(acc, s_x, s_c, M, N, Y, (cudaStream_t)stream));
 }
 
 int qoq_w4a8_linear(const uint16_t *X, int M, int N, int K, int group_size, const uint8_t *Wp,
@@ -210,6 +289,13 @@ int qoq_set_gemm_cta_pairs(int enable)
 {
     if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;
     qoq::set_cta_pairs(enable != 0);
+    return QOQ_OK;
+}
+
+int qoq_set_gemm_half_ctas(int enable)
+{
+    if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;
+    qoq::set_half_ctas(enable != 0);
     return QOQ_OK;
 }
 

@@ -102,6 +102,13 @@ struct GemmArgs {
     uint16_t *s_xw;    // = s_x
     int32_t *ws_ready; // token rows quantized and stored (one-launch layer call)
     int32_t *ws_done;  // CTAs finished; the last one resets both counters
+    // Output-side fusion (kEpiPlain, kEpiResidual, kEpiSiluMul): with
+    // kEpiResidual Y = fp16(y + R) for the layer output y; with kEpiSiluMul
+    // the packed panels hold 64 gate then 64 up channels and Y[m][j] =
+    // fp16(silu(g) * u) over N/2 columns.  ldy is Y's row stride.
+    int epi;
+    const uint16_t *R;
+    int ldy;
     int M, N, K, G;
     int m_tiles;
     int ks;            // K / KST units per tile
@@ -138,7 +145,11 @@ __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
 // PAIR: a 2-CTA cluster computes a 256-channel x BN-token tile with one
 // M = 256 MMA per K step (tcgen05 cta_group::2): each CTA dequantizes its
 // own 128-channel panel into its TMEM and holds half of the X8 tile.
-template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false>
+// HALF: a CTA that takes at most half of an SM (registers, shared memory,
+// tensor memory), so that the next GEMM's CTA can be resident beside it and
+// stream and dequantize its weights while this one finishes (token tiles up
+// to 64, K blocks of 128).
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false, bool HALF = false>
 struct GemmCfg {
     static constexpr int kChunks = KST / kBlockK;        // packed 8 KB chunks per K block
     static constexpr int kXRows = PAIR ? BN / 2 : BN;    // token rows of X8 this CTA holds
@@ -160,9 +171,10 @@ struct GemmCfg {
     static constexpr int kAccBufs = (2 * BN + (A_TMEM ? SX * (int)kACols : 0) <= 512) ? 2 : 1;
     static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * kAccBufs + 2;
     static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
-    // at least ~120 KB so that exactly one CTA (and one TMEM allocation)
-    // lives on each SM; +1024 for manual alignment of the dynamic base
-    static constexpr int kSmemBytes = (kUsed > 120 * 1024 ? kUsed : 120 * 1024) + 1024;
+    // full CTAs: at least ~120 KB so that exactly one CTA (and one TMEM
+    // allocation) lives on each SM; +1024 for manual alignment of the
+    // dynamic base
+    static constexpr int kSmemBytes = (HALF || kUsed > 120 * 1024 ? kUsed : 120 * 1024) + 1024;
     static constexpr uint32_t kACol0 = kAccBufs * BN;    // first TMEM column of the A ring
     static constexpr uint32_t kTmemCols = pow2_cols(kACol0 + (A_TMEM ? SX * kACols : 0));
     static constexpr int kSx = (BN + 31) / 32;           // s_x registers per lane
@@ -180,6 +192,9 @@ struct GemmCfg {
     // sufficient rule: each weight slot belongs to one group.
     static_assert(SW % dequant_groups(BN) == 0, "each weight slot belongs to one dequant group");
     static_assert(kXSlot % 1024 == 0 && kAOff % 1024 == 0 && kWOff % 1024 == 0, "swizzle atoms");
+    // two half CTAs per SM: 228 KB of shared memory (1 KB reserved per CTA)
+    // and 512 TMEM columns between them
+    static_assert(!HALF || (kSmemBytes <= 113 * 1024 && kTmemCols <= 256 && !PAIR && A_TMEM), "half CTA");
 };
 
 // The CTA whose stream-K range contains unit i (ranges: [c*T/P, (c+1)*T/P)).
@@ -238,16 +253,57 @@ __device__ __forceinline__ uint16_t scale_to_half(int32_t acc, float sx, float s
     return __half_as_ushort(__float2half_rn(y));
 }
 
-// FP16 outputs (and optionally the INT32 accumulators) of the 16
+// FP16 outputs (and optionally the INT32 accumulators; with kEpiI32 only
+// those) of the 16
 // consecutive tokens m0.. of chunk `cc` for this lane's channel n0 + lane.
 // The token scales come from the lanes' registers: lane l of sx holds
 // s_x[m0 - 16*(cc&1) + l].  The warp stages its 16 x 32 block in its own
 // 1 KB of shared memory ([token][32 channels], 64 bytes per token) and then
 // writes Y with 16-byte stores: in store j, lane l writes token 8*j + l/4,
 // channels 8*(l%4) .. 8*(l%4)+7.
-__device__ __forceinline__ void store_outputs(const GemmArgs &a, uint8_t *stg, int m0, int cc, int n0, int lane,
-                                              float sc, float sx, const int32_t *acc)
+//
+// Output-side fusion happens on the staged FP16 values, so the layer's own
+// output is rounded exactly as without it:
+//   residual: each stored value becomes fp16((float)y + (float)R[m][n]);
+//   SiLU-gated pair: the four epilogue warps of the group (quarters 0-1 hold
+//     gate channels, 2-3 the up channels of the same outputs) meet at a
+//     named barrier; quarters 0-1 read the up values from the staging block
+//     two warps on and store fp16(silu(g) * u), silu in FP32 with IEEE
+//     division; a second barrier frees the staging blocks for the next chunk.
+__device__ __forceinline__ uint32_t add_half2(uint32_t y, uint32_t r)
 {
+    const float lo = __fadd_rn(__half2float(__ushort_as_half((unsigned short)(y & 0xFFFFu))),
+                               __half2float(__ushort_as_half((unsigned short)(r & 0xFFFFu))));
+    const float hi = __fadd_rn(__half2float(__ushort_as_half((unsigned short)(y >> 16))),
+                               __half2float(__ushort_as_half((unsigned short)(r >> 16))));
+    return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
+}
+
+__device__ __forceinline__ uint16_t silu_mul_half(uint16_t gb, uint16_t ub)
+{
+    const float g = __half2float(__ushort_as_half(gb));
+    const float u = __half2float(__ushort_as_half(ub));
+    const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+    return __half_as_ushort(__float2half_rn(__fmul_rn(silu, u)));
+}
+
+__device__ __forceinline__ uint32_t silu_mul_half2(uint32_t g, uint32_t u)
+{
+    return (uint32_t)silu_mul_half((uint16_t)(g & 0xFFFFu), (uint16_t)(u & 0xFFFFu)) |
+           ((uint32_t)silu_mul_half((uint16_t)(g >> 16), (uint16_t)(u >> 16)) << 16);
+}
+
+__device__ __forceinline__ void store_outputs(const GemmArgs &a, uint8_t *stg, int m0, int cc, int n0, int lane,
+                                              float sc, float sx, const int32_t *acc, int quarter, int bar_id)
+{
+    if (a.epi == kEpiI32) {
+        // INT32 partial sums only (the K-split layer scales them after its
+        // all-reduce)
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            if (m0 + q < a.M) a.acc_dbg[(size_t)(m0 + q) * a.N + n0 + lane] = acc[q];
+        return;
+    }
     __syncwarp();  // the previous chunk's reads of the staging block are done
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
@@ -255,12 +311,39 @@ __device__ __forceinline__ void store_outputs(const GemmArgs &a, uint8_t *stg, i
         *reinterpret_cast<uint16_t *>(stg + q * 64 + lane * 2) = scale_to_half(acc[q], sxq, sc);
     }
     __syncwarp();
+    if (a.epi == kEpiSiluMul) {
+        named_barrier(bar_id, 128);  // the group's four warps have staged their chunk
+        if (quarter < 2) {
+            // output column of this warp's first gate channel: 64 per panel
+            const int o0 = (n0 / 128) * 64 + quarter * 32;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int q = 8 * j + (lane >> 2);
-        const int m = m0 + q;
-        const uint4 v = *reinterpret_cast<const uint4 *>(stg + q * 64 + (lane & 3) * 16);
-        if (m < a.M) *reinterpret_cast<uint4 *>(a.Y + (size_t)m * a.N + n0 + (lane & 3) * 8) = v;
+            for (int j = 0; j < 2; ++j) {
+                const int q = 8 * j + (lane >> 2);
+                const int m = m0 + q;
+                const uint4 g = *reinterpret_cast<const uint4 *>(stg + q * 64 + (lane & 3) * 16);
+                const uint4 u = *reinterpret_cast<const uint4 *>(stg + 2048 + q * 64 + (lane & 3) * 16);
+                const uint4 v = make_uint4(silu_mul_half2(g.x, u.x), silu_mul_half2(g.y, u.y),
+                                           silu_mul_half2(g.z, u.z), silu_mul_half2(g.w, u.w));
+                if (m < a.M) *reinterpret_cast<uint4 *>(a.Y + (size_t)m * a.ldy + o0 + (lane & 3) * 8) = v;
+            }
+        }
+        named_barrier(bar_id, 128);  // the up values have been read
+    } else {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int q = 8 * j + (lane >> 2);
+            const int m = m0 + q;
+            uint4 v = *reinterpret_cast<const uint4 *>(stg + q * 64 + (lane & 3) * 16);
+            if (m < a.M) {
+                const size_t o = (size_t)m * a.ldy + n0 + (lane & 3) * 8;
+                if (a.epi == kEpiResidual) {
+                    // a plain load: R may be Y itself (this thread reads o before it writes o)
+                    const uint4 r = *reinterpret_cast<const uint4 *>(a.R + o);
+                    v = make_uint4(add_half2(v.x, r.x), add_half2(v.y, r.y), add_half2(v.z, r.z), add_half2(v.w, r.w));
+                }
+                *reinterpret_cast<uint4 *>(a.Y + o) = v;
+            }
+        }
     }
     if (a.acc_dbg) {
 #pragma unroll
@@ -284,11 +367,11 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *v)
     }
 }
 
-template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR>
-__global__ void __launch_bounds__(gemm_threads(BN), 1)
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR, bool HALF>
+__global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs a)
 {
-    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR>;
+    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR, HALF>;
     static_assert(!PAIR || (A_TMEM && BN == 256), "pairs: 256-token tiles, A in TMEM");
     constexpr int kCh = C::kChunks;
     constexpr int kDq = dequant_groups(BN);
@@ -747,9 +830,10 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
 #pragma unroll
             for (int q = 0; q < C::kSx; ++q) {
                 const int m = m0 + q * 32 + lane;
-                sx_reg[q] = (q * 32 + lane < BN && m < a.M) ? half_bits_to_float(__ldcg(a.s_x + m)) : 0.0f;
+                sx_reg[q] = (a.epi != kEpiI32 && q * 32 + lane < BN && m < a.M) ? half_bits_to_float(__ldcg(a.s_x + m))
+                                                                                   : 0.0f;
             }
-            const float sc = half_bits_to_float(__ldg(a.s_c + n));
+            const float sc = a.epi != kEpiI32 ? half_bits_to_float(__ldg(a.s_c + n)) : 0.0f;
             // (scheduled units: CTAs, or CTA pairs; cta_index maps one to
             // the CTA that holds this CTA's panel)
             const int c_lo = partial ? cta_of(t * ks, P, T) : sched;
@@ -760,10 +844,10 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
             // theirs: wait for the count and sum their partials now, while
             // this CTA's own MMAs for the tile are still running.
             bool ready = true;
-            constexpr bool kPresum = (BN <= 64);
+            constexpr bool kPresum = (BN <= 64) && !HALF;  // (registers: 64 per thread in a half CTA)
             // accumulator columns per TMEM load (16 where the pre-summed
             // partials of a 64-wide tile already hold 64 registers)
-            constexpr int kGrp = BN < 64 ? BN : (kPresum ? 16 : (kEpi == 2 ? 32 : 64));
+            constexpr int kGrp = HALF ? 16 : BN < 64 ? BN : (kPresum ? 16 : (kEpi == 2 ? 32 : 64));
             int32_t pre[kPresum ? BN : 1];
             if (finisher) {
                 // Every lane of every later contributor counts its own
@@ -908,7 +992,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), 1)
 #pragma unroll
                         for (int q = 1; q < C::kSx; ++q)
                             if ((cc >> 1) == q) sxr = sx_reg[q];
-                        store_outputs(a, stg, m0 + cc * 16, cc, n - lane, lane, sc, sxr, acc);
+                        store_outputs(a, stg, m0 + cc * 16, cc, n - lane, lane, sc, sxr, acc, quarter, 2 + eg);
                     }
                     }
                 }
@@ -1006,11 +1090,11 @@ EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false>
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false, bool HALF = false>
 cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR>;
-    auto kern = w4a8_gemm_kernel<BN, KST, SW, SX, A_TMEM, PAIR>;
+    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR, HALF>;
+    auto kern = w4a8_gemm_kernel<BN, KST, SW, SX, A_TMEM, PAIR, HALF>;
     // the shared-memory opt-in is per device and per kernel: set it once
     static std::atomic<unsigned long long> opted_in{0};
     int dev = 0;
@@ -1054,10 +1138,19 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
 // allows (A in shared memory); the weight ring fills the rest of the
 // ~227 KB of shared memory, since it is what streams from HBM.
 template <bool A_TMEM>
-cudaError_t dispatch(int BN, int KST, bool pair, const CUtensorMap &tmap, const GemmArgs &args, int grid,
-                     cudaStream_t stream)
+cudaError_t dispatch(int BN, int KST, bool pair, bool half, const CUtensorMap &tmap, const GemmArgs &args,
+                     int grid, cudaStream_t stream)
 {
     if constexpr (A_TMEM) {
+        // half CTAs (two per SM, consecutive GEMMs overlap): 128-wide K
+        // blocks, rings sized to half the SM
+        if (half) {
+            switch (BN) {
+            case 16: return launch_cfg<16, 128, 10, 7, true, false, true>(tmap, args, grid, stream);
+            case 32: return launch_cfg<32, 128, 8, 6, true, false, true>(tmap, args, grid, stream);
+            default: return launch_cfg<64, 128, 8, 4, true, false, true>(tmap, args, grid, stream);
+            }
+        }
         // 256-token tiles on CTA pairs: half the X8 tile per CTA, so a ring
         // of 8 stages fits beside 10 weight stages
         if (pair) {
@@ -1082,6 +1175,7 @@ cudaError_t dispatch(int BN, int KST, bool pair, const CUtensorMap &tmap, const 
 }
 
 std::atomic<int> g_cta_pairs{1};
+std::atomic<int> g_half_ctas{0};
 std::atomic<int> g_narrow_tiles{1};
 
 // SMs of the current device, looked up once per device.
@@ -1119,6 +1213,11 @@ void set_narrow_tiles(bool enable)
     g_narrow_tiles.store(enable ? 1 : 0);
 }
 
+void set_half_ctas(bool enable)
+{
+    g_half_ctas.store(enable ? 1 : 0);
+}
+
 // Token tile width.  Up to 128 tokens one tile covers M.  Beyond that,
 // 256-token tiles unless they are so few that stream-K shares each among
 // many CTAs: every extra CTA on a tile costs a full INT32 partial that the
@@ -1138,10 +1237,12 @@ static int block_n_for(int M, int N, int K, bool narrow)
     }
 }
 
+// The most stream-K units a tile width can give: 128-wide K blocks (the
+// narrowest stage any configuration uses), so that sizes derived from it
+// hold for every stage width, CTA pairs and half CTAs included.
 static long long units_for(int M, int N, int K, int BN)
 {
-    const int KST = (BN <= 64 && K % 256 == 0) ? 256 : 128;
-    return (long long)((M + BN - 1) / BN) * (N / kPanelRows) * (K / KST);
+    return (long long)((M + BN - 1) / BN) * (N / kPanelRows) * (K / 128);
 }
 
 int gemm_block_n(int M, int N, int K)
@@ -1170,7 +1271,7 @@ size_t gemm_workspace_bytes(int M, int N, int K)
 cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
                         const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
                         int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream, int *tmap_status,
-                        const uint16_t *X)
+                        const uint16_t *X, int epi, const uint16_t *R, int ldx)
 {
     *tmap_status = 0;
     const int BN = gemm_block_n(M, N, K);
@@ -1178,7 +1279,9 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     // panels, each CTA holding half of the X8 tile) when N allows it, with
     // 256-wide K stages where K allows them
     const bool pair = a_in_tmem && g_cta_pairs.load(std::memory_order_relaxed) && BN == 256 && N % 256 == 0;
-    const int KST = (pair && K % 256 == 0) ? 256 : (BN <= 64 && K % 256 == 0) ? 256 : 128;
+    // token tiles up to 64 in half CTAs (two per SM) when selected
+    const bool half = a_in_tmem && !pair && BN <= 64 && g_half_ctas.load(std::memory_order_relaxed);
+    const int KST = half ? 128 : (pair && K % 256 == 0) ? 256 : (BN <= 64 && K % 256 == 0) ? 256 : 128;
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) {
         *tmap_status = -1;
@@ -1186,7 +1289,8 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     }
     CUtensorMap tmap;
     const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    const cuuint64_t gstride[1] = {(cuuint64_t)K};
+    // X8 rows are ldx bytes apart (K, or the full row of a K-split layer's slice)
+    const cuuint64_t gstride[1] = {(cuuint64_t)(ldx > 0 ? ldx : K)};
     const cuuint32_t box[2] = {(cuuint32_t)kBlockK, (cuuint32_t)(pair ? BN / 2 : BN)};
     const cuuint32_t estride[2] = {1, 1};
     CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(X8), gdim, gstride, box, estride,
@@ -1198,7 +1302,8 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     }
     const int sms = sm_count();
     // stream-K units: (tile, K block) per CTA, or per CTA pair
-    const long long units = pair ? (long long)((M + BN - 1) / BN) * (N / 256) * (K / KST) : units_for(M, N, K, BN);
+    const long long units = pair ? (long long)((M + BN - 1) / BN) * (N / 256) * (K / KST)
+                                 : (long long)((M + BN - 1) / BN) * (N / kPanelRows) * (K / KST);
     // Stream-K over the SMs, except when the tiles alone fill at least 70%
     // of them: then one whole tile per CTA (or pair), so that no tile is
     // split and no CTA waits at the end for another's partial sums (the
@@ -1216,6 +1321,9 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     args.s_c = s_c;
     args.Y = Y;
     args.acc_dbg = acc_dbg;
+    args.epi = epi;
+    args.R = R;
+    args.ldy = (epi == kEpiSiluMul) ? N / 2 : N;
     args.ws_cnt = reinterpret_cast<int32_t *>(workspace);
     args.X = X;
     args.X8w = const_cast<int8_t *>(X8);
@@ -1232,8 +1340,8 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     args.ngroups = K / G;
     args.total = (int)units;
     args.timeout_ns = 2000000000ull;  // 2 s for one wait: far beyond any legitimate one
-    return a_in_tmem ? dispatch<true>(BN, KST, pair, tmap, args, (int)grid, stream)
-                     : dispatch<false>(BN, KST, false, tmap, args, (int)grid, stream);
+    return a_in_tmem ? dispatch<true>(BN, KST, pair, half, tmap, args, (int)grid, stream)
+                     : dispatch<false>(BN, KST, false, false, tmap, args, (int)grid, stream);
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value)

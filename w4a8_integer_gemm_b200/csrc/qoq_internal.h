@@ -19,9 +19,11 @@ constexpr size_t kCounterBytes = 8192;
 // split-tile counters: kMaxCtas CTAs x 2 epilogue groups x 4 quarters
 static_assert(kMaxCtas * 2 * 4 * 4 <= kCounterBytes - 64, "counter region");
 
-// z_dbg and q_dbg may be null (optional inspection outputs).
+// z_dbg and q_dbg may be null (optional inspection outputs).  With gate_up
+// set, W holds a gate/up pair ([N/2 gate rows; N/2 up rows]) and packed
+// panel p takes gate rows 64p..64p+63 then up rows 64p..64p+63.
 cudaError_t launch_pack(const float *W, int N, int K, int G, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g,
-                        uint8_t *zs, uint8_t *z_dbg, uint8_t *q_dbg, cudaStream_t stream);
+                        uint8_t *zs, uint8_t *z_dbg, uint8_t *q_dbg, cudaStream_t stream, bool gate_up = false);
 
 // rowsum may be null.
 cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16_t *s_x, int32_t *rowsum,
@@ -49,6 +51,10 @@ void set_cta_pairs(bool enable);
 // default on.
 void set_narrow_tiles(bool enable);
 
+// Whether token tiles up to 64 run in half-SM CTAs (two per SM, so that
+// consecutive GEMMs overlap).
+void set_half_ctas(bool enable);
+
 // Word offsets, in the workspace's counter region, of the two counters of
 // the one-launch layer call (after the split-tile counters of up to kMaxCtas CTAs).
 constexpr int kFusedReadyWord = 2000;
@@ -56,14 +62,28 @@ constexpr int kFusedDoneWord = 2001;
 // Largest M for which the layer call can quantize inside the GEMM kernel.
 constexpr int kFusedMaxRows = kMaxCtas;
 
+// ldx: bytes between rows of X8 (0 means K).
 // Returns cudaSuccess or the launch / tensor-map error.  `tmap_status`
 // receives the driver status of the tensor-map encode (0 on success).
 // With X non-null the kernel first quantizes X into X8 and s_x (the one-launch
 // call); otherwise it reads them.
+// Output-side fusion kinds of the GEMM epilogue (the values of
+// qoq_epilogue_kind in qoq.h).
+constexpr int kEpiPlain = 0;
+constexpr int kEpiResidual = 1;
+constexpr int kEpiSiluMul = 2;
+// (internal) INT32 sums only, into acc_dbg: the partial GEMM of a K-split layer
+constexpr int kEpiI32 = 3;
+
+// Y[m][n] = fp16(((float)acc[m][n] * s_x[m]) * s_c[n]) over [M][N].
+cudaError_t launch_epilogue_i32(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_c, int M, int N,
+                                uint16_t *Y, cudaStream_t stream);
+
 cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
                         const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
                         int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream,
-                        int *tmap_status, const uint16_t *X = nullptr);
+                        int *tmap_status, const uint16_t *X = nullptr, int epi = kEpiPlain,
+                        const uint16_t *R = nullptr, int ldx = 0);
 
 
 // Device error flag of the current device: read and clear (synchronous).

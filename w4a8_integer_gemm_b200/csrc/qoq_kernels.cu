@@ -59,12 +59,17 @@ __device__ __forceinline__ uint32_t stage2_code(int w8, float sgf, int z)
 __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, int N, int K, int G,
                                                    uint8_t *__restrict__ Wp, uint16_t *__restrict__ s_c,
                                                    uint8_t *__restrict__ s_g, uint8_t *__restrict__ zs,
-                                                   uint8_t *__restrict__ z_dbg, uint8_t *__restrict__ q_dbg)
+                                                   uint8_t *__restrict__ z_dbg, uint8_t *__restrict__ q_dbg,
+                                                   bool gate_up)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n = blockIdx.x * 8 + warp;
+    const int n = blockIdx.x * 8 + warp;  // packed row (output channel position)
     if (n >= N) return;
-    const float *w = W + (size_t)n * K;
+    // the source row: itself, or for a gate/up pair, gate row 64p + r (r < 64)
+    // or up row N/2 + 64p + r - 64 of packed panel p
+    const int pr = n % kPanelRows, pp = n / kPanelRows;
+    const int src = !gate_up ? n : (pr < 64 ? 64 * pp + pr : N / 2 + 64 * pp + pr - 64);
+    const float *w = W + (size_t)src * K;
 
     float amax = 0.0f;
     for (int k = lane * 4; k < K; k += 128) {
@@ -235,12 +240,45 @@ __global__ void dequant_kernel(const uint8_t *__restrict__ Wp, const uint8_t *__
     dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
 }
 
+// ------------------------------------------------ stand-alone epilogue --
+// The output rescaling on INT32 sums that were computed elsewhere (the
+// all-reduced partials of a K-split layer): one thread per 8 consecutive
+// outputs of a row, 16-byte loads and stores, the GEMM epilogue's rounding
+// order.  HBM-bound: 4 + 2 bytes per output.
+__global__ void __launch_bounds__(256) epilogue_i32_kernel(const int32_t *__restrict__ acc,
+                                                           const uint16_t *__restrict__ s_x,
+                                                           const uint16_t *__restrict__ s_c, int M, int N,
+                                                           uint16_t *__restrict__ Y)
+{
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int per_row = N / 8;
+    if (idx >= (size_t)M * per_row) return;
+    const int m = (int)(idx / per_row);
+    const int n0 = (int)(idx % per_row) * 8;
+    const int4 a0 = __ldcs(reinterpret_cast<const int4 *>(acc + (size_t)m * N + n0));
+    const int4 a1 = __ldcs(reinterpret_cast<const int4 *>(acc + (size_t)m * N + n0 + 4));
+    const uint4 c = __ldg(reinterpret_cast<const uint4 *>(s_c + n0));
+    const float sx = half_bits_to_float(__ldg(s_x + m));
+    const int av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = __fmul_rn(__fmul_rn(__int2float_rn(av[2 * i]), sx),
+                                   half_bits_to_float((uint16_t)(cw[i] & 0xFFFFu)));
+        const float hi = __fmul_rn(__fmul_rn(__int2float_rn(av[2 * i + 1]), sx),
+                                   half_bits_to_float((uint16_t)(cw[i] >> 16)));
+        o[i] = (uint32_t)float_to_half_bits(lo) | ((uint32_t)float_to_half_bits(hi) << 16);
+    }
+    *reinterpret_cast<uint4 *>(Y + (size_t)m * N + n0) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 }  // namespace
 
 cudaError_t launch_pack(const float *W, int N, int K, int G, uint8_t *Wp, uint16_t *s_c, uint8_t *s_g, uint8_t *zs,
-                        uint8_t *z_dbg, uint8_t *q_dbg, cudaStream_t stream)
+                        uint8_t *z_dbg, uint8_t *q_dbg, cudaStream_t stream, bool gate_up)
 {
-    pack_kernel<<<(N + 7) / 8, 256, 0, stream>>>(W, N, K, G, Wp, s_c, s_g, zs, z_dbg, q_dbg);
+    pack_kernel<<<(N + 7) / 8, 256, 0, stream>>>(W, N, K, G, Wp, s_c, s_g, zs, z_dbg, q_dbg, gate_up);
     return cudaGetLastError();
 }
 
@@ -262,6 +300,14 @@ cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, X, K, X8, s_x, rowsum);
     if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_epilogue_i32(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_c, int M, int N,
+                                uint16_t *Y, cudaStream_t stream)
+{
+    const size_t threads = (size_t)M * (N / 8);
+    epilogue_i32_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(acc, s_x, s_c, M, N, Y);
     return cudaGetLastError();
 }
 
