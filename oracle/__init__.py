@@ -84,6 +84,8 @@ def _load():
         lib.oracle_gemm_i32.restype = None
         lib.oracle_epilogue.argtypes = [_P, _P, _P, _I64, _I64, _P]
         lib.oracle_epilogue.restype = None
+        lib.oracle_quantize_weights_w8.argtypes = [_P, _I64, _I64, _P, _P]
+        lib.oracle_quantize_weights_w8.restype = None
         lib.oracle_double_to_half_rn.argtypes = [ctypes.c_double]
         lib.oracle_double_to_half_rn.restype = ctypes.c_uint16
         lib.oracle_epilogue_residual.argtypes = [_P, _P, _P, _I64, _I64, _P, _P]
@@ -261,6 +263,25 @@ def epilogue_silu_mul(acc: np.ndarray, s_x: np.ndarray, s_c: np.ndarray) -> np.n
     Out = np.zeros((M, N2 // 2), np.uint16)
     _load().oracle_epilogue_silu_mul(_ptr(acc), _ptr(s_x), _ptr(s_c), M, N2, _ptr(Out))
     return Out
+
+
+def quantize_weights_w8(W: np.ndarray):
+    """The W8A8 yardstick's weights: (W8 int8 [N][K], s_w uint16 FP16 bits [N])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    W8 = np.zeros((N, K), np.int8)
+    s_w = np.zeros(N, np.uint16)
+    _load().oracle_quantize_weights_w8(_ptr(W), N, K, _ptr(s_w), _ptr(W8))
+    return W8, s_w
+
+
+def linear_w8a8(X_half: np.ndarray, W: np.ndarray) -> dict:
+    """The W8A8 yardstick layer on the CPU."""
+    W8, s_w = quantize_weights_w8(W)
+    X8, s_x = quant_act(X_half)
+    acc = gemm_i32(X8, W8)
+    Y = epilogue(acc, s_x, s_w)
+    return dict(W8=W8, s_w=s_w, X8=X8, s_x=s_x, acc=acc, Y=Y)
 
 
 # ------------------------------------------------------------ chains ----

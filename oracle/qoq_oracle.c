@@ -272,6 +272,39 @@ void oracle_epilogue(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_
 }
 
 /* ------------------------------------------------------------------------ */
+/* The W8A8 yardstick's weights ("QServe: Low Bit Width Does Not Guarantee   */
+/* High Throughput", section 2 "Motivation": W8A8 keeps 8-bit weights and    */
+/* 8-bit activations on INT8 tensor cores; the same page's Figure 3 roofline */
+/* compares it with W4A16 and W4A8).  Reading: per-channel symmetric INT8    */
+/* over the full range, s_w = fp16(max|W_n| / 127), W8 = clamp(round(W /    */
+/* s_w), -127, 127), round half to even, with the stored FP16 scale; a zero  */
+/* scale gives a zero row.  The product and the epilogue are the W4A8        */
+/* layer's (oracle_gemm_i32, oracle_epilogue) with W8 in place of W8hat.      */
+/* ------------------------------------------------------------------------ */
+void oracle_quantize_weights_w8(const float *W, int64_t N, int64_t K, uint16_t *s_w, int8_t *W8)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const float *w = W + n * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(w[k]);
+            if (a > amax) amax = a;
+        }
+        uint16_t bits = oracle_float_to_half_rn(amax / 127.0f);
+        float sw = oracle_half_to_float(bits);
+        s_w[n] = bits;
+        for (int64_t k = 0; k < K; ++k) {
+            if (sw == 0.0f) { W8[n * K + k] = 0; continue; }
+            float r = rintf(w[k] / sw);
+            if (r > 127.0f) r = 127.0f;
+            if (r < -127.0f) r = -127.0f;
+            W8[n * K + k] = (int8_t)r;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* binary64 -> binary16, round to nearest, ties to even, from the format     */
 /* definition (11 significant bits; subnormals in units of 2^-24).            */
 /* ------------------------------------------------------------------------ */
