@@ -89,6 +89,8 @@ def parse():
                     help="restrict the workload to one shape name (for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-w8a8", action="store_true",
+                    help="skip the W8A8 yardstick (the same kernel with INT8 weights) beside each point")
     ap.add_argument("--eager", action="store_true",
                     help="launch every kernel from Python in the timed steps instead of replaying a CUDA graph")
     ap.add_argument("--a-smem", action="store_true",
@@ -274,7 +276,10 @@ def run_ours(args, rank, world, local, dist):
     cases = []
     for i, s in enumerate(work.shapes):
         X, W = wl.make_case(work, i)
-        packed = q.qoq_pack_weights(W.to(dev), s.G)
+        Wd = W.to(dev)
+        packed = q.qoq_pack_weights(Wd, s.G)
+        w8 = None if args.no_w8a8 else q.qoq_quantize_weights_w8(Wd)
+        del Wd
         Xd = X.to(dev)
         X8 = torch.empty(s.M, s.K, dtype=torch.int8, device=dev)
         s_x = torch.empty(max(s.M, 8), dtype=torch.int16, device=dev)
@@ -282,7 +287,7 @@ def run_ours(args, rank, world, local, dist):
         ws = torch.zeros(q.qoq_gemm_workspace_bytes(s.M, s.N, s.K, s.G), dtype=torch.uint8, device=dev)
         Xh = X.pin_memory()
         Yh = torch.empty(s.M, s.N, dtype=torch.float16, pin_memory=True)
-        cases.append(dict(s=s, packed=packed, X=Xd, X8=X8, s_x=s_x, Y=Y, ws=ws, Xh=Xh, Yh=Yh,
+        cases.append(dict(s=s, packed=packed, w8=w8, X=Xd, X8=X8, s_x=s_x, Y=Y, ws=ws, Xh=Xh, Yh=Yh,
                           bound=roofline.bound(s.M, s.N, s.K, s.G, P8, BW)))
         del W
     torch.cuda.synchronize()
@@ -309,10 +314,12 @@ def run_ours(args, rank, world, local, dist):
 
     def enqueue(st, subset, layer=True):
         """Launch on stream st, per shape of `subset`, the layer call
-        (qoq_w4a8_linear: the quantizer kernel, then the GEMM kernel), or
-        the GEMM kernel alone."""
+        (qoq_w4a8_linear: the quantizer kernel, then the GEMM kernel), the
+        GEMM kernel alone, or (layer="w8a8") the W8A8 yardstick's GEMM."""
         for c in subset:
-            if layer:
+            if layer == "w8a8":
+                q.qoq_w8a8_gemm(c["X8"], c["s_x"], c["w8"][0], c["w8"][1], Y=c["Y"], workspace=c["ws"], stream=st)
+            elif layer:
                 q.qoq_w4a8_linear(c["X"], c["packed"], X8=c["X8"], s_x=c["s_x"], Y=c["Y"], workspace=c["ws"],
                                   stream=st)
             else:
@@ -344,11 +351,19 @@ def run_ours(args, rank, world, local, dist):
         return tot
 
     def isolated(reps=3):
-        """Per shape, L2 flushed, kernel(s) alone: the per-point breakdown."""
+        """Per shape, L2 flushed, kernel(s) alone: the per-point breakdown
+        (layer call, GEMM, and the W8A8 yardstick's GEMM)."""
         out = []
         for j, c in enumerate(cases):
-            st = gm = 0.0
+            st = gm = w8 = 0.0
             for _ in range(reps):
+                if c["w8"] is not None:
+                    flush.zero_()
+                    ev[j][0].record(stream)
+                    enqueue(stream, [c], "w8a8")
+                    ev[j][1].record(stream)
+                    torch.cuda.synchronize()
+                    w8 += ev[j][0].elapsed_time(ev[j][1])
                 flush.zero_()
                 ev[j][0].record(stream)
                 enqueue(stream, [c], True)
@@ -360,12 +375,14 @@ def run_ours(args, rank, world, local, dist):
                 torch.cuda.synchronize()
                 st += ev[j][0].elapsed_time(ev[j][1])
                 gm += ev[j][2].elapsed_time(ev[j][3])
-            out.append((st / reps, gm / reps))
+            out.append((st / reps, gm / reps, w8 / reps if c["w8"] is not None else None))
         return out
 
     chains = {"step": (cases, True)}
     for b, sub in regimes.items():
         chains["gemm_" + b] = (sub, False)
+        if not args.no_w8a8:
+            chains["w8a8_" + b] = (sub, "w8a8")
     for _ in range(max(3, args.warmup)):
         for name, (sub, layer) in chains.items():
             timed(name, sub, layer)
@@ -405,6 +422,8 @@ def run_ours(args, rank, world, local, dist):
     clocks = clk.summary()
     chain_ms = {b: statistics.median(timed("gemm_" + b, sub, False) for _ in range(args.steps))
                 for b, sub in regimes.items()}
+    w8_chain_ms = {} if args.no_w8a8 else {
+        b: statistics.median(timed("w8a8_" + b, sub, "w8a8") for _ in range(args.steps)) for b, sub in regimes.items()}
     iso = isolated()
     if q.qoq_device_error() != q.QOQ_OK:
         raise RuntimeError("device error in the timed region")
@@ -413,7 +432,7 @@ def run_ours(args, rank, world, local, dist):
     tot_ops = 0.0
     for j, c in enumerate(cases):
         s = c["s"]
-        pair_ms, gm_ms = iso[j]
+        pair_ms, gm_ms, w8_ms = iso[j]
         ops = roofline.ops(s.M, s.N, s.K)
         byt = roofline.algorithmic_bytes(s.M, s.N, s.K, s.G)
         roof = roofline.roofline_ops_per_s(s.M, s.N, s.K, s.G, P8, BW)
@@ -422,6 +441,14 @@ def run_ours(args, rank, world, local, dist):
                     "isolated_step_us": round(pair_ms * 1e3, 2), "isolated_gemm_us": round(gm_ms * 1e3, 2),
                     "isolated_gemm_tops": round(tops, 2), "isolated_gemm_gbs": round(byt / (gm_ms * 1e-3) / 1e9, 1),
                     "roofline_tops": round(roof / 1e12, 2), "isolated_frac": round(tops * 1e12 / roof, 4)})
+        if w8_ms is not None:
+            b8 = roofline.algorithmic_bytes_w8(s.M, s.N, s.K)
+            roof8 = min(P8, ops * BW / b8)
+            per[-1].update({"w8a8_isolated_gemm_us": round(w8_ms * 1e3, 2),
+                            "w8a8_isolated_gemm_tops": round(ops / (w8_ms * 1e-3) / 1e12, 2),
+                            "w8a8_roofline_tops": round(roof8 / 1e12, 2),
+                            "w8a8_isolated_frac": round(ops / (w8_ms * 1e-3) / roof8, 4),
+                            "w4a8_speedup_over_w8a8": round(w8_ms / gm_ms, 3)})
         tot_ops += ops
     tot_ms = statistics.median(step_ms)
     ms_step, value = aggregate(tot_ops, tot_ms, world, dist)
@@ -432,6 +459,28 @@ def run_ours(args, rank, world, local, dist):
     dom = max(by_bound, key=lambda b: by_bound[b]["chain_us"])
     rl = dict(by_bound[dom])
     rl["by_bound"] = by_bound
+    # the W8A8 yardstick over the same chains (its own algorithmic bytes:
+    # INT8 weights, N*K), and where it overtakes W4A8 (isolated points)
+    w8a8 = None
+    if w8_chain_ms:
+        w8a8 = {"kernel": "w4a8_gemm_kernel (W8 variant: INT8 weights by TMA, no dequantization)", "by_bound": {}}
+        for b, sub in regimes.items():
+            shp = [c["s"] for c in sub]
+            ms = w8_chain_ms[b]
+            ops_b = sum(roofline.ops(x.M, x.N, x.K) for x in shp)
+            byt_b = sum(roofline.algorithmic_bytes_w8(x.M, x.N, x.K) for x in shp)
+            ent = {"chain_us": round(ms * 1e3, 2), "tops": round(ops_b / (ms * 1e-3) / 1e12, 1),
+                   "w4a8_chain_us": round(chain_ms[b] * 1e3, 2),
+                   "w4a8_speedup": round(ms / chain_ms[b], 3)}
+            if b == "hbm":
+                ach = byt_b / (ms * 1e-3) / 1e9
+                ent.update({"achieved_gbs": round(ach, 1), "frac_of_hbm": round(ach / peaks["hbm_gbs"], 4)})
+            else:
+                ach = ops_b / (ms * 1e-3) / 1e12
+                ent.update({"frac_of_int8_peak": round(ach / peaks["int8_tops"], 4)})
+            w8a8["by_bound"][b] = ent
+        cross = [p["M"] for p in per if "w4a8_speedup_over_w8a8" in p and p["w4a8_speedup_over_w8a8"] < 1.0]
+        w8a8["first_M_where_w8a8_is_faster"] = min(cross) if cross else None
 
     # end to end through the public API from pinned host memory
     e2e = None
@@ -479,7 +528,7 @@ def run_ours(args, rank, world, local, dist):
                    "eager_ms_per_step": None if eager_ms is None else round(eager_ms, 5),
                    "kernels": ("per shape qoq_w4a8_linear: the per-token quantizer kernel, then the GEMM kernel "
                                "(programmatic dependent launch)")},
-        "roofline": rl, "points": per, "clocks": clocks, "e2e": e2e,
+        "roofline": rl, "points": per, "clocks": clocks, "e2e": e2e, "w8a8_yardstick": w8a8,
         "gpu_launches": 2 * n_sh * args.steps,
         "a_operand": "smem" if args.a_smem else "tmem",
     }

@@ -308,6 +308,39 @@ QOQ_API int qoq_w4a8_gemm_i32(const int8_t *X8, int ldx, const uint8_t *Wp, cons
 QOQ_API int qoq_epilogue_i32(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_c,
                      int M, int N, uint16_t *Y, void *stream);
 
+/* ------------------------------------------------------------------------
+ * The W8A8 yardstick (the pages have no kernel for it; they use W8A8 as the
+ * INT8-peak side of their roofline argument, "QServe: Low Bit Width Does Not
+ * Guarantee High Throughput", section 2 "Motivation", Figure 3). The same
+ * GEMM kernel with 8-bit weights loaded by TMA straight into the tensor
+ * cores' operand slots: no unpacking and no dequantization, twice the weight
+ * bytes. Comparing it with qoq_w4a8_gemm measures what the 4-bit stream saves
+ * at small M and what the dequantization costs at large M.
+ * ------------------------------------------------------------------------ */
+
+/* Per-channel symmetric INT8 weights: s_w[n] = fp16(max_k |W[n][k]| / 127),
+ * W8[n][k] = clamp(round(W[n][k] / s_w[n]), -127, 127), IEEE division, round
+ * half to even, with the stored FP16 scale; a zero scale gives a zero row.
+ *   W    device, float32 [N][K], read only (finite).
+ *   W8   device, int8_t [N][K], written.
+ *   s_w  device, uint16_t [N] FP16 bits, written.
+ * N and K follow the GEMM limits. */
+QOQ_API int qoq_quantize_weights_w8(const float *W, int N, int K, int8_t *W8, uint16_t *s_w,
+                            void *stream);
+
+/* Y[m][n] = fp16( ((float)acc * s_x[m]) * s_w[n] ), acc = sum_k X8[m][k] * W8[n][k]
+ * (INT32, exact), the epilogue of qoq_w4a8_gemm.
+ *   X8, s_x   device, from qoq_quant_act_per_token.
+ *   W8, s_w   device, from qoq_quantize_weights_w8.
+ *   Y         device, uint16_t [M][N] FP16 bits, written.
+ *   acc_dbg   device int32_t [M][N] or NULL: the raw INT32 sums.
+ *   workspace, workspace_bytes  as for qoq_w4a8_gemm, sized by
+ *             qoq_gemm_workspace_bytes(M, N, K, 128).
+ * Limits as for qoq_w4a8_gemm. */
+QOQ_API int qoq_w8a8_gemm(const int8_t *X8, const uint16_t *s_x, const int8_t *W8, const uint16_t *s_w,
+                  int M, int N, int K, uint16_t *Y, int32_t *acc_dbg,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
 /* The whole W4A8 linear layer in one call: the per-token quantization of
  * qoq_quant_act_per_token followed by qoq_w4a8_gemm.
  *

@@ -55,6 +55,8 @@ SIGNATURES = {
     "qoq_w4a8_gemm_fused": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "qoq_w4a8_gemm_i32": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "qoq_epilogue_i32": (_I, [_P, _P, _P, _I, _I, _P, _P]),
+    "qoq_quantize_weights_w8": (_I, [_P, _I, _I, _P, _P, _P]),
+    "qoq_w8a8_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "qoq_w4a8_linear": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "qoq_dequant_weights_i8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "qoq_set_gemm_a_in_tmem": (_I, [_I]),
@@ -336,6 +338,37 @@ def qoq_epilogue_i32(acc: torch.Tensor, s_x: torch.Tensor, s_c: torch.Tensor, Y:
         Y = torch.empty(M, N, dtype=torch.float16, device=acc.device)
     st = lib().qoq_epilogue_i32(_ptr(acc), _ptr(s_x), _ptr(s_c), M, N, _ptr(Y), _stream(stream))
     _check("qoq_epilogue_i32", st)
+    return Y
+
+
+def qoq_quantize_weights_w8(W: torch.Tensor, stream=None):
+    """W fp32 [N, K] -> (W8 int8 [N, K], s_w int16 [N] FP16 bits): the W8A8 yardstick's weights."""
+    _need(W, torch.float32, "W")
+    N, K = W.shape
+    W8 = torch.empty(N, K, dtype=torch.int8, device=W.device)
+    s_w = torch.empty(max(N, 8), dtype=torch.int16, device=W.device)
+    st = lib().qoq_quantize_weights_w8(_ptr(W), N, K, _ptr(W8), _ptr(s_w), _stream(stream))
+    _check("qoq_quantize_weights_w8", st)
+    return W8, s_w
+
+
+def qoq_w8a8_gemm(X8: torch.Tensor, s_x: torch.Tensor, W8: torch.Tensor, s_w: torch.Tensor,
+                  Y: Optional[torch.Tensor] = None, acc_dbg: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The W8A8 yardstick: Y fp16 [M, N] = fp16(((float)(X8 . W8^T) * s_x) * s_w)."""
+    _need(X8, torch.int8, "X8")
+    _need(W8, torch.int8, "W8")
+    M, K = X8.shape
+    N, K2 = W8.shape
+    if K != K2:
+        raise ValueError("K mismatch between X8 and W8")
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float16, device=X8.device)
+    if workspace is None:
+        workspace = gemm_workspace(max(M, 1), N, K, 128, X8.device)
+    st = lib().qoq_w8a8_gemm(_ptr(X8), _ptr(s_x), _ptr(W8), _ptr(s_w), M, N, K, _ptr(Y), _ptr(acc_dbg),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("qoq_w8a8_gemm", st)
     return Y
 
 

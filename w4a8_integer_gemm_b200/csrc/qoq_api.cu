@@ -229,6 +229,36 @@ int qoq_epilogue_i32(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_
     return from_cuda(qoq::launch_epilogue_i32(acc, s_x, s_c, M, N, Y, (cudaStream_t)stream));
 }
 
+int qoq_quantize_weights_w8(const float *W, int N, int K, int8_t *W8, uint16_t *s_w, void *stream)
+{
+    if (!valid_nk(N, K)) return QOQ_ERR_INVALID_ARG;
+    if (!W || !W8 || !s_w || !aligned16(W) || !aligned16(W8) || !aligned16(s_w)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(qoq::launch_quantize_w8(W, N, K, W8, s_w, (cudaStream_t)stream));
+}
+
+int qoq_w8a8_gemm(const int8_t *X8, const uint16_t *s_x, const int8_t *W8, const uint16_t *s_w, int M, int N, int K,
+                  uint16_t *Y, int32_t *acc_dbg, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (M < 0 || M > kMaxM || !valid_nk(N, K)) return QOQ_ERR_INVALID_ARG;
+    if (M == 0) return QOQ_OK;
+    if (!X8 || !s_x || !W8 || !s_w || !Y || !workspace) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(X8) || !aligned16(s_x) || !aligned16(W8) || !aligned16(s_w) || !aligned16(Y) ||
+        !aligned16(workspace) || (acc_dbg && !aligned16(acc_dbg)))
+        return QOQ_ERR_INVALID_ARG;
+    if (!qoq::gemm_shape_supported(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    if (workspace_bytes < qoq::gemm_workspace_bytes(M, N, K)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    int tmap_status = 0;
+    cudaError_t e = qoq::launch_gemm(X8, s_x, nullptr, s_w, nullptr, nullptr, M, N, K, 128, Y, acc_dbg, workspace,
+                                     false, (cudaStream_t)stream, &tmap_status, nullptr, qoq::kEpiPlain, nullptr, 0,
+                                     W8);
+    if (tmap_status == -1) return QOQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
 int qoq_w4a8_linear(const uint16_t *X, int M, int N, int K, int group_size, const uint8_t *Wp,
                     const uint16_t *s_c, const uint8_t *s_g, const uint8_t *zs, int8_t *X8, uint16_t *s_x,
                     uint16_t *Y, void *workspace, size_t workspace_bytes, void *stream)

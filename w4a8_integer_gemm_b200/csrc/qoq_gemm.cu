@@ -127,14 +127,16 @@ constexpr int kPrologueStages = 2;
 // stage, and one group's barrier waits and TMEM stores overlap the other's
 // arithmetic.  Wider tiles keep one group (384 threads, 168 registers) for
 // their larger epilogue.
-__host__ __device__ constexpr int dequant_groups(int BN) { return BN <= 64 ? 2 : 1; }
+// The W8A8 yardstick (W8) has no dequantization: its INT8 weights go
+// straight from HBM into the MMA's A slots.
+__host__ __device__ constexpr int dequant_groups(int BN, bool W8 = false) { return W8 ? 0 : BN <= 64 ? 2 : 1; }
 // 256-token tiles drain their accumulator with two epilogue warpgroups (one
 // per 128 tokens): with one accumulator in TMEM the MMAs of the next tile
 // wait for the epilogue, so its length is lost tensor time.
 __host__ __device__ constexpr int epilogue_groups(int BN) { return BN == 256 ? 2 : 1; }
-__host__ __device__ constexpr int gemm_threads(int BN)
+__host__ __device__ constexpr int gemm_threads(int BN, bool W8 = false)
 {
-    return 128 * (1 + dequant_groups(BN) + epilogue_groups(BN));
+    return 128 * (1 + dequant_groups(BN, W8) + epilogue_groups(BN));
 }
 
 __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
@@ -149,7 +151,10 @@ __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
 // tensor memory), so that the next GEMM's CTA can be resident beside it and
 // stream and dequantize its weights while this one finishes (token tiles up
 // to 64, K blocks of 128).
-template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false, bool HALF = false>
+// W8: the W8A8 yardstick: INT8 weights [N][K] loaded by 2-D tiled TMA into
+// shared-memory A slots (one per X8 slot, SW == SX), no weight ring and no
+// dequant warps.
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false, bool HALF = false, bool W8 = false>
 struct GemmCfg {
     static constexpr int kChunks = KST / kBlockK;        // packed 8 KB chunks per K block
     static constexpr int kXRows = PAIR ? BN / 2 : BN;    // token rows of X8 this CTA holds
@@ -159,7 +164,7 @@ struct GemmCfg {
     static constexpr int kABytes = A_TMEM ? 0 : kChunks * kATile;
     // one W slot: the K block's packed chunks, each followed by its group
     // tables when G = 128 (the layout of the packed buffer itself)
-    static constexpr int kWSlot = kChunks * (kChunkBytes + kChunkTabBytes);
+    static constexpr int kWSlot = W8 ? 0 : kChunks * (kChunkBytes + kChunkTabBytes);
     // shared memory: [X8 ring][A ring (A in shared memory only)][W ring][barriers]
     static constexpr int kAOff = SX * kXSlot;
     static constexpr int kWOff = kAOff + SX * kABytes;
@@ -190,7 +195,8 @@ struct GemmCfg {
     // completed one (unless SW >= SX + 2, when the group's own previous A-slot
     // wait already proves that fill consumed).  The kernel keeps the simpler
     // sufficient rule: each weight slot belongs to one group.
-    static_assert(SW % dequant_groups(BN) == 0, "each weight slot belongs to one dequant group");
+    static_assert(W8 || SW % dequant_groups(BN) == 0, "each weight slot belongs to one dequant group");
+    static_assert(!W8 || (!A_TMEM && !PAIR && !HALF && SW == SX), "W8A8: A slots in shared memory, one per X8 slot");
     static_assert(kXSlot % 1024 == 0 && kAOff % 1024 == 0 && kWOff % 1024 == 0, "swizzle atoms");
     // two half CTAs per SM: 228 KB of shared memory (1 KB reserved per CTA)
     // and 512 TMEM columns between them
@@ -367,14 +373,15 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *v)
     }
 }
 
-template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR, bool HALF>
-__global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
-    w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs a)
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR, bool HALF, bool W8>
+__global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
+    w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                     const GemmArgs a)
 {
-    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR, HALF>;
+    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR, HALF, W8>;
     static_assert(!PAIR || (A_TMEM && BN == 256), "pairs: 256-token tiles, A in TMEM");
     constexpr int kCh = C::kChunks;
-    constexpr int kDq = dequant_groups(BN);
+    constexpr int kDq = dequant_groups(BN, W8);
     constexpr int kEpiWarp0 = 4 + 4 * kDq;  // first epilogue warp
     constexpr int kEpi = epilogue_groups(BN);
     extern __shared__ uint8_t smem_raw[];
@@ -438,10 +445,20 @@ __global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
         const int t = u / ks;
         const int kb = u - t * ks;
         const int n_tile = panel_of(t);
-        const uint32_t st = sbase + C::kWOff + s * C::kWSlot;
-        const uint32_t bytes = (uint32_t)(kCh * cstride);
-        mbar_arrive_expect_tx(wfull_bar(s), bytes);
-        bulk_load(st, a.Wp + chunk_offset(n_tile, kb * kCh, a.K, a.G), bytes, wfull_bar(s));
+        if constexpr (W8) {
+            // W8A8: the K block's [128 channels][KST] INT8 tile, straight
+            // into A slot s (128-byte swizzled K-major, as the MMA reads it)
+            mbar_arrive_expect_tx(wfull_bar(s), (uint32_t)C::kABytes);
+#pragma unroll
+            for (int c = 0; c < kCh; ++c)
+                tma_load_2d(sbase + C::kAOff + s * C::kABytes + c * C::kATile, &tmap_w, (kb * kCh + c) * kBlockK,
+                            n_tile * kPanelRows, wfull_bar(s));
+        } else {
+            const uint32_t st = sbase + C::kWOff + s * C::kWSlot;
+            const uint32_t bytes = (uint32_t)(kCh * cstride);
+            mbar_arrive_expect_tx(wfull_bar(s), bytes);
+            bulk_load(st, a.Wp + chunk_offset(n_tile, kb * kCh, a.K, a.G), bytes, wfull_bar(s));
+        }
         issued |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
     };
@@ -457,7 +474,8 @@ __global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
         for (int s = 0; s < SX; ++s) {
             // 4 dequant warps (of each CTA of a pair) + the X8 producer (of
             // CTA 0 of a pair, whose expected bytes cover both halves)
-            mbar_init(afull_bar(s), PAIR ? 9 : 5);
+            // (W8A8: the X8 producer alone)
+            mbar_init(afull_bar(s), W8 ? 1 : PAIR ? 9 : 5);
             mbar_init(xaempty_bar(s), 1);    // MMA commit
         }
         for (int b = 0; b < C::kAccBufs; ++b) {
@@ -474,6 +492,9 @@ __global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
         }
     }
     if (threadIdx.x == 64) prefetch_tmap(&tmap_x);
+    if constexpr (W8) {
+        if (threadIdx.x == 32) prefetch_tmap(&tmap_w);
+    }
     // The next kernel in the stream may launch now; whatever it reads from
     // this GEMM it must read after its own griddepcontrol.wait.
     grid_launch_dependents();
@@ -507,7 +528,9 @@ __global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
             int s = n_pro == SW ? 0 : n_pro;
             uint32_t ph = (n_pro == SW) ? 1u : 0u;
             for (int u = i_begin + n_pro; u < i_end; ++u) {
-                if (!wait_bounded(wempty_bar(s), ph ^ 1u, abort_flag, budget)) break;
+                // a weight slot is free once the dequant warps have read it
+                // (W8A8: once the MMAs reading the A slot have completed)
+                if (!wait_bounded(W8 ? xaempty_bar(s) : wempty_bar(s), ph ^ 1u, abort_flag, budget)) break;
                 issue_weights(u, s, ph);
                 if (++s == SW) {
                     s = 0;
@@ -585,6 +608,13 @@ __global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
                         ok = false;
                         break;
                     }
+                    if constexpr (W8) {
+                        // W8A8: the weight tile of this slot has landed too
+                        if (!wait_x(wfull_bar(s), ph)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                     tc_fence_after();
                     const uint32_t st = sbase + s * C::kXSlot;
 #pragma unroll
@@ -632,6 +662,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
             drain_wait(mmadone_bar, 0, 200000000ull);
         }
     } else if (warp >= 4 && warp < kEpiWarp0) {
+      if constexpr (!W8) {
         // ------------------------------------------------------ dequant --
         // With two groups of four warps, group 0 takes the CTA's even
         // stages and group 1 the odd ones.
@@ -740,6 +771,7 @@ __global__ void __launch_bounds__(gemm_threads(BN), HALF ? 2 : 1)
                 px ^= 1u;
             }
         }
+      }
     } else if (warp >= kEpiWarp0) {
         // ----------------------------------------------------- epilogue --
         const int quarter = warp & 3;
@@ -1090,11 +1122,12 @@ EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false, bool HALF = false>
-cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream)
+template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR = false, bool HALF = false, bool W8 = false>
+cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, cudaStream_t stream,
+                       const CUtensorMap *tmap_w = nullptr)
 {
-    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR, HALF>;
-    auto kern = w4a8_gemm_kernel<BN, KST, SW, SX, A_TMEM, PAIR, HALF>;
+    using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR, HALF, W8>;
+    auto kern = w4a8_gemm_kernel<BN, KST, SW, SX, A_TMEM, PAIR, HALF, W8>;
     // the shared-memory opt-in is per device and per kernel: set it once
     static std::atomic<unsigned long long> opted_in{0};
     int dev = 0;
@@ -1112,7 +1145,7 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     // touches X8 or s_x.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(gemm_threads(BN));
+    cfg.blockDim = dim3(gemm_threads(BN, W8));
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -1128,7 +1161,7 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
         attr[1].val.clusterDim.z = 1;
         cfg.numAttrs = 2;
     }
-    e = cudaLaunchKernelEx(&cfg, kern, tmap, args);
+    e = cudaLaunchKernelEx(&cfg, kern, tmap, tmap_w ? *tmap_w : tmap, args);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1171,6 +1204,27 @@ cudaError_t dispatch(int BN, int KST, bool pair, bool half, const CUtensorMap &t
     case 64: return launch_cfg<64, 128, A_TMEM ? 16 : 12, A_TMEM ? 8 : 4, A_TMEM>(tmap, args, grid, stream);
     case 128: return launch_cfg<128, 128, A_TMEM ? 10 : 10, A_TMEM ? 8 : 3, A_TMEM>(tmap, args, grid, stream);
     default: return launch_cfg<256, 128, A_TMEM ? 6 : 8, A_TMEM ? 5 : 3, A_TMEM>(tmap, args, grid, stream);
+    }
+}
+
+// The W8A8 yardstick: A and X8 slots in pairs (one stage each), as many as
+// shared memory holds.
+cudaError_t dispatch_w8(int BN, int KST, const CUtensorMap &tmap, const CUtensorMap &tmap_w, const GemmArgs &args,
+                        int grid, cudaStream_t stream)
+{
+    if (KST == 256) {
+        switch (BN) {
+        case 16: return launch_cfg<16, 256, 5, 5, false, false, false, true>(tmap, args, grid, stream, &tmap_w);
+        case 32: return launch_cfg<32, 256, 5, 5, false, false, false, true>(tmap, args, grid, stream, &tmap_w);
+        default: return launch_cfg<64, 256, 4, 4, false, false, false, true>(tmap, args, grid, stream, &tmap_w);
+        }
+    }
+    switch (BN) {
+    case 16: return launch_cfg<16, 128, 8, 8, false, false, false, true>(tmap, args, grid, stream, &tmap_w);
+    case 32: return launch_cfg<32, 128, 8, 8, false, false, false, true>(tmap, args, grid, stream, &tmap_w);
+    case 64: return launch_cfg<64, 128, 8, 8, false, false, false, true>(tmap, args, grid, stream, &tmap_w);
+    case 128: return launch_cfg<128, 128, 6, 6, false, false, false, true>(tmap, args, grid, stream, &tmap_w);
+    default: return launch_cfg<256, 128, 4, 4, false, false, false, true>(tmap, args, grid, stream, &tmap_w);
     }
 }
 
@@ -1271,10 +1325,13 @@ size_t gemm_workspace_bytes(int M, int N, int K)
 cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
                         const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
                         int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream, int *tmap_status,
-                        const uint16_t *X, int epi, const uint16_t *R, int ldx)
+                        const uint16_t *X, int epi, const uint16_t *R, int ldx, const int8_t *W8)
 {
     *tmap_status = 0;
     const int BN = gemm_block_n(M, N, K);
+    // W8A8 yardstick: INT8 weights in shared-memory A slots, single CTAs
+    const bool w8 = W8 != nullptr;
+    if (w8) a_in_tmem = false;
     // 256-token tiles run on CTA pairs (one M = 256 MMA over two weight
     // panels, each CTA holding half of the X8 tile) when N allows it, with
     // 256-wide K stages where K allows them
@@ -1299,6 +1356,20 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     if (r != CUDA_SUCCESS) {
         *tmap_status = (int)r;
         return cudaErrorInvalidValue;
+    }
+    CUtensorMap tmap_w;
+    if (w8) {
+        // [N][K] INT8 weights, [128 channels][128 K] boxes, 128-byte swizzle
+        const cuuint64_t wdim[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        const cuuint64_t wstride[1] = {(cuuint64_t)K};
+        const cuuint32_t wbox[2] = {(cuuint32_t)kBlockK, (cuuint32_t)kPanelRows};
+        r = enc(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(W8), wdim, wstride, wbox, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            *tmap_status = (int)r;
+            return cudaErrorInvalidValue;
+        }
     }
     const int sms = sm_count();
     // stream-K units: (tile, K block) per CTA, or per CTA pair
@@ -1340,6 +1411,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     args.ngroups = K / G;
     args.total = (int)units;
     args.timeout_ns = 2000000000ull;  // 2 s for one wait: far beyond any legitimate one
+    if (w8) return dispatch_w8(BN, KST, tmap, tmap_w, args, (int)grid, stream);
     return a_in_tmem ? dispatch<true>(BN, KST, pair, half, tmap, args, (int)grid, stream)
                      : dispatch<false>(BN, KST, false, false, tmap, args, (int)grid, stream);
 }

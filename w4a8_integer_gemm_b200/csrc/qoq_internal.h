@@ -62,7 +62,9 @@ constexpr int kFusedDoneWord = 2001;
 // Largest M for which the layer call can quantize inside the GEMM kernel.
 constexpr int kFusedMaxRows = kMaxCtas;
 
-// ldx: bytes between rows of X8 (0 means K).
+// ldx: bytes between rows of X8 (0 means K).  W8 non-null: the W8A8
+// yardstick, INT8 weights [N][K] in place of the packed ones (Wp, s_g, zs
+// unused; s_c holds the weights' per-channel scales).
 // Returns cudaSuccess or the launch / tensor-map error.  `tmap_status`
 // receives the driver status of the tensor-map encode (0 on success).
 // With X non-null the kernel first quantizes X into X8 and s_x (the one-launch
@@ -75,6 +77,9 @@ constexpr int kEpiSiluMul = 2;
 // (internal) INT32 sums only, into acc_dbg: the partial GEMM of a K-split layer
 constexpr int kEpiI32 = 3;
 
+// W8A8 yardstick weights: per-channel symmetric INT8, s_w = fp16(max|W|/127).
+cudaError_t launch_quantize_w8(const float *W, int N, int K, int8_t *W8, uint16_t *s_w, cudaStream_t stream);
+
 // Y[m][n] = fp16(((float)acc[m][n] * s_x[m]) * s_c[n]) over [M][N].
 cudaError_t launch_epilogue_i32(const int32_t *acc, const uint16_t *s_x, const uint16_t *s_c, int M, int N,
                                 uint16_t *Y, cudaStream_t stream);
@@ -83,7 +88,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
                         const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
                         int32_t *acc_dbg, void *workspace, bool a_in_tmem, cudaStream_t stream,
                         int *tmap_status, const uint16_t *X = nullptr, int epi = kEpiPlain,
-                        const uint16_t *R = nullptr, int ldx = 0);
+                        const uint16_t *R = nullptr, int ldx = 0, const int8_t *W8 = nullptr);
 
 
 // Device error flag of the current device: read and clear (synchronous).

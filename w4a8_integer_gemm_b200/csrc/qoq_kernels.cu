@@ -240,6 +240,39 @@ __global__ void dequant_kernel(const uint8_t *__restrict__ Wp, const uint8_t *__
     dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
 }
 
+// ------------------------------------------- W8A8 yardstick weights --
+// One warp per output channel: s_w = fp16(max|W| / 127), then
+// W8 = clamp(round(W / s_w), -127, 127) with IEEE division and round half to
+// even, using the stored FP16 scale (a zero scale gives a zero row).
+__global__ void __launch_bounds__(256) quantize_w8_kernel(const float *__restrict__ W, int N, int K,
+                                                          int8_t *__restrict__ W8, uint16_t *__restrict__ s_w)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = blockIdx.x * 8 + warp;
+    if (n >= N) return;
+    const float *w = W + (size_t)n * K;
+    float amax = 0.0f;
+    for (int k = lane * 4; k < K; k += 128) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(w + k));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    amax = warp_max(amax);
+    const uint16_t bits = float_to_half_bits(__fdiv_rn(amax, 127.0f));
+    const float sw = half_bits_to_float(bits);
+    if (lane == 0) s_w[n] = bits;
+    for (int k = lane * 4; k < K; k += 128) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(w + k));
+        const float e[4] = {v.x, v.y, v.z, v.w};
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int c = sw == 0.0f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(e[i], sw)), -127.0f), 127.0f);
+            word |= (uint32_t)(c & 0xFF) << (8 * i);
+        }
+        *reinterpret_cast<uint32_t *>(W8 + (size_t)n * K + k) = word;
+    }
+}
+
 // ------------------------------------------------ stand-alone epilogue --
 // The output rescaling on INT32 sums that were computed elsewhere (the
 // all-reduced partials of a K-split layer): one thread per 8 consecutive
@@ -300,6 +333,12 @@ cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, X, K, X8, s_x, rowsum);
     if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_w8(const float *W, int N, int K, int8_t *W8, uint16_t *s_w, cudaStream_t stream)
+{
+    quantize_w8_kernel<<<(N + 7) / 8, 256, 0, stream>>>(W, N, K, W8, s_w);
     return cudaGetLastError();
 }
 

@@ -25,6 +25,12 @@ def algorithmic_bytes(M: int, N: int, K: int, G: int) -> int:
     return N * K // 2 + 2 * N * (K // G) + 2 * N + M * K + 2 * M + 2 * M * N
 
 
+def algorithmic_bytes_w8(M: int, N: int, K: int) -> int:
+    """The W8A8 yardstick: INT8 weights and their FP16 channel scales, X8 with
+    its token scales, FP16 Y."""
+    return N * K + 2 * N + M * K + 2 * M + 2 * M * N
+
+
 def act_quant_bytes(M: int, K: int) -> int:
     """FP16 X read, INT8 X8 written, FP16 s_x written."""
     return 2 * M * K + M * K + 2 * M
