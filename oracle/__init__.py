@@ -86,6 +86,12 @@ def _load():
         lib.oracle_epilogue.restype = None
         lib.oracle_quantize_weights_w8.argtypes = [_P, _I64, _I64, _P, _P]
         lib.oracle_quantize_weights_w8.restype = None
+        lib.oracle_smooth_lambda.argtypes = [_P, _I64, _I64, ctypes.c_double, _P]
+        lib.oracle_smooth_lambda.restype = None
+        lib.oracle_kv4_quantize.argtypes = [_P, _I64, _I64, _P, _P, _P]
+        lib.oracle_kv4_quantize.restype = None
+        lib.oracle_kv4_attention.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]
+        lib.oracle_kv4_attention.restype = None
         lib.oracle_double_to_half_rn.argtypes = [ctypes.c_double]
         lib.oracle_double_to_half_rn.restype = ctypes.c_uint16
         lib.oracle_epilogue_residual.argtypes = [_P, _P, _P, _I64, _I64, _P, _P]
@@ -282,6 +288,62 @@ def linear_w8a8(X_half: np.ndarray, W: np.ndarray) -> dict:
     acc = gemm_i32(X8, W8)
     Y = epilogue(acc, s_x, s_w)
     return dict(W8=W8, s_w=s_w, X8=X8, s_x=s_x, acc=acc, Y=Y)
+
+
+# ---------------------------------------------------- KV4 attention ----
+def _bits16(x):
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float16:
+        x = x.view(np.uint16)
+    return np.ascontiguousarray(x, np.uint16)
+
+
+def smooth_lambda(K: np.ndarray, alpha: float = 0.5) -> np.ndarray:
+    """SmoothAttention factors of one KV head: K [L][d] FP16 -> lambda [d] FP16 bits."""
+    K = _bits16(K)
+    L, d = K.shape
+    lam = np.zeros(d, np.uint16)
+    _load().oracle_smooth_lambda(_ptr(K), L, d, float(alpha), _ptr(lam))
+    return lam
+
+
+def kv4_quantize(X: np.ndarray, lam: np.ndarray = None):
+    """X [L][d] FP16 -> (codes int8 [L][d] in -8..7, s uint16 FP16 bits [d]); with lam,
+    X is divided by it first (the smoothed keys)."""
+    X = _bits16(X)
+    L, d = X.shape
+    codes = np.zeros((L, d), np.int8)
+    s = np.zeros(d, np.uint16)
+    lp = None if lam is None else _bits16(lam)
+    _load().oracle_kv4_quantize(_ptr(X), L, d, None if lp is None else _ptr(lp), _ptr(codes), _ptr(s))
+    return codes, s
+
+
+def kv4_attention(q: np.ndarray, k_codes: np.ndarray, s_k: np.ndarray, v_codes: np.ndarray,
+                  s_v: np.ndarray, lam: np.ndarray) -> np.ndarray:
+    """One sequence: q [Hq][d] FP16; codes [Hkv][L][d]; s_k, s_v, lam [Hkv][d] FP16 bits.
+    Returns out [Hq][d] FP16 bits."""
+    q = _bits16(q)
+    Hq, d = q.shape
+    Hkv, L, d2 = k_codes.shape
+    assert d2 == d and Hq % Hkv == 0
+    out = np.zeros((Hq, d), np.uint16)
+    _load().oracle_kv4_attention(_ptr(q), _ptr(np.ascontiguousarray(k_codes, np.int8)), _ptr(_bits16(s_k)),
+                                 _ptr(np.ascontiguousarray(v_codes, np.int8)), _ptr(_bits16(s_v)),
+                                 _ptr(_bits16(lam)), Hq, Hkv, L, d, _ptr(out))
+    return out
+
+
+def kv4_decode(q: np.ndarray, K: np.ndarray, V: np.ndarray, alpha: float = 0.5) -> dict:
+    """The whole KV4 step for one sequence on the CPU: q [Hq][d], K, V [Hkv][L][d] FP16."""
+    Hkv, L, d = K.shape
+    lam = np.stack([smooth_lambda(K[g], alpha) for g in range(Hkv)])
+    kq = [kv4_quantize(K[g], lam[g]) for g in range(Hkv)]
+    vq = [kv4_quantize(V[g]) for g in range(Hkv)]
+    k_codes = np.stack([c for c, _ in kq]); s_k = np.stack([s for _, s in kq])
+    v_codes = np.stack([c for c, _ in vq]); s_v = np.stack([s for _, s in vq])
+    out = kv4_attention(q, k_codes, s_k, v_codes, s_v, lam)
+    return dict(lam=lam, k_codes=k_codes, s_k=s_k, v_codes=v_codes, s_v=s_v, out=out)
 
 
 # ------------------------------------------------------------ chains ----

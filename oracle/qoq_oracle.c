@@ -47,6 +47,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #ifdef _OPENMP
@@ -370,6 +371,115 @@ void oracle_epilogue_silu_mul(const int32_t *acc, const uint16_t *s_x, const uin
             double silu = gd / (1.0 + exp(-gd));
             Out[m * I + j] = oracle_double_to_half_rn(silu * ud);
         }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* KV4 decode attention with SmoothAttention.                                 */
+/*                                                                            */
+/* [LBW] section 4 (the SmoothAttention paragraph) and [GUIDE] "The           */
+/* Architecture" subsection 3: a per-channel factor lambda_c moves the        */
+/* outliers of the cached keys into the (uncached) query, K'_c = K_c /        */
+/* lambda_c and Q'_c = Q_c * lambda_c, so Q'K'^T = QK^T; lambda_c =           */
+/* max|K_c|^alpha, alpha = 0.5.  The smoothed keys and the values are stored */
+/* as 4-bit integers with per-channel scales.  Readings where the pages are   */
+/* silent:                                                                    */
+/*   - the statistics are per (sequence, KV head, channel c), over the       */
+/*     cached tokens; lambda is stored in FP16, floored at 1e-5 (a zero      */
+/*     channel keeps a finite factor), computed as fp16(sqrt(max|K|)) for    */
+/*     alpha = 0.5 and as fp16(pow(max|K|, alpha)) otherwise, in binary64;   */
+/*   - K' = (float)K / (float)lambda in FP32 (IEEE division);                */
+/*   - 4-bit codes are symmetric: s_c = fp16(max_l |X'[l][c]| / 7) in FP32,  */
+/*     code = clamp(round(X' / s_c), -8, 7), round half to even; a zero      */
+/*     scale gives zero codes (the same rule as the guide's illustration,    */
+/*     applied per channel);                                                  */
+/*   - attention for one new query token per sequence and query head h      */
+/*     (KV head h / G, G = Hq / Hkv): score_l = sum_c Q'_c K^_lc / sqrt(d)    */
+/*     with K^ = s_k * code, softmax over the L cached tokens, out_c =      */
+/*     sum_l p_l V^_lc, all in binary64, output rounded once to FP16.        */
+/* ------------------------------------------------------------------------ */
+void oracle_smooth_lambda(const uint16_t *K, int64_t L, int64_t d, double alpha, uint16_t *lambda)
+{
+    for (int64_t c = 0; c < d; ++c) {
+        float m = 0.0f;
+        for (int64_t l = 0; l < L; ++l) {
+            float a = fabsf(oracle_half_to_float(K[l * d + c]));
+            if (a > m) m = a;
+        }
+        double v = (alpha == 0.5) ? sqrt((double)m) : pow((double)m, alpha);
+        if (v < 1e-5) v = 1e-5;
+        lambda[c] = oracle_double_to_half_rn(v);
+    }
+}
+
+/* X [L][d] FP16 bits -> codes [L][d] (int8 in -8..7) and s [d] FP16 bits.
+ * lambda (FP16 bits [d]) or NULL: the keys are divided by it first. */
+void oracle_kv4_quantize(const uint16_t *X, int64_t L, int64_t d, const uint16_t *lambda,
+                         int8_t *codes, uint16_t *s)
+{
+    for (int64_t c = 0; c < d; ++c) {
+        float lam = lambda ? oracle_half_to_float(lambda[c]) : 1.0f;
+        float m = 0.0f;
+        for (int64_t l = 0; l < L; ++l) {
+            float x = oracle_half_to_float(X[l * d + c]);
+            if (lambda) x = x / lam;
+            float a = fabsf(x);
+            if (a > m) m = a;
+        }
+        uint16_t sb = oracle_float_to_half_rn(m / 7.0f);
+        float sc = oracle_half_to_float(sb);
+        s[c] = sb;
+        for (int64_t l = 0; l < L; ++l) {
+            float x = oracle_half_to_float(X[l * d + c]);
+            if (lambda) x = x / lam;
+            if (sc == 0.0f) { codes[l * d + c] = 0; continue; }
+            float r = rintf(x / sc);
+            if (r > 7.0f) r = 7.0f;
+            if (r < -8.0f) r = -8.0f;
+            codes[l * d + c] = (int8_t)r;
+        }
+    }
+}
+
+/* One sequence: q [Hq][d] FP16 bits (the unsmoothed query), per KV head g:
+ * k_codes/v_codes [Hkv][L][d], s_k/s_v/lambda [Hkv][d] FP16 bits.
+ * out [Hq][d] FP16 bits. */
+void oracle_kv4_attention(const uint16_t *q, const int8_t *k_codes, const uint16_t *s_k,
+                          const int8_t *v_codes, const uint16_t *s_v, const uint16_t *lambda,
+                          int64_t Hq, int64_t Hkv, int64_t L, int64_t d, uint16_t *out)
+{
+    int64_t G = Hq / Hkv;
+    double inv = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(static)
+    for (int64_t h = 0; h < Hq; ++h) {
+        int64_t g = h / G;
+        const int8_t *kc = k_codes + g * L * d;
+        const int8_t *vc = v_codes + g * L * d;
+        double *sc = (double *)malloc(sizeof(double) * (size_t)L);
+        double mx = -INFINITY;
+        for (int64_t l = 0; l < L; ++l) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < d; ++c) {
+                double qs = (double)oracle_half_to_float(q[h * d + c]) *
+                            (double)oracle_half_to_float(lambda[g * d + c]);         /* Q' = Q lambda */
+                double kh = (double)oracle_half_to_float(s_k[g * d + c]) * (double)kc[l * d + c];
+                acc += qs * kh;
+            }
+            sc[l] = acc * inv;
+            if (sc[l] > mx) mx = sc[l];
+        }
+        double den = 0.0;
+        for (int64_t l = 0; l < L; ++l) {
+            sc[l] = exp(sc[l] - mx);
+            den += sc[l];
+        }
+        for (int64_t c = 0; c < d; ++c) {
+            double num = 0.0;
+            for (int64_t l = 0; l < L; ++l)
+                num += sc[l] * (double)oracle_half_to_float(s_v[g * d + c]) * (double)vc[l * d + c];
+            out[h * d + c] = oracle_double_to_half_rn(num / den);
+        }
+        free(sc);
     }
 }
 

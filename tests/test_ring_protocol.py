@@ -11,10 +11,15 @@ issue order, and the roles of the kernel:
   * D dequant groups take the units in turn (group u % D).  Each waits for
     its weight fill (wfull), reads it, frees the slot (wempty), waits for a
     free A slot (xaempty), writes it and arrives on afull;
-  * the X8 producer waits for a free X8 slot (xaempty) and issues its copy
-    (afull completes on its bytes);
-  * the MMA waits on afull, consumes unit u, and its commit (after a delay)
-    frees the X8/A slot (xaempty).
+  * the X8 producer waits for a free X8 slot (xaempty) and issues its copy,
+    which completes on the slot's own x8full (the producer's arrival plus
+    the copy's bytes, nothing else);
+  * the MMA waits on afull and x8full, consumes unit u, and its commit
+    (after a delay) frees the X8/A slot (xaempty).
+A second model (run_pair) covers two CTAs of a pair with an abort injected
+at any step: CTA 1 forwards the landing of its X8 half to CTA 0 (x8peer),
+and every producer drains only barriers its own copies complete, so every
+issued copy has landed before the CTA exits.
 Every consumer checks that what it reads is the unit it waited for, so a
 wait that passes on another phase (aliasing) fails the test.  The model is
 shown to catch the weight-slot race of an odd ring shared by two groups.
@@ -66,7 +71,8 @@ def run_rings(SW, SX, D, units, seed, steps=200000, ks=None, acc_bufs=2, epi=1, 
     rng = random.Random(seed)
     wfull = [Barrier(1) for _ in range(SW)]
     wempty = [Barrier(D and 1) for _ in range(SW)]
-    afull = [Barrier(2) for _ in range(SX)]    # the dequant group + the X8 producer (and its bytes)
+    afull = [Barrier(1) for _ in range(SX)]    # the dequant group
+    x8full = [Barrier(1) for _ in range(SX)]   # the X8 producer and its copy's bytes
     xaempty = [Barrier(1) for _ in range(SX)]  # the MMA's commit
     wslot = [None] * SW                        # unit whose weights a slot holds
     xslot = [None] * SX                        # unit whose X8 tile an X8 slot holds
@@ -125,11 +131,11 @@ def run_rings(SW, SX, D, units, seed, steps=200000, ks=None, acc_bufs=2, epi=1, 
             while not xaempty[a].passes((j & 1) ^ 1):
                 yield
             assert xslot[a] is None, f"X8 slot {a} overwritten before the MMA read unit {xslot[a]}"
-            afull[a].arrive(tx=1)
+            x8full[a].arrive(tx=1)
 
             def land(a=a, u=u):
                 xslot[a] = u
-                afull[a].complete_tx(1)
+                x8full[a].complete_tx(1)
             later(land, copy_delay())
             yield
 
@@ -143,7 +149,7 @@ def run_rings(SW, SX, D, units, seed, steps=200000, ks=None, acc_bufs=2, epi=1, 
                 assert acc[b] is None or acc[b][2] == epi, f"tile {t} overwrites accumulator {b} before it was drained"
                 acc[b] = [t, 0, 0]
             a, j = u % SX, u // SX
-            while not afull[a].passes(j & 1):
+            while not (afull[a].passes(j & 1) and x8full[a].passes(j & 1)):
                 yield
             assert aslot[a] == u and xslot[a] == u, f"MMA of unit {u} read A {aslot[a]} and X8 {xslot[a]}"
             acc[b][1] += 1
@@ -277,3 +283,263 @@ def test_the_model_catches_a_weight_slot_shared_by_two_groups():
     with pytest.raises(AssertionError, match="read weight slot"):
         for seed in range(400):
             run_rings(7, 6, 2, units=40, seed=seed)
+
+
+# ------------------------------------------------------------------------
+# CTA pairs and aborts
+# ------------------------------------------------------------------------
+def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_barrier=True,
+             drain_ticks=40, steps=300000):
+    """Two CTAs (or one, pair=False) of the kernel's rings with an abort.
+
+    Each CTA has a weight producer, one dequant group and an X8 producer;
+    CTA 0 issues the MMAs and multicasts each commit to both CTAs' xaempty.
+    Both CTAs' dequant groups arrive on CTA 0's afull.  With
+    own_x8_barrier (the kernel's design) each CTA's X8 copies complete on
+    its own x8full; CTA 1's forwarder waits for its x8full and arrives on
+    CTA 0's x8peer, and the MMA waits on afull, x8full and x8peer.  Without
+    it (the earlier design), both halves' bytes and the producer's arrival
+    counted on CTA 0's afull.
+
+    At step abort_at, CTA abort_cta raises its abort flag (as a timed-out
+    wait does).  A role whose wait is not yet satisfied leaves when its
+    CTA's flag is up; a wait that stays unsatisfied for 2000 ticks raises
+    the flag (the kernel's per-wait budget).  Every role then meets the
+    others at the CTA's final barrier (a pair: both CTAs, the cluster
+    barrier).  After it, if the CTA's flag is up, each producer waits for
+    the barrier phases of the copies it issued: for at most drain_ticks
+    when that phase also needs other roles (the earlier design's bounded
+    grace), until completion when only its own copy completes it.  The
+    model checks that no copy into a CTA lands after that CTA's exit."""
+    rng = random.Random(seed)
+    ncta = 2 if pair else 1
+    clock = [0, 0]
+    inflight = []
+    last_commit = [0]
+    abort = [False] * ncta
+    finished = [0] * ncta
+    nroles = [0] * ncta
+    arrived = [0] * ncta
+    exited = [False] * ncta
+    drains = [[] for _ in range(ncta)]   # per CTA: (barrier, parity, bounded) of issued copies
+
+    def later(action, delay):
+        clock[1] += 1
+        inflight.append([clock[0] + delay, clock[1], action])
+
+    def copy_delay():
+        return rng.randint(1, 30) if rng.random() < 0.9 else rng.randint(60, 400)
+
+    wfull = [[Barrier(1) for _ in range(SW)] for _ in range(ncta)]
+    wempty = [[Barrier(1) for _ in range(SW)] for _ in range(ncta)]
+    x8full = [[Barrier(1) for _ in range(SX)] for _ in range(ncta)]
+    x8peer = [Barrier(1) for _ in range(SX)]
+    if own_x8_barrier:
+        afull = [Barrier(ncta) for _ in range(SX)]            # both CTAs' dequant groups
+    else:
+        afull = [Barrier(ncta + 1) for _ in range(SX)]        # + CTA 0's producer (both halves' bytes)
+    xaempty = [[Barrier(1) for _ in range(SX)] for _ in range(ncta)]
+    wslot = [[None] * SW for _ in range(ncta)]
+    xslot = [[None] * SX for _ in range(ncta)]
+    aslot = [[None] * SX for _ in range(ncta)]
+
+    def landing(c, fn):
+        def act():
+            assert not exited[c], f"a copy landed in CTA {c} after it exited"
+            fn()
+        return act
+
+    def waiting(c, cond, budget=2000):
+        """Yield until cond() holds; return False if the CTA aborts first."""
+        t0 = clock[0]
+        while not cond():
+            if abort[c]:
+                return
+            if clock[0] - t0 > budget:
+                abort[c] = True
+                return
+            yield
+        return True
+
+    def role(c, gen, producer=False):
+        nroles[c] += 1
+
+        def run():
+            yield from gen
+            arrived[c] += 1
+            while sum(arrived) < sum(nroles):          # the final (cluster) barrier
+                yield
+            if producer and abort[c]:
+                for bar, par, bounded, _ in [d for d in drains[c] if d[3] == id(gen)]:
+                    waited = 0
+                    while not bar.passes(par):
+                        if bounded and waited >= drain_ticks:
+                            break
+                        waited += 1
+                        yield
+            finished[c] += 1
+            if finished[c] == nroles[c]:
+                exited[c] = True
+        return run()
+
+    def w_producer(c, me):
+        issued = {}
+        for u in range(units):
+            s, k = u % SW, u // SW
+            ok = yield from waiting(c, lambda s=s, k=k: wempty[c][s].passes((k & 1) ^ 1))
+            if not ok:
+                break
+            wfull[c][s].arrive(tx=1)
+            issued[s] = k & 1
+
+            def land(s=s, u=u):
+                wslot[c][s] = u
+                wfull[c][s].complete_tx(1)
+            later(landing(c, land), copy_delay())
+            yield
+        # wfull: the producer's own arrival and its own copy's bytes only
+        drains[c].extend((wfull[c][s], par, False, me[0]) for s, par in issued.items())
+
+    def dequant(c):
+        for u in range(units):
+            s, k = u % SW, u // SW
+            ok = yield from waiting(c, lambda s=s, k=k: wfull[c][s].passes(k & 1))
+            if not ok:
+                return
+            assert wslot[c][s] == u
+            yield
+            wempty[c][s].arrive()
+            a, j = u % SX, u // SX
+            ok = yield from waiting(c, lambda a=a, j=j: xaempty[c][a].passes((j & 1) ^ 1))
+            if not ok:
+                return
+            aslot[c][a] = u
+            yield
+            afull[a].arrive()
+
+    def x_producer(c, me):
+        issued = {}
+        for u in range(units):
+            a, j = u % SX, u // SX
+            ok = yield from waiting(c, lambda a=a, j=j: xaempty[c][a].passes((j & 1) ^ 1))
+            if not ok:
+                break
+            if own_x8_barrier:
+                bar = x8full[c][a]
+                bar.arrive(tx=1)
+            else:
+                bar = afull[a]
+                if c == 0:
+                    bar.arrive(tx=ncta)            # both halves' bytes
+            issued[a] = (bar, j & 1)
+
+            def land(a=a, u=u, bar=bar):
+                xslot[c][a] = u
+                bar.complete_tx(1)
+            later(landing(c, land), copy_delay())
+            yield
+        # own x8full: exact; the earlier afull also needed the dequant
+        # arrivals, so its drain was bounded by a grace period
+        drains[c].extend((bar, par, not own_x8_barrier, me[0]) for a, (bar, par) in issued.items())
+
+    def forwarder(c):
+        for u in range(units):
+            a, j = u % SX, u // SX
+            ok = yield from waiting(c, lambda a=a, j=j: x8full[c][a].passes(j & 1))
+            if not ok:
+                return
+            yield
+            x8peer[a].arrive()
+
+    def mma():
+        for u in range(units):
+            a, j = u % SX, u // SX
+
+            def ready(a=a, j=j):
+                if not afull[a].passes(j & 1):
+                    return False
+                if own_x8_barrier:
+                    if not x8full[0][a].passes(j & 1):
+                        return False
+                    if pair and not x8peer[a].passes(j & 1):
+                        return False
+                return True
+            ok = yield from waiting(0, ready)
+            if not ok:
+                return
+            for c in range(ncta):
+                assert aslot[c][a] == u and xslot[c][a] == u, f"MMA of unit {u}: CTA {c} A {aslot[c][a]} X8 {xslot[c][a]}"
+            yield
+
+            def commit(a=a):
+                for c in range(ncta):
+                    aslot[c][a] = None
+                    xslot[c][a] = None
+                    xaempty[c][a].arrive()
+            due = max(last_commit[0] + 1, clock[0] + rng.randint(1, 20))
+            last_commit[0] = due
+            later(commit, due - clock[0])
+
+    def producer_role(c, fn):
+        me = [None]
+        gen = fn(c, me)
+        me[0] = id(gen)
+        return role(c, gen, producer=True)
+
+    live = []
+    for c in range(ncta):
+        live += [producer_role(c, w_producer), role(c, dequant(c)), producer_role(c, x_producer)]
+        if pair and own_x8_barrier and c == 1:
+            live.append(role(c, forwarder(c)))
+    live.append(role(0, mma()))
+    step = 0
+    while live or inflight:
+        step += 1
+        if step > steps:
+            raise AssertionError("the model did not finish (a wait that never passes)")
+        if abort_at is not None and step == abort_at:
+            abort[abort_cta] = True
+        # time moves on (landing what is due) about every other step, also
+        # while nothing is in flight (the per-wait budgets run on it)
+        if not live or rng.random() < 0.5:
+            clock[0] += 1
+            done = sorted((f for f in inflight if f[0] <= clock[0]), key=lambda f: (f[0], f[1]))
+            inflight[:] = [f for f in inflight if f[0] > clock[0]]
+            for f in done:
+                f[2]()
+            continue
+        r = rng.choice(live)
+        try:
+            next(r)
+        except StopIteration:
+            live.remove(r)
+    return abort
+
+
+@pytest.mark.parametrize("pair", [False, True], ids=["single", "pair"])
+def test_pair_rings_without_abort(pair):
+    for seed in range(30):
+        run_pair(4, 4, units=23, seed=seed, pair=pair)
+
+
+@pytest.mark.parametrize("pair", [False, True], ids=["single", "pair"])
+@pytest.mark.parametrize("abort_cta", [0, 1])
+def test_abort_at_every_step_lets_every_copy_land(pair, abort_cta):
+    """An abort at any step, in either CTA: every issued copy lands before
+    its CTA exits, and no role waits forever."""
+    if not pair and abort_cta == 1:
+        pytest.skip("one CTA")
+    for seed in range(6):
+        for at in range(1, 400, 3):
+            run_pair(4, 4, units=18, seed=seed, abort_at=at, abort_cta=abort_cta, pair=pair)
+
+
+def test_the_model_catches_the_earlier_x8_drain():
+    """With X8 bytes counted on afull (which also needs the dequant
+    arrivals) and a bounded grace period, some abort leaves a copy landing
+    after the CTA exited."""
+    with pytest.raises(AssertionError, match="landed in CTA"):
+        for seed in range(60):
+            for at in range(1, 300, 2):
+                run_pair(4, 4, units=18, seed=seed, abort_at=at, pair=False, own_x8_barrier=False,
+                         drain_ticks=5)

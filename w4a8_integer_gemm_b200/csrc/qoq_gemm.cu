@@ -38,10 +38,13 @@
 //                   packed chunks with their group tables; also TMEM.
 //       warp 1      MMA issuer (one thread): one barrier wait, KST/32
 //                   tcgen05.mma (K = 32) and one tcgen05.commit per stage.
-//       warp 2      X8 producer: tiled TMA loads of the activation tiles.
-//                   It and the epilogue alone wait for the preceding kernel
+//       warp 2      X8 producer: tiled TMA loads of the activation tiles,
+//                   completing on this CTA's own x8full barrier.  It and
+//                   the epilogue alone wait for the preceding kernel
 //                   (programmatic dependent launch), so weights stream in
 //                   and are dequantized while that kernel still runs.
+//       warp 3      (CTA 1 of a pair) X8 forwarder: once its half of a
+//                   stage's X8 tile has landed, it tells CTA 0's MMA issuer.
 //       dequant     one or two groups of four warps (two for tiles up to 64
 //                   tokens, taking alternate stages): thread r owns output
 //                   channel r of the panel, reads its packed bytes with
@@ -58,17 +61,22 @@
 //     as soon as the dequant warps hold them in registers; with two dequant
 //     groups each slot belongs to one group); an X8/A ring
 //     (slot s holds the X8 tiles of a K block in shared memory and its
-//     dequantized weights in A slot s; one barrier says both are ready, one
-//     commit frees both); and one or two TMEM accumulators, so the MMAs of
-//     the next tile need not wait for the epilogue of the last one.
+//     dequantized weights in A slot s; the MMA waits for the dequant warps'
+//     barrier and for the X8 copies' own barrier, and one commit frees
+//     both); and one or two TMEM accumulators, so the MMAs of the next tile
+//     need not wait for the epilogue of the last one.  Every copy completes
+//     on a barrier that only its issuer's arrival and its own bytes
+//     complete, so an aborted CTA can wait for exactly its own copies.
 //   * CTA pairs (256-token tiles): a cluster of two CTAs computes a
 //     256-channel tile with one M = 256 MMA per K step (cta_group::2);
 //     each CTA dequantizes its own 128-channel panel into its TMEM and
 //     loads half of the X8 tile, CTA 0 issues the MMAs and multicasts the
-//     commits, and the other CTA's warps arrive on CTA 0's barriers.
+//     commits, and the other CTA's dequant warps and X8 forwarder arrive on
+//     CTA 0's barriers.
 //   * Every wait is bounded (per wait, global timer); on expiry the CTA
-//     stops, drains its own in-flight copies and MMAs, frees TMEM, and
-//     raises the device error flag that qoq_device_error() reports.
+//     stops, waits for its own in-flight copies (on their own barriers) and
+//     MMAs, frees TMEM, and raises the device error flag that
+//     qoq_device_error() reports.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -129,14 +137,18 @@ constexpr int kPrologueStages = 2;
 // their larger epilogue.
 // The W8A8 yardstick (W8) has no dequantization: its INT8 weights go
 // straight from HBM into the MMA's A slots.
-__host__ __device__ constexpr int dequant_groups(int BN, bool W8 = false) { return W8 ? 0 : BN <= 64 ? 2 : 1; }
+// Half-SM CTAs (HALF) keep one group, for registers.
+__host__ __device__ constexpr int dequant_groups(int BN, bool W8 = false, bool HALF = false)
+{
+    return W8 ? 0 : (BN <= 64 && !HALF) ? 2 : 1;
+}
 // 256-token tiles drain their accumulator with two epilogue warpgroups (one
 // per 128 tokens): with one accumulator in TMEM the MMAs of the next tile
 // wait for the epilogue, so its length is lost tensor time.
 __host__ __device__ constexpr int epilogue_groups(int BN) { return BN == 256 ? 2 : 1; }
-__host__ __device__ constexpr int gemm_threads(int BN, bool W8 = false)
+__host__ __device__ constexpr int gemm_threads(int BN, bool W8 = false, bool HALF = false)
 {
-    return 128 * (1 + dequant_groups(BN, W8) + epilogue_groups(BN));
+    return 128 * (1 + dequant_groups(BN, W8, HALF) + epilogue_groups(BN));
 }
 
 __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c)
@@ -174,7 +186,7 @@ struct GemmCfg {
     // two accumulators (the MMAs of the next tile run while the epilogue
     // drains the last one) wherever TMEM has room for them
     static constexpr int kAccBufs = (2 * BN + (A_TMEM ? SX * (int)kACols : 0) <= 512) ? 2 : 1;
-    static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * kAccBufs + 2;
+    static constexpr int kNumBars = 2 * SW + 4 * SX + 2 * kAccBufs + 2;
     static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
     // full CTAs: at least ~120 KB so that exactly one CTA (and one TMEM
     // allocation) lives on each SM; +1024 for manual alignment of the
@@ -195,7 +207,7 @@ struct GemmCfg {
     // completed one (unless SW >= SX + 2, when the group's own previous A-slot
     // wait already proves that fill consumed).  The kernel keeps the simpler
     // sufficient rule: each weight slot belongs to one group.
-    static_assert(W8 || SW % dequant_groups(BN) == 0, "each weight slot belongs to one dequant group");
+    static_assert(W8 || SW % dequant_groups(BN, W8, HALF) == 0, "each weight slot belongs to one dequant group");
     static_assert(!W8 || (!A_TMEM && !PAIR && !HALF && SW == SX), "W8A8: A slots in shared memory, one per X8 slot");
     static_assert(kXSlot % 1024 == 0 && kAOff % 1024 == 0 && kWOff % 1024 == 0, "swizzle atoms");
     // two half CTAs per SM: 228 KB of shared memory (1 KB reserved per CTA)
@@ -374,14 +386,14 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *v)
 }
 
 template <int BN, int KST, int SW, int SX, bool A_TMEM, bool PAIR, bool HALF, bool W8>
-__global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
+__global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const GemmArgs a)
 {
     using C = GemmCfg<BN, KST, SW, SX, A_TMEM, PAIR, HALF, W8>;
     static_assert(!PAIR || (A_TMEM && BN == 256), "pairs: 256-token tiles, A in TMEM");
     constexpr int kCh = C::kChunks;
-    constexpr int kDq = dequant_groups(BN, W8);
+    constexpr int kDq = dequant_groups(BN, W8, HALF);
     constexpr int kEpiWarp0 = 4 + 4 * kDq;  // first epilogue warp
     constexpr int kEpi = epilogue_groups(BN);
     extern __shared__ uint8_t smem_raw[];
@@ -391,9 +403,13 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
     // W ring (packed weights + group tables of one K block):
     //   wfull (bulk copy landed), wempty (the dequant warps have read it)
     // X8/A ring (X8 tiles in shared memory, dequantized weights in A slot):
-    //   afull (the slot is ready for the MMAs: the 4 dequant warps of the
-    //   stage have written the A slot, and the X8 producer's arrival plus
-    //   its copies' transaction bytes say the X8 tiles have landed),
+    //   afull (the 4 dequant warps of the stage -- of each CTA of a pair --
+    //   have written the A slot),
+    //   x8full (this CTA's X8 tiles have landed: the X8 producer's arrival
+    //   plus its own copies' bytes, and nothing else, so the producer can
+    //   always wait for its own copies),
+    //   x8peer (pairs, in CTA 0: the other CTA's X8 half has landed; its
+    //   forwarder arrives once that CTA's own x8full completes),
     //   xaempty (the MMAs reading the slot have completed: both the X8
     //   slot and the A slot are free)
     auto wfull_bar = [&](int s) { return bar0 + 8u * s; };
@@ -405,6 +421,8 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
     auto accfull_bar = [&](int b) { return bar0 + 8u * (2 * SW + 2 * SX + b); };
     auto accempty_bar = [&](int b) { return bar0 + 8u * (2 * SW + 2 * SX + C::kAccBufs + b); };
     const uint32_t mmadone_bar = bar0 + 8u * (2 * SW + 2 * SX + 2 * C::kAccBufs);
+    auto x8full_bar = [&](int s) { return mmadone_bar + 16u + 8u * s; };
+    auto x8peer_bar = [&](int s) { return mmadone_bar + 16u + 8u * (SX + s); };
     // one-launch layer call: every token row of X8 and s_x is in memory (the X8
     // producer, the one thread of the CTA that polls the grid-wide count,
     // passes it on to the epilogue warps)
@@ -472,11 +490,11 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
             mbar_init(wempty_bar(s), 4);     // 4 dequant warps
         }
         for (int s = 0; s < SX; ++s) {
-            // 4 dequant warps (of each CTA of a pair) + the X8 producer (of
-            // CTA 0 of a pair, whose expected bytes cover both halves)
-            // (W8A8: the X8 producer alone)
-            mbar_init(afull_bar(s), W8 ? 1 : PAIR ? 9 : 5);
+            // 4 dequant warps (of each CTA of a pair; unused in W8A8)
+            mbar_init(afull_bar(s), PAIR ? 8 : 4);
             mbar_init(xaempty_bar(s), 1);    // MMA commit
+            mbar_init(x8full_bar(s), 1);     // this CTA's X8 producer, plus its bytes
+            mbar_init(x8peer_bar(s), 1);     // (pairs) the other CTA's forwarder
         }
         for (int b = 0; b < C::kAccBufs; ++b) {
             mbar_init(accfull_bar(b), 1);
@@ -560,23 +578,14 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
                         ok = false;
                         break;
                     }
+                    // this CTA's token rows of the tile (a pair: its half),
+                    // completing on its own x8full
                     const uint32_t st = sbase + s * C::kXSlot;
-                    if constexpr (PAIR) {
-                        // each CTA loads its half of the tile's tokens; the
-                        // bytes of both count on CTA 0's barrier
-                        if (rank == 0) mbar_arrive_expect_tx(afull_bar(s), 2 * C::kXSlot);
-                        const uint32_t fb = leader(afull_bar(s));
+                    mbar_arrive_expect_tx(x8full_bar(s), C::kXSlot);
 #pragma unroll
-                        for (int c = 0; c < kCh; ++c)
-                            tma_load_2d_pair(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK,
-                                             m_tile * BN + (int)rank * C::kXRows, fb);
-                    } else {
-                        mbar_arrive_expect_tx(afull_bar(s), C::kXSlot);
-#pragma unroll
-                        for (int c = 0; c < kCh; ++c)
-                            tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN,
-                                        afull_bar(s));
-                    }
+                    for (int c = 0; c < kCh; ++c)
+                        tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK,
+                                    m_tile * BN + (int)rank * C::kXRows, x8full_bar(s));
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
                     if (++s == SX) {
@@ -585,6 +594,33 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
                     }
                 }
                 i = t * ks + ks1;
+            }
+        }
+    } else if (warp == 3) {
+        // -------------------------------------- X8 forwarder (pairs) --
+        // CTA 1 of a pair: once its half of a stage's X8 tile has landed
+        // (its own x8full), tell CTA 0's MMA issuer (x8peer there).
+        if constexpr (PAIR) {
+            if (lane == 0 && rank == 1) {
+                int s = 0;
+                uint32_t ph = 0;
+                bool ok = true;
+                for (int i = i_begin; i < i_end && ok;) {
+                    const int t = i / ks;
+                    const int ks1 = min(ks, i_end - t * ks);
+                    for (int kb = i - t * ks; kb < ks1; ++kb) {
+                        if (!wait_x(x8full_bar(s), ph)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_release_cluster(leader(x8peer_bar(s)));
+                        if (++s == SX) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                    i = t * ks + ks1;
+                }
             }
         }
     } else if (warp == 1) {
@@ -604,13 +640,14 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
                 tc_fence_after();
                 const uint32_t dacc = tmem_base + (uint32_t)(ab * BN);
                 for (int kb = ks0; kb < ks1; ++kb) {
-                    if (!wait_x(afull_bar(s), ph)) {
+                    // the stage is ready: its A slot written (W8A8: its weight
+                    // tile landed) and its X8 tiles landed (a pair: both halves)
+                    if (!wait_x(W8 ? wfull_bar(s) : afull_bar(s), ph) || !wait_x(x8full_bar(s), ph)) {
                         ok = false;
                         break;
                     }
-                    if constexpr (W8) {
-                        // W8A8: the weight tile of this slot has landed too
-                        if (!wait_x(wfull_bar(s), ph)) {
+                    if constexpr (PAIR) {
+                        if (!wait_bounded_cluster(x8peer_bar(s), ph, abort_flag, budget)) {
                             ok = false;
                             break;
                         }
@@ -1055,20 +1092,18 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8), HALF ? 2 : 1)
     }
     if ((threadIdx.x == 0 || threadIdx.x == 64) && *abort_flag) {
         // the producers: let their own copies land before the CTA exits
+        // (each waits on barriers whose phase only its own arrival and its
+        // own copies' bytes complete, so an issued copy cannot be missed;
+        // the bound is a last resort that a landing copy never reaches)
         if (threadIdx.x == 0) {
             atomicExch(&g_dev_error, 1);
             for (int q = 0; q < SW; ++q)
                 if (issued & (1u << q)) drain_wait(wfull_bar(q), (issued_par >> q) & 1u, 200000000ull);
         } else {
-            // An X8 slot's phase also needs the dequant warps' arrivals,
-            // which an aborted stage may lack: wait briefly for each, then
-            // give any copy still in flight a fixed grace period (a tile
-            // lands within microseconds).
+            // x8full's phase needs only this thread's arrival and its own
+            // copies' bytes: once it completes, the copy has landed
             for (int q = 0; q < SX; ++q)
-                if (issued & (1u << q)) drain_wait(afull_bar(q), (issued_par >> q) & 1u, 1000000ull);
-            const uint64_t until = global_timer_ns() + 200000ull;
-            while (global_timer_ns() < until) {
-            }
+                if (issued & (1u << q)) drain_wait(x8full_bar(q), (issued_par >> q) & 1u, 200000000ull);
         }
     }
     if (warp == 0) {
@@ -1145,7 +1180,7 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     // touches X8 or s_x.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(gemm_threads(BN, W8));
+    cfg.blockDim = dim3(gemm_threads(BN, W8, HALF));
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -1175,13 +1210,13 @@ cudaError_t dispatch(int BN, int KST, bool pair, bool half, const CUtensorMap &t
                      int grid, cudaStream_t stream)
 {
     if constexpr (A_TMEM) {
-        // half CTAs (two per SM, consecutive GEMMs overlap): 128-wide K
-        // blocks, rings sized to half the SM
+        // half CTAs (two per SM, consecutive GEMMs overlap): one dequant
+        // group, 256-wide K blocks, rings sized to half the SM
         if (half) {
             switch (BN) {
-            case 16: return launch_cfg<16, 128, 10, 7, true, false, true>(tmap, args, grid, stream);
-            case 32: return launch_cfg<32, 128, 8, 6, true, false, true>(tmap, args, grid, stream);
-            default: return launch_cfg<64, 128, 8, 4, true, false, true>(tmap, args, grid, stream);
+            case 16: return launch_cfg<16, 256, 4, 3, true, false, true>(tmap, args, grid, stream);
+            case 32: return launch_cfg<32, 256, 4, 3, true, false, true>(tmap, args, grid, stream);
+            default: return launch_cfg<64, 256, 4, 2, true, false, true>(tmap, args, grid, stream);
             }
         }
         // 256-token tiles on CTA pairs: half the X8 tile per CTA, so a ring
@@ -1337,8 +1372,8 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
     // 256-wide K stages where K allows them
     const bool pair = a_in_tmem && g_cta_pairs.load(std::memory_order_relaxed) && BN == 256 && N % 256 == 0;
     // token tiles up to 64 in half CTAs (two per SM) when selected
-    const bool half = a_in_tmem && !pair && BN <= 64 && g_half_ctas.load(std::memory_order_relaxed);
-    const int KST = half ? 128 : (pair && K % 256 == 0) ? 256 : (BN <= 64 && K % 256 == 0) ? 256 : 128;
+    const bool half = a_in_tmem && !pair && BN <= 64 && K % 256 == 0 && g_half_ctas.load(std::memory_order_relaxed);
+    const int KST = (pair && K % 256 == 0) ? 256 : (BN <= 64 && K % 256 == 0) ? 256 : 128;
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) {
         *tmap_status = -1;
