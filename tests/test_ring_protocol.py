@@ -289,39 +289,42 @@ def test_the_model_catches_a_weight_slot_shared_by_two_groups():
 # CTA pairs and aborts
 # ------------------------------------------------------------------------
 def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_barrier=True,
-             drain_ticks=40, steps=300000):
+             drain_ticks=5000, steps=400000):
     """Two CTAs (or one, pair=False) of the kernel's rings with an abort.
 
     Each CTA has a weight producer, one dequant group and an X8 producer;
-    CTA 0 issues the MMAs and multicasts each commit to both CTAs' xaempty.
-    Both CTAs' dequant groups arrive on CTA 0's afull.  With
-    own_x8_barrier (the kernel's design) each CTA's X8 copies complete on
-    its own x8full; CTA 1's forwarder waits for its x8full and arrives on
-    CTA 0's x8peer, and the MMA waits on afull, x8full and x8peer.  Without
-    it (the earlier design), both halves' bytes and the producer's arrival
-    counted on CTA 0's afull.
+    CTA 0 issues the MMAs and multicasts each commit to both CTAs' xaempty,
+    and both CTAs' dequant groups arrive on CTA 0's afull.  With
+    own_x8_barrier (the kernel's design): CTA 0's X8 copies complete on its
+    own x8full; CTA 0's producer then arms x8peer with CTA 1's half and
+    arrives on CTA 1's go barrier; CTA 1 issues a stage only after that go,
+    and its copy completes on CTA 0's x8peer; the MMA waits on afull,
+    x8full and x8peer.  Without it (the earlier design), the producer's
+    arrival and the copy's bytes counted on afull, which also needs the
+    dequant arrivals.
 
     At step abort_at, CTA abort_cta raises its abort flag (as a timed-out
     wait does).  A role whose wait is not yet satisfied leaves when its
     CTA's flag is up; a wait that stays unsatisfied for 2000 ticks raises
-    the flag (the kernel's per-wait budget).  Every role then meets the
-    others at the CTA's final barrier (a pair: both CTAs, the cluster
-    barrier).  After it, if the CTA's flag is up, each producer waits for
-    the barrier phases of the copies it issued: for at most drain_ticks
-    when that phase also needs other roles (the earlier design's bounded
-    grace), until completion when only its own copy completes it.  The
-    model checks that no copy into a CTA lands after that CTA's exit."""
+    the flag (the kernel's per-wait budget).  End of the kernel, as in the
+    source: the CTA's roles meet (block barrier); if its flag is up, its
+    producers wait for their own copies' barrier phases (the earlier
+    design: for at most drain_ticks, its grace period); a pair then meets
+    at a cluster barrier, CTA 0 (if aborted) waits for the x8peer phases it
+    armed (bounded by drain_ticks: a phase that never completes is one
+    whose copy CTA 1 never issued), and the pair meets again before
+    exiting.  The model checks that no copy lands in a CTA after it exited."""
     rng = random.Random(seed)
     ncta = 2 if pair else 1
     clock = [0, 0]
     inflight = []
     last_commit = [0]
     abort = [False] * ncta
-    finished = [0] * ncta
     nroles = [0] * ncta
-    arrived = [0] * ncta
+    done_roles = [0] * ncta      # roles past the block barrier
+    drained = [0] * ncta         # roles past their own drains
+    peer_drained = [False]
     exited = [False] * ncta
-    drains = [[] for _ in range(ncta)]   # per CTA: (barrier, parity, bounded) of issued copies
 
     def later(action, delay):
         clock[1] += 1
@@ -332,8 +335,9 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
 
     wfull = [[Barrier(1) for _ in range(SW)] for _ in range(ncta)]
     wempty = [[Barrier(1) for _ in range(SW)] for _ in range(ncta)]
-    x8full = [[Barrier(1) for _ in range(SX)] for _ in range(ncta)]
-    x8peer = [Barrier(1) for _ in range(SX)]
+    x8full = [Barrier(1) for _ in range(SX)]          # CTA 0's own X8 copies
+    x8peer = [Barrier(1) for _ in range(SX)]          # in CTA 0: CTA 1's half
+    go = [Barrier(1) for _ in range(SX)]              # in CTA 1: CTA 0 armed the stage
     if own_x8_barrier:
         afull = [Barrier(ncta) for _ in range(SX)]            # both CTAs' dequant groups
     else:
@@ -342,6 +346,8 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
     wslot = [[None] * SW for _ in range(ncta)]
     xslot = [[None] * SX for _ in range(ncta)]
     aslot = [[None] * SX for _ in range(ncta)]
+    drains = [[] for _ in range(ncta)]   # (barrier, parity, bounded, owner)
+    peer_armed = {}                      # CTA 0: x8peer slot -> parity of its latest arming
 
     def landing(c, fn):
         def act():
@@ -350,7 +356,6 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
         return act
 
     def waiting(c, cond, budget=2000):
-        """Yield until cond() holds; return False if the CTA aborts first."""
         t0 = clock[0]
         while not cond():
             if abort[c]:
@@ -361,28 +366,45 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
             yield
         return True
 
-    def role(c, gen, producer=False):
+    def drain(bar, par, bounded):
+        waited = 0
+        while not bar.passes(par):
+            if bounded and waited >= drain_ticks:
+                return
+            waited += 1
+            yield
+
+    def role(c, gen, owner=None):
         nroles[c] += 1
 
         def run():
             yield from gen
-            arrived[c] += 1
-            while sum(arrived) < sum(nroles):          # the final (cluster) barrier
+            done_roles[c] += 1
+            while done_roles[c] < nroles[c]:                   # block barrier
                 yield
-            if producer and abort[c]:
-                for bar, par, bounded, _ in [d for d in drains[c] if d[3] == id(gen)]:
-                    waited = 0
-                    while not bar.passes(par):
-                        if bounded and waited >= drain_ticks:
-                            break
-                        waited += 1
-                        yield
-            finished[c] += 1
-            if finished[c] == nroles[c]:
-                exited[c] = True
+            if abort[c] and owner is not None:
+                for bar, par, bounded, o in drains[c]:
+                    if o == owner:
+                        yield from drain(bar, par, bounded)
+            drained[c] += 1
+            if pair:
+                while sum(drained) < sum(nroles):              # cluster barrier 1
+                    yield
+                if c == 0 and owner == "x8" and abort[0]:
+                    for a, par in peer_armed.items():
+                        yield from drain(x8peer[a], par, True)
+                    peer_drained[0] = True
+                elif c == 0 and owner == "x8":
+                    peer_drained[0] = True
+                while not peer_drained[0]:                     # cluster barrier 2
+                    yield
+            else:
+                while drained[c] < nroles[c]:
+                    yield
+            exited[c] = True
         return run()
 
-    def w_producer(c, me):
+    def w_producer(c):
         issued = {}
         for u in range(units):
             s, k = u % SW, u // SW
@@ -397,8 +419,7 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
                 wfull[c][s].complete_tx(1)
             later(landing(c, land), copy_delay())
             yield
-        # wfull: the producer's own arrival and its own copy's bytes only
-        drains[c].extend((wfull[c][s], par, False, me[0]) for s, par in issued.items())
+        drains[c].extend((wfull[c][s], par, False, "w") for s, par in issued.items())
 
     def dequant(c):
         for u in range(units):
@@ -417,39 +438,39 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
             yield
             afull[a].arrive()
 
-    def x_producer(c, me):
+    def x_producer(c):
         issued = {}
         for u in range(units):
             a, j = u % SX, u // SX
             ok = yield from waiting(c, lambda a=a, j=j: xaempty[c][a].passes((j & 1) ^ 1))
             if not ok:
                 break
-            if own_x8_barrier:
-                bar = x8full[c][a]
-                bar.arrive(tx=1)
-            else:
+            if not own_x8_barrier:
                 bar = afull[a]
                 if c == 0:
                     bar.arrive(tx=ncta)            # both halves' bytes
-            issued[a] = (bar, j & 1)
+                issued[a] = (bar, j & 1, True)
+            elif c == 0:
+                bar = x8full[a]
+                bar.arrive(tx=1)
+                issued[a] = (bar, j & 1, False)
+            else:
+                # CTA 1: only a stage CTA 0 has armed; the bytes complete there
+                ok = yield from waiting(c, lambda a=a, j=j: go[a].passes(j & 1))
+                if not ok:
+                    break
+                bar = x8peer[a]
 
             def land(a=a, u=u, bar=bar):
                 xslot[c][a] = u
                 bar.complete_tx(1)
             later(landing(c, land), copy_delay())
+            if own_x8_barrier and c == 0 and pair:
+                x8peer[a].arrive(tx=1)             # arm CTA 1's half, then let CTA 1 issue it
+                peer_armed[a] = j & 1
+                go[a].arrive()
             yield
-        # own x8full: exact; the earlier afull also needed the dequant
-        # arrivals, so its drain was bounded by a grace period
-        drains[c].extend((bar, par, not own_x8_barrier, me[0]) for a, (bar, par) in issued.items())
-
-    def forwarder(c):
-        for u in range(units):
-            a, j = u % SX, u // SX
-            ok = yield from waiting(c, lambda a=a, j=j: x8full[c][a].passes(j & 1))
-            if not ok:
-                return
-            yield
-            x8peer[a].arrive()
+        drains[c].extend((bar, par, bounded, "x8") for a, (bar, par, bounded) in issued.items())
 
     def mma():
         for u in range(units):
@@ -459,7 +480,7 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
                 if not afull[a].passes(j & 1):
                     return False
                 if own_x8_barrier:
-                    if not x8full[0][a].passes(j & 1):
+                    if not x8full[a].passes(j & 1):
                         return False
                     if pair and not x8peer[a].passes(j & 1):
                         return False
@@ -480,17 +501,9 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
             last_commit[0] = due
             later(commit, due - clock[0])
 
-    def producer_role(c, fn):
-        me = [None]
-        gen = fn(c, me)
-        me[0] = id(gen)
-        return role(c, gen, producer=True)
-
     live = []
     for c in range(ncta):
-        live += [producer_role(c, w_producer), role(c, dequant(c)), producer_role(c, x_producer)]
-        if pair and own_x8_barrier and c == 1:
-            live.append(role(c, forwarder(c)))
+        live += [role(c, w_producer(c), "w"), role(c, dequant(c)), role(c, x_producer(c), "x8")]
     live.append(role(0, mma()))
     step = 0
     while live or inflight:
@@ -498,7 +511,8 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
         if step > steps:
             raise AssertionError("the model did not finish (a wait that never passes)")
         if abort_at is not None and step == abort_at:
-            abort[abort_cta] = True
+            for c in (range(ncta) if abort_cta == "both" else (abort_cta,)):
+                abort[c] = True
         # time moves on (landing what is due) about every other step, also
         # while nothing is in flight (the per-wait budgets run on it)
         if not live or rng.random() < 0.5:
@@ -523,14 +537,14 @@ def test_pair_rings_without_abort(pair):
 
 
 @pytest.mark.parametrize("pair", [False, True], ids=["single", "pair"])
-@pytest.mark.parametrize("abort_cta", [0, 1])
+@pytest.mark.parametrize("abort_cta", [0, 1, "both"])
 def test_abort_at_every_step_lets_every_copy_land(pair, abort_cta):
-    """An abort at any step, in either CTA: every issued copy lands before
-    its CTA exits, and no role waits forever."""
-    if not pair and abort_cta == 1:
+    """An abort at any step, in either CTA or both: every issued copy lands
+    before its CTA exits, and no role waits forever."""
+    if not pair and abort_cta != 0:
         pytest.skip("one CTA")
-    for seed in range(6):
-        for at in range(1, 400, 3):
+    for seed in range(4):
+        for at in range(1, 400, 4):
             run_pair(4, 4, units=18, seed=seed, abort_at=at, abort_cta=abort_cta, pair=pair)
 
 
@@ -543,3 +557,12 @@ def test_the_model_catches_the_earlier_x8_drain():
             for at in range(1, 300, 2):
                 run_pair(4, 4, units=18, seed=seed, abort_at=at, pair=False, own_x8_barrier=False,
                          drain_ticks=5)
+
+
+def test_the_model_catches_a_pair_leaving_before_the_peer_drain():
+    """Without CTA 0's wait for the x8peer phases it armed (drain bound 0),
+    CTA 1 can exit while its last copy is still landing."""
+    with pytest.raises(AssertionError, match="landed in CTA 1"):
+        for seed in range(80):
+            for at in range(1, 300, 3):
+                run_pair(4, 4, units=18, seed=seed, abort_at=at, abort_cta="both", pair=True, drain_ticks=0)

@@ -39,12 +39,11 @@
 //       warp 1      MMA issuer (one thread): one barrier wait, KST/32
 //                   tcgen05.mma (K = 32) and one tcgen05.commit per stage.
 //       warp 2      X8 producer: tiled TMA loads of the activation tiles,
-//                   completing on this CTA's own x8full barrier.  It and
-//                   the epilogue alone wait for the preceding kernel
+//                   completing on this CTA's own x8full barrier (CTA 1 of
+//                   a pair: on CTA 0's x8peer, which CTA 0 arms first).  It
+//                   and the epilogue alone wait for the preceding kernel
 //                   (programmatic dependent launch), so weights stream in
 //                   and are dequantized while that kernel still runs.
-//       warp 3      (CTA 1 of a pair) X8 forwarder: once its half of a
-//                   stage's X8 tile has landed, it tells CTA 0's MMA issuer.
 //       dequant     one or two groups of four warps (two for tiles up to 64
 //                   tokens, taking alternate stages): thread r owns output
 //                   channel r of the panel, reads its packed bytes with
@@ -71,7 +70,7 @@
 //     256-channel tile with one M = 256 MMA per K step (cta_group::2);
 //     each CTA dequantizes its own 128-channel panel into its TMEM and
 //     loads half of the X8 tile, CTA 0 issues the MMAs and multicasts the
-//     commits, and the other CTA's dequant warps and X8 forwarder arrive on
+//     commits, and the other CTA's dequant warps and X8 copies arrive on
 //     CTA 0's barriers.
 //   * Every wait is bounded (per wait, global timer); on expiry the CTA
 //     stops, waits for its own in-flight copies (on their own barriers) and
@@ -408,8 +407,10 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
     //   x8full (this CTA's X8 tiles have landed: the X8 producer's arrival
     //   plus its own copies' bytes, and nothing else, so the producer can
     //   always wait for its own copies),
-    //   x8peer (pairs, in CTA 0: the other CTA's X8 half has landed; its
-    //   forwarder arrives once that CTA's own x8full completes),
+    //   x8peer (pairs) in CTA 0: CTA 1's X8 half has landed (CTA 0's
+    //   producer arms it with that half's bytes; CTA 1's copies complete on
+    //   it); in CTA 1: CTA 0 has armed the stage, so CTA 1 may issue its
+    //   half (CTA 0's producer arrives on it after arming),
     //   xaempty (the MMAs reading the slot have completed: both the X8
     //   slot and the A slot are free)
     auto wfull_bar = [&](int s) { return bar0 + 8u * s; };
@@ -494,7 +495,7 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
             mbar_init(afull_bar(s), PAIR ? 8 : 4);
             mbar_init(xaempty_bar(s), 1);    // MMA commit
             mbar_init(x8full_bar(s), 1);     // this CTA's X8 producer, plus its bytes
-            mbar_init(x8peer_bar(s), 1);     // (pairs) the other CTA's forwarder
+            mbar_init(x8peer_bar(s), 1);     // (pairs) CTA 0's X8 producer
         }
         for (int b = 0; b < C::kAccBufs; ++b) {
             mbar_init(accfull_bar(b), 1);
@@ -578,14 +579,33 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
                         ok = false;
                         break;
                     }
-                    // this CTA's token rows of the tile (a pair: its half),
-                    // completing on its own x8full
                     const uint32_t st = sbase + s * C::kXSlot;
-                    mbar_arrive_expect_tx(x8full_bar(s), C::kXSlot);
+                    if (rank == 0) {
+                        // this CTA's token rows of the tile (a pair: its
+                        // half), completing on its own x8full
+                        mbar_arrive_expect_tx(x8full_bar(s), C::kXSlot);
 #pragma unroll
-                    for (int c = 0; c < kCh; ++c)
-                        tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK,
-                                    m_tile * BN + (int)rank * C::kXRows, x8full_bar(s));
+                        for (int c = 0; c < kCh; ++c)
+                            tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN,
+                                        x8full_bar(s));
+                        if constexpr (PAIR) {
+                            // arm CTA 1's half on x8peer here, then let CTA 1 issue it
+                            mbar_arrive_expect_tx(x8peer_bar(s), C::kXSlot);
+                            mbar_arrive_release_cluster(mapa_shared(x8peer_bar(s), 1));
+                        }
+                    } else {
+                        // CTA 1 of a pair: only stages CTA 0 has armed (so
+                        // CTA 0's drain covers every copy issued here); the
+                        // bytes complete on CTA 0's x8peer
+                        if (!wait_x(x8peer_bar(s), ph)) {
+                            ok = false;
+                            break;
+                        }
+#pragma unroll
+                        for (int c = 0; c < kCh; ++c)
+                            tma_load_2d_pair(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK,
+                                             m_tile * BN + C::kXRows, leader(x8peer_bar(s)));
+                    }
                     issued |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
                     if (++s == SX) {
@@ -594,33 +614,6 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
                     }
                 }
                 i = t * ks + ks1;
-            }
-        }
-    } else if (warp == 3) {
-        // -------------------------------------- X8 forwarder (pairs) --
-        // CTA 1 of a pair: once its half of a stage's X8 tile has landed
-        // (its own x8full), tell CTA 0's MMA issuer (x8peer there).
-        if constexpr (PAIR) {
-            if (lane == 0 && rank == 1) {
-                int s = 0;
-                uint32_t ph = 0;
-                bool ok = true;
-                for (int i = i_begin; i < i_end && ok;) {
-                    const int t = i / ks;
-                    const int ks1 = min(ks, i_end - t * ks);
-                    for (int kb = i - t * ks; kb < ks1; ++kb) {
-                        if (!wait_x(x8full_bar(s), ph)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_release_cluster(leader(x8peer_bar(s)));
-                        if (++s == SX) {
-                            s = 0;
-                            ph ^= 1u;
-                        }
-                    }
-                    i = t * ks + ks1;
-                }
             }
         }
     } else if (warp == 1) {
@@ -647,7 +640,7 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
                         break;
                     }
                     if constexpr (PAIR) {
-                        if (!wait_bounded_cluster(x8peer_bar(s), ph, abort_flag, budget)) {
+                        if (!wait_x(x8peer_bar(s), ph)) {  // CTA 1's half
                             ok = false;
                             break;
                         }
@@ -1078,9 +1071,38 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
     __syncwarp();
     tc_fence_before();
     __syncthreads();
-    // a pair: CTA 0's MMAs write both CTAs' TMEM and the CTAs arrive on
-    // each other's barriers; neither leaves before both are done
-    if constexpr (PAIR) cluster_sync_all();
+    // An aborted CTA first lets its producers' own copies land: each waits on
+    // barriers whose phase only its own arrival and its own copies' bytes
+    // complete, so an issued copy cannot be missed (the bound is a last
+    // resort that a landing copy never reaches).
+    if (*abort_flag) {
+        if (threadIdx.x == 0) {
+            atomicExch(&g_dev_error, 1);
+            for (int q = 0; q < SW; ++q)
+                if (issued & (1u << q)) drain_wait(wfull_bar(q), (issued_par >> q) & 1u, 200000000ull);
+        } else if (threadIdx.x == 64 && rank == 0) {
+            for (int q = 0; q < SX; ++q)
+                if (issued & (1u << q)) drain_wait(x8full_bar(q), (issued_par >> q) & 1u, 200000000ull);
+        }
+    }
+    if constexpr (PAIR) {
+        // CTA 0's MMAs write both CTAs' TMEM and the CTAs arrive on each
+        // other's barriers: neither leaves before both are done.  After this
+        // barrier neither CTA issues anything.
+        __syncthreads();
+        cluster_sync_all();
+        // CTA 1's X8 copies complete on CTA 0's x8peer, armed by CTA 0 for
+        // every stage it issued; CTA 1 issued only armed stages.  So an
+        // armed phase that never completes is one whose copy was never
+        // issued, and waiting on the armed phases (bounded) sees every issued
+        // copy land.  CTA 1 waits at the second barrier until then.
+        if (*abort_flag && rank == 0 && threadIdx.x == 64) {
+            for (int q = 0; q < SX; ++q)
+                if (issued & (1u << q)) drain_wait(x8peer_bar(q), (issued_par >> q) & 1u, 200000000ull);
+        }
+        __syncthreads();
+        cluster_sync_all();
+    }
     tc_fence_after();
     if (a.X && threadIdx.x == 0) {
         // every CTA is past its waits on ws_ready: the last one to get here
@@ -1088,22 +1110,6 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
         if (atomicAdd(a.ws_done, 1) == (int)gridDim.x - 1) {
             *a.ws_ready = 0;
             *a.ws_done = 0;
-        }
-    }
-    if ((threadIdx.x == 0 || threadIdx.x == 64) && *abort_flag) {
-        // the producers: let their own copies land before the CTA exits
-        // (each waits on barriers whose phase only its own arrival and its
-        // own copies' bytes complete, so an issued copy cannot be missed;
-        // the bound is a last resort that a landing copy never reaches)
-        if (threadIdx.x == 0) {
-            atomicExch(&g_dev_error, 1);
-            for (int q = 0; q < SW; ++q)
-                if (issued & (1u << q)) drain_wait(wfull_bar(q), (issued_par >> q) & 1u, 200000000ull);
-        } else {
-            // x8full's phase needs only this thread's arrival and its own
-            // copies' bytes: once it completes, the copy has landed
-            for (int q = 0; q < SX; ++q)
-                if (issued & (1u << q)) drain_wait(x8full_bar(q), (issued_par >> q) & 1u, 200000000ull);
         }
     }
     if (warp == 0) {

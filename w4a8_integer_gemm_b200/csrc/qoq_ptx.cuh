@@ -248,37 +248,6 @@ __device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_add
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// mbar_try_wait with acquire semantics at cluster scope (for phases that
-// another CTA of the cluster completes).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait (as wait_bounded) with acquire at cluster scope.
-__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile int *abort,
-                                                     uint64_t budget_ns)
-{
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t start = global_timer_ns();
-    for (;;) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (*abort) return false;
-        if (global_timer_ns() - start > budget_ns) {
-            *abort = 1;
-            return false;
-        }
-        __nanosleep(64);
-    }
-}
 
 // Both CTAs of the cluster: release, then wait (acquire) for the other.
 __device__ __forceinline__ void cluster_sync_all()
