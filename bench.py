@@ -89,6 +89,8 @@ def parse():
                     help="restrict the workload to one shape name (for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-kv4", action="store_true",
+                    help="skip the KV4 decode-attention measurement reported beside the GEMM")
     ap.add_argument("--no-w8a8", action="store_true",
                     help="skip the W8A8 yardstick (the same kernel with INT8 weights) beside each point")
     ap.add_argument("--eager", action="store_true",
@@ -208,6 +210,61 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]), "reasons": reasons,
                 "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3] != "[N/A]")}
+
+
+# ----------------------------------------------------- KV4 attention leg --
+KV4_SHAPES = (  # (name, sequences, query heads, KV heads, cached tokens); head dimension 128
+    ("llama3_8b_gqa4_B32_L4096", 32, 32, 8, 4096),
+    ("qwen15_72b_mha_B8_L4096", 8, 64, 64, 4096),
+)
+
+
+def run_kv4(dev, peaks, flush, reps=20):
+    """KV4 decode attention over a synthetic 4-bit cache: device time of the
+    two kernels (chunks + combine) per call, L2 flushed before each call,
+    against the HBM roofline of its algorithmic bytes (the 4-bit codes of K
+    and V, their per-channel factors, the query and the output)."""
+    import w4a8_integer_gemm_b200 as q
+    out = []
+    stream = torch.cuda.current_stream()
+    for name, B, Hq, Hkv, L in KV4_SHAPES:
+        d = 128
+        K, V = wl.make_kv(B, Hkv, L, d, seed=7 + L)
+        Q = wl.make_queries(B, Hq, d, seed=8 + L).to(dev)
+        cache = q.qoq_kv4_cache_quantize(K.to(dev), V.to(dev))
+        del K, V
+        ws = torch.empty(q.qoq_kv4_attention_workspace_bytes(B, Hq, Hkv, L, d), dtype=torch.uint8, device=dev)
+        o = torch.empty(B, Hq, d, dtype=torch.float16, device=dev)
+        for _ in range(3):
+            q.qoq_kv4_decode_attention(Q, cache, out=o, workspace=ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0.record(stream)
+            q.qoq_kv4_decode_attention(Q, cache, out=o, workspace=ws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        byt = B * Hkv * L * d + 3 * B * Hkv * d * 2 + 2 * B * Hq * d * 2
+        gbs = byt / (ms * 1e-3) / 1e9
+        G = Hq // Hkv
+        # FP32 issue bound: G fused multiply-adds per cached element (K and
+        # V), 128 lanes x 2 flops per SM per clock at the maximum SM clock
+        fp32_flops = 2.0 * 2 * G * B * Hkv * L * d
+        fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6
+        out.append({"shape": name, "B": B, "Hq": Hq, "Hkv": Hkv, "L": L, "d": d, "us": round(ms * 1e3, 2),
+                    "algorithmic_bytes": byt, "achieved_gbs": round(gbs, 1),
+                    "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                    "fp32_fma_time_floor_us": round(fp32_flops / fp32_peak * 1e6, 2),
+                    "bound": "hbm" if byt / (peaks["hbm_gbs"] * 1e9) >= fp32_flops / fp32_peak else "alu"})
+        del cache, ws
+    torch.cuda.synchronize()
+    if q.qoq_device_error() != q.QOQ_OK:
+        raise RuntimeError("device error in the KV4 attention leg")
+    return {"kernels": "kv4_attn_chunk_kernel + kv4_combine_kernel", "timing": "isolated, L2 flushed, median of %d" % reps,
+            "points": out}
 
 
 # --------------------------------------------------------------- our arm --
@@ -529,6 +586,8 @@ def run_ours(args, rank, world, local, dist):
                    "kernels": ("per shape qoq_w4a8_linear: the per-token quantizer kernel, then the GEMM kernel "
                                "(programmatic dependent launch)")},
         "roofline": rl, "points": per, "clocks": clocks, "e2e": e2e, "w8a8_yardstick": w8a8,
+        "kv4_attention": None if args.no_kv4 else run_kv4(dev, dict(peaks, sm_max_mhz=clocks.get("sm_max_mhz") or 1965.0),
+                                                          flush),
         "gpu_launches": 2 * n_sh * args.steps,
         "a_operand": "smem" if args.a_smem else "tmem",
     }

@@ -406,6 +406,54 @@ QOQ_API int qoq_w4a8_gemm_noalloc(const int8_t *X8, const uint16_t *s_x,
                                   int M, int N, int K, int group_size,
                                   uint16_t *Y, void *stream);
 
+/* ------------------------------------------------------------------------
+ * KV4 decode attention with SmoothAttention
+ * ------------------------------------------------------------------------
+ * Sources: "QServe: Low Bit Width Does Not Guarantee High Throughput",
+ * section 4 (SmoothAttention: K' = K / lambda, Q' = Q * lambda, so
+ * Q'K'^T = QK^T, with lambda = max|K|^alpha, alpha = 0.5); "QServe Guide:
+ * W4A8KV4 Quantization for LLM Serving", The Architecture, subsection 3
+ * (the smoothed keys and the values stored as 4-bit integers with
+ * per-channel scale factors). Choices where the pages are silent:
+ *   - statistics per (sequence, KV head, channel), over the cached tokens;
+ *   - lambda = fp16(max(sqrt(max_l |K[l][c]|), 1e-5));
+ *   - K'[l][c] = K / lambda (FP32); s = fp16(max_l |X'| / 7); code =
+ *     clamp(round(X' / s), -8, 7), round half to even, for X' = K' (s_k)
+ *     and X' = V (s_v); a zero scale gives zero codes.
+ * Layouts (head dimension d = 128):
+ *   K, V      FP16 [B][Hkv][L][d];   q, out   FP16 [B][Hq][d];
+ *   K4, V4    uint8 [B][Hkv][L][d/2]: byte j of a token row holds channel
+ *             2j (low nibble) and 2j+1 (high nibble), each as code + 8;
+ *   lam, s_k, s_v   FP16 bits [B][Hkv][d].
+ * Query head h attends with KV head h / (Hq / Hkv) (grouped-query
+ * attention; Hq / Hkv in {1, 2, 4, 8}).
+ */
+
+/* Fills a KV4 cache from FP16 keys and values (the cache writer).
+ * B >= 0 (0 does nothing), 1 <= Hkv <= 1024, 1 <= L <= 2^20, d = 128;
+ * 16-byte aligned pointers. */
+QOQ_API int qoq_kv4_cache_quantize(const uint16_t *K, const uint16_t *V, int B, int Hkv, int L, int d,
+                           uint8_t *K4, uint8_t *V4, uint16_t *lam, uint16_t *s_k, uint16_t *s_v,
+                           void *stream);
+
+/* Bytes of scratch qoq_kv4_decode_attention needs (per-chunk partial
+ * results); 0 for an invalid or empty shape. */
+QOQ_API size_t qoq_kv4_attention_workspace_bytes(int B, int Hq, int Hkv, int L, int d);
+
+/* Attention of one new query token per sequence over its L cached tokens:
+ *   score[l] = sum_c (q[c] * lam[c]) * (s_k[c] * code_k[l][c]) / sqrt(d)
+ *   p = softmax(score);  out[c] = sum_l p[l] * s_v[c] * code_v[l][c]
+ * rounded to FP16 once. The kernel folds lam, s_k and 1/sqrt(d) into the
+ * query and s_v into the final sum, and computes in FP32: within 2 FP16 ulp
+ * (plus 1e-3 of the output row's largest value) of the binary64 result.
+ *   workspace   device, qoq_kv4_attention_workspace_bytes bytes, any
+ *               contents (every call overwrites what it reads).
+ * Limits as for qoq_kv4_cache_quantize, plus Hq a multiple of Hkv. */
+QOQ_API int qoq_kv4_decode_attention(const uint16_t *q, const uint8_t *K4, const uint8_t *V4,
+                             const uint16_t *lam, const uint16_t *s_k, const uint16_t *s_v,
+                             int B, int Hq, int Hkv, int L, int d, uint16_t *out,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* Expands the packed codes to the INT8 weights the GEMM multiplies,
  * W8hat[n][k] = q*s_g - zs. It runs the same device routine as the GEMM's
  * in-register dequantization. Use it for parity tests and inspection; it is

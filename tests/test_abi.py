@@ -27,7 +27,7 @@ def declared():
 def test_exports_every_declared_symbol(L):
     import w4a8_integer_gemm_b200 as q
     names = declared()
-    assert len(names) == 22
+    assert len(names) == 25
     for n in names:
         assert hasattr(L, n), n
     assert names == set(q.SIGNATURES)

@@ -289,19 +289,18 @@ def test_the_model_catches_a_weight_slot_shared_by_two_groups():
 # CTA pairs and aborts
 # ------------------------------------------------------------------------
 def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_barrier=True,
-             drain_ticks=5000, steps=400000):
+             drain_ticks=5000, peer_drain=True, steps=400000):
     """Two CTAs (or one, pair=False) of the kernel's rings with an abort.
 
     Each CTA has a weight producer, one dequant group and an X8 producer;
     CTA 0 issues the MMAs and multicasts each commit to both CTAs' xaempty,
     and both CTAs' dequant groups arrive on CTA 0's afull.  With
     own_x8_barrier (the kernel's design): CTA 0's X8 copies complete on its
-    own x8full; CTA 0's producer then arms x8peer with CTA 1's half and
-    arrives on CTA 1's go barrier; CTA 1 issues a stage only after that go,
-    and its copy completes on CTA 0's x8peer; the MMA waits on afull,
-    x8full and x8peer.  Without it (the earlier design), the producer's
-    arrival and the copy's bytes counted on afull, which also needs the
-    dequant arrivals.
+    own x8full; CTA 1's producer arms CTA 0's x8peer itself (a remote
+    arrival expecting its half's bytes) and its copy completes there; the
+    MMA waits on afull, x8full and x8peer.  Without it (the earlier
+    design), the producer's arrival and the copy's bytes counted on afull,
+    which also needs the dequant arrivals.
 
     At step abort_at, CTA abort_cta raises its abort flag (as a timed-out
     wait does).  A role whose wait is not yet satisfied leaves when its
@@ -310,10 +309,11 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
     source: the CTA's roles meet (block barrier); if its flag is up, its
     producers wait for their own copies' barrier phases (the earlier
     design: for at most drain_ticks, its grace period); a pair then meets
-    at a cluster barrier, CTA 0 (if aborted) waits for the x8peer phases it
-    armed (bounded by drain_ticks: a phase that never completes is one
-    whose copy CTA 1 never issued), and the pair meets again before
-    exiting.  The model checks that no copy lands in a CTA after it exited."""
+    at a cluster barrier (CTA 1 has stated how many stages it issued),
+    CTA 0 (if aborted) waits for the latest x8peer phase of every slot CTA 1
+    used (each completes exactly when its copy lands; peer_drain=False
+    skips this), and the pair meets again before exiting.  The model
+    checks that no copy lands in a CTA after it exited."""
     rng = random.Random(seed)
     ncta = 2 if pair else 1
     clock = [0, 0]
@@ -336,8 +336,8 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
     wfull = [[Barrier(1) for _ in range(SW)] for _ in range(ncta)]
     wempty = [[Barrier(1) for _ in range(SW)] for _ in range(ncta)]
     x8full = [Barrier(1) for _ in range(SX)]          # CTA 0's own X8 copies
-    x8peer = [Barrier(1) for _ in range(SX)]          # in CTA 0: CTA 1's half
-    go = [Barrier(1) for _ in range(SX)]              # in CTA 1: CTA 0 armed the stage
+    x8peer = [Barrier(1) for _ in range(SX)]          # in CTA 0: CTA 1's half (armed by CTA 1)
+    n_peer = [0]                                      # stages CTA 1 issued
     if own_x8_barrier:
         afull = [Barrier(ncta) for _ in range(SX)]            # both CTAs' dequant groups
     else:
@@ -347,7 +347,6 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
     xslot = [[None] * SX for _ in range(ncta)]
     aslot = [[None] * SX for _ in range(ncta)]
     drains = [[] for _ in range(ncta)]   # (barrier, parity, bounded, owner)
-    peer_armed = {}                      # CTA 0: x8peer slot -> parity of its latest arming
 
     def landing(c, fn):
         def act():
@@ -390,9 +389,11 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
             if pair:
                 while sum(drained) < sum(nroles):              # cluster barrier 1
                     yield
-                if c == 0 and owner == "x8" and abort[0]:
-                    for a, par in peer_armed.items():
-                        yield from drain(x8peer[a], par, True)
+                if c == 0 and owner == "x8" and abort[0] and peer_drain:
+                    n1 = n_peer[0]
+                    for a in range(min(SX, n1)):
+                        j = a + (n1 - 1 - a) // SX * SX       # CTA 1's last stage in slot a
+                        yield from drain(x8peer[a], (j // SX) & 1, False)
                     peer_drained[0] = True
                 elif c == 0 and owner == "x8":
                     peer_drained[0] = True
@@ -455,20 +456,15 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
                 bar.arrive(tx=1)
                 issued[a] = (bar, j & 1, False)
             else:
-                # CTA 1: only a stage CTA 0 has armed; the bytes complete there
-                ok = yield from waiting(c, lambda a=a, j=j: go[a].passes(j & 1))
-                if not ok:
-                    break
+                # CTA 1: arms CTA 0's x8peer itself; its bytes complete there
                 bar = x8peer[a]
+                bar.arrive(tx=1)
+                n_peer[0] += 1
 
             def land(a=a, u=u, bar=bar):
                 xslot[c][a] = u
                 bar.complete_tx(1)
             later(landing(c, land), copy_delay())
-            if own_x8_barrier and c == 0 and pair:
-                x8peer[a].arrive(tx=1)             # arm CTA 1's half, then let CTA 1 issue it
-                peer_armed[a] = j & 1
-                go[a].arrive()
             yield
         drains[c].extend((bar, par, bounded, "x8") for a, (bar, par, bounded) in issued.items())
 
@@ -560,9 +556,9 @@ def test_the_model_catches_the_earlier_x8_drain():
 
 
 def test_the_model_catches_a_pair_leaving_before_the_peer_drain():
-    """Without CTA 0's wait for the x8peer phases it armed (drain bound 0),
-    CTA 1 can exit while its last copy is still landing."""
+    """Without CTA 0's wait for CTA 1's x8peer phases, CTA 1 can exit while
+    its last copy is still landing."""
     with pytest.raises(AssertionError, match="landed in CTA 1"):
         for seed in range(80):
             for at in range(1, 300, 3):
-                run_pair(4, 4, units=18, seed=seed, abort_at=at, abort_cta="both", pair=True, drain_ticks=0)
+                run_pair(4, 4, units=18, seed=seed, abort_at=at, abort_cta="both", pair=True, peer_drain=False)

@@ -56,6 +56,9 @@ SIGNATURES = {
     "qoq_w4a8_gemm_i32": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "qoq_epilogue_i32": (_I, [_P, _P, _P, _I, _I, _P, _P]),
     "qoq_quantize_weights_w8": (_I, [_P, _I, _I, _P, _P, _P]),
+    "qoq_kv4_cache_quantize": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "qoq_kv4_attention_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "qoq_kv4_decode_attention": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "qoq_w8a8_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "qoq_w4a8_linear": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "qoq_dequant_weights_i8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
@@ -429,6 +432,56 @@ def qoq_dequant_weights_i8(packed: PackedWeights, out: Optional[torch.Tensor] = 
     st = lib().qoq_dequant_weights_i8(_ptr(packed.Wp), _ptr(packed.s_g), _ptr(packed.zs), packed.N,
                                       packed.K, packed.group_size, _ptr(out), _stream(stream))
     _check("qoq_dequant_weights_i8", st)
+    return out
+
+
+# -------------------------------------------------------- KV4 attention ----
+@dataclass
+class KV4Cache:
+    """A 4-bit KV cache with SmoothAttention factors (layouts of include/qoq.h)."""
+    K4: torch.Tensor     # uint8 [B, Hkv, L, d/2]
+    V4: torch.Tensor     # uint8 [B, Hkv, L, d/2]
+    lam: torch.Tensor    # int16 [B, Hkv, d] FP16 bits
+    s_k: torch.Tensor    # int16 [B, Hkv, d] FP16 bits
+    s_v: torch.Tensor    # int16 [B, Hkv, d] FP16 bits
+
+
+def qoq_kv4_cache_quantize(K: torch.Tensor, V: torch.Tensor, stream=None) -> KV4Cache:
+    """K, V fp16 [B, Hkv, L, d] -> KV4Cache."""
+    _need(K, torch.float16, "K")
+    _need(V, torch.float16, "V")
+    B, Hkv, L, d = K.shape
+    dev = K.device
+    c = KV4Cache(torch.empty(B, Hkv, L, d // 2, dtype=torch.uint8, device=dev),
+                 torch.empty(B, Hkv, L, d // 2, dtype=torch.uint8, device=dev),
+                 torch.empty(B, Hkv, d, dtype=torch.int16, device=dev),
+                 torch.empty(B, Hkv, d, dtype=torch.int16, device=dev),
+                 torch.empty(B, Hkv, d, dtype=torch.int16, device=dev))
+    st = lib().qoq_kv4_cache_quantize(_ptr(K), _ptr(V), B, Hkv, L, d, _ptr(c.K4), _ptr(c.V4), _ptr(c.lam),
+                                      _ptr(c.s_k), _ptr(c.s_v), _stream(stream))
+    _check("qoq_kv4_cache_quantize", st)
+    return c
+
+
+def qoq_kv4_attention_workspace_bytes(B: int, Hq: int, Hkv: int, L: int, d: int) -> int:
+    return int(lib().qoq_kv4_attention_workspace_bytes(int(B), int(Hq), int(Hkv), int(L), int(d)))
+
+
+def qoq_kv4_decode_attention(q: torch.Tensor, cache: KV4Cache, out: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """q fp16 [B, Hq, d] -> out fp16 [B, Hq, d]: attention over the KV4 cache."""
+    _need(q, torch.float16, "q")
+    B, Hq, d = q.shape
+    _, Hkv, L, _ = cache.K4.shape
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float16, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(qoq_kv4_attention_workspace_bytes(B, Hq, Hkv, L, d), 16),
+                                dtype=torch.uint8, device=q.device)
+    st = lib().qoq_kv4_decode_attention(_ptr(q), _ptr(cache.K4), _ptr(cache.V4), _ptr(cache.lam), _ptr(cache.s_k),
+                                        _ptr(cache.s_v), B, Hq, Hkv, L, d, _ptr(out), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("qoq_kv4_decode_attention", st)
     return out
 
 

@@ -259,6 +259,50 @@ int qoq_w8a8_gemm(const int8_t *X8, const uint16_t *s_x, const int8_t *W8, const
     return from_cuda(e);
 }
 
+static bool valid_kv4(int B, int Hq, int Hkv, int L, int d)
+{
+    if (B < 0 || B > (1 << 16) || Hkv < 1 || Hkv > 1024 || Hq < Hkv || Hq % Hkv != 0 || d != 128) return false;
+    const int G = Hq / Hkv;
+    return (G == 1 || G == 2 || G == 4 || G == 8) && L >= 1 && L <= (1 << 20);
+}
+
+int qoq_kv4_cache_quantize(const uint16_t *K, const uint16_t *V, int B, int Hkv, int L, int d, uint8_t *K4,
+                           uint8_t *V4, uint16_t *lam, uint16_t *s_k, uint16_t *s_v, void *stream)
+{
+    if (!valid_kv4(B, Hkv, Hkv, L, d)) return QOQ_ERR_INVALID_ARG;
+    if (B == 0) return QOQ_OK;
+    if (!K || !V || !K4 || !V4 || !lam || !s_k || !s_v) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(K4) || !aligned16(V4) || !aligned16(lam) || !aligned16(s_k) ||
+        !aligned16(s_v))
+        return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(qoq::launch_kv4_cache(K, V, B, Hkv, L, K4, V4, lam, s_k, s_v, (cudaStream_t)stream));
+}
+
+size_t qoq_kv4_attention_workspace_bytes(int B, int Hq, int Hkv, int L, int d)
+{
+    if (!valid_kv4(B, Hq, Hkv, L, d) || B == 0) return 0;
+    return qoq::kv4_workspace_bytes(B, Hq, Hkv, L);
+}
+
+int qoq_kv4_decode_attention(const uint16_t *q, const uint8_t *K4, const uint8_t *V4, const uint16_t *lam,
+                             const uint16_t *s_k, const uint16_t *s_v, int B, int Hq, int Hkv, int L, int d,
+                             uint16_t *out, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!valid_kv4(B, Hq, Hkv, L, d)) return QOQ_ERR_INVALID_ARG;
+    if (B == 0) return QOQ_OK;
+    if (!q || !K4 || !V4 || !lam || !s_k || !s_v || !out || !workspace) return QOQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(K4) || !aligned16(V4) || !aligned16(lam) || !aligned16(s_k) || !aligned16(s_v) ||
+        !aligned16(out) || !aligned16(workspace))
+        return QOQ_ERR_INVALID_ARG;
+    if (workspace_bytes < qoq::kv4_workspace_bytes(B, Hq, Hkv, L)) return QOQ_ERR_INVALID_ARG;
+    const int dev = check_device();
+    if (dev != QOQ_OK) return dev;
+    return from_cuda(
+        qoq::launch_kv4_attention(q, K4, V4, lam, s_k, s_v, B, Hq, Hkv, L, out, workspace, (cudaStream_t)stream));
+}
+
 int qoq_w4a8_linear(const uint16_t *X, int M, int N, int K, int group_size, const uint8_t *Wp,
                     const uint16_t *s_c, const uint8_t *s_g, const uint8_t *zs, int8_t *X8, uint16_t *s_x,
                     uint16_t *Y, void *workspace, size_t workspace_bytes, void *stream)

@@ -40,7 +40,7 @@
 //                   tcgen05.mma (K = 32) and one tcgen05.commit per stage.
 //       warp 2      X8 producer: tiled TMA loads of the activation tiles,
 //                   completing on this CTA's own x8full barrier (CTA 1 of
-//                   a pair: on CTA 0's x8peer, which CTA 0 arms first).  It
+//                   a pair: on CTA 0's x8peer, which it arms itself).  It
 //                   and the epilogue alone wait for the preceding kernel
 //                   (programmatic dependent launch), so weights stream in
 //                   and are dequantized while that kernel still runs.
@@ -186,7 +186,7 @@ struct GemmCfg {
     // drains the last one) wherever TMEM has room for them
     static constexpr int kAccBufs = (2 * BN + (A_TMEM ? SX * (int)kACols : 0) <= 512) ? 2 : 1;
     static constexpr int kNumBars = 2 * SW + 4 * SX + 2 * kAccBufs + 2;
-    static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;
+    static constexpr int kUsed = kBarOff + kNumBars * 8 + 16;  // + TMEM base, abort flag, peer count
     // full CTAs: at least ~120 KB so that exactly one CTA (and one TMEM
     // allocation) lives on each SM; +1024 for manual alignment of the
     // dynamic base
@@ -407,10 +407,9 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
     //   x8full (this CTA's X8 tiles have landed: the X8 producer's arrival
     //   plus its own copies' bytes, and nothing else, so the producer can
     //   always wait for its own copies),
-    //   x8peer (pairs) in CTA 0: CTA 1's X8 half has landed (CTA 0's
-    //   producer arms it with that half's bytes; CTA 1's copies complete on
-    //   it); in CTA 1: CTA 0 has armed the stage, so CTA 1 may issue its
-    //   half (CTA 0's producer arrives on it after arming),
+    //   x8peer (pairs, in CTA 0): CTA 1's X8 half has landed -- CTA 1's
+    //   producer's remote arrival (with the half's bytes expected) plus its
+    //   copies' bytes, and nothing else,
     //   xaempty (the MMAs reading the slot have completed: both the X8
     //   slot and the A slot are free)
     auto wfull_bar = [&](int s) { return bar0 + 8u * s; };
@@ -430,6 +429,8 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
     const uint32_t xready_bar = mmadone_bar + 8u;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    // (pairs, CTA 0) the number of X8 stages CTA 1 issued, written by CTA 1
+    uint32_t *peer_count = tmem_slot + 2;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -495,7 +496,7 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
             mbar_init(afull_bar(s), PAIR ? 8 : 4);
             mbar_init(xaempty_bar(s), 1);    // MMA commit
             mbar_init(x8full_bar(s), 1);     // this CTA's X8 producer, plus its bytes
-            mbar_init(x8peer_bar(s), 1);     // (pairs) CTA 0's X8 producer
+            mbar_init(x8peer_bar(s), 1);     // (pairs) CTA 1's X8 producer
         }
         for (int b = 0; b < C::kAccBufs; ++b) {
             mbar_init(accfull_bar(b), 1);
@@ -504,6 +505,7 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
         mbar_init(mmadone_bar, 1);
         mbar_init(xready_bar, 1);
         *abort_flag = 0;
+        *peer_count = 0;
         fence_mbar_init();
         // weights stream from here on, while the rest of the CTA sets up
         for (int j = 0; j < n_pro; ++j) {
@@ -570,6 +572,7 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
             }
             int s = 0;
             uint32_t ph = 0;
+            uint32_t n_peer = 0;  // (CTA 1 of a pair) stages issued
             for (int i = i_begin; i < i_end && ok;) {
                 const int t = i / ks;
                 const int ks1 = min(ks, i_end - t * ks);
@@ -588,19 +591,12 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
                         for (int c = 0; c < kCh; ++c)
                             tma_load_2d(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK, m_tile * BN,
                                         x8full_bar(s));
-                        if constexpr (PAIR) {
-                            // arm CTA 1's half on x8peer here, then let CTA 1 issue it
-                            mbar_arrive_expect_tx(x8peer_bar(s), C::kXSlot);
-                            mbar_arrive_release_cluster(mapa_shared(x8peer_bar(s), 1));
-                        }
                     } else {
-                        // CTA 1 of a pair: only stages CTA 0 has armed (so
-                        // CTA 0's drain covers every copy issued here); the
-                        // bytes complete on CTA 0's x8peer
-                        if (!wait_x(x8peer_bar(s), ph)) {
-                            ok = false;
-                            break;
-                        }
+                        // CTA 1 of a pair: its half completes on CTA 0's
+                        // x8peer, which only this arrival and these bytes
+                        // complete
+                        mbar_arrive_expect_tx_cluster(leader(x8peer_bar(s)), C::kXSlot);
+                        ++n_peer;
 #pragma unroll
                         for (int c = 0; c < kCh; ++c)
                             tma_load_2d_pair(st + c * C::kXTile, &tmap_x, (kb * kCh + c) * kBlockK,
@@ -614,6 +610,11 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
                     }
                 }
                 i = t * ks + ks1;
+            }
+            // CTA 1 of a pair tells CTA 0 how many stages it issued (read
+            // after the cluster barrier at the end, when no more are issued)
+            if constexpr (PAIR) {
+                if (rank == 1) st_shared_cluster_u32(mapa_shared(smem_addr(peer_count), 0), n_peer);
             }
         }
     } else if (warp == 1) {
@@ -1091,14 +1092,18 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
         // barrier neither CTA issues anything.
         __syncthreads();
         cluster_sync_all();
-        // CTA 1's X8 copies complete on CTA 0's x8peer, armed by CTA 0 for
-        // every stage it issued; CTA 1 issued only armed stages.  So an
-        // armed phase that never completes is one whose copy was never
-        // issued, and waiting on the armed phases (bounded) sees every issued
-        // copy land.  CTA 1 waits at the second barrier until then.
+        // CTA 1's X8 copies complete on CTA 0's x8peer, each phase armed by
+        // CTA 1 itself: the latest phase of every slot CTA 1 used completes
+        // exactly when its copy has landed.  CTA 0 waits for those (CTA 1
+        // stated their number before the barrier); CTA 1 waits at the second
+        // barrier until then.
         if (*abort_flag && rank == 0 && threadIdx.x == 64) {
-            for (int q = 0; q < SX; ++q)
-                if (issued & (1u << q)) drain_wait(x8peer_bar(q), (issued_par >> q) & 1u, 200000000ull);
+            const uint32_t n1 = *reinterpret_cast<volatile uint32_t *>(peer_count);
+            for (uint32_t q = 0; q < (uint32_t)SX && q < n1; ++q) {
+                // stage j = the last one CTA 1 issued into slot q
+                const uint32_t j = q + (n1 - 1 - q) / SX * SX;
+                drain_wait(x8peer_bar((int)q), (j / SX) & 1u, 200000000ull);
+            }
         }
         __syncthreads();
         cluster_sync_all();

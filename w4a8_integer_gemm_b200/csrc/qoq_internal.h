@@ -91,6 +91,16 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
                         const uint16_t *R = nullptr, int ldx = 0, const int8_t *W8 = nullptr);
 
 
+// KV4 cache (head dimension 128): per (sequence, KV head) lambda, s_k, s_v
+// and the packed 4-bit codes of K' = K / lambda and V.
+cudaError_t launch_kv4_cache(const uint16_t *K, const uint16_t *V, int B, int Hkv, int L, uint8_t *K4, uint8_t *V4,
+                             uint16_t *lam, uint16_t *s_k, uint16_t *s_v, cudaStream_t stream);
+// Decode attention over a KV4 cache: chunk kernel, then combine kernel.
+size_t kv4_workspace_bytes(int B, int Hq, int Hkv, int L);
+cudaError_t launch_kv4_attention(const uint16_t *q, const uint8_t *K4, const uint8_t *V4, const uint16_t *lam,
+                                 const uint16_t *s_k, const uint16_t *s_v, int B, int Hq, int Hkv, int L,
+                                 uint16_t *out, void *workspace, cudaStream_t stream);
+
 // Device error flag of the current device: read and clear (synchronous).
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value);
 

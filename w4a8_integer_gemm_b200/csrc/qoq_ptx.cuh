@@ -240,13 +240,22 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// Remote arrive with release semantics at cluster scope: what this thread
-// observed (the landing of its CTA's copies) is visible to the thread of the
-// other CTA that acquires the barrier's phase at cluster scope.
-__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr)
+// Remote arrive that also expects `tx` bytes on that barrier's current
+// phase (release at cluster scope): the arriving thread's copies, which
+// complete on the same barrier, may land before or after it.
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr, uint32_t tx)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
+                 "r"(tx)
+                 : "memory");
 }
+
+// 32-bit store into another CTA's shared memory (shared::cluster address).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
 
 
 // Both CTAs of the cluster: release, then wait (acquire) for the other.

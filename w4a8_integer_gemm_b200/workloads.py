@@ -114,6 +114,28 @@ def make_activations(M: int, K: int, dist: Dist, seed: int) -> torch.Tensor:
     return X.to(torch.float16)
 
 
+def make_kv(B: int, Hkv: int, L: int, d: int, seed: int, k_frac: float = 0.02, k_scale: float = 25.0):
+    """FP16 keys and values [B, Hkv, L, d] of a synthetic KV cache: normal
+    draws, with round(k_frac * d) key channels per KV head (picked without
+    replacement) scaled by k_scale, the outlier channels SmoothAttention is
+    for."""
+    gen = torch.Generator(device="cpu").manual_seed(int(seed))
+    K = torch.randn(B, Hkv, L, d, generator=gen, dtype=torch.float32)
+    V = torch.randn(B, Hkv, L, d, generator=gen, dtype=torch.float32)
+    count = int(round(k_frac * d))
+    for h in range(Hkv):
+        cols = torch.randperm(d, generator=gen)[:count]
+        if count:
+            K[:, h, :, cols] *= k_scale
+    return K.to(torch.float16), V.to(torch.float16)
+
+
+def make_queries(B: int, Hq: int, d: int, seed: int):
+    """FP16 queries [B, Hq, d] (one new token per sequence)."""
+    gen = torch.Generator(device="cpu").manual_seed(int(seed))
+    return torch.randn(B, Hq, d, generator=gen, dtype=torch.float32).to(torch.float16)
+
+
 def make_case(workload: Workload, i: int, shape: Shape = None):
     """(X fp16 [M][K], W fp32 [N][K]) for shape i of a workload."""
     s = shape or workload.shapes[i]
