@@ -310,7 +310,7 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
     producers wait for their own copies' barrier phases (the earlier
     design: for at most drain_ticks, its grace period); a pair then meets
     at a cluster barrier (CTA 1 has stated how many stages it issued),
-    CTA 0 (if aborted) waits for the latest x8peer phase of every slot CTA 1
+    CTA 0 (if either CTA aborted) waits for the latest x8peer phase of every slot CTA 1
     used (each completes exactly when its copy lands; peer_drain=False
     skips this), and the pair meets again before exiting.  The model
     checks that no copy lands in a CTA after it exited."""
@@ -389,7 +389,7 @@ def run_pair(SW, SX, units, seed, abort_at=None, abort_cta=0, pair=True, own_x8_
             if pair:
                 while sum(drained) < sum(nroles):              # cluster barrier 1
                     yield
-                if c == 0 and owner == "x8" and abort[0] and peer_drain:
+                if c == 0 and owner == "x8" and any(abort) and peer_drain:
                     n1 = n_peer[0]
                     for a in range(min(SX, n1)):
                         j = a + (n1 - 1 - a) // SX * SX       # CTA 1's last stage in slot a

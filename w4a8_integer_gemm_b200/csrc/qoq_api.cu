@@ -390,9 +390,10 @@ int qoq_set_linear_in_kernel_quant(int enable)
 
 int qoq_device_error(void *stream)
 {
-    int v = 0;
+    int v = 0, w = 0;
     if (qoq::read_and_clear_device_error((cudaStream_t)stream, &v) != cudaSuccess) return QOQ_ERR_CUDA;
-    return v ? QOQ_ERR_TIMEOUT : QOQ_OK;
+    if (qoq::read_and_clear_kv4_error(&w) != cudaSuccess) return QOQ_ERR_CUDA;
+    return (v || w) ? QOQ_ERR_TIMEOUT : QOQ_OK;
 }
 
 }  // extern "C"

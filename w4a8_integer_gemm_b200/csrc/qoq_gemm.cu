@@ -1090,23 +1090,26 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
         // CTA 0's MMAs write both CTAs' TMEM and the CTAs arrive on each
         // other's barriers: neither leaves before both are done.  After this
         // barrier neither CTA issues anything.
-        __syncthreads();
         cluster_sync_all();
         // CTA 1's X8 copies complete on CTA 0's x8peer, each phase armed by
         // CTA 1 itself: the latest phase of every slot CTA 1 used completes
-        // exactly when its copy has landed.  CTA 0 waits for those (CTA 1
-        // stated their number before the barrier); CTA 1 waits at the second
-        // barrier until then.
-        if (*abort_flag && rank == 0 && threadIdx.x == 64) {
-            const uint32_t n1 = *reinterpret_cast<volatile uint32_t *>(peer_count);
-            for (uint32_t q = 0; q < (uint32_t)SX && q < n1; ++q) {
-                // stage j = the last one CTA 1 issued into slot q
-                const uint32_t j = q + (n1 - 1 - q) / SX * SX;
-                drain_wait(x8peer_bar((int)q), (j / SX) & 1u, 200000000ull);
+        // exactly when its copy has landed.  If either CTA stopped early,
+        // CTA 0 waits for those (CTA 1 stated their number before the
+        // barrier) and CTA 1 waits at a second barrier until then; both read
+        // the same two flags, so both take the same branch.
+        const bool any_abort =
+            *abort_flag || ld_shared_cluster_u32(mapa_shared(smem_addr((void *)abort_flag), rank ^ 1u)) != 0;
+        if (any_abort) {
+            if (rank == 0 && threadIdx.x == 64) {
+                const uint32_t n1 = *reinterpret_cast<volatile uint32_t *>(peer_count);
+                for (uint32_t q = 0; q < (uint32_t)SX && q < n1; ++q) {
+                    // stage j = the last one CTA 1 issued into slot q
+                    const uint32_t j = q + (n1 - 1 - q) / SX * SX;
+                    drain_wait(x8peer_bar((int)q), (j / SX) & 1u, 200000000ull);
+                }
             }
+            cluster_sync_all();
         }
-        __syncthreads();
-        cluster_sync_all();
     }
     tc_fence_after();
     if (a.X && threadIdx.x == 0) {

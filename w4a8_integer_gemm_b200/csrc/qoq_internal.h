@@ -103,6 +103,8 @@ cudaError_t launch_kv4_attention(const uint16_t *q, const uint8_t *K4, const uin
 
 // Device error flag of the current device: read and clear (synchronous).
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value);
+// The KV4 kernels' own flag (read after that synchronization).
+cudaError_t read_and_clear_kv4_error(int *value);
 
 // The argument checks every GEMM entry point shares (qoq_api.cu).
 bool valid_nk(int N, int K);

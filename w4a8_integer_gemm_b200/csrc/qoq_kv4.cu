@@ -87,43 +87,75 @@ __global__ void __launch_bounds__(kD) kv4_cache_kernel(const uint16_t *__restric
     }
 }
 
-// 16 nibbles of a 64-bit word -> the codes as floats (nibble - 8).
+// 16 nibbles of a 64-bit word -> the codes as floats (nibble - 8).  The
+// nibble is placed in the low mantissa bits of 2^23 (exactly 2^23 + n) and
+// 2^23 + 8 is subtracted: one logic op and one add per value, exact, at
+// full rate (an integer-to-float conversion is a quarter-rate instruction).
+__device__ __forceinline__ float nib_to_float(uint32_t w, int i)
+{
+    return __int_as_float((int)(0x4B000000u | ((w >> (4 * i)) & 0xFu))) - 8388616.0f;
+}
+
 __device__ __forceinline__ void unpack16(uint2 w, float *f)
 {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = (float)(int)((w.x >> (4 * i)) & 0xFu) - 8.0f;
+    for (int i = 0; i < 8; ++i) f[i] = nib_to_float(w.x, i);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) f[8 + i] = (float)(int)((w.y >> (4 * i)) & 0xFu) - 8.0f;
+    for (int i = 0; i < 8; ++i) f[8 + i] = nib_to_float(w.y, i);
 }
 
-constexpr int kThreads = 128;    // 4 warps; a warp covers 4 tokens per load (8 lanes a token)
+constexpr int kThreads = 256;    // 8 warps; a warp covers 4 token rows per step (8 lanes a row)
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunk = 512;      // tokens per CTA: 32 KB of K codes and 32 KB of V codes
+
+__device__ int g_kv4_error;      // non-zero after a bounded wait of this file's kernels ran out
 
 // ------------------------------------------------- attention, one chunk --
-// CTA (sequence b, KV head g, chunk s) over tokens [s*Lc, min(L, (s+1)*Lc)):
-// pass 1 scores every token for the G query heads, the chunk's softmax
-// numerators follow, pass 2 sums the codes of V weighted by them.  The
-// chunk's (max, sum, weighted sums) go to the workspace for the combine.
+// CTA (sequence b, KV head g, chunk s) over tokens [s*kChunk, min(L, ...)):
+// the chunk's K and V codes are contiguous in the cache, so one bulk copy
+// each brings them into shared memory at the start (64 KB in flight per
+// CTA).  Pass 1 scores every token for the G query heads (from shared
+// memory), the chunk's softmax numerators follow, pass 2 sums the value
+// codes weighted by them.  The chunk's (max, sum, weighted sums) go to the
+// workspace for the combine.
 template <int G>
 __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
     const uint16_t *__restrict__ q, const uint8_t *__restrict__ K4, const uint8_t *__restrict__ V4,
-    const uint16_t *__restrict__ lam, const uint16_t *__restrict__ s_k, int Hkv, int L, int Lc,
+    const uint16_t *__restrict__ lam, const uint16_t *__restrict__ s_k, int Hkv, int L,
     float *__restrict__ part)
 {
-    extern __shared__ float sm[];                // [G][Lc] scores, then numerators
-    __shared__ float red[G][kThreads / 32];
+    extern __shared__ __align__(128) uint8_t dyn[];
+    uint8_t *ks = dyn;                                   // [kChunk][64] K codes
+    uint8_t *vs = dyn + kChunk * kRowBytes;              // [kChunk][64] V codes
+    float *sm = reinterpret_cast<float *>(dyn + 2 * kChunk * kRowBytes);   // [G][kChunk]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G * kChunk);        // K landed, V landed
+    __shared__ float red[G][kWarps];
     __shared__ float gmax[G], gsum[G];
-    __shared__ float osum[kThreads / 32][G][kD];
+    __shared__ float osum[kWarps][G][kD];
+    __shared__ int abort_flag;
     const int bh = blockIdx.x;                   // b * Hkv + kv head
     const int b = bh / Hkv, hk = bh % Hkv;
     const int S = gridDim.y, s = blockIdx.y;
-    const int l0 = s * Lc, l1 = min(L, l0 + Lc);
-    const int n = l1 - l0;
+    const int l0 = s * kChunk, n = min(L - l0, kChunk);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cb = lane & 7;                     // channel block: channels 16*cb .. 16*cb+15
-    const int tw = lane >> 3;                    // token within the warp's 4
+    const int tw = lane >> 3;                    // row within the warp's 4
     const size_t head = (size_t)bh;
+    const uint32_t kbar = smem_addr(bars), vbar = smem_addr(bars + 1);
+    const uint32_t bytes = (uint32_t)n * kRowBytes;
+    if (threadIdx.x == 0) {
+        mbar_init(kbar, 1);
+        mbar_init(vbar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        mbar_arrive_expect_tx(kbar, bytes);
+        bulk_load(smem_addr(ks), K4 + (head * L + l0) * kRowBytes, bytes, kbar);
+        mbar_arrive_expect_tx(vbar, bytes);
+        bulk_load(smem_addr(vs), V4 + (head * L + l0) * kRowBytes, bytes, vbar);
+    }
+    // the query of each of the G heads, with lambda, s_k and 1/sqrt(d)
+    // folded in (while the copies are in flight)
     const float inv_sqrt_d = 0.08838834764831845f;   // 1 / sqrt(128)
-    // the query of each of the G heads, with lambda, s_k and 1/sqrt(d) folded in
     float qf[G][16];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
@@ -137,11 +169,14 @@ __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
             qf[gi][i] = __fmul_rn(half_bits_to_float(__ldg(q + qh + c)), f);
         }
     }
+    __syncthreads();
+    const uint64_t budget = 2000000000ull;
+    bool ok = wait_bounded(kbar, 0u, &abort_flag, budget);
     // pass 1: scores
-    const uint2 *krow = reinterpret_cast<const uint2 *>(K4 + head * (size_t)L * kRowBytes);
-    for (int t0 = 4 * warp + tw; t0 < ((n + 15) & ~15); t0 += 16) {
-        const bool live = t0 < n;
-        const uint2 w = live ? __ldcs(krow + (size_t)(l0 + t0) * (kRowBytes / 8) + cb) : make_uint2(0x88888888u, 0x88888888u);
+    const int nr = (n + 4 * kWarps - 1) / (4 * kWarps) * (4 * kWarps);
+    for (int t0 = 4 * warp + tw; t0 < nr && ok; t0 += 4 * kWarps) {
+        const uint2 w = t0 < n ? *reinterpret_cast<const uint2 *>(ks + t0 * kRowBytes + 8 * cb)
+                               : make_uint2(0x88888888u, 0x88888888u);
         float kc[16];
         unpack16(w, kc);
         float acc[G];
@@ -158,9 +193,9 @@ __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
             acc[gi] += __shfl_xor_sync(0xffffffffu, acc[gi], 2);
             acc[gi] += __shfl_xor_sync(0xffffffffu, acc[gi], 1);
         }
-        if (cb == 0 && live) {
+        if (cb == 0 && t0 < n) {
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) sm[gi * Lc + t0] = acc[gi];
+            for (int gi = 0; gi < G; ++gi) sm[gi * kChunk + t0] = acc[gi];
         }
     }
     __syncthreads();
@@ -168,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
         float m = -INFINITY;
-        for (int t = threadIdx.x; t < n; t += kThreads) m = fmaxf(m, sm[gi * Lc + t]);
+        for (int t = threadIdx.x; t < n; t += kThreads) m = fmaxf(m, sm[gi * kChunk + t]);
         m = warp_max(m);
         if (lane == 0) red[gi][warp] = m;
     }
@@ -176,7 +211,7 @@ __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
     if (threadIdx.x < G) {
         float m = red[threadIdx.x][0];
 #pragma unroll
-        for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[threadIdx.x][w]);
+        for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[threadIdx.x][w]);
         gmax[threadIdx.x] = m;
     }
     __syncthreads();
@@ -184,8 +219,8 @@ __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
     for (int gi = 0; gi < G; ++gi) {
         float sum = 0.0f;
         for (int t = threadIdx.x; t < n; t += kThreads) {
-            const float p = expf(sm[gi * Lc + t] - gmax[gi]);
-            sm[gi * Lc + t] = p;
+            const float p = expf(sm[gi * kChunk + t] - gmax[gi]);
+            sm[gi * kChunk + t] = p;
             sum += p;
         }
 #pragma unroll
@@ -196,7 +231,7 @@ __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
     if (threadIdx.x < G) {
         float t = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) t += red[threadIdx.x][w];
+        for (int w = 0; w < kWarps; ++w) t += red[threadIdx.x][w];
         gsum[threadIdx.x] = t;
     }
     // pass 2: the numerator-weighted sums of the value codes
@@ -205,20 +240,20 @@ __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
     for (int gi = 0; gi < G; ++gi)
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc2[gi][i] = 0.0f;
-    const uint2 *vrow = reinterpret_cast<const uint2 *>(V4 + head * (size_t)L * kRowBytes);
-    for (int t0 = 4 * warp + tw; t0 < ((n + 15) & ~15); t0 += 16) {
-        const bool live = t0 < n;
-        const uint2 w = live ? __ldcs(vrow + (size_t)(l0 + t0) * (kRowBytes / 8) + cb) : make_uint2(0x88888888u, 0x88888888u);
+    ok = ok && wait_bounded(vbar, 0u, &abort_flag, budget);
+    for (int t0 = 4 * warp + tw; t0 < nr && ok; t0 += 4 * kWarps) {
+        const uint2 w = t0 < n ? *reinterpret_cast<const uint2 *>(vs + t0 * kRowBytes + 8 * cb)
+                               : make_uint2(0x88888888u, 0x88888888u);
         float vc[16];
         unpack16(w, vc);
 #pragma unroll
         for (int gi = 0; gi < G; ++gi) {
-            const float p = live ? sm[gi * Lc + t0] : 0.0f;
+            const float p = t0 < n ? sm[gi * kChunk + t0] : 0.0f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) acc2[gi][i] = fmaf(p, vc[i], acc2[gi][i]);
         }
     }
-    // sum over the warp's 4 token lanes (same channel block), then the warps
+    // sum over the warp's 4 row lanes (same channel block), then the warps
 #pragma unroll
     for (int gi = 0; gi < G; ++gi)
 #pragma unroll
@@ -239,12 +274,21 @@ __global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
         const int gi = e / kD, c = e % kD;
         float t = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) t += osum[w][gi][c];
+        for (int w = 0; w < kWarps; ++w) t += osum[w][gi][c];
         rec[gi * (kD + 2) + 2 + c] = t;
     }
     if (threadIdx.x < G) {
         rec[threadIdx.x * (kD + 2)] = gmax[threadIdx.x];
         rec[threadIdx.x * (kD + 2) + 1] = gsum[threadIdx.x];
+    }
+    if (threadIdx.x == 0 && abort_flag) {
+        // a wait ran out: report it, and let both copies land before leaving
+        atomicExch(&g_kv4_error, 1);
+        const uint64_t end = global_timer_ns() + 200000000ull;
+        while (!mbar_try_wait(kbar, 0u) && global_timer_ns() < end) {
+        }
+        while (!mbar_try_wait(vbar, 0u) && global_timer_ns() < end) {
+        }
     }
 }
 
@@ -277,24 +321,9 @@ __global__ void __launch_bounds__(kD) kv4_combine_kernel(const float *__restrict
 
 }  // namespace
 
-// chunk length (tokens, a multiple of 16) for a problem: about two CTAs per
-// SM over all (sequence, KV head, chunk), at most 1024 tokens per chunk
-static int kv4_chunk(int B, int Hkv, int L)
-{
-    const long long heads = (long long)B * Hkv;
-    long long S = (2 * kMaxCtas + heads - 1) / heads;
-    if (S < 1) S = 1;
-    long long Lc = (L + S - 1) / S;
-    Lc = (Lc + 15) / 16 * 16;
-    if (Lc < 64) Lc = 64;
-    if (Lc > 1024) Lc = 1024;
-    return (int)Lc;
-}
-
 size_t kv4_workspace_bytes(int B, int Hq, int Hkv, int L)
 {
-    const int Lc = kv4_chunk(B, Hkv, L);
-    const long long S = (L + Lc - 1) / Lc;
+    const long long S = (L + kChunk - 1) / kChunk;
     return (size_t)B * Hq * S * (kD + 2) * sizeof(float);
 }
 
@@ -310,13 +339,12 @@ static cudaError_t launch_attn_g(const uint16_t *q, const uint8_t *K4, const uin
                                  const uint16_t *s_k, const uint16_t *s_v, int B, int Hkv, int L, uint16_t *out,
                                  float *part, cudaStream_t stream)
 {
-    const int Lc = kv4_chunk(B, Hkv, L);
-    const int S = (L + Lc - 1) / Lc;
-    const size_t smem = (size_t)G * Lc * sizeof(float);
+    const int S = (L + kChunk - 1) / kChunk;
+    const size_t smem = 2 * (size_t)kChunk * kRowBytes + (size_t)G * kChunk * sizeof(float) + 16;
     auto k1 = kv4_attn_chunk_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k1<<<dim3((unsigned)(B * Hkv), (unsigned)S), kThreads, smem, stream>>>(q, K4, V4, lam, s_k, Hkv, L, Lc, part);
+    k1<<<dim3((unsigned)(B * Hkv), (unsigned)S), kThreads, smem, stream>>>(q, K4, V4, lam, s_k, Hkv, L, part);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     kv4_combine_kernel<G><<<(unsigned)(B * Hkv * G), kD, 0, stream>>>(part, s_v, Hkv, S, out);
@@ -334,6 +362,20 @@ cudaError_t launch_kv4_attention(const uint16_t *q, const uint8_t *K4, const uin
     case 4: return launch_attn_g<4>(q, K4, V4, lam, s_k, s_v, B, Hkv, L, out, part, stream);
     default: return launch_attn_g<8>(q, K4, V4, lam, s_k, s_v, B, Hkv, L, out, part, stream);
     }
+}
+
+cudaError_t read_and_clear_kv4_error(int *value)
+{
+    *value = 0;
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_kv4_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_kv4_error, &zero, sizeof(int));
+    }
+    *value = v;
+    return e;
 }
 
 }  // namespace qoq
