@@ -538,6 +538,15 @@ def run_ours(args, rank, world, local, dist):
             w8a8["by_bound"][b] = ent
         cross = [p["M"] for p in per if "w4a8_speedup_over_w8a8" in p and p["w4a8_speedup_over_w8a8"] < 1.0]
         w8a8["first_M_where_w8a8_is_faster"] = min(cross) if cross else None
+        # the pages' roofline argument ("QServe: Low Bit Width Does Not
+        # Guarantee High Throughput", section 2, Figure 3) redone with this
+        # GPU's measured peaks: per weight element, W4A16 moves 0.5 byte at
+        # the FP16 peak (half the INT8 peak), W8A8 1 byte at the INT8 peak,
+        # W4A8 0.5 byte at the INT8 peak
+        w4a16, w8, w4 = (P8 / 2, 0.5), (P8, 1.0), (P8, 0.5)
+        w8a8["roofline_model_crossovers_m"] = {
+            "w4a16_vs_w8a8": roofline.crossover_m(w4a16, w8, BW),
+            "w4a8_vs_w8a8_equal_from": roofline.crossover_m(w4, w8, BW)}
 
     # end to end through the public API from pinned host memory
     e2e = None
