@@ -444,8 +444,11 @@ QOQ_API size_t qoq_kv4_attention_workspace_bytes(int B, int Hq, int Hkv, int L, 
  *   score[l] = sum_c (q[c] * lam[c]) * (s_k[c] * code_k[l][c]) / sqrt(d)
  *   p = softmax(score);  out[c] = sum_l p[l] * s_v[c] * code_v[l][c]
  * rounded to FP16 once. The kernel folds lam, s_k and 1/sqrt(d) into the
- * query and s_v into the final sum, and computes in FP32: within 2 FP16 ulp
- * (plus 1e-3 of the output row's largest value) of the binary64 result.
+ * query and s_v into the final sum. Both products run on the tensor cores
+ * with the codes exact in FP16 and each FP32 factor (the folded query, the
+ * softmax numerators) split into two FP16 parts, summed in FP32: within
+ * 2 FP16 ulp (plus 1e-3 of the output row's largest value) of the binary64
+ * result.
  *   workspace   device, qoq_kv4_attention_workspace_bytes bytes, any
  *               contents (every call overwrites what it reads).
  * Limits as for qoq_kv4_cache_quantize, plus Hq a multiple of Hkv. */

@@ -100,10 +100,9 @@ PAIR_SHAPES = [(200, 1024, 512, 128), (256, 4096, 4096, 128), (513, 512, 256, 51
 
 @pytest.mark.parametrize("M,K,N,G", PAIR_SHAPES, ids=[f"M{m}_K{k}_N{n}_G{g}" for m, k, n, g in PAIR_SHAPES])
 def test_cta_pairs_match_single(M, K, N, G):
-    """256-token tiles on CTA pairs (2-SM MMA) give the same bits as on
-    single CTAs, and as the narrower tiles the default rule picks for few
-    tiles; all equal the exact product."""
-    q.qoq_set_gemm_a_in_tmem(True)
+    """256-token tiles on CTA pairs (2-SM MMA, A in TMEM or in shared
+    memory) give the same bits as on single CTAs, and as the narrower tiles
+    the default rule picks for few tiles; all equal the exact product."""
     dev = torch.device("cuda")
     X = wl.make_activations(M, K, wl.LLAMA, seed=5300 + M)
     W = wl.make_weights(N, K, wl.LLAMA, seed=5400 + M)
@@ -112,18 +111,21 @@ def test_cta_pairs_match_single(M, K, N, G):
     ref = _ref_acc(X8, q.qoq_dequant_weights_i8(packed))
     out = {}
     try:
-        for narrow, pairs in ((False, False), (False, True), (True, True)):
-            q.qoq_set_gemm_narrow_tiles(narrow)
-            q.qoq_set_gemm_cta_pairs(pairs)
-            for run in range(3):
-                acc = torch.full((M, N), -7, dtype=torch.int32, device=dev)
-                Y = q.qoq_w4a8_gemm(X8, s_x, packed, acc_dbg=acc)
-                torch.cuda.synchronize()
-                assert q.qoq_device_error() == q.QOQ_OK
-                assert torch.equal(acc, ref), f"narrow={narrow} pairs={pairs} run {run}: INT32 mismatch"
-            out[(narrow, pairs)] = Y
+        for a_tmem in (True, False):
+            q.qoq_set_gemm_a_in_tmem(a_tmem)
+            for narrow, pairs in ((False, False), (False, True), (True, True)):
+                q.qoq_set_gemm_narrow_tiles(narrow)
+                q.qoq_set_gemm_cta_pairs(pairs)
+                for run in range(3):
+                    acc = torch.full((M, N), -7, dtype=torch.int32, device=dev)
+                    Y = q.qoq_w4a8_gemm(X8, s_x, packed, acc_dbg=acc)
+                    torch.cuda.synchronize()
+                    assert q.qoq_device_error() == q.QOQ_OK
+                    assert torch.equal(acc, ref), f"a_tmem={a_tmem} narrow={narrow} pairs={pairs} run {run}"
+                out[(a_tmem, narrow, pairs)] = Y
     finally:
         q.qoq_set_gemm_cta_pairs(True)
         q.qoq_set_gemm_narrow_tiles(True)
+        q.qoq_set_gemm_a_in_tmem(True)
     for k in out:
-        assert torch.equal(out[k].view(torch.int16), out[(False, False)].view(torch.int16)), k
+        assert torch.equal(out[k].view(torch.int16), out[(True, False, False)].view(torch.int16)), k

@@ -1186,6 +1186,11 @@ cudaError_t launch_cfg(const CUtensorMap &tmap, const GemmArgs &args, int grid, 
     if (!(opted_in.load(std::memory_order_acquire) & bit)) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
         if (e != cudaSuccess) return e;
+        // all of the unified L1/shared storage as shared memory, so that two
+        // half CTAs (or a GEMM CTA and a neighbour) fit on one SM
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         opted_in.fetch_or(bit, std::memory_order_acq_rel);
     }
     // programmatic dependent launch: the GEMM may start (and stream weights)

@@ -21,10 +21,11 @@
 // the final weighted sum.  Design for B200 (the pages' A100 kernel with
 // FP16 QK/SV products is prior art): flash-decoding over token chunks, one
 // CTA per (sequence, KV head, chunk) serving the G query heads that share
-// the KV head, FP32 products and sums on the CUDA cores, 8-byte coalesced
-// loads (a warp reads 4 whole token rows per load), a second small kernel
-// combining the chunks.  The path is HBM-bound for G = 1 and bound by the
-// FP32 issue rate for larger G (G FMAs per cached element).
+// the KV head, the chunk's codes brought into shared memory by bulk copies,
+// both products on the tensor cores as warp-level MMAs with the codes
+// expanded to FP16 in registers (exact) and the FP32 factors split into
+// two FP16 parts, a second small kernel combining the chunks.  The path is
+// HBM-bound: the expansion costs about 1.5 instructions per code.
 #include <cuda_fp16.h>
 
 #include <cstdint>
@@ -87,208 +88,375 @@ __global__ void __launch_bounds__(kD) kv4_cache_kernel(const uint16_t *__restric
     }
 }
 
-// 16 nibbles of a 64-bit word -> the codes as floats (nibble - 8).  The
-// nibble is placed in the low mantissa bits of 2^23 (exactly 2^23 + n) and
-// 2^23 + 8 is subtracted: one logic op and one add per value, exact, at
-// full rate (an integer-to-float conversion is a quarter-rate instruction).
-__device__ __forceinline__ float nib_to_float(uint32_t w, int i)
+// Two 4-bit codes as an FP16 pair: the nibbles in bits 0-3 and 16-19 of x
+// are placed in the mantissa of 1024 (exactly 1024 + n) and 1032 is
+// subtracted, giving the codes n - 8 exactly: one logic op and one FP16 pair
+// subtraction per two codes (an integer-to-float conversion is a
+// quarter-rate instruction).
+__device__ __forceinline__ uint32_t codes_h2(uint32_t x)
 {
-    return __int_as_float((int)(0x4B000000u | ((w >> (4 * i)) & 0xFu))) - 8388616.0f;
+    const uint32_t h = (x & 0x000F000Fu) | 0x64006400u;
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64086408u));
+    return r;
 }
 
-__device__ __forceinline__ void unpack16(uint2 w, float *f)
+// D (16 x 8, FP32) += A (16 x 16, FP16, row) * B (16 x 8, FP16, col): the
+// warp-level tensor-core product.  Fragment of lane (g = lane / 4, c = lane
+// % 4): A rows g and g + 8 at columns 2c, 2c + 1 and 2c + 8, 2c + 9; B
+// column g at rows 2c, 2c + 1 and 2c + 8, 2c + 9; D rows g and g + 8 at
+// columns 2c, 2c + 1.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = nib_to_float(w.x, i);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f[8 + i] = nib_to_float(w.y, i);
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-constexpr int kThreads = 256;    // 8 warps; a warp covers 4 token rows per step (8 lanes a row)
+__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi)
+{
+    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+constexpr int kThreads = 256;    // 8 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = 512;      // tokens per CTA: 32 KB of K codes and 32 KB of V codes
+constexpr int kWarpTok = kChunk / kWarps;   // 64 tokens per warp: four 16-token MMA steps
+constexpr int kSub = 128;        // tokens per bulk copy (two warps' share)
+constexpr int kNumSub = kChunk / kSub;
+constexpr int kPStride = kChunk + 8;        // FP16 elements per row of P (rows 4 banks apart)
 
 __device__ int g_kv4_error;      // non-zero after a bounded wait of this file's kernels ran out
 
 // ------------------------------------------------- attention, one chunk --
 // CTA (sequence b, KV head g, chunk s) over tokens [s*kChunk, min(L, ...)):
-// the chunk's K and V codes are contiguous in the cache, so one bulk copy
-// each brings them into shared memory at the start (64 KB in flight per
-// CTA).  Pass 1 scores every token for the G query heads (from shared
-// memory), the chunk's softmax numerators follow, pass 2 sums the value
-// codes weighted by them.  The chunk's (max, sum, weighted sums) go to the
-// workspace for the combine.
+// the chunk's K and V codes are contiguous in the cache and arrive by bulk
+// copies of 128 tokens, each on its own barrier, so the products start as
+// soon as the first 8 KB has landed.  Both products run on the tensor cores
+// (mma.sync m16n8k16, FP16 operands, FP32 sums), eight columns per MMA:
+// up to four query heads, each as a high and a low FP16 part, so that the
+// operands carry FP32-level precision (hi + lo) while the codes are exact
+// in FP16.
+//   scores:  S[token][col] = sum_c K[token][c] * q'[col][c]   (A = codes, rows = tokens)
+//   values:  O^T[c][col]   = sum_t V[t][c] * p[col][t]        (A = codes^T, rows = channels)
+// Each head's q' is scaled by a power of two that brings its largest
+// element into [2^13, 2^14) (no FP16 overflow, full precision in the
+// parts), undone exactly on the score.  The softmax numerators of the
+// chunk, split the same way, go through shared memory (the score fragment
+// holds tokens by row, the value product needs them by column).  Each
+// warp takes 64 tokens in both passes; the warps' weighted sums are added in
+// shared memory (over the K codes, dead by then), and the chunk's (max, sum,
+// weighted sums) per query head go to the workspace for the combine.
 template <int G>
-__global__ void __launch_bounds__(kThreads) kv4_attn_chunk_kernel(
+__global__ void __launch_bounds__(kThreads, G > 4 ? 1 : 2) kv4_attn_chunk_kernel(
     const uint16_t *__restrict__ q, const uint8_t *__restrict__ K4, const uint8_t *__restrict__ V4,
     const uint16_t *__restrict__ lam, const uint16_t *__restrict__ s_k, int Hkv, int L,
     float *__restrict__ part)
 {
+    constexpr int HT = (G + 3) / 4;             // column tiles of 8 (4 heads x hi/lo)
     extern __shared__ __align__(128) uint8_t dyn[];
     uint8_t *ks = dyn;                                   // [kChunk][64] K codes
     uint8_t *vs = dyn + kChunk * kRowBytes;              // [kChunk][64] V codes
-    float *sm = reinterpret_cast<float *>(dyn + 2 * kChunk * kRowBytes);   // [G][kChunk]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G * kChunk);        // K landed, V landed
-    __shared__ float red[G][kWarps];
+    __half *ps = reinterpret_cast<__half *>(dyn + 2 * kChunk * kRowBytes);  // [HT][8][kPStride]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ps + HT * 8 * kPStride);  // K parts, V parts
+    float *osum = reinterpret_cast<float *>(ks);         // [kWarps][G][kD], over the K codes
+    __shared__ float red[kWarps][G];
     __shared__ float gmax[G], gsum[G];
-    __shared__ float osum[kWarps][G][kD];
     __shared__ int abort_flag;
     const int bh = blockIdx.x;                   // b * Hkv + kv head
     const int b = bh / Hkv, hk = bh % Hkv;
     const int S = gridDim.y, s = blockIdx.y;
     const int l0 = s * kChunk, n = min(L - l0, kChunk);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int cb = lane & 7;                     // channel block: channels 16*cb .. 16*cb+15
-    const int tw = lane >> 3;                    // row within the warp's 4
+    const int g = lane >> 2, c = lane & 3;
     const size_t head = (size_t)bh;
-    const uint32_t kbar = smem_addr(bars), vbar = smem_addr(bars + 1);
-    const uint32_t bytes = (uint32_t)n * kRowBytes;
+    const uint32_t bar0 = smem_addr(bars);
+    auto kbar = [&](int j) { return bar0 + 8u * j; };
+    auto vbar = [&](int j) { return bar0 + 8u * (kNumSub + j); };
     if (threadIdx.x == 0) {
-        mbar_init(kbar, 1);
-        mbar_init(vbar, 1);
+        for (int j = 0; j < 2 * kNumSub; ++j) mbar_init(bar0 + 8u * j, 1);
         abort_flag = 0;
         fence_mbar_init();
-        mbar_arrive_expect_tx(kbar, bytes);
-        bulk_load(smem_addr(ks), K4 + (head * L + l0) * kRowBytes, bytes, kbar);
-        mbar_arrive_expect_tx(vbar, bytes);
-        bulk_load(smem_addr(vs), V4 + (head * L + l0) * kRowBytes, bytes, vbar);
+        for (int pass = 0; pass < 2; ++pass) {
+            const uint8_t *src = (pass ? V4 : K4) + (head * L + l0) * kRowBytes;
+            uint8_t *dst = pass ? vs : ks;
+            for (int j = 0; j < kNumSub; ++j) {
+                const int rows = max(0, min(n - j * kSub, kSub));
+                const uint32_t bar = pass ? vbar(j) : kbar(j);
+                if (rows > 0) {
+                    mbar_arrive_expect_tx(bar, (uint32_t)rows * kRowBytes);
+                    bulk_load(smem_addr(dst + j * kSub * kRowBytes), src + (size_t)j * kSub * kRowBytes,
+                              (uint32_t)rows * kRowBytes, bar);
+                } else {
+                    mbar_arrive(bar);
+                }
+            }
+        }
     }
-    // the query of each of the G heads, with lambda, s_k and 1/sqrt(d)
-    // folded in (while the copies are in flight)
+    // B fragments of the score product (while the copies are in flight):
+    // column g of tile t is query head 4t + g % 4, its high part for g < 4
+    // and its low part for g >= 4; lane c holds channels 32c .. 32c + 31.
+    // The K codes' word j of those channels holds channel 32c + 8j + i in
+    // nibble i; MMA step 2j + h pairs nibbles (2h, 2h + 4) at columns
+    // 2c, 2c + 1 and (2h + 1, 2h + 5) at 2c + 8, 2c + 9.
     const float inv_sqrt_d = 0.08838834764831845f;   // 1 / sqrt(128)
-    float qf[G][16];
+    uint32_t qb[HT][8][2];
+    float escale[HT][2];                         // 2^e of heads 4t + 2(c % 2) + {0, 1}
+    {
+        float fold[32];
+        {
+            const uint4 *lp = reinterpret_cast<const uint4 *>(lam + head * kD + 32 * c);
+            const uint4 *sp = reinterpret_cast<const uint4 *>(s_k + head * kD + 32 * c);
 #pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
-        const size_t qh = ((size_t)b * Hkv * G + (size_t)hk * G + gi) * kD;
+            for (int v = 0; v < 4; ++v) {
+                const uint4 lw = __ldg(lp + v), sw = __ldg(sp + v);
+                const uint32_t la[4] = {lw.x, lw.y, lw.z, lw.w}, sa[4] = {sw.x, sw.y, sw.z, sw.w};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int c = 16 * cb + i;
-            const float f = __fmul_rn(__fmul_rn(half_bits_to_float(__ldg(lam + head * kD + c)),
-                                                half_bits_to_float(__ldg(s_k + head * kD + c))),
-                                      inv_sqrt_d);
-            qf[gi][i] = __fmul_rn(half_bits_to_float(__ldg(q + qh + c)), f);
+                for (int e = 0; e < 8; ++e) {
+                    const float lf = half_bits_to_float((uint16_t)(la[e / 2] >> (16 * (e % 2))));
+                    const float sf = half_bits_to_float((uint16_t)(sa[e / 2] >> (16 * (e % 2))));
+                    fold[8 * v + e] = __fmul_rn(__fmul_rn(lf, sf), inv_sqrt_d);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < HT; ++t) {
+            const int hq = 4 * t + (g & 3);
+            float f[32];
+            float m = 0.0f;
+            if (hq < G) {
+                const uint4 *qp = reinterpret_cast<const uint4 *>(q + ((size_t)bh * G + hq) * kD + 32 * c);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 qw = __ldg(qp + v);
+                    const uint32_t qa[4] = {qw.x, qw.y, qw.z, qw.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        f[8 * v + e] = __fmul_rn(half_bits_to_float((uint16_t)(qa[e / 2] >> (16 * (e % 2)))),
+                                                 fold[8 * v + e]);
+                        m = fmaxf(m, fabsf(f[8 * v + e]));
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) f[i] = 0.0f;
+            }
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            // m in [2^E, 2^(E+1)) with E its biased exponent field - 127 (a
+            // zero or subnormal m takes E = -126); e = E - 13 brings the
+            // largest |q'| * 2^-e into [2^13, 2^14), and both powers of two
+            // are exact FP32 numbers for e in [-126, 114]
+            const int E = max((int)((__float_as_uint(m) >> 23) & 0xFFu), 1) - 127;
+            const int e = max(E - 13, -126);
+            const float down = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e
+            __half part_v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float x = f[i] * down;
+                const __half hi = __float2half_rn(x);
+                part_v[i] = g < 4 ? hi : __float2half_rn(x - __half2float(hi));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    qb[t][2 * j + h][0] = pack_h2(part_v[8 * j + 2 * h], part_v[8 * j + 2 * h + 4]);
+                    qb[t][2 * j + h][1] = pack_h2(part_v[8 * j + 2 * h + 1], part_v[8 * j + 2 * h + 5]);
+                }
+            // the exponents of the two heads whose scores this lane ends up with
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                escale[t][i] = __uint_as_float((uint32_t)(127 + __shfl_sync(0xffffffffu, e, 4 * (2 * (c & 1) + i))) << 23);
         }
     }
     __syncthreads();
     const uint64_t budget = 2000000000ull;
-    bool ok = wait_bounded(kbar, 0u, &abort_flag, budget);
-    // pass 1: scores
-    const int nr = (n + 4 * kWarps - 1) / (4 * kWarps) * (4 * kWarps);
-    for (int t0 = 4 * warp + tw; t0 < nr && ok; t0 += 4 * kWarps) {
-        const uint2 w = t0 < n ? *reinterpret_cast<const uint2 *>(ks + t0 * kRowBytes + 8 * cb)
-                               : make_uint2(0x88888888u, 0x88888888u);
-        float kc[16];
-        unpack16(w, kc);
-        float acc[G];
+    const int T0 = warp * kWarpTok;
+    bool ok = wait_bounded(kbar(T0 / kSub), 0u, &abort_flag, budget);
+    // pass 1: scores of the warp's 64 tokens (rows g and g + 8 of each
+    // 16-token step), all columns
+    float sc[4][HT][4];
 #pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
-            float a = 0.0f;
+    for (int st = 0; st < 4; ++st) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) a = fmaf(qf[gi][i], kc[i], a);
-            acc[gi] = a;
-        }
+        for (int t = 0; t < HT; ++t)
 #pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
-            acc[gi] += __shfl_xor_sync(0xffffffffu, acc[gi], 4);
-            acc[gi] += __shfl_xor_sync(0xffffffffu, acc[gi], 2);
-            acc[gi] += __shfl_xor_sync(0xffffffffu, acc[gi], 1);
-        }
-        if (cb == 0 && t0 < n) {
+            for (int r = 0; r < 4; ++r) sc[st][t][r] = 0.0f;
+        if (!ok) continue;
+        const int r0 = T0 + 16 * st + g;
+        const uint4 k0 = *reinterpret_cast<const uint4 *>(ks + r0 * kRowBytes + 16 * c);
+        const uint4 k1 = *reinterpret_cast<const uint4 *>(ks + (r0 + 8) * kRowBytes + 16 * c);
+        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) sm[gi * kChunk + t0] = acc[gi];
-        }
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t a[4] = {codes_h2(w0[j] >> (8 * h)), codes_h2(w1[j] >> (8 * h)),
+                                       codes_h2(w0[j] >> (8 * h + 4)), codes_h2(w1[j] >> (8 * h + 4))};
+#pragma unroll
+                for (int t = 0; t < HT; ++t) mma_f16_16816(sc[st][t], a, qb[t][2 * j + h][0], qb[t][2 * j + h][1]);
+            }
     }
-    __syncthreads();
+    // high + low columns (lanes c and c ^ 2), power of two undone; lane c
+    // then holds heads 4t + 2(c % 2) + i for rows g and g + 8 of each step
+    float lmax[HT][2];
+#pragma unroll
+    for (int t = 0; t < HT; ++t) lmax[t][0] = lmax[t][1] = -INFINITY;
+#pragma unroll
+    for (int st = 0; st < 4; ++st)
+#pragma unroll
+        for (int t = 0; t < HT; ++t)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int i = r & 1;
+                const int tok = T0 + 16 * st + g + 8 * (r >> 1);
+                const int hq = 4 * t + 2 * (c & 1) + i;
+                const float v = (sc[st][t][r] + __shfl_xor_sync(0xffffffffu, sc[st][t][r], 2)) * escale[t][i];
+                sc[st][t][r] = (tok < n && hq < G) ? v : -INFINITY;
+                lmax[t][i] = fmaxf(lmax[t][i], sc[st][t][r]);
+            }
     // the chunk's softmax numerators: exp(score - chunk max), and their sum
 #pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
-        float m = -INFINITY;
-        for (int t = threadIdx.x; t < n; t += kThreads) m = fmaxf(m, sm[gi * kChunk + t]);
-        m = warp_max(m);
-        if (lane == 0) red[gi][warp] = m;
-    }
+    for (int t = 0; t < HT; ++t)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            float m = lmax[t][i];
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+            const int hq = 4 * t + 2 * (c & 1) + i;
+            if (lane < 2 && hq < G) red[warp][hq] = m;
+        }
     __syncthreads();
     if (threadIdx.x < G) {
-        float m = red[threadIdx.x][0];
+        float m = red[0][threadIdx.x];
 #pragma unroll
-        for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[threadIdx.x][w]);
+        for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w][threadIdx.x]);
         gmax[threadIdx.x] = m;
     }
     __syncthreads();
+    float lsum[HT][2];
 #pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
-        float sum = 0.0f;
-        for (int t = threadIdx.x; t < n; t += kThreads) {
-            const float p = expf(sm[gi * kChunk + t] - gmax[gi]);
-            sm[gi * kChunk + t] = p;
-            sum += p;
+    for (int t = 0; t < HT; ++t) lsum[t][0] = lsum[t][1] = 0.0f;
+#pragma unroll
+    for (int st = 0; st < 4; ++st)
+#pragma unroll
+        for (int t = 0; t < HT; ++t)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int i = r & 1;
+                const int tok = T0 + 16 * st + g + 8 * (r >> 1);
+                const int hq = 4 * t + 2 * (c & 1) + i;
+                const float p = sc[st][t][r] == -INFINITY ? 0.0f : expf(sc[st][t][r] - gmax[hq < G ? hq : 0]);
+                lsum[t][i] += p;
+                // column (c / 2) * 4 + 2(c % 2) + i: the high part from lanes c < 2,
+                // the low part from lanes c >= 2
+                const __half hi = __float2half_rn(p);
+                ps[(t * 8 + (c >> 1) * 4 + 2 * (c & 1) + i) * kPStride + tok] =
+                    c < 2 ? hi : __float2half_rn(p - __half2float(hi));
+            }
+    __syncthreads();   // red is reused below; P complete; the K codes are dead
+#pragma unroll
+    for (int t = 0; t < HT; ++t)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            float v = lsum[t][i];
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 16);
+            const int hq = 4 * t + 2 * (c & 1) + i;
+            if (lane < 2 && hq < G) red[warp][hq] = v;
+        }
+    // pass 2: O^T[channel][column] over the warp's 64 tokens; m-tile mt
+    // row g is channel 16g + 2mt (a low nibble), row g + 8 channel
+    // 16g + 2mt + 1 (the high nibble of the same byte)
+    float o[HT][8][4];
+#pragma unroll
+    for (int t = 0; t < HT; ++t)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) o[t][mt][r] = 0.0f;
+    ok = ok && wait_bounded(vbar(T0 / kSub), 0u, &abort_flag, budget);
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+        if (!ok) break;
+        const int tA = T0 + 16 * st + 2 * c;    // tokens tA, tA + 1, tA + 8, tA + 9
+        const int odd = c & 1;
+        // each load instruction of the warp touches rows of both parities
+        const uint2 x0 = *reinterpret_cast<const uint2 *>(vs + (tA + odd) * kRowBytes + 8 * g);
+        const uint2 x1 = *reinterpret_cast<const uint2 *>(vs + (tA + 1 - odd) * kRowBytes + 8 * g);
+        const uint2 y0 = *reinterpret_cast<const uint2 *>(vs + (tA + 8 + odd) * kRowBytes + 8 * g);
+        const uint2 y1 = *reinterpret_cast<const uint2 *>(vs + (tA + 9 - odd) * kRowBytes + 8 * g);
+        const uint2 vA = odd ? x1 : x0, vB = odd ? x0 : x1, vC = odd ? y1 : y0, vD = odd ? y0 : y1;
+        uint32_t pb[HT][2];
+#pragma unroll
+        for (int t = 0; t < HT; ++t) {
+            pb[t][0] = *reinterpret_cast<const uint32_t *>(ps + (t * 8 + g) * kPStride + tA);
+            pb[t][1] = *reinterpret_cast<const uint32_t *>(ps + (t * 8 + g) * kPStride + tA + 8);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) red[gi][warp] = sum;
+        for (int wi = 0; wi < 2; ++wi) {
+            const uint32_t wa = wi ? vA.y : vA.x, wb = wi ? vB.y : vB.x;
+            const uint32_t wc = wi ? vC.y : vC.x, wd = wi ? vD.y : vD.x;
+#pragma unroll
+            for (int bp = 0; bp < 2; ++bp) {
+                // bytes 2bp, 2bp + 1 of the first token over those of the second
+                const uint32_t sel = (2 * bp) | ((2 * bp + 1) << 4) | ((2 * bp + 4) << 8) | ((2 * bp + 5) << 12);
+                const uint32_t xab = __byte_perm(wa, wb, sel), xcd = __byte_perm(wc, wd, sel);
+                const int mt = 4 * wi + 2 * bp;
+                const uint32_t a0[4] = {codes_h2(xab), codes_h2(xab >> 4), codes_h2(xcd), codes_h2(xcd >> 4)};
+                const uint32_t a1[4] = {codes_h2(xab >> 8), codes_h2(xab >> 12), codes_h2(xcd >> 8),
+                                        codes_h2(xcd >> 12)};
+#pragma unroll
+                for (int t = 0; t < HT; ++t) {
+                    mma_f16_16816(o[t][mt], a0, pb[t][0], pb[t][1]);
+                    mma_f16_16816(o[t][mt + 1], a1, pb[t][0], pb[t][1]);
+                }
+            }
+        }
     }
+    // high + low columns, then the warps' sums in shared memory
+#pragma unroll
+    for (int t = 0; t < HT; ++t)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float v = o[t][mt][r] + __shfl_xor_sync(0xffffffffu, o[t][mt][r], 2);
+                const int hq = 4 * t + 2 * c + (r & 1);
+                if (c < 2 && hq < G) osum[(warp * G + hq) * kD + 16 * g + 2 * mt + (r >> 1)] = v;
+            }
     __syncthreads();
     if (threadIdx.x < G) {
         float t = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) t += red[threadIdx.x][w];
+        for (int w = 0; w < kWarps; ++w) t += red[w][threadIdx.x];
         gsum[threadIdx.x] = t;
     }
-    // pass 2: the numerator-weighted sums of the value codes
-    float acc2[G][16];
-#pragma unroll
-    for (int gi = 0; gi < G; ++gi)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) acc2[gi][i] = 0.0f;
-    ok = ok && wait_bounded(vbar, 0u, &abort_flag, budget);
-    for (int t0 = 4 * warp + tw; t0 < nr && ok; t0 += 4 * kWarps) {
-        const uint2 w = t0 < n ? *reinterpret_cast<const uint2 *>(vs + t0 * kRowBytes + 8 * cb)
-                               : make_uint2(0x88888888u, 0x88888888u);
-        float vc[16];
-        unpack16(w, vc);
-#pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
-            const float p = t0 < n ? sm[gi * kChunk + t0] : 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc2[gi][i] = fmaf(p, vc[i], acc2[gi][i]);
-        }
-    }
-    // sum over the warp's 4 row lanes (same channel block), then the warps
-#pragma unroll
-    for (int gi = 0; gi < G; ++gi)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            acc2[gi][i] += __shfl_xor_sync(0xffffffffu, acc2[gi][i], 8);
-            acc2[gi][i] += __shfl_xor_sync(0xffffffffu, acc2[gi][i], 16);
-        }
-    if (tw == 0) {
-#pragma unroll
-        for (int gi = 0; gi < G; ++gi)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) osum[warp][gi][16 * cb + i] = acc2[gi][i];
-    }
-    __syncthreads();
     // partial record per query head: [max, sum, kD weighted sums]
     float *rec = part + (((size_t)bh * S + s) * G) * (kD + 2);
     for (int e = threadIdx.x; e < G * kD; e += kThreads) {
-        const int gi = e / kD, c = e % kD;
+        const int gi = e / kD, ch = e % kD;
         float t = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) t += osum[w][gi][c];
-        rec[gi * (kD + 2) + 2 + c] = t;
+        for (int w = 0; w < kWarps; ++w) t += osum[(w * G + gi) * kD + ch];
+        rec[gi * (kD + 2) + 2 + ch] = t;
     }
+    __syncthreads();
     if (threadIdx.x < G) {
         rec[threadIdx.x * (kD + 2)] = gmax[threadIdx.x];
         rec[threadIdx.x * (kD + 2) + 1] = gsum[threadIdx.x];
     }
     if (threadIdx.x == 0 && abort_flag) {
-        // a wait ran out: report it, and let both copies land before leaving
+        // a wait ran out: report it, and let every copy land before leaving
         atomicExch(&g_kv4_error, 1);
         const uint64_t end = global_timer_ns() + 200000000ull;
-        while (!mbar_try_wait(kbar, 0u) && global_timer_ns() < end) {
-        }
-        while (!mbar_try_wait(vbar, 0u) && global_timer_ns() < end) {
-        }
+        for (int j = 0; j < 2 * kNumSub; ++j)
+            while (!mbar_try_wait(bar0 + 8u * j, 0u) && global_timer_ns() < end) {
+            }
     }
 }
 
@@ -306,14 +474,32 @@ __global__ void __launch_bounds__(kD) kv4_combine_kernel(const float *__restrict
     const int hk = h / G, gi = h % G;
     const size_t bh = (size_t)b * Hkv + hk;
     const int c = threadIdx.x;
+    const float *rec0 = part + (bh * S * G + gi) * (kD + 2);   // chunk s at rec0 + s * G * (kD + 2)
+    const size_t step = (size_t)G * (kD + 2);
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, part[((bh * S + s) * G + gi) * (kD + 2)]);
+    for (int s = 0; s < S; s += 8) {
+        float m[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m[u] = s + u < S ? rec0[(s + u) * step] : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) M = fmaxf(M, m[u]);
+    }
     float den = 0.0f, num = 0.0f;
-    for (int s = 0; s < S; ++s) {
-        const float *rec = part + ((bh * S + s) * G + gi) * (kD + 2);
-        const float w = expf(rec[0] - M);
-        den = fmaf(rec[1], w, den);
-        num = fmaf(rec[2 + c], w, num);
+    for (int s = 0; s < S; s += 8) {
+        float mx[8], sm[8], x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const bool in = s + u < S;
+            mx[u] = in ? rec0[(s + u) * step] : -INFINITY;
+            sm[u] = in ? rec0[(s + u) * step + 1] : 0.0f;
+            x[u] = in ? rec0[(s + u) * step + 2 + c] : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float w = s + u < S ? expf(mx[u] - M) : 0.0f;
+            den = fmaf(sm[u], w, den);
+            num = fmaf(x[u], w, num);
+        }
     }
     const float sv = half_bits_to_float(__ldg(s_v + bh * kD + c));
     out[(size_t)bq * kD + c] = float_to_half_bits(__fmul_rn(__fdiv_rn(num, den), sv));
@@ -340,9 +526,14 @@ static cudaError_t launch_attn_g(const uint16_t *q, const uint8_t *K4, const uin
                                  float *part, cudaStream_t stream)
 {
     const int S = (L + kChunk - 1) / kChunk;
-    const size_t smem = 2 * (size_t)kChunk * kRowBytes + (size_t)G * kChunk * sizeof(float) + 16;
+    const size_t smem = 2 * (size_t)kChunk * kRowBytes + (size_t)((G + 3) / 4) * 8 * kPStride * sizeof(__half) +
+                        2 * kNumSub * sizeof(uint64_t);
     auto k1 = kv4_attn_chunk_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // all of the unified L1/shared storage as shared memory: three CTAs
+    // (two for G = 8) per SM keep their copies in flight together
+    e = cudaFuncSetAttribute(k1, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     k1<<<dim3((unsigned)(B * Hkv), (unsigned)S), kThreads, smem, stream>>>(q, K4, V4, lam, s_k, Hkv, L, part);
     e = cudaGetLastError();
