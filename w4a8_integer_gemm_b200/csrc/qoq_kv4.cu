@@ -28,6 +28,7 @@
 // HBM-bound: the expansion costs about 1.5 instructions per code.
 #include <cuda_fp16.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "qoq_internal.h"
@@ -114,11 +115,6 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi)
-{
-    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-}
-
 constexpr int kThreads = 256;    // 8 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = 512;      // tokens per CTA: 32 KB of K codes and 32 KB of V codes
@@ -129,334 +125,371 @@ constexpr int kPStride = kChunk + 8;        // FP16 elements per row of P (rows 
 
 __device__ int g_kv4_error;      // non-zero after a bounded wait of this file's kernels ran out
 
-// ------------------------------------------------- attention, one chunk --
-// CTA (sequence b, KV head g, chunk s) over tokens [s*kChunk, min(L, ...)):
-// the chunk's K and V codes are contiguous in the cache and arrive by bulk
-// copies of 128 tokens, each on its own barrier, so the products start as
-// soon as the first 8 KB has landed.  Both products run on the tensor cores
-// (mma.sync m16n8k16, FP16 operands, FP32 sums), eight columns per MMA:
-// up to four query heads, each as a high and a low FP16 part, so that the
-// operands carry FP32-level precision (hi + lo) while the codes are exact
-// in FP16.
-//   scores:  S[token][col] = sum_c K[token][c] * q'[col][c]   (A = codes, rows = tokens)
-//   values:  O^T[c][col]   = sum_t V[t][c] * p[col][t]        (A = codes^T, rows = channels)
-// Each head's q' is scaled by a power of two that brings its largest
+// ------------------------------------------------------------ attention --
+// A persistent CTA per resident slot.  The work items are the (sequence, KV
+// head, chunk) triples in that order; CTA k of P takes items [k*I/P,
+// (k+1)*I/P), so consecutive items mostly share a KV head.  Per item, over
+// tokens [s*kChunk, min(L, ...)) of the chunk:
+//   - the K and V codes are contiguous in the cache and arrive by bulk
+//     copies of 128 tokens, each on its own barrier; the next item's K codes
+//     are requested as soon as this item's scores are computed, its V codes
+//     once this item's weighted sums are out of shared memory;
+//   - both products run on the tensor cores (mma.sync m16n8k16, FP16
+//     operands, FP32 sums), eight columns per MMA: up to four query heads,
+//     each as a high and a low FP16 part, so that the operands carry
+//     FP32-level precision (hi + lo) while the codes are exact in FP16:
+//       scores:  S[token][col] = sum_c K[token][c] * q'[col][c]  (A = codes, rows = tokens)
+//       values:  O^T[c][col]   = sum_t V[t][c] * p[col][t]       (A = codes^T, rows = channels)
+//   - the softmax numerators of the chunk, split the same way, go through
+//     shared memory (the score fragment holds tokens by row, the value
+//     product needs them by column);
+//   - each warp takes 64 tokens in both passes; the warps' weighted sums are
+//     added in shared memory (over the V codes, read by then), and the
+//     chunk's (max, sum, weighted sums) per query head go to the workspace
+//     for the combine.
+// The folded query q' of a KV head is built once per change of head: warp h
+// folds query head h, scales it by the power of two that brings its largest
 // element into [2^13, 2^14) (no FP16 overflow, full precision in the
-// parts), undone exactly on the score.  The softmax numerators of the
-// chunk, split the same way, go through shared memory (the score fragment
-// holds tokens by row, the value product needs them by column).  Each
-// warp takes 64 tokens in both passes; the warps' weighted sums are added in
-// shared memory (over the K codes, dead by then), and the chunk's (max, sum,
-// weighted sums) per query head go to the workspace for the combine.
+// parts; the score undoes it exactly) and writes the high and low parts
+// into shared memory in the order of the MMA's B fragments.
 template <int G>
-__global__ void __launch_bounds__(kThreads, G > 4 ? 1 : 2) kv4_attn_chunk_kernel(
+__global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
     const uint16_t *__restrict__ q, const uint8_t *__restrict__ K4, const uint8_t *__restrict__ V4,
-    const uint16_t *__restrict__ lam, const uint16_t *__restrict__ s_k, int Hkv, int L,
+    const uint16_t *__restrict__ lam, const uint16_t *__restrict__ s_k, int Hkv, int L, int S, int items,
     float *__restrict__ part)
 {
     constexpr int HT = (G + 3) / 4;             // column tiles of 8 (4 heads x hi/lo)
     extern __shared__ __align__(128) uint8_t dyn[];
     uint8_t *ks = dyn;                                   // [kChunk][64] K codes
     uint8_t *vs = dyn + kChunk * kRowBytes;              // [kChunk][64] V codes
-    __half *ps = reinterpret_cast<__half *>(dyn + 2 * kChunk * kRowBytes);  // [HT][8][kPStride]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ps + HT * 8 * kPStride);  // K parts, V parts
-    float *osum = reinterpret_cast<float *>(ks);         // [kWarps][G][kD], over the K codes
-    __shared__ float red[kWarps][G];
-    __shared__ float gmax[G], gsum[G];
+    __half *ps = reinterpret_cast<__half *>(dyn + 2 * kChunk * kRowBytes);   // [HT][8][kPStride]
+    uint2 *qfrag = reinterpret_cast<uint2 *>(ps + HT * 8 * kPStride);        // [HT][8 steps][32 lanes]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(qfrag + HT * 8 * 32);      // K parts, V parts
+    float *osum = reinterpret_cast<float *>(vs);         // [kWarps][G][kD], over the V codes once read
+    __shared__ float red[kWarps][G], red2[kWarps][G];
+    __shared__ float gmax[G], escl[4 * HT];
     __shared__ int abort_flag;
-    const int bh = blockIdx.x;                   // b * Hkv + kv head
-    const int b = bh / Hkv, hk = bh % Hkv;
-    const int S = gridDim.y, s = blockIdx.y;
-    const int l0 = s * kChunk, n = min(L - l0, kChunk);
+    const int P = gridDim.x;
+    const int it_begin = (int)((long long)blockIdx.x * items / P);
+    const int it_end = (int)((long long)(blockIdx.x + 1) * items / P);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
-    const size_t head = (size_t)bh;
     const uint32_t bar0 = smem_addr(bars);
     auto kbar = [&](int j) { return bar0 + 8u * j; };
     auto vbar = [&](int j) { return bar0 + 8u * (kNumSub + j); };
+    // (thread 0) one item's K or V codes, in parts of kSub tokens
+    auto issue = [&](int it, bool val) {
+        const int bh_ = it / S, s_ = it % S;
+        const int l0_ = s_ * kChunk, n_ = min(L - l0_, kChunk);
+        const uint8_t *src = (val ? V4 : K4) + ((size_t)bh_ * L + l0_) * kRowBytes;
+        uint8_t *dst = val ? vs : ks;
+        for (int j = 0; j < kNumSub; ++j) {
+            const int rows = max(0, min(n_ - j * kSub, kSub));
+            const uint32_t bar = val ? vbar(j) : kbar(j);
+            if (rows > 0) {
+                mbar_arrive_expect_tx(bar, (uint32_t)rows * kRowBytes);
+                bulk_load(smem_addr(dst + j * kSub * kRowBytes), src + (size_t)j * kSub * kRowBytes,
+                          (uint32_t)rows * kRowBytes, bar);
+            } else {
+                mbar_arrive(bar);
+            }
+        }
+    };
+    int k_issued = 0, v_issued = 0;              // (thread 0) items whose copies went out
     if (threadIdx.x == 0) {
         for (int j = 0; j < 2 * kNumSub; ++j) mbar_init(bar0 + 8u * j, 1);
         abort_flag = 0;
         fence_mbar_init();
-        for (int pass = 0; pass < 2; ++pass) {
-            const uint8_t *src = (pass ? V4 : K4) + (head * L + l0) * kRowBytes;
-            uint8_t *dst = pass ? vs : ks;
-            for (int j = 0; j < kNumSub; ++j) {
-                const int rows = max(0, min(n - j * kSub, kSub));
-                const uint32_t bar = pass ? vbar(j) : kbar(j);
-                if (rows > 0) {
-                    mbar_arrive_expect_tx(bar, (uint32_t)rows * kRowBytes);
-                    bulk_load(smem_addr(dst + j * kSub * kRowBytes), src + (size_t)j * kSub * kRowBytes,
-                              (uint32_t)rows * kRowBytes, bar);
-                } else {
-                    mbar_arrive(bar);
-                }
-            }
-        }
-    }
-    // B fragments of the score product (while the copies are in flight):
-    // column g of tile t is query head 4t + g % 4, its high part for g < 4
-    // and its low part for g >= 4; lane c holds channels 32c .. 32c + 31.
-    // The K codes' word j of those channels holds channel 32c + 8j + i in
-    // nibble i; MMA step 2j + h pairs nibbles (2h, 2h + 4) at columns
-    // 2c, 2c + 1 and (2h + 1, 2h + 5) at 2c + 8, 2c + 9.
-    const float inv_sqrt_d = 0.08838834764831845f;   // 1 / sqrt(128)
-    uint32_t qb[HT][8][2];
-    float escale[HT][2];                         // 2^e of heads 4t + 2(c % 2) + {0, 1}
-    {
-        float fold[32];
-        {
-            const uint4 *lp = reinterpret_cast<const uint4 *>(lam + head * kD + 32 * c);
-            const uint4 *sp = reinterpret_cast<const uint4 *>(s_k + head * kD + 32 * c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const uint4 lw = __ldg(lp + v), sw = __ldg(sp + v);
-                const uint32_t la[4] = {lw.x, lw.y, lw.z, lw.w}, sa[4] = {sw.x, sw.y, sw.z, sw.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float lf = half_bits_to_float((uint16_t)(la[e / 2] >> (16 * (e % 2))));
-                    const float sf = half_bits_to_float((uint16_t)(sa[e / 2] >> (16 * (e % 2))));
-                    fold[8 * v + e] = __fmul_rn(__fmul_rn(lf, sf), inv_sqrt_d);
-                }
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < HT; ++t) {
-            const int hq = 4 * t + (g & 3);
-            float f[32];
-            float m = 0.0f;
-            if (hq < G) {
-                const uint4 *qp = reinterpret_cast<const uint4 *>(q + ((size_t)bh * G + hq) * kD + 32 * c);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const uint4 qw = __ldg(qp + v);
-                    const uint32_t qa[4] = {qw.x, qw.y, qw.z, qw.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        f[8 * v + e] = __fmul_rn(half_bits_to_float((uint16_t)(qa[e / 2] >> (16 * (e % 2)))),
-                                                 fold[8 * v + e]);
-                        m = fmaxf(m, fabsf(f[8 * v + e]));
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) f[i] = 0.0f;
-            }
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            // m in [2^E, 2^(E+1)) with E its biased exponent field - 127 (a
-            // zero or subnormal m takes E = -126); e = E - 13 brings the
-            // largest |q'| * 2^-e into [2^13, 2^14), and both powers of two
-            // are exact FP32 numbers for e in [-126, 114]
-            const int E = max((int)((__float_as_uint(m) >> 23) & 0xFFu), 1) - 127;
-            const int e = max(E - 13, -126);
-            const float down = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e
-            __half part_v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float x = f[i] * down;
-                const __half hi = __float2half_rn(x);
-                part_v[i] = g < 4 ? hi : __float2half_rn(x - __half2float(hi));
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    qb[t][2 * j + h][0] = pack_h2(part_v[8 * j + 2 * h], part_v[8 * j + 2 * h + 4]);
-                    qb[t][2 * j + h][1] = pack_h2(part_v[8 * j + 2 * h + 1], part_v[8 * j + 2 * h + 5]);
-                }
-            // the exponents of the two heads whose scores this lane ends up with
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                escale[t][i] = __uint_as_float((uint32_t)(127 + __shfl_sync(0xffffffffu, e, 4 * (2 * (c & 1) + i))) << 23);
+        if (it_begin < it_end) {
+            issue(it_begin, false);
+            issue(it_begin, true);
+            k_issued = v_issued = 1;
         }
     }
     __syncthreads();
     const uint64_t budget = 2000000000ull;
+    const float inv_sqrt_d = 0.08838834764831845f;   // 1 / sqrt(128)
     const int T0 = warp * kWarpTok;
-    bool ok = wait_bounded(kbar(T0 / kSub), 0u, &abort_flag, budget);
-    // pass 1: scores of the warp's 64 tokens (rows g and g + 8 of each
-    // 16-token step), all columns
-    float sc[4][HT][4];
+    int cur_bh = -1;
+    for (int it = it_begin; it < it_end; ++it) {
+        const uint32_t ph = (uint32_t)((it - it_begin) & 1);
+        const int bh = it / S, s = it % S;
+        const int l0 = s * kChunk, n = min(L - l0, kChunk);
+        if (bh != cur_bh) {                      // the same for every thread of the CTA
+            cur_bh = bh;
+            if (warp < 4 * HT) {
+                // query head `warp` (zeros past G): lane l folds channels 4l .. 4l + 3
+                float f[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                float m = 0.0f;
+                if (warp < G) {
+                    const uint2 lw = __ldg(reinterpret_cast<const uint2 *>(lam + (size_t)bh * kD) + lane);
+                    const uint2 sw = __ldg(reinterpret_cast<const uint2 *>(s_k + (size_t)bh * kD) + lane);
+                    const uint2 qw = __ldg(reinterpret_cast<const uint2 *>(q + ((size_t)bh * G + warp) * kD) + lane);
+                    const uint32_t la[2] = {lw.x, lw.y}, sa[2] = {sw.x, sw.y}, qa[2] = {qw.x, qw.y};
 #pragma unroll
-    for (int st = 0; st < 4; ++st) {
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const int sh = 16 * (e4 & 1);
+                        const float fold = __fmul_rn(__fmul_rn(half_bits_to_float((uint16_t)(la[e4 >> 1] >> sh)),
+                                                               half_bits_to_float((uint16_t)(sa[e4 >> 1] >> sh))),
+                                                     inv_sqrt_d);
+                        f[e4] = __fmul_rn(half_bits_to_float((uint16_t)(qa[e4 >> 1] >> sh)), fold);
+                        m = fmaxf(m, fabsf(f[e4]));
+                    }
+                }
+                m = warp_max(m);
+                // m in [2^E, 2^(E+1)) with E its biased exponent field - 127 (a
+                // zero or subnormal m takes E = -126); e = E - 13 brings the
+                // largest |q'| * 2^-e into [2^13, 2^14), and both powers of
+                // two are exact FP32 numbers for e in [-126, 114]
+                const int E = max((int)((__float_as_uint(m) >> 23) & 0xFFu), 1) - 127;
+                const int e = max(E - 13, -126);
+                const float down = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e
+                // channel 32c + 8j + i goes to step 2j + h, register r, half hf
+                // of lane (column, c), where i = 2h + r + 4hf; the column is
+                // the head's slot (high part) or slot + 4 (low part)
+                const int t = warp >> 2, slot = warp & 3;
+                const int cc = lane >> 3, j = (lane & 7) >> 1, ib = 4 * (lane & 1);
 #pragma unroll
-        for (int t = 0; t < HT; ++t)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) sc[st][t][r] = 0.0f;
-        if (!ok) continue;
-        const int r0 = T0 + 16 * st + g;
-        const uint4 k0 = *reinterpret_cast<const uint4 *>(ks + r0 * kRowBytes + 16 * c);
-        const uint4 k1 = *reinterpret_cast<const uint4 *>(ks + (r0 + 8) * kRowBytes + 16 * c);
-        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t a[4] = {codes_h2(w0[j] >> (8 * h)), codes_h2(w1[j] >> (8 * h)),
-                                       codes_h2(w0[j] >> (8 * h + 4)), codes_h2(w1[j] >> (8 * h + 4))};
-#pragma unroll
-                for (int t = 0; t < HT; ++t) mma_f16_16816(sc[st][t], a, qb[t][2 * j + h][0], qb[t][2 * j + h][1]);
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const int i = ib + e4;
+                    const int hf = i >> 2, h = (i & 3) >> 1, r = i & 1;
+                    const float x = f[e4] * down;
+                    const __half hi = __float2half_rn(x);
+                    const __half lo = __float2half_rn(x - __half2float(hi));
+                    uint16_t *fr = reinterpret_cast<uint16_t *>(qfrag + (t * 8 + 2 * j + h) * 32);
+                    fr[(slot * 4 + cc) * 4 + 2 * r + hf] = __half_as_ushort(hi);
+                    fr[((slot + 4) * 4 + cc) * 4 + 2 * r + hf] = __half_as_ushort(lo);
+                }
+                if (lane == 0) escl[warp] = __uint_as_float((uint32_t)(127 + e) << 23);   // 2^e
             }
-    }
-    // high + low columns (lanes c and c ^ 2), power of two undone; lane c
-    // then holds heads 4t + 2(c % 2) + i for rows g and g + 8 of each step
-    float lmax[HT][2];
-#pragma unroll
-    for (int t = 0; t < HT; ++t) lmax[t][0] = lmax[t][1] = -INFINITY;
-#pragma unroll
-    for (int st = 0; st < 4; ++st)
-#pragma unroll
-        for (int t = 0; t < HT; ++t)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int i = r & 1;
-                const int tok = T0 + 16 * st + g + 8 * (r >> 1);
-                const int hq = 4 * t + 2 * (c & 1) + i;
-                const float v = (sc[st][t][r] + __shfl_xor_sync(0xffffffffu, sc[st][t][r], 2)) * escale[t][i];
-                sc[st][t][r] = (tok < n && hq < G) ? v : -INFINITY;
-                lmax[t][i] = fmaxf(lmax[t][i], sc[st][t][r]);
-            }
-    // the chunk's softmax numerators: exp(score - chunk max), and their sum
-#pragma unroll
-    for (int t = 0; t < HT; ++t)
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            float m = lmax[t][i];
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-            const int hq = 4 * t + 2 * (c & 1) + i;
-            if (lane < 2 && hq < G) red[warp][hq] = m;
+            __syncthreads();
         }
-    __syncthreads();
-    if (threadIdx.x < G) {
-        float m = red[0][threadIdx.x];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w][threadIdx.x]);
-        gmax[threadIdx.x] = m;
-    }
-    __syncthreads();
-    float lsum[HT][2];
-#pragma unroll
-    for (int t = 0; t < HT; ++t) lsum[t][0] = lsum[t][1] = 0.0f;
-#pragma unroll
-    for (int st = 0; st < 4; ++st)
-#pragma unroll
-        for (int t = 0; t < HT; ++t)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int i = r & 1;
-                const int tok = T0 + 16 * st + g + 8 * (r >> 1);
-                const int hq = 4 * t + 2 * (c & 1) + i;
-                const float p = sc[st][t][r] == -INFINITY ? 0.0f : expf(sc[st][t][r] - gmax[hq < G ? hq : 0]);
-                lsum[t][i] += p;
-                // column (c / 2) * 4 + 2(c % 2) + i: the high part from lanes c < 2,
-                // the low part from lanes c >= 2
-                const __half hi = __float2half_rn(p);
-                ps[(t * 8 + (c >> 1) * 4 + 2 * (c & 1) + i) * kPStride + tok] =
-                    c < 2 ? hi : __float2half_rn(p - __half2float(hi));
-            }
-    __syncthreads();   // red is reused below; P complete; the K codes are dead
-#pragma unroll
-    for (int t = 0; t < HT; ++t)
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            float v = lsum[t][i];
-            v += __shfl_xor_sync(0xffffffffu, v, 4);
-            v += __shfl_xor_sync(0xffffffffu, v, 8);
-            v += __shfl_xor_sync(0xffffffffu, v, 16);
-            const int hq = 4 * t + 2 * (c & 1) + i;
-            if (lane < 2 && hq < G) red[warp][hq] = v;
-        }
-    // pass 2: O^T[channel][column] over the warp's 64 tokens; m-tile mt
-    // row g is channel 16g + 2mt (a low nibble), row g + 8 channel
-    // 16g + 2mt + 1 (the high nibble of the same byte)
-    float o[HT][8][4];
-#pragma unroll
-    for (int t = 0; t < HT; ++t)
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) o[t][mt][r] = 0.0f;
-    ok = ok && wait_bounded(vbar(T0 / kSub), 0u, &abort_flag, budget);
-#pragma unroll
-    for (int st = 0; st < 4; ++st) {
-        if (!ok) break;
-        const int tA = T0 + 16 * st + 2 * c;    // tokens tA, tA + 1, tA + 8, tA + 9
-        const int odd = c & 1;
-        // each load instruction of the warp touches rows of both parities
-        const uint2 x0 = *reinterpret_cast<const uint2 *>(vs + (tA + odd) * kRowBytes + 8 * g);
-        const uint2 x1 = *reinterpret_cast<const uint2 *>(vs + (tA + 1 - odd) * kRowBytes + 8 * g);
-        const uint2 y0 = *reinterpret_cast<const uint2 *>(vs + (tA + 8 + odd) * kRowBytes + 8 * g);
-        const uint2 y1 = *reinterpret_cast<const uint2 *>(vs + (tA + 9 - odd) * kRowBytes + 8 * g);
-        const uint2 vA = odd ? x1 : x0, vB = odd ? x0 : x1, vC = odd ? y1 : y0, vD = odd ? y0 : y1;
-        uint32_t pb[HT][2];
+        // this lane's B fragments (reloaded per item: registers are what
+        // bounds the CTAs per SM)
+        uint32_t qb[HT][8][2];
+        float escale[HT][2];
 #pragma unroll
         for (int t = 0; t < HT; ++t) {
-            pb[t][0] = *reinterpret_cast<const uint32_t *>(ps + (t * 8 + g) * kPStride + tA);
-            pb[t][1] = *reinterpret_cast<const uint32_t *>(ps + (t * 8 + g) * kPStride + tA + 8);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint2 v = qfrag[(t * 8 + kk) * 32 + lane];
+                qb[t][kk][0] = v.x;
+                qb[t][kk][1] = v.y;
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) escale[t][i] = escl[4 * t + 2 * (c & 1) + i];
         }
+        bool ok = wait_bounded(kbar(T0 / kSub), ph, &abort_flag, budget);
+        // pass 1: scores of the warp's 64 tokens (rows g and g + 8 of each
+        // 16-token step), all columns; the K codes' word j of lane c's 32
+        // channels holds channel 32c + 8j + i in nibble i, and MMA step 2j + h
+        // pairs nibbles (2h, 2h + 4) at columns 2c, 2c + 1 and (2h + 1,
+        // 2h + 5) at 2c + 8, 2c + 9 (the order of q' in qb)
+        float sc[4][HT][4];
 #pragma unroll
-        for (int wi = 0; wi < 2; ++wi) {
-            const uint32_t wa = wi ? vA.y : vA.x, wb = wi ? vB.y : vB.x;
-            const uint32_t wc = wi ? vC.y : vC.x, wd = wi ? vD.y : vD.x;
+        for (int st = 0; st < 4; ++st) {
 #pragma unroll
-            for (int bp = 0; bp < 2; ++bp) {
-                // bytes 2bp, 2bp + 1 of the first token over those of the second
-                const uint32_t sel = (2 * bp) | ((2 * bp + 1) << 4) | ((2 * bp + 4) << 8) | ((2 * bp + 5) << 12);
-                const uint32_t xab = __byte_perm(wa, wb, sel), xcd = __byte_perm(wc, wd, sel);
-                const int mt = 4 * wi + 2 * bp;
-                const uint32_t a0[4] = {codes_h2(xab), codes_h2(xab >> 4), codes_h2(xcd), codes_h2(xcd >> 4)};
-                const uint32_t a1[4] = {codes_h2(xab >> 8), codes_h2(xab >> 12), codes_h2(xcd >> 8),
-                                        codes_h2(xcd >> 12)};
+            for (int t = 0; t < HT; ++t)
 #pragma unroll
-                for (int t = 0; t < HT; ++t) {
-                    mma_f16_16816(o[t][mt], a0, pb[t][0], pb[t][1]);
-                    mma_f16_16816(o[t][mt + 1], a1, pb[t][0], pb[t][1]);
+                for (int r = 0; r < 4; ++r) sc[st][t][r] = 0.0f;
+            if (!ok) continue;
+            const int r0 = T0 + 16 * st + g;
+            const uint4 k0 = *reinterpret_cast<const uint4 *>(ks + r0 * kRowBytes + 16 * c);
+            const uint4 k1 = *reinterpret_cast<const uint4 *>(ks + (r0 + 8) * kRowBytes + 16 * c);
+            const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t a[4] = {codes_h2(w0[j] >> (8 * h)), codes_h2(w1[j] >> (8 * h)),
+                                           codes_h2(w0[j] >> (8 * h + 4)), codes_h2(w1[j] >> (8 * h + 4))};
+#pragma unroll
+                    for (int t = 0; t < HT; ++t)
+                        mma_f16_16816(sc[st][t], a, qb[t][2 * j + h][0], qb[t][2 * j + h][1]);
+                }
+        }
+        // high + low columns (lanes c and c ^ 2), power of two undone; lane c
+        // then holds heads 4t + 2(c % 2) + i for rows g and g + 8 of each step
+        float lmax[HT][2];
+#pragma unroll
+        for (int t = 0; t < HT; ++t) lmax[t][0] = lmax[t][1] = -INFINITY;
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+#pragma unroll
+            for (int t = 0; t < HT; ++t)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int i = r & 1;
+                    const int tok = T0 + 16 * st + g + 8 * (r >> 1);
+                    const int hq = 4 * t + 2 * (c & 1) + i;
+                    const float v = (sc[st][t][r] + __shfl_xor_sync(0xffffffffu, sc[st][t][r], 2)) * escale[t][i];
+                    sc[st][t][r] = (tok < n && hq < G) ? v : -INFINITY;
+                    lmax[t][i] = fmaxf(lmax[t][i], sc[st][t][r]);
+                }
+#pragma unroll
+        for (int t = 0; t < HT; ++t)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float m = lmax[t][i];
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                const int hq = 4 * t + 2 * (c & 1) + i;
+                if (lane < 2 && hq < G) red[warp][hq] = m;
+            }
+        // the K codes were read through the generic proxy; the next item's
+        // bulk copies write them through the async proxy
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (threadIdx.x == 0 && it + 1 < it_end && !abort_flag) {
+            issue(it + 1, false);
+            ++k_issued;
+        }
+        if (threadIdx.x < G) {
+            float m = red[0][threadIdx.x];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w][threadIdx.x]);
+            gmax[threadIdx.x] = m;
+        }
+        __syncthreads();
+        // the chunk's softmax numerators exp(score - chunk max), their sum,
+        // and their high and low FP16 parts at column (c / 2) * 4 + 2(c % 2) + i
+        float lsum[HT][2];
+#pragma unroll
+        for (int t = 0; t < HT; ++t) lsum[t][0] = lsum[t][1] = 0.0f;
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+#pragma unroll
+            for (int t = 0; t < HT; ++t)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int i = r & 1;
+                    const int tok = T0 + 16 * st + g + 8 * (r >> 1);
+                    const int hq = 4 * t + 2 * (c & 1) + i;
+                    const float p = sc[st][t][r] == -INFINITY ? 0.0f : expf(sc[st][t][r] - gmax[hq < G ? hq : 0]);
+                    lsum[t][i] += p;
+                    const __half hi = __float2half_rn(p);
+                    ps[(t * 8 + (c >> 1) * 4 + 2 * (c & 1) + i) * kPStride + tok] =
+                        c < 2 ? hi : __float2half_rn(p - __half2float(hi));
+                }
+#pragma unroll
+        for (int t = 0; t < HT; ++t)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float v = lsum[t][i];
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                const int hq = 4 * t + 2 * (c & 1) + i;
+                if (lane < 2 && hq < G) red2[warp][hq] = v;
+            }
+        __syncthreads();   // P complete
+        // pass 2: O^T[channel][column] over the warp's 64 tokens; m-tile mt
+        // row g is channel 16g + 2mt (a low nibble), row g + 8 channel
+        // 16g + 2mt + 1 (the high nibble of the same byte)
+        float o[HT][8][4];
+#pragma unroll
+        for (int t = 0; t < HT; ++t)
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) o[t][mt][r] = 0.0f;
+        ok = ok && wait_bounded(vbar(T0 / kSub), ph, &abort_flag, budget);
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+            if (!ok) break;
+            const int tA = T0 + 16 * st + 2 * c;    // tokens tA, tA + 1, tA + 8, tA + 9
+            const int odd = c & 1;
+            // each load instruction of the warp touches rows of both parities
+            const uint2 x0 = *reinterpret_cast<const uint2 *>(vs + (tA + odd) * kRowBytes + 8 * g);
+            const uint2 x1 = *reinterpret_cast<const uint2 *>(vs + (tA + 1 - odd) * kRowBytes + 8 * g);
+            const uint2 y0 = *reinterpret_cast<const uint2 *>(vs + (tA + 8 + odd) * kRowBytes + 8 * g);
+            const uint2 y1 = *reinterpret_cast<const uint2 *>(vs + (tA + 9 - odd) * kRowBytes + 8 * g);
+            const uint2 vA = odd ? x1 : x0, vB = odd ? x0 : x1, vC = odd ? y1 : y0, vD = odd ? y0 : y1;
+            uint32_t pb[HT][2];
+#pragma unroll
+            for (int t = 0; t < HT; ++t) {
+                pb[t][0] = *reinterpret_cast<const uint32_t *>(ps + (t * 8 + g) * kPStride + tA);
+                pb[t][1] = *reinterpret_cast<const uint32_t *>(ps + (t * 8 + g) * kPStride + tA + 8);
+            }
+#pragma unroll
+            for (int wi = 0; wi < 2; ++wi) {
+                const uint32_t wa = wi ? vA.y : vA.x, wb = wi ? vB.y : vB.x;
+                const uint32_t wc = wi ? vC.y : vC.x, wd = wi ? vD.y : vD.x;
+#pragma unroll
+                for (int bp = 0; bp < 2; ++bp) {
+                    // bytes 2bp, 2bp + 1 of the first token over those of the second
+                    const uint32_t sel = (2 * bp) | ((2 * bp + 1) << 4) | ((2 * bp + 4) << 8) | ((2 * bp + 5) << 12);
+                    const uint32_t xab = __byte_perm(wa, wb, sel), xcd = __byte_perm(wc, wd, sel);
+                    const int mt = 4 * wi + 2 * bp;
+                    const uint32_t a0[4] = {codes_h2(xab), codes_h2(xab >> 4), codes_h2(xcd), codes_h2(xcd >> 4)};
+                    const uint32_t a1[4] = {codes_h2(xab >> 8), codes_h2(xab >> 12), codes_h2(xcd >> 8),
+                                            codes_h2(xcd >> 12)};
+#pragma unroll
+                    for (int t = 0; t < HT; ++t) {
+                        mma_f16_16816(o[t][mt], a0, pb[t][0], pb[t][1]);
+                        mma_f16_16816(o[t][mt + 1], a1, pb[t][0], pb[t][1]);
+                    }
                 }
             }
         }
-    }
-    // high + low columns, then the warps' sums in shared memory
 #pragma unroll
-    for (int t = 0; t < HT; ++t)
+        for (int t = 0; t < HT; ++t)
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
+            for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float v = o[t][mt][r] + __shfl_xor_sync(0xffffffffu, o[t][mt][r], 2);
-                const int hq = 4 * t + 2 * c + (r & 1);
-                if (c < 2 && hq < G) osum[(warp * G + hq) * kD + 16 * g + 2 * mt + (r >> 1)] = v;
-            }
-    __syncthreads();
-    if (threadIdx.x < G) {
-        float t = 0.0f;
+                for (int r = 0; r < 4; ++r) o[t][mt][r] += __shfl_xor_sync(0xffffffffu, o[t][mt][r], 2);
+        __syncthreads();   // every warp is done with the V codes
+        // high + low columns, then the warps' sums in shared memory
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) t += red[w][threadIdx.x];
-        gsum[threadIdx.x] = t;
-    }
-    // partial record per query head: [max, sum, kD weighted sums]
-    float *rec = part + (((size_t)bh * S + s) * G) * (kD + 2);
-    for (int e = threadIdx.x; e < G * kD; e += kThreads) {
-        const int gi = e / kD, ch = e % kD;
-        float t = 0.0f;
+        for (int t = 0; t < HT; ++t)
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) t += osum[(w * G + gi) * kD + ch];
-        rec[gi * (kD + 2) + 2 + ch] = t;
-    }
-    __syncthreads();
-    if (threadIdx.x < G) {
-        rec[threadIdx.x * (kD + 2)] = gmax[threadIdx.x];
-        rec[threadIdx.x * (kD + 2) + 1] = gsum[threadIdx.x];
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int hq = 4 * t + 2 * c + (r & 1);
+                    if (c < 2 && hq < G) osum[(warp * G + hq) * kD + 16 * g + 2 * mt + (r >> 1)] = o[t][mt][r];
+                }
+        __syncthreads();
+        // partial record per query head: [max, sum, kD weighted sums]
+        float *rec = part + (size_t)it * G * (kD + 2);
+        for (int e = threadIdx.x; e < G * kD; e += kThreads) {
+            const int gi = e / kD, ch = e % kD;
+            float t = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) t += osum[(w * G + gi) * kD + ch];
+            rec[gi * (kD + 2) + 2 + ch] = t;
+        }
+        if (threadIdx.x < G) {
+            float t = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) t += red2[w][threadIdx.x];
+            rec[threadIdx.x * (kD + 2)] = gmax[threadIdx.x];
+            rec[threadIdx.x * (kD + 2) + 1] = t;
+        }
+        // the V codes' bytes were used through the generic proxy; the next
+        // item's bulk copies write them through the async proxy
+        fence_proxy_async_smem();
+        if (__syncthreads_or(abort_flag != 0)) break;
+        if (threadIdx.x == 0 && it + 1 < it_end) {
+            issue(it + 1, true);
+            ++v_issued;
+        }
     }
     if (threadIdx.x == 0 && abort_flag) {
-        // a wait ran out: report it, and let every copy land before leaving
+        // a wait ran out: report it, and let every copy issued land before
+        // leaving (the last item issued on each barrier completes its phase
+        // last)
         atomicExch(&g_kv4_error, 1);
         const uint64_t end = global_timer_ns() + 200000000ull;
-        for (int j = 0; j < 2 * kNumSub; ++j)
-            while (!mbar_try_wait(bar0 + 8u * j, 0u) && global_timer_ns() < end) {
-            }
+        for (int j = 0; j < kNumSub; ++j) {
+            if (k_issued > 0)
+                while (!mbar_try_wait(kbar(j), (uint32_t)((k_issued - 1) & 1)) && global_timer_ns() < end) {
+                }
+            if (v_issued > 0)
+                while (!mbar_try_wait(vbar(j), (uint32_t)((v_issued - 1) & 1)) && global_timer_ns() < end) {
+                }
+        }
     }
 }
 
@@ -520,22 +553,43 @@ cudaError_t launch_kv4_cache(const uint16_t *K, const uint16_t *V, int B, int Hk
     return cudaGetLastError();
 }
 
+// SMs of the current device, looked up once per device.
+static int kv4_sm_count()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
 template <int G>
 static cudaError_t launch_attn_g(const uint16_t *q, const uint8_t *K4, const uint8_t *V4, const uint16_t *lam,
                                  const uint16_t *s_k, const uint16_t *s_v, int B, int Hkv, int L, uint16_t *out,
                                  float *part, cudaStream_t stream)
 {
+    constexpr int HT = (G + 3) / 4;
     const int S = (L + kChunk - 1) / kChunk;
-    const size_t smem = 2 * (size_t)kChunk * kRowBytes + (size_t)((G + 3) / 4) * 8 * kPStride * sizeof(__half) +
-                        2 * kNumSub * sizeof(uint64_t);
-    auto k1 = kv4_attn_chunk_kernel<G>;
+    const long long items = (long long)B * Hkv * S;
+    const size_t smem = 2 * (size_t)kChunk * kRowBytes + (size_t)HT * 8 * kPStride * sizeof(__half) +
+                        (size_t)HT * 8 * 32 * sizeof(uint2) + 2 * kNumSub * sizeof(uint64_t);
+    auto k1 = kv4_attn_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // all of the unified L1/shared storage as shared memory: three CTAs
     // (two for G = 8) per SM keep their copies in flight together
     e = cudaFuncSetAttribute(k1, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    k1<<<dim3((unsigned)(B * Hkv), (unsigned)S), kThreads, smem, stream>>>(q, K4, V4, lam, s_k, Hkv, L, part);
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k1, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    const long long slots = (long long)kv4_sm_count() * (per_sm > 0 ? per_sm : 1);
+    const int grid = (int)(items < slots ? items : slots);
+    k1<<<grid, kThreads, smem, stream>>>(q, K4, V4, lam, s_k, Hkv, L, S, (int)items, part);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     kv4_combine_kernel<G><<<(unsigned)(B * Hkv * G), kD, 0, stream>>>(part, s_v, Hkv, S, out);
