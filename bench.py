@@ -263,7 +263,7 @@ def run_kv4(dev, peaks, flush, reps=20):
     torch.cuda.synchronize()
     if q.qoq_device_error() != q.QOQ_OK:
         raise RuntimeError("device error in the KV4 attention leg")
-    return {"kernels": "kv4_attn_chunk_kernel + kv4_combine_kernel", "timing": "isolated, L2 flushed, median of %d" % reps,
+    return {"kernels": "kv4_attn_kernel + kv4_combine_kernel", "timing": "isolated, L2 flushed, median of %d" % reps,
             "points": out}
 
 
