@@ -89,16 +89,27 @@ __global__ void __launch_bounds__(kD) kv4_cache_kernel(const uint16_t *__restric
     }
 }
 
-// Two 4-bit codes as an FP16 pair: the nibbles in bits 0-3 and 16-19 of x
-// are placed in the mantissa of 1024 (exactly 1024 + n) and 1032 is
-// subtracted, giving the codes n - 8 exactly: one logic op and one FP16 pair
-// subtraction per two codes (an integer-to-float conversion is a
-// quarter-rate instruction).
+// Two 4-bit codes as an FP16 pair, without conversion instructions.  A
+// nibble pair in bits 0-3 and 16-19 of x goes into the mantissa of 1024
+// (exactly 1024 + n), and 1032 is subtracted: the codes n - 8, exact.  A
+// pair in bits 4-7 and 20-23 lands one hex digit higher (1024 + 16n), and
+// 1152 is subtracted: 16 (n - 8), exact, so two of every four nibble pairs
+// need no shift; the factor 16 is taken out of the other operand (the
+// query) or of the result (the weighted sums).  One logic op and one FP16
+// pair subtraction per two codes.
 __device__ __forceinline__ uint32_t codes_h2(uint32_t x)
 {
     const uint32_t h = (x & 0x000F000Fu) | 0x64006400u;
     uint32_t r;
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64086408u));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t codes16_h2(uint32_t x)
+{
+    const uint32_t h = (x & 0x00F000F0u) | 0x64006400u;
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64806480u));
     return r;
 }
 
@@ -253,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
                 for (int e4 = 0; e4 < 4; ++e4) {
                     const int i = ib + e4;
                     const int hf = i >> 2, h = (i & 3) >> 1, r = i & 1;
-                    const float x = f[e4] * down;
+                    // register 1 meets codes scaled by 16 (codes16_h2): 1/16 here
+                    const float x = f[e4] * down * (r ? 0.0625f : 1.0f);
                     const __half hi = __float2half_rn(x);
                     const __half lo = __float2half_rn(x - __half2float(hi));
                     uint16_t *fr = reinterpret_cast<uint16_t *>(qfrag + (t * 8 + 2 * j + h) * 32);
@@ -284,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
         // 16-token step), all columns; the K codes' word j of lane c's 32
         // channels holds channel 32c + 8j + i in nibble i, and MMA step 2j + h
         // pairs nibbles (2h, 2h + 4) at columns 2c, 2c + 1 and (2h + 1,
-        // 2h + 5) at 2c + 8, 2c + 9 (the order of q' in qb)
+        // 2h + 5) at 2c + 8, 2c + 9, the latter scaled by 16 (the order of
+        // q' in qb, whose second register carries the factor 1/16)
         float sc[4][HT][4];
 #pragma unroll
         for (int st = 0; st < 4; ++st) {
@@ -301,8 +314,8 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const uint32_t a[4] = {codes_h2(w0[j] >> (8 * h)), codes_h2(w1[j] >> (8 * h)),
-                                           codes_h2(w0[j] >> (8 * h + 4)), codes_h2(w1[j] >> (8 * h + 4))};
+                    const uint32_t x0 = w0[j] >> (8 * h), x1 = w1[j] >> (8 * h);
+                    const uint32_t a[4] = {codes_h2(x0), codes_h2(x1), codes16_h2(x0), codes16_h2(x1)};
 #pragma unroll
                     for (int t = 0; t < HT; ++t)
                         mma_f16_16816(sc[st][t], a, qb[t][2 * j + h][0], qb[t][2 * j + h][1]);
@@ -422,9 +435,10 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
                     const uint32_t sel = (2 * bp) | ((2 * bp + 1) << 4) | ((2 * bp + 4) << 8) | ((2 * bp + 5) << 12);
                     const uint32_t xab = __byte_perm(wa, wb, sel), xcd = __byte_perm(wc, wd, sel);
                     const int mt = 4 * wi + 2 * bp;
-                    const uint32_t a0[4] = {codes_h2(xab), codes_h2(xab >> 4), codes_h2(xcd), codes_h2(xcd >> 4)};
-                    const uint32_t a1[4] = {codes_h2(xab >> 8), codes_h2(xab >> 12), codes_h2(xcd >> 8),
-                                            codes_h2(xcd >> 12)};
+                    // rows g + 8 (the high nibbles) come out scaled by 16
+                    const uint32_t xab8 = xab >> 8, xcd8 = xcd >> 8;
+                    const uint32_t a0[4] = {codes_h2(xab), codes16_h2(xab), codes_h2(xcd), codes16_h2(xcd)};
+                    const uint32_t a1[4] = {codes_h2(xab8), codes16_h2(xab8), codes_h2(xcd8), codes16_h2(xcd8)};
 #pragma unroll
                     for (int t = 0; t < HT; ++t) {
                         mma_f16_16816(o[t][mt], a0, pb[t][0], pb[t][1]);
@@ -438,7 +452,10 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-                for (int r = 0; r < 4; ++r) o[t][mt][r] += __shfl_xor_sync(0xffffffffu, o[t][mt][r], 2);
+                for (int r = 0; r < 4; ++r) {
+                    o[t][mt][r] += __shfl_xor_sync(0xffffffffu, o[t][mt][r], 2);
+                    if (r >= 2) o[t][mt][r] *= 0.0625f;   // rows g + 8: codes scaled by 16
+                }
         __syncthreads();   // every warp is done with the V codes
         // high + low columns, then the warps' sums in shared memory
 #pragma unroll
