@@ -909,8 +909,11 @@ __global__ void __launch_bounds__(gemm_threads(BN, W8, HALF), HALF ? 2 : 1)
             bool ready = true;
             constexpr bool kPresum = (BN <= 64) && !HALF;  // (registers: 64 per thread in a half CTA)
             // accumulator columns per TMEM load (16 where the pre-summed
-            // partials of a 64-wide tile already hold 64 registers)
-            constexpr int kGrp = HALF ? 16 : BN < 64 ? BN : (kPresum ? 16 : (kEpi == 2 ? 32 : 64));
+            // partials of a 64-wide tile already hold 64 registers); 64 for
+            // the 256-token tiles, so that each epilogue warp has its last
+            // columns in registers (and the accumulator back with the MMA)
+            // after one group of four chunks instead of three groups of two
+            constexpr int kGrp = HALF ? 16 : BN < 64 ? BN : (kPresum ? 16 : 64);
             int32_t pre[kPresum ? BN : 1];
             if (finisher) {
                 // Every lane of every later contributor counts its own
