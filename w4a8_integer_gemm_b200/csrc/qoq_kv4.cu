@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
     uint64_t *bars = reinterpret_cast<uint64_t *>(qfrag + HT * 8 * 32);      // K parts, V parts
     float *osum = reinterpret_cast<float *>(vs);         // [kWarps][G][kD], over the V codes once read
     __shared__ float red[kWarps][G], red2[kWarps][G];
-    __shared__ float gmax[G], escl[4 * HT];
+    __shared__ float escl[4 * HT];
     __shared__ int abort_flag;
     const int P = gridDim.x;
     const int it_begin = (int)((long long)blockIdx.x * items / P);
@@ -221,6 +221,9 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
     const uint64_t budget = 2000000000ull;
     const float inv_sqrt_d = 0.08838834764831845f;   // 1 / sqrt(128)
     const int T0 = warp * kWarpTok;
+    // byte selectors of the value pass (see there): even lanes hold token
+    // tA in the first operand, odd lanes in the second
+    const uint32_t psel_even[2] = {0x5410u, 0x7632u}, psel_odd[2] = {0x1054u, 0x3276u};
     int cur_bh = -1;
     for (int it = it_begin; it < it_end; ++it) {
         const uint32_t ph = (uint32_t)((it - it_begin) & 1);
@@ -358,13 +361,21 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
             issue(it + 1, false);
             ++k_issued;
         }
-        if (threadIdx.x < G) {
-            float m = red[0][threadIdx.x];
+        // the chunk max of each head this lane holds (every lane reads the
+        // warps' maxima itself: no second barrier)
+        float cmax[HT][2];
 #pragma unroll
-            for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w][threadIdx.x]);
-            gmax[threadIdx.x] = m;
-        }
-        __syncthreads();
+        for (int t = 0; t < HT; ++t)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int hq = 4 * t + 2 * (c & 1) + i;
+                float m = -INFINITY;
+                if (hq < G) {
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w][hq]);
+                }
+                cmax[t][i] = m;
+            }
         // the chunk's softmax numerators exp(score - chunk max), their sum,
         // and their high and low FP16 parts at column (c / 2) * 4 + 2(c % 2) + i
         float lsum[HT][2];
@@ -379,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
                     const int i = r & 1;
                     const int tok = T0 + 16 * st + g + 8 * (r >> 1);
                     const int hq = 4 * t + 2 * (c & 1) + i;
-                    const float p = sc[st][t][r] == -INFINITY ? 0.0f : expf(sc[st][t][r] - gmax[hq < G ? hq : 0]);
+                    const float p = sc[st][t][r] == -INFINITY ? 0.0f : expf(sc[st][t][r] - cmax[t][i]);
                     lsum[t][i] += p;
                     const __half hi = __float2half_rn(p);
                     ps[(t * 8 + (c >> 1) * 4 + 2 * (c & 1) + i) * kPStride + tok] =
@@ -414,11 +425,12 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
             const int tA = T0 + 16 * st + 2 * c;    // tokens tA, tA + 1, tA + 8, tA + 9
             const int odd = c & 1;
             // each load instruction of the warp touches rows of both parities
+            // (odd lanes load token tA + 1 first; their byte selectors below
+            // take the second operand first, so no register is swapped)
             const uint2 x0 = *reinterpret_cast<const uint2 *>(vs + (tA + odd) * kRowBytes + 8 * g);
             const uint2 x1 = *reinterpret_cast<const uint2 *>(vs + (tA + 1 - odd) * kRowBytes + 8 * g);
             const uint2 y0 = *reinterpret_cast<const uint2 *>(vs + (tA + 8 + odd) * kRowBytes + 8 * g);
             const uint2 y1 = *reinterpret_cast<const uint2 *>(vs + (tA + 9 - odd) * kRowBytes + 8 * g);
-            const uint2 vA = odd ? x1 : x0, vB = odd ? x0 : x1, vC = odd ? y1 : y0, vD = odd ? y0 : y1;
             uint32_t pb[HT][2];
 #pragma unroll
             for (int t = 0; t < HT; ++t) {
@@ -427,12 +439,13 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
             }
 #pragma unroll
             for (int wi = 0; wi < 2; ++wi) {
-                const uint32_t wa = wi ? vA.y : vA.x, wb = wi ? vB.y : vB.x;
-                const uint32_t wc = wi ? vC.y : vC.x, wd = wi ? vD.y : vD.x;
+                const uint32_t wa = wi ? x0.y : x0.x, wb = wi ? x1.y : x1.x;
+                const uint32_t wc = wi ? y0.y : y0.x, wd = wi ? y1.y : y1.x;
 #pragma unroll
                 for (int bp = 0; bp < 2; ++bp) {
-                    // bytes 2bp, 2bp + 1 of the first token over those of the second
-                    const uint32_t sel = (2 * bp) | ((2 * bp + 1) << 4) | ((2 * bp + 4) << 8) | ((2 * bp + 5) << 12);
+                    // bytes 2bp, 2bp + 1 of token tA (resp. tA + 8) over those
+                    // of tA + 1 (tA + 9)
+                    const uint32_t sel = odd ? psel_odd[bp] : psel_even[bp];
                     const uint32_t xab = __byte_perm(wa, wb, sel), xcd = __byte_perm(wc, wd, sel);
                     const int mt = 4 * wi + 2 * bp;
                     // rows g + 8 (the high nibbles) come out scaled by 16
@@ -481,7 +494,10 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
             float t = 0.0f;
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) t += red2[w][threadIdx.x];
-            rec[threadIdx.x * (kD + 2)] = gmax[threadIdx.x];
+            float m = red[0][threadIdx.x];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w][threadIdx.x]);
+            rec[threadIdx.x * (kD + 2)] = m;
             rec[threadIdx.x * (kD + 2) + 1] = t;
         }
         // the V codes' bytes were used through the generic proxy; the next
