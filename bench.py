@@ -50,7 +50,7 @@ from w4a8_integer_gemm_b200 import roofline, workloads as wl  # noqa: E402
 
 FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20
-GEMM_SOURCES = ("qoq_gemm.cu", "qoq_layout.cuh", "qoq_ptx.cuh", "qoq_internal.h", "qoq_quant.cuh")
+GEMM_SOURCES = ("qoq_gemm.cu", "qoq_epilogue.cuh", "qoq_layout.cuh", "qoq_ptx.cuh", "qoq_internal.h", "qoq_quant.cuh")
 
 
 def code_only(text: str) -> str:

@@ -494,6 +494,20 @@ QOQ_API int qoq_set_gemm_cta_pairs(int enable);
  * identical either way. Returns QOQ_ERR_INVALID_ARG for other values. */
 QOQ_API int qoq_set_gemm_half_ctas(int enable);
 
+/* Selects the kernel for M <= 8 tokens (decode):
+ *   1 (default): a decode kernel without the GEMM's per-launch machinery:
+ *      the codes expand to INT8 in registers as in the GEMM, straight into
+ *      the fragments of warp-level INT8 MMAs (m16n8k32, INT32 sums, the
+ *      tokens as the 8-wide N dimension); each CTA owns 16 output channels
+ *      and all of K, so no tensor memory, barrier ring or split-tile handoff
+ *      is set up per launch;
+ *   0: the tensor-core GEMM with a 16-token tile.
+ * It does not apply to the SiLU-gated gate/up epilogue or to the one-launch
+ * layer call, which keep the GEMM. The choice applies to later GEMM calls
+ * from every thread. Results are identical either way. Returns
+ * QOQ_ERR_INVALID_ARG for other values. */
+QOQ_API int qoq_set_gemm_gemv(int enable);
+
 /* Selects the token-tile width rule for M > 64:
  *   1 (default): 256 tokens per tile (128 for M <= 128), narrowed to 128 and
  *      then 64 while the tiles are so few that stream-K would share each

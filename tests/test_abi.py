@@ -27,7 +27,7 @@ def declared():
 def test_exports_every_declared_symbol(L):
     import w4a8_integer_gemm_b200 as q
     names = declared()
-    assert len(names) == 25
+    assert len(names) == 26
     for n in names:
         assert hasattr(L, n), n
     assert names == set(q.SIGNATURES)
@@ -117,6 +117,7 @@ def test_invalid_arguments_rejected_on_host(L):
     assert L.qoq_set_gemm_cta_pairs(2) == INVALID
     assert L.qoq_set_gemm_narrow_tiles(-1) == INVALID
     assert L.qoq_set_gemm_half_ctas(3) == INVALID
+    assert L.qoq_set_gemm_gemv(2) == INVALID
     assert L.qoq_set_linear_in_kernel_quant(2) == INVALID
     assert L.qoq_selftest_wait_timeout(ctypes.c_ulonglong(10), None) == INVALID          # budget too short
     assert L.qoq_selftest_wait_timeout(ctypes.c_ulonglong(10 ** 12), None) == INVALID    # too long

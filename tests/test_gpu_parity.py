@@ -173,6 +173,7 @@ def test_gemm_bit_exact_half_ctas(M, K, N, G):
     X = wl.make_activations(M, K, wl.LLAMA, seed=410 + M)
     W = wl.make_weights(N, K, wl.LLAMA, seed=510 + N + K)
     q.qoq_set_gemm_half_ctas(True)
+    q.qoq_set_gemm_gemv(False)   # M <= 8 would otherwise take the decode kernel
     try:
         _, X8, s_x, Y, acc = run_layer(X, W, G, True)
         # several launches in a row on the stream: CTAs of consecutive GEMMs
@@ -186,6 +187,7 @@ def test_gemm_bit_exact_half_ctas(M, K, N, G):
         assert q.qoq_device_error() == q.QOQ_OK
     finally:
         q.qoq_set_gemm_half_ctas(False)
+        q.qoq_set_gemm_gemv(True)
     r = oracle.linear(X.numpy(), W.numpy(), G)
     assert np.array_equal(acc.cpu().numpy(), r["acc"])
     assert_half_within_1ulp(_u16(Y), r["Y"])

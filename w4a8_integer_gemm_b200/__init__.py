@@ -66,6 +66,7 @@ SIGNATURES = {
     "qoq_set_gemm_cta_pairs": (_I, [_I]),
     "qoq_set_gemm_narrow_tiles": (_I, [_I]),
     "qoq_set_gemm_half_ctas": (_I, [_I]),
+    "qoq_set_gemm_gemv": (_I, [_I]),
     "qoq_set_linear_in_kernel_quant": (_I, [_I]),
     "qoq_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "qoq_device_error": (_I, [_P]),
@@ -148,6 +149,11 @@ def qoq_set_gemm_narrow_tiles(enable: bool) -> None:
 
 def qoq_set_gemm_half_ctas(enable: bool) -> None:
     _check("qoq_set_gemm_half_ctas", lib().qoq_set_gemm_half_ctas(1 if enable else 0))
+
+
+def qoq_set_gemm_gemv(enable: bool) -> None:
+    """M <= 8 tokens: the decode kernel (warp-level INT8 MMAs; True, the default) or the tensor-core GEMM."""
+    _check("qoq_set_gemm_gemv", lib().qoq_set_gemm_gemv(1 if enable else 0))
 
 
 def qoq_set_linear_in_kernel_quant(enable: bool) -> None:

@@ -373,6 +373,13 @@ int qoq_set_gemm_half_ctas(int enable)
     return QOQ_OK;
 }
 
+int qoq_set_gemm_gemv(int enable)
+{
+    if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;
+    qoq::set_gemv(enable != 0);
+    return QOQ_OK;
+}
+
 int qoq_set_gemm_narrow_tiles(int enable)
 {
     if (enable != 0 && enable != 1) return QOQ_ERR_INVALID_ARG;

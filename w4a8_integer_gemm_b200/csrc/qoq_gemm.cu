@@ -84,6 +84,7 @@
 #include <mutex>
 
 #include "qoq_internal.h"
+#include "qoq_epilogue.cuh"
 #include "qoq_layout.cuh"
 #include "qoq_ptx.cuh"
 #include "qoq_quant.cuh"
@@ -264,12 +265,6 @@ __device__ __forceinline__ void red_release_gpu_add(int *p, int v)
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ uint16_t scale_to_half(int32_t acc, float sx, float sc)
-{
-    const float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sx), sc);
-    return __half_as_ushort(__float2half_rn(y));
-}
-
 // FP16 outputs (and optionally the INT32 accumulators; with kEpiI32 only
 // those) of the 16
 // consecutive tokens m0.. of chunk `cc` for this lane's channel n0 + lane.
@@ -287,29 +282,7 @@ __device__ __forceinline__ uint16_t scale_to_half(int32_t acc, float sx, float s
 //     named barrier; quarters 0-1 read the up values from the staging block
 //     two warps on and store fp16(silu(g) * u), silu in FP32 with IEEE
 //     division; a second barrier frees the staging blocks for the next chunk.
-__device__ __forceinline__ uint32_t add_half2(uint32_t y, uint32_t r)
-{
-    const float lo = __fadd_rn(__half2float(__ushort_as_half((unsigned short)(y & 0xFFFFu))),
-                               __half2float(__ushort_as_half((unsigned short)(r & 0xFFFFu))));
-    const float hi = __fadd_rn(__half2float(__ushort_as_half((unsigned short)(y >> 16))),
-                               __half2float(__ushort_as_half((unsigned short)(r >> 16))));
-    return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
-}
-
-__device__ __forceinline__ uint16_t silu_mul_half(uint16_t gb, uint16_t ub)
-{
-    const float g = __half2float(__ushort_as_half(gb));
-    const float u = __half2float(__ushort_as_half(ub));
-    const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
-    return __half_as_ushort(__float2half_rn(__fmul_rn(silu, u)));
-}
-
-__device__ __forceinline__ uint32_t silu_mul_half2(uint32_t g, uint32_t u)
-{
-    return (uint32_t)silu_mul_half((uint16_t)(g & 0xFFFFu), (uint16_t)(u & 0xFFFFu)) |
-           ((uint32_t)silu_mul_half((uint16_t)(g >> 16), (uint16_t)(u >> 16)) << 16);
-}
-
+// (The rounding of each step is in qoq_epilogue.cuh.)
 __device__ __forceinline__ void store_outputs(const GemmArgs &a, uint8_t *stg, int m0, int cc, int n0, int lane,
                                               float sc, float sx, const int32_t *acc, int quarter, int bar_id)
 {
@@ -1287,6 +1260,7 @@ cudaError_t dispatch_w8(int BN, int KST, const CUtensorMap &tmap, const CUtensor
 
 std::atomic<int> g_cta_pairs{1};
 std::atomic<int> g_half_ctas{0};
+std::atomic<int> g_gemv{1};
 std::atomic<int> g_narrow_tiles{1};
 
 // SMs of the current device, looked up once per device.
@@ -1327,6 +1301,11 @@ void set_narrow_tiles(bool enable)
 void set_half_ctas(bool enable)
 {
     g_half_ctas.store(enable ? 1 : 0);
+}
+
+void set_gemv(bool enable)
+{
+    g_gemv.store(enable ? 1 : 0);
 }
 
 // Token tile width.  Up to 128 tokens one tile covers M.  Beyond that,
@@ -1385,6 +1364,9 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
                         const uint16_t *X, int epi, const uint16_t *R, int ldx, const int8_t *W8)
 {
     *tmap_status = 0;
+    // a few tokens: the matrix-vector kernel on the CUDA cores
+    if (W8 == nullptr && g_gemv.load(std::memory_order_relaxed) && gemv_applies(M, epi, X != nullptr))
+        return launch_gemv(X8, ldx, s_x, Wp, s_c, s_g, zs, M, N, K, G, Y, acc_dbg, epi, R, stream);
     const int BN = gemm_block_n(M, N, K);
     // W8A8 yardstick: INT8 weights in shared-memory A slots, single CTAs
     const bool w8 = W8 != nullptr;

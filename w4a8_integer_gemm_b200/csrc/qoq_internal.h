@@ -54,6 +54,10 @@ void set_narrow_tiles(bool enable);
 // Whether token tiles up to 64 run in half-SM CTAs (two per SM, so that
 // consecutive GEMMs overlap).
 void set_half_ctas(bool enable);
+// Up to kGemvMaxM tokens: the decode kernel (warp-level MMAs, the default)
+// or the tensor-core GEMM.
+constexpr int kGemvMaxM = 8;
+void set_gemv(bool enable);
 
 // Word offsets, in the workspace's counter region, of the two counters of
 // the one-launch layer call (after the split-tile counters of up to kMaxCtas CTAs).
@@ -114,5 +118,14 @@ bool aligned16(const void *p);
 bool gemm_a_in_tmem();
 // QOQ_OK when the current device is compute capability 10.0 (cached per device).
 int check_device();
+
+// The layer for M <= kGemvMaxM tokens on the CUDA cores (same inputs,
+// outputs and rounding as launch_gemm; no workspace).  gemv_applies says
+// whether a call can take it (not the SiLU-gated pair, not the one-launch
+// layer call).
+bool gemv_applies(int M, int epi, bool one_launch);
+cudaError_t launch_gemv(const int8_t *X8, int ldx, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
+                        const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
+                        int32_t *acc_dbg, int epi, const uint16_t *R, cudaStream_t stream);
 
 }  // namespace qoq
