@@ -302,7 +302,9 @@ def regime_roofline(bound, shapes, ms, peaks, traffic):
               "unit": "TOPS", "frac": round(achieved / peaks["int8_tops"], 4), "traffic": None,
               "peak_source": peaks["source"] + " (2 x bf16 cuBLAS burst)",
               "frac_of_sustained_peak": round(achieved / peaks["int8_tops_sustained"], 4)}
-    rl.update({"kernel": "w4a8_gemm_kernel", "launches": n, "chain_us": round(ms * 1e3, 2),
+    small = [x.name for x in shapes if x.M <= 8]
+    kern = "w4a8_gemm_kernel" + (f" (w4a8_gemv_kernel for {', '.join(small)})" if small else "")
+    rl.update({"kernel": kern, "launches": n, "chain_us": round(ms * 1e3, 2),
                "us_per_launch": round(ms * 1e3 / n, 3), "shapes": [x.name for x in shapes],
                "algorithmic_bytes_per_launch": int(byt / n), "ops_per_launch": int(ops / n)})
     rep = [k for k in traffic if k in {x.name for x in shapes}]
