@@ -502,8 +502,10 @@ QOQ_API int qoq_set_gemm_half_ctas(int enable);
  *      and all of K, so no tensor memory, barrier ring or split-tile handoff
  *      is set up per launch;
  *   0: the tensor-core GEMM with a 16-token tile.
- * It does not apply to the SiLU-gated gate/up epilogue or to the one-launch
- * layer call, which keep the GEMM. The choice applies to later GEMM calls
+ * It does not apply to the SiLU-gated gate/up epilogue, to the one-launch
+ * layer call, or to N above 128 channels per SM (18944 on 148 SMs), where
+ * the GEMM's bulk-copy weight stream is faster; those keep the GEMM. For
+ * small N the decode kernel splits K over a cluster of 2 or 4 CTAs. The choice applies to later GEMM calls
  * from every thread. Results are identical either way. Returns
  * QOQ_ERR_INVALID_ARG for other values. */
 QOQ_API int qoq_set_gemm_gemv(int enable);

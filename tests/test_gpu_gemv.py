@@ -4,7 +4,8 @@ tensor-core GEMM, through the C ABI.
 Both kernels compute the same INT32 sums (exact in any order) and round the
 output through the same epilogue, so every case is bit-identical between
 them; the oracle pins both.  Cases span 1-8 tokens (and 9-16, which take
-the GEMM whatever the switch says), both table layouts
+the GEMM whatever the switch says), K split over clusters of 1, 2 and 4
+CTAs (by N), an N above the decode kernel's limit (the GEMM), both table layouts
 (128-wide groups, per channel), K from one block to 64 blocks (fewer blocks
 than the CTA's warps, and several per warp), N from one CTA of 32 channels
 up, back-to-back launches on one stream and in a CUDA graph.
@@ -36,7 +37,8 @@ def _u16(t):
 CASES = [(1, 128, 128, 128), (1, 512, 384, 512), (2, 1024, 256, 128), (3, 4096, 640, 128),
          (4, 2048, 1024, 2048), (5, 8192, 512, 128), (7, 1536, 128, 1536), (8, 4096, 2048, 128),
          (8, 8192, 256, 8192), (9, 1024, 384, 128), (12, 2048, 128, 2048), (16, 4096, 1024, 128),
-         (16, 8192, 512, 8192)]
+         (16, 8192, 512, 8192), (3, 2048, 4096, 128), (6, 14336, 4096, 128), (2, 4096, 8192, 128),
+         (4, 1024, 20480, 128)]
 
 
 @pytest.mark.parametrize("M,K,N,G", CASES)

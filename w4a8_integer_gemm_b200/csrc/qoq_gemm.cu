@@ -1365,7 +1365,7 @@ cudaError_t launch_gemm(const int8_t *X8, const uint16_t *s_x, const uint8_t *Wp
 {
     *tmap_status = 0;
     // a few tokens: the matrix-vector kernel on the CUDA cores
-    if (W8 == nullptr && g_gemv.load(std::memory_order_relaxed) && gemv_applies(M, epi, X != nullptr))
+    if (W8 == nullptr && g_gemv.load(std::memory_order_relaxed) && gemv_applies(M, N, epi, X != nullptr, sm_count()))
         return launch_gemv(X8, ldx, s_x, Wp, s_c, s_g, zs, M, N, K, G, Y, acc_dbg, epi, R, stream);
     const int BN = gemm_block_n(M, N, K);
     // W8A8 yardstick: INT8 weights in shared-memory A slots, single CTAs

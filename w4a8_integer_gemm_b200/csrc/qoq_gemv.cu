@@ -14,8 +14,10 @@
 // coalesced loads, and the next layer's CTAs fit beside this layer's on an
 // SM (programmatic dependent launch).
 //
-// CTA: 16 output channels (one MMA tile) and all of K; its 8 warps take the
-// 128-wide K blocks in turn (block b to warp b % 8).  The
+// CTA: 16 output channels (one MMA tile) and all of K, or for small N (too
+// few channel groups to give every SM three CTAs) a 1/2 or 1/4 share of the
+// K blocks, the shares' INT32 sums added through distributed shared memory
+// in a cluster; its 8 warps take the 128-wide K blocks in turn.  The
 // products are warp-level INT8 MMAs (m16n8k32, INT32 sums) with the tokens
 // as the 8-wide N dimension, so up to 8 tokens cost one MMA per 32 K per 16
 // channels, whatever M is.  The packed
@@ -95,17 +97,21 @@ __device__ __forceinline__ void load_block(const GemvArgs &a, int panel, int r0,
 }
 
 // NT: token tiles of 8 (M <= 8 NT; the layer calls use one); PG: 128-wide
-// groups (tables in the chunks), else per-channel tables.
-template <int NT, bool PG>
+// groups (tables in the chunks), else per-channel tables; S: CTAs (a
+// cluster) that split the K blocks of one channel group, their INT32 sums
+// added through distributed shared memory by the cluster's first CTA.
+template <int NT, bool PG, int S>
 __global__ void __launch_bounds__(kGvThreads, 4) w4a8_gemv_kernel(GemvArgs a)
 {
     __shared__ int32_t red[kGvWarps][16][8 * NT];   // [warp][channel][token]
+    __shared__ int32_t part[16][8 * NT];            // the CTA's sums
     // the next kernel in the stream may launch now; it waits for this grid
     // before it reads anything this kernel writes
     grid_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
-    const int n0 = blockIdx.x * 16;
+    const int q = S > 1 ? (int)cluster_ctarank() : 0;   // this CTA's share of the K blocks
+    const int n0 = (blockIdx.x / S) * 16;
     const int panel = n0 / kPanelRows, r0 = n0 % kPanelRows;
     const int nb = a.K / kBlockK;
     uint32_t sg[2] = {0, 0}, bias[2] = {0, 0};
@@ -122,13 +128,14 @@ __global__ void __launch_bounds__(kGvThreads, 4) w4a8_gemv_kernel(GemvArgs a)
     for (int u = 0; u < NT; ++u)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[u][i] = 0;
+    constexpr int kStep = kGvWarps * S;
     Block cur;
-    int b = warp;
+    int b = q * kGvWarps + warp;
     if (b < nb) load_block<PG>(a, panel, r0, g, c, b, cur);
     grid_dependency_wait();  // X8 and s_x come from the preceding kernel
-    for (; b < nb; b += kGvWarps) {
+    for (; b < nb; b += kStep) {
         Block nxt;
-        if (b + kGvWarps < nb) load_block<PG>(a, panel, r0, g, c, b + kGvWarps, nxt);
+        if (b + kStep < nb) load_block<PG>(a, panel, r0, g, c, b + kStep, nxt);
         uint32_t gs[2], bs[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(kGvThreads, 4) w4a8_gemv_kernel(GemvArgs a)
                 mma_s8_16832(acc[u], af, xlo[s], xhi[s]);
             }
         }
-        if (b + kGvWarps < nb) cur = nxt;
+        if (b + kStep < nb) cur = nxt;
     }
     // the warps' sums: lane (g, c) holds rows (channels) g and g + 8,
     // columns (tokens) 8u + 2c and 8u + 2c + 1
@@ -177,13 +184,22 @@ __global__ void __launch_bounds__(kGvThreads, 4) w4a8_gemv_kernel(GemvArgs a)
         red[warp][g + 8][8 * u + 2 * c + 1] = acc[u][3];
     }
     __syncthreads();
-    // outputs: thread i of the CTA takes channel i % 16 of tokens i / 16,
-    // i / 16 + 16, ...
     for (int e = threadIdx.x; e < 16 * a.M; e += kGvThreads) {
         const int m = e >> 4, ch = e & 15;
         int32_t s = 0;
 #pragma unroll
         for (int w = 0; w < kGvWarps; ++w) s += red[w][ch][m];
+        part[ch][m] = s;
+    }
+    if constexpr (S > 1) cluster_sync_all();   // every CTA's sums are in its shared memory
+    else __syncthreads();
+    // outputs (the cluster's first CTA): thread i takes channel i % 16 of
+    // tokens i / 16, i / 16 + 16, ...
+    for (int e = threadIdx.x; e < 16 * a.M && q == 0; e += kGvThreads) {
+        const int m = e >> 4, ch = e & 15;
+        int32_t s = part[ch][m];
+#pragma unroll
+        for (int r = 1; r < S; ++r) s += (int32_t)ld_shared_cluster_u32(mapa_shared(smem_addr(&part[ch][m]), r));
         const int n = n0 + ch;
         const size_t o = (size_t)m * a.N + n;
         if (a.acc_dbg) a.acc_dbg[o] = s;
@@ -193,32 +209,56 @@ __global__ void __launch_bounds__(kGvThreads, 4) w4a8_gemv_kernel(GemvArgs a)
             a.Y[o] = y;
         }
     }
+    // the other CTAs' shared memory stays until the first one has read it
+    if constexpr (S > 1) cluster_sync_all();
 }
 
-template <int NT>
-cudaError_t launch_nt(const GemvArgs &a, cudaStream_t stream)
+template <int NT, int S>
+cudaError_t launch_nts(const GemvArgs &a, cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(a.N / 16));
+    cfg.gridDim = dim3((unsigned)(a.N / 16 * S));
     cfg.blockDim = dim3(kGvThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = a.G == kBlockK ? cudaLaunchKernelEx(&cfg, w4a8_gemv_kernel<NT, true>, a)
-                                   : cudaLaunchKernelEx(&cfg, w4a8_gemv_kernel<NT, false>, a);
+    if (S > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = S;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    cudaError_t e = a.G == kBlockK ? cudaLaunchKernelEx(&cfg, w4a8_gemv_kernel<NT, true, S>, a)
+                                   : cudaLaunchKernelEx(&cfg, w4a8_gemv_kernel<NT, false, S>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
+// K split over S CTAs (1, 2 or 4) so that the grid gives every SM at least
+// about three CTAs: 16-channel groups alone are too few for small N.
+template <int NT>
+cudaError_t launch_nt(const GemvArgs &a, cudaStream_t stream)
+{
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long groups = a.N / 16;
+    int S = 1;
+    while (S < 4 && groups * S < 3LL * sms) S *= 2;
+    if (S == 1) return launch_nts<NT, 1>(a, stream);
+    if (S == 2) return launch_nts<NT, 2>(a, stream);
+    return launch_nts<NT, 4>(a, stream);
+}
+
 }  // namespace
 
-bool gemv_applies(int M, int epi, bool one_launch)
+bool gemv_applies(int M, int N, int epi, bool one_launch, int sms)
 {
-    return M >= 1 && M <= kGemvMaxM && epi != kEpiSiluMul && !one_launch;
+    return M >= 1 && M <= kGemvMaxM && epi != kEpiSiluMul && !one_launch && (long long)(N / 16) <= 8LL * sms;
 }
 
 cudaError_t launch_gemv(const int8_t *X8, int ldx, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,

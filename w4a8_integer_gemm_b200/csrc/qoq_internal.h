@@ -119,11 +119,12 @@ bool gemm_a_in_tmem();
 // QOQ_OK when the current device is compute capability 10.0 (cached per device).
 int check_device();
 
-// The layer for M <= kGemvMaxM tokens on the CUDA cores (same inputs,
-// outputs and rounding as launch_gemm; no workspace).  gemv_applies says
-// whether a call can take it (not the SiLU-gated pair, not the one-launch
-// layer call).
-bool gemv_applies(int M, int epi, bool one_launch);
+// The decode kernel for M <= kGemvMaxM tokens (same inputs, outputs and
+// rounding as launch_gemm; no workspace).  gemv_applies says whether a call
+// takes it: not the SiLU-gated pair, not the one-launch layer call, and not
+// N above 8 channel groups of 16 per SM, where the GEMM's bulk-copy weight
+// stream is faster than the decode kernel's loads.
+bool gemv_applies(int M, int N, int epi, bool one_launch, int sms);
 cudaError_t launch_gemv(const int8_t *X8, int ldx, const uint16_t *s_x, const uint8_t *Wp, const uint16_t *s_c,
                         const uint8_t *s_g, const uint8_t *zs, int M, int N, int K, int G, uint16_t *Y,
                         int32_t *acc_dbg, int epi, const uint16_t *R, cudaStream_t stream);
