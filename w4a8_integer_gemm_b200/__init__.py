@@ -12,7 +12,8 @@ calls raise.
     Y = qoq_w4a8_gemm(X8, s_x, packed)                        # per forward
 
 `W4A8Linear` wraps the three for a layer; `w4a8_linear_host` is the end to
-end call a user makes with host tensors.
+end call a user makes with host tensors, and `w4a8_linear_host_many` runs
+several of them with their host copies overlapping the kernels.
 """
 from __future__ import annotations
 
@@ -505,6 +506,52 @@ class W4A8Linear:
         """y = fp16 W4A8 linear of x (fp16 [M, in_features]) through the layer call."""
         Y, _, _ = qoq_w4a8_linear(x_fp16, self.packed, stream=stream)
         return Y
+
+
+_HOST_STREAMS = {}
+_HOST_STREAMS_LOCK = threading.Lock()
+
+
+def w4a8_linear_host_many(calls, stream=None) -> list:
+    """Several end-to-end calls from host memory, pipelined.  `calls` is a
+    list of (x_host, layer, y_host): FP16 X in host memory (ideally pinned),
+    a W4A8Linear, and a host tensor for Y (ideally pinned).  Call i's copy of
+    X to the device, its layer call and its copy of Y back run on three
+    streams chained by events, so that one call's copies overlap the other
+    calls' kernels (the host link is full duplex).  Returns the y_host
+    tensors once all of them hold their results; `stream` waits for all of
+    the work, so events on it bracket the whole pipeline."""
+    s = stream or torch.cuda.current_stream()
+    dev = s.device
+    with _HOST_STREAMS_LOCK:
+        if dev not in _HOST_STREAMS:
+            _HOST_STREAMS[dev] = tuple(torch.cuda.Stream(device=dev) for _ in range(3))
+        s_in, s_cmp, s_out = _HOST_STREAMS[dev]
+    start = torch.cuda.Event()
+    start.record(s)
+    for t in (s_in, s_cmp, s_out):
+        t.wait_event(start)
+    for x_host, layer, y_host in calls:
+        with torch.cuda.stream(s_in):
+            x = x_host.to(dev, non_blocking=True)
+        ready = torch.cuda.Event()
+        ready.record(s_in)
+        s_cmp.wait_event(ready)
+        x.record_stream(s_cmp)
+        with torch.cuda.stream(s_cmp):
+            y = layer(x, stream=s_cmp)
+        done = torch.cuda.Event()
+        done.record(s_cmp)
+        s_out.wait_event(done)
+        y.record_stream(s_out)
+        with torch.cuda.stream(s_out):
+            y_host.copy_(y, non_blocking=True)
+    for t in (s_in, s_cmp, s_out):
+        e = torch.cuda.Event()
+        e.record(t)
+        s.wait_event(e)
+    s.synchronize()
+    return [c[2] for c in calls]
 
 
 def w4a8_linear_host(x_host: torch.Tensor, layer: W4A8Linear, y_host: Optional[torch.Tensor] = None,
