@@ -126,22 +126,23 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
 }
 
 // ---------------------------------------------------- activation quant --
-// A small CTA (128 threads, few registers) so that the quantizer of the
-// next layer fits on an SM beside a running GEMM CTA: it can then start,
-// and trigger the launch of its own GEMM, before the current GEMM ends.
-constexpr int kActThreads = 128;
-constexpr int kActCache = 4;   // 16-byte vectors per thread kept in registers (K <= 4096)
-
 // One CTA per token row: read the row once (kept in registers up to
-// kActCache vectors per thread), reduce max|x|, then quantize.
+// T * CACHE * 8 values), reduce max|x|, then quantize.  Short rows
+// (K <= 4096) take a small CTA (128 threads, few registers) so that the
+// quantizer of the next layer fits on an SM beside a running GEMM CTA: it
+// can then start, and trigger the launch of its own GEMM, before the
+// current GEMM ends.  Longer rows take 256 threads with 8 vectors each
+// (K <= 16384 in registers), so that every load of the row is in flight at
+// once: the quantizer of a large batch is on the step's critical path.
 // With rowsum non-null it also writes rowsum[m] = sum_k X8[m][k] (INT32).
-__global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16_t *__restrict__ X, int K,
-                                                                 int8_t *__restrict__ X8,
-                                                                 uint16_t *__restrict__ s_x,
-                                                                 int32_t *__restrict__ rowsum)
+template <int T, int CACHE>
+__global__ void __launch_bounds__(T, T == 128 ? 12 : 4) act_quant_kernel(const uint16_t *__restrict__ X, int K,
+                                                                        int8_t *__restrict__ X8,
+                                                                        uint16_t *__restrict__ s_x,
+                                                                        int32_t *__restrict__ rowsum)
 {
-    __shared__ float red[kActThreads / 32];
-    __shared__ int rsum[kActThreads / 32];
+    __shared__ float red[T / 32];
+    __shared__ int rsum[T / 32];
     // the GEMM that consumes X8 may launch now and start streaming weights;
     // it waits for this grid to finish before it reads X8 or s_x
     grid_launch_dependents();
@@ -153,23 +154,25 @@ __global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16
     const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)m * K);
     uint2 *out = reinterpret_cast<uint2 *>(X8 + (size_t)m * K);
     const int nvec = K / 8;
-    uint4 cache[kActCache];
+    uint4 cache[CACHE];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kActCache; ++i) {
-        const int idx = threadIdx.x + i * kActThreads;
-        if (idx < nvec) {
-            cache[i] = __ldcs(row + idx);
-            amax = fmaxf(amax, absmax8(cache[i]));
-        }
+    for (int i = 0; i < CACHE; ++i) {
+        const int idx = threadIdx.x + i * T;
+        if (idx < nvec) cache[i] = __ldcs(row + idx);
     }
-    for (int idx = threadIdx.x + kActCache * kActThreads; idx < nvec; idx += kActThreads)
+#pragma unroll
+    for (int i = 0; i < CACHE; ++i) {
+        const int idx = threadIdx.x + i * T;
+        if (idx < nvec) amax = fmaxf(amax, absmax8(cache[i]));
+    }
+    for (int idx = threadIdx.x + CACHE * T; idx < nvec; idx += T)
         amax = fmaxf(amax, absmax8(__ldg(row + idx)));
     amax = warp_max(amax);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     if (threadIdx.x < 32) {
-        float v = threadIdx.x < kActThreads / 32 ? red[threadIdx.x] : 0.0f;
+        float v = threadIdx.x < T / 32 ? red[threadIdx.x] : 0.0f;
         v = warp_max(v);
         if (threadIdx.x == 0) red[0] = v;
     }
@@ -180,15 +183,15 @@ __global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16
     if (threadIdx.x == 0) s_x[m] = sxh;
     int sum = 0;  // sum of this thread's INT8 codes (rowsum only)
 #pragma unroll
-    for (int i = 0; i < kActCache; ++i) {
-        const int idx = threadIdx.x + i * kActThreads;
+    for (int i = 0; i < CACHE; ++i) {
+        const int idx = threadIdx.x + i * T;
         if (idx < nvec) {
             const uint2 v = quant8(cache[i], sx);
             out[idx] = v;
             if (rowsum) sum = __dp4a((int)v.y, 0x01010101, __dp4a((int)v.x, 0x01010101, sum));
         }
     }
-    for (int idx = threadIdx.x + kActCache * kActThreads; idx < nvec; idx += kActThreads) {
+    for (int idx = threadIdx.x + CACHE * T; idx < nvec; idx += T) {
         const uint2 v = quant8(__ldg(row + idx), sx);
         out[idx] = v;
         if (rowsum) sum = __dp4a((int)v.y, 0x01010101, __dp4a((int)v.x, 0x01010101, sum));
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(kActThreads, 12) act_quant_kernel(const uint16
         if (threadIdx.x == 0) {
             int t = 0;
 #pragma unroll
-            for (int w = 0; w < kActThreads / 32; ++w) t += rsum[w];
+            for (int w = 0; w < T / 32; ++w) t += rsum[w];
             rowsum[m] = t;
         }
     }
@@ -321,9 +324,10 @@ cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16
     // programmatic dependent launch: the CTAs may be scheduled while the
     // previous kernel (for instance the previous layer's GEMM) finishes;
     // they wait for it at the top of the kernel
+    const bool wide = K > 4096;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)M);
-    cfg.blockDim = dim3(kActThreads);
+    cfg.blockDim = dim3(wide ? 256 : 128);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -331,7 +335,8 @@ cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, X, K, X8, s_x, rowsum);
+    cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, act_quant_kernel<256, 8>, X, K, X8, s_x, rowsum)
+                         : cudaLaunchKernelEx(&cfg, act_quant_kernel<128, 4>, X, K, X8, s_x, rowsum);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
