@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
 // once: the quantizer of a large batch is on the step's critical path.
 // With rowsum non-null it also writes rowsum[m] = sum_k X8[m][k] (INT32).
 template <int T, int CACHE>
-__global__ void __launch_bounds__(T, T == 128 ? 12 : 4) act_quant_kernel(const uint16_t *__restrict__ X, int K,
+__global__ void __launch_bounds__(T, T == 128 ? 12 : CACHE <= 4 ? 6 : 4) act_quant_kernel(const uint16_t *__restrict__ X, int K,
                                                                         int8_t *__restrict__ X8,
                                                                         uint16_t *__restrict__ s_x,
                                                                         int32_t *__restrict__ rowsum)
@@ -328,6 +328,7 @@ cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)M);
     cfg.blockDim = dim3(wide ? 256 : 128);
+    // (K <= 8192: four vectors per thread, few registers, six CTAs per SM)
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -335,8 +336,9 @@ cudaError_t launch_act_quant(const uint16_t *X, int M, int K, int8_t *X8, uint16
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, act_quant_kernel<256, 8>, X, K, X8, s_x, rowsum)
-                         : cudaLaunchKernelEx(&cfg, act_quant_kernel<128, 4>, X, K, X8, s_x, rowsum);
+    cudaError_t e = !wide     ? cudaLaunchKernelEx(&cfg, act_quant_kernel<128, 4>, X, K, X8, s_x, rowsum)
+                    : K <= 8192 ? cudaLaunchKernelEx(&cfg, act_quant_kernel<256, 4>, X, K, X8, s_x, rowsum)
+                                : cudaLaunchKernelEx(&cfg, act_quant_kernel<256, 8>, X, K, X8, s_x, rowsum);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
