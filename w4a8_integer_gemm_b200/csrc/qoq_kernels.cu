@@ -125,6 +125,36 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
     }
 }
 
+// quant_x(x, sx) = clamp(rint(fl(x / sx))) without a division for almost
+// every x.  With r = fl(1/sx), qa = fl(x * r) differs from fl(x / sx) by at
+// most |x/sx| * 3 * 2^-24 (two roundings of r and qa, one of the quotient):
+// under 2.3e-5 for the quotients that survive the clamp, and under 2.5e-4
+// up to |x/sx| = 1300, beyond which both clamp alike.  So when qa is farther
+// than 2^-12 from the nearest half-integer, no half-integer lies between qa
+// and fl(x / sx), and rint(qa) is rint(fl(x / sx)); only the rare x within
+// 2^-12 of a rounding boundary take the IEEE division itself.
+__device__ __forceinline__ int quant_x_fast(float x, float sx, float rsx)
+{
+    if (sx == 0.0f) return 0;
+    const float qa = x * rsx;
+    const float f = qa - floorf(qa);
+    if (fabsf(f - 0.5f) > 0.000244140625f) return (int)fminf(fmaxf(rintf(qa), -128.0f), 127.0f);
+    return quant_x(x, sx);
+}
+
+__device__ __forceinline__ uint2 quant8_fast(const uint4 &v, float sx, float rsx)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[2] = {0, 0};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = (uint32_t)quant_x_fast(half_bits_to_float((uint16_t)(w[i] & 0xFFFFu)), sx, rsx) & 0xFFu;
+        const uint32_t hi = (uint32_t)quant_x_fast(half_bits_to_float((uint16_t)(w[i] >> 16)), sx, rsx) & 0xFFu;
+        o[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
+    }
+    return make_uint2(o[0], o[1]);
+}
+
 // ---------------------------------------------------- activation quant --
 // One CTA per token row: read the row once (kept in registers up to
 // T * CACHE * 8 values), reduce max|x|, then quantize.  Short rows
@@ -180,19 +210,20 @@ __global__ void __launch_bounds__(T, T == 128 ? 12 : CACHE <= 4 ? 6 : 4) act_qua
     amax = red[0];
     const uint16_t sxh = token_scale_bits(amax);
     const float sx = half_bits_to_float(sxh);
+    const float rsx = sx == 0.0f ? 0.0f : __frcp_rn(sx);
     if (threadIdx.x == 0) s_x[m] = sxh;
     int sum = 0;  // sum of this thread's INT8 codes (rowsum only)
 #pragma unroll
     for (int i = 0; i < CACHE; ++i) {
         const int idx = threadIdx.x + i * T;
         if (idx < nvec) {
-            const uint2 v = quant8(cache[i], sx);
+            const uint2 v = quant8_fast(cache[i], sx, rsx);
             out[idx] = v;
             if (rowsum) sum = __dp4a((int)v.y, 0x01010101, __dp4a((int)v.x, 0x01010101, sum));
         }
     }
     for (int idx = threadIdx.x + CACHE * T; idx < nvec; idx += T) {
-        const uint2 v = quant8(__ldg(row + idx), sx);
+        const uint2 v = quant8_fast(__ldg(row + idx), sx, rsx);
         out[idx] = v;
         if (rowsum) sum = __dp4a((int)v.y, 0x01010101, __dp4a((int)v.x, 0x01010101, sum));
     }
