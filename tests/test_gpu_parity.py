@@ -84,6 +84,41 @@ def test_act_quant_degenerate_rows():
     assert np.array_equal(_u16(s_x)[:4], rs)
 
 
+def _boundary_rows(K):
+    """Rows whose values sit on and next to the rounding boundaries of the
+    INT8 grid: x near (k + 1/2) * s_x for k = -127 .. 126 and their FP16
+    neighbours up to 3 ulps away, with max |x| fixed by element 0 (several
+    row maxima, among them ones that make s_x a power of two, so that the
+    ties are exact)."""
+    rows = []
+    for A in (127.0, 63.5, 1.0, 3.3, 0.0137, 1000.0, 17.25):
+        sx = float(np.float16(np.float32(A) / np.float32(127.0)))
+        vals = []
+        for k in range(-127, 127):
+            v = np.float16((k + 0.5) * sx)
+            lo = hi = v
+            vals.append(v)
+            for _ in range(3):
+                lo = np.nextafter(lo, np.float16(-np.inf))
+                hi = np.nextafter(hi, np.float16(np.inf))
+                vals += [lo, hi]
+        row = np.resize(np.array(vals, dtype=np.float16), K)
+        row[0] = np.float16(A) if A < 65504 else row[0]
+        rows.append(row)
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("K", [2048, 8192, 24576])
+def test_act_quant_rounding_boundaries(K):
+    """Values within a few ulps of x / s_x = k + 1/2: the quantizer's
+    reciprocal shortcut must round them exactly as the IEEE division does."""
+    X = torch.from_numpy(_boundary_rows(K))
+    X8, s_x = q.qoq_quant_act_per_token(X.cuda())
+    rX8, rs = oracle.quant_act(X.numpy())
+    assert np.array_equal(_u16(s_x)[:X.shape[0]], rs)
+    assert np.array_equal(X8.cpu().numpy(), rX8)
+
+
 # ----------------------------------------------------------- packing ----
 @pytest.mark.parametrize("N,K,G", [(128, 128, 128), (512, 512, 128), (512, 512, 512), (384, 4096, 128),
                                    (256, 4096, 4096)])

@@ -129,13 +129,15 @@ __global__ void __launch_bounds__(kGvThreads, 4) w4a8_gemv_kernel(GemvArgs a)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[u][i] = 0;
     constexpr int kStep = kGvWarps * S;
-    Block cur;
+    // weights two K blocks ahead of the products
+    Block cur, nxt;
     int b = q * kGvWarps + warp;
     if (b < nb) load_block<PG>(a, panel, r0, g, c, b, cur);
+    if (b + kStep < nb) load_block<PG>(a, panel, r0, g, c, b + kStep, nxt);
     grid_dependency_wait();  // X8 and s_x come from the preceding kernel
     for (; b < nb; b += kStep) {
-        Block nxt;
-        if (b + kStep < nb) load_block<PG>(a, panel, r0, g, c, b + kStep, nxt);
+        Block nx2;
+        if (b + 2 * kStep < nb) load_block<PG>(a, panel, r0, g, c, b + 2 * kStep, nx2);
         uint32_t gs[2], bs[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -172,7 +174,8 @@ __global__ void __launch_bounds__(kGvThreads, 4) w4a8_gemv_kernel(GemvArgs a)
                 mma_s8_16832(acc[u], af, xlo[s], xhi[s]);
             }
         }
-        if (b + kStep < nb) cur = nxt;
+        cur = nxt;
+        nxt = nx2;
     }
     // the warps' sums: lane (g, c) holds rows (channels) g and g + 8,
     // columns (tokens) 8u + 2c and 8u + 2c + 1
