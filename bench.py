@@ -589,8 +589,9 @@ def run_ours(args, rank, world, local, dist):
         e2e = {"value": round(world * tot_ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e2e_ms, 4),
-               "call": "w4a8_linear_host_many over the step's shapes: X pinned host -> device, layer call, "
-                       "Y -> pinned host on three streams chained by events, one synchronize at the end",
+               "call": "w4a8_linear_host_many over the step's shapes, cut into row blocks of about 16 MB: "
+                       "X pinned host -> device, layer call, Y -> pinned host on three streams chained by "
+                       "events, one synchronize at the end",
                "serial": {"value": round(world * tot_ops / (serial_ms * 1e-3) / 1e12, 3), "ms_per_step":
                           round(serial_ms, 4), "call": "w4a8_linear_host per shape, each synchronized"}}
 

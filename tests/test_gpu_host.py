@@ -35,3 +35,21 @@ def test_host_calls_match_device_layer():
         assert q.qoq_device_error() == q.QOQ_OK
         for y, ref in zip(outs, refs):
             assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("chunk_rows", [None, 128, 1000])
+def test_host_many_row_blocks(chunk_rows):
+    """Calls cut into row blocks (ragged last block, and a call smaller than
+    one block) return the bits of the whole device-resident layer call."""
+    shapes = [(2500, 4096, 4096), (7, 1024, 512), (4500, 2048, 1024)]
+    calls, refs = [], []
+    for i, (M, K, N) in enumerate(shapes):
+        W = wl.make_weights(N, K, wl.LLAMA, seed=6300 + i)
+        layer = q.W4A8Linear(W.cuda(), group_size=128)
+        X = wl.make_activations(M, K, wl.LLAMA, seed=6400 + i)
+        refs.append(layer(X.cuda()).cpu())
+        calls.append((X.pin_memory(), layer, torch.full((M, N), float("nan"), dtype=torch.float16).pin_memory()))
+    outs = q.w4a8_linear_host_many(calls, chunk_rows=chunk_rows)
+    assert q.qoq_device_error() == q.QOQ_OK
+    for y, ref in zip(outs, refs):
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16))

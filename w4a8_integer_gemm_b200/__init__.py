@@ -512,15 +512,44 @@ _HOST_STREAMS = {}
 _HOST_STREAMS_LOCK = threading.Lock()
 
 
-def w4a8_linear_host_many(calls, stream=None) -> list:
+_HOST_CHUNK_BYTES = 16 << 20
+
+
+def _host_pieces(calls, chunk_rows):
+    """The calls cut into row blocks: the layer is row-wise (each output row
+    depends on its own input row only, per-token scale included), so a block
+    of rows is a call of its own with the same bits.  Blocks of about 16 MB
+    of X or Y let one block's copy in overlap the previous block's kernels
+    and copy out."""
+    out = []
+    for x_host, layer, y_host in calls:
+        M = x_host.shape[0] if x_host.dim() == 2 else 0
+        rows = chunk_rows
+        if rows is None:
+            width = max(x_host.shape[-1], y_host.shape[-1])
+            rows = max(128, _HOST_CHUNK_BYTES // (2 * width) // 128 * 128)
+        if M <= rows or y_host.dim() != 2 or y_host.shape[0] != M:
+            out.append((x_host, layer, y_host))
+            continue
+        for r in range(0, M, rows):
+            out.append((x_host[r:r + rows], layer, y_host[r:r + rows]))
+    return out
+
+
+def w4a8_linear_host_many(calls, stream=None, chunk_rows: Optional[int] = None) -> list:
     """Several end-to-end calls from host memory, pipelined.  `calls` is a
-    list of (x_host, layer, y_host): FP16 X in host memory (ideally pinned),
-    a W4A8Linear, and a host tensor for Y (ideally pinned).  Call i's copy of
-    X to the device, its layer call and its copy of Y back run on three
-    streams chained by events, so that one call's copies overlap the other
-    calls' kernels (the host link is full duplex).  Returns the y_host
-    tensors once all of them hold their results; `stream` waits for all of
-    the work, so events on it bracket the whole pipeline."""
+    list of (x_host, layer, y_host): FP16 X [M][K] in host memory (ideally
+    pinned), a W4A8Linear, and a host tensor for Y [M][N] (ideally pinned).
+    Each call is cut into blocks of `chunk_rows` token rows (by default about
+    16 MB of X or Y per block; the outputs are the same bits).  Block i's copy
+    of X to the device, its layer call and its copy of Y back run on three
+    streams chained by events, so that one block's copies overlap the other
+    blocks' kernels and copies in the other direction (the host link is full
+    duplex).  Returns the y_host tensors once all of them hold their results;
+    `stream` waits for all of the work, so events on it bracket the whole
+    pipeline."""
+    if chunk_rows is not None and chunk_rows < 1:
+        raise ValueError("chunk_rows must be positive")
     s = stream or torch.cuda.current_stream()
     dev = s.device
     with _HOST_STREAMS_LOCK:
@@ -531,7 +560,7 @@ def w4a8_linear_host_many(calls, stream=None) -> list:
     start.record(s)
     for t in (s_in, s_cmp, s_out):
         t.wait_event(start)
-    for x_host, layer, y_host in calls:
+    for x_host, layer, y_host in _host_pieces(calls, chunk_rows):
         with torch.cuda.stream(s_in):
             x = x_host.to(dev, non_blocking=True)
         ready = torch.cuda.Event()
