@@ -407,7 +407,8 @@ __global__ void __launch_bounds__(kThreads, G > 4 ? 2 : 3) kv4_attn_kernel(
                 const int hq = 4 * t + 2 * (c & 1) + i;
                 if (lane < 2 && hq < G) red2[warp][hq] = v;
             }
-        __syncthreads();   // P complete
+        // each warp reads back only the numerators of its own 64 tokens
+        __syncwarp();
         // pass 2: O^T[channel][column] over the warp's 64 tokens; m-tile mt
         // row g is channel 16g + 2mt (a low nibble), row g + 8 channel
         // 16g + 2mt + 1 (the high nibble of the same byte)
