@@ -127,32 +127,54 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
 
 // quant_x(x, sx) = clamp(rint(fl(x / sx))) without a division for almost
 // every x.  With r = fl(1/sx), qa = fl(x * r) differs from fl(x / sx) by at
-// most |x/sx| * 3 * 2^-24 (two roundings of r and qa, one of the quotient):
-// under 2.3e-5 for the quotients that survive the clamp, and under 2.5e-4
-// up to |x/sx| = 1300, beyond which both clamp alike.  So when qa is farther
-// than 2^-12 from the nearest half-integer, no half-integer lies between qa
-// and fl(x / sx), and rint(qa) is rint(fl(x / sx)); only the rare x within
-// 2^-12 of a rounding boundary take the IEEE division itself.
-__device__ __forceinline__ int quant_x_fast(float x, float sx, float rsx)
-{
-    if (sx == 0.0f) return 0;
-    const float qa = x * rsx;
-    const float f = qa - floorf(qa);
-    if (fabsf(f - 0.5f) > 0.000244140625f) return (int)fminf(fmaxf(rintf(qa), -128.0f), 127.0f);
-    return quant_x(x, sx);
-}
+// most |x/sx| * 3 * 2^-24 (two roundings of r and qa, one of the quotient),
+// under 2.3e-5 for every x of the row (|x| <= max|x| keeps |x/sx| below
+// 127.1).  So when qa is farther than 2^-12 from the nearest half-integer,
+// no half-integer lies between qa and fl(x / sx), and both round to the
+// same integer; and clamping first to [-128, 127] (whose ends are integers)
+// changes neither result.  The rounding itself: adding 1.5 * 2^23 to a
+// float of magnitude below 2^22 leaves a float of unit spacing, so the sum
+// is rounded to an integer, ties to even as rint rounds, and that integer's
+// low byte (two's complement) is the low byte of the sum's bits.
+constexpr float kRoundMagic = 12582912.0f;        // 1.5 * 2^23
+constexpr float kFarFromHalf = 0.499755859375f;   // 1/2 - 2^-12
 
+// 8 FP16 values -> 8 INT8 codes (lowest address in the lowest byte).  The
+// rare vector with an element within 2^-12 of a rounding boundary (or any
+// vector of a row with s_x = 0) is redone with the IEEE division.
 __device__ __forceinline__ uint2 quant8_fast(const uint4 &v, float sx, float rsx)
 {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[2] = {0, 0};
+    uint32_t y[8];
+    bool near = false;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = (uint32_t)quant_x_fast(half_bits_to_float((uint16_t)(w[i] & 0xFFFFu)), sx, rsx) & 0xFFu;
-        const uint32_t hi = (uint32_t)quant_x_fast(half_bits_to_float((uint16_t)(w[i] >> 16)), sx, rsx) & 0xFFu;
-        o[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
+    for (int i = 0; i < 8; ++i) {
+        const float c = fminf(fmaxf(half_bits_to_float((uint16_t)(w[i >> 1] >> (16 * (i & 1)))) * rsx, -128.0f),
+                              127.0f);
+        const float r = c + kRoundMagic;
+        near |= fabsf(c - (r - kRoundMagic)) >= kFarFromHalf;
+        y[i] = __float_as_uint(r);
     }
-    return make_uint2(o[0], o[1]);
+    if (near || sx == 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            y[i] = (uint32_t)quant_x(half_bits_to_float((uint16_t)(w[i >> 1] >> (16 * (i & 1)))), sx);
+    }
+    // the low byte of each: two per half word, then the halves side by side
+    const uint32_t a = __byte_perm(y[0], y[1], 0x0040u), b = __byte_perm(y[2], y[3], 0x0040u);
+    const uint32_t c = __byte_perm(y[4], y[5], 0x0040u), d = __byte_perm(y[6], y[7], 0x0040u);
+    return make_uint2(__byte_perm(a, b, 0x5410u), __byte_perm(c, d, 0x5410u));
+}
+
+// max |x| of 8 FP16 values, taken in FP16 (exact), returned as a float
+__device__ __forceinline__ float absmax8_h2(const uint4 &v)
+{
+    __half2 m = __habs2(__halves2half2(__ushort_as_half((uint16_t)v.x), __ushort_as_half((uint16_t)(v.x >> 16))));
+    const uint32_t w[3] = {v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+        m = __hmax2(m, __habs2(__halves2half2(__ushort_as_half((uint16_t)w[i]), __ushort_as_half((uint16_t)(w[i] >> 16)))));
+    return fmaxf(__low2float(m), __high2float(m));
 }
 
 // ---------------------------------------------------- activation quant --
@@ -166,7 +188,7 @@ __device__ __forceinline__ uint2 quant8_fast(const uint4 &v, float sx, float rsx
 // once: the quantizer of a large batch is on the step's critical path.
 // With rowsum non-null it also writes rowsum[m] = sum_k X8[m][k] (INT32).
 template <int T, int CACHE>
-__global__ void __launch_bounds__(T, T == 128 ? 12 : CACHE <= 4 ? 6 : 4) act_quant_kernel(const uint16_t *__restrict__ X, int K,
+__global__ void __launch_bounds__(T, T == 128 ? 10 : CACHE <= 4 ? 5 : 4) act_quant_kernel(const uint16_t *__restrict__ X, int K,
                                                                         int8_t *__restrict__ X8,
                                                                         uint16_t *__restrict__ s_x,
                                                                         int32_t *__restrict__ rowsum)
@@ -194,10 +216,10 @@ __global__ void __launch_bounds__(T, T == 128 ? 12 : CACHE <= 4 ? 6 : 4) act_qua
 #pragma unroll
     for (int i = 0; i < CACHE; ++i) {
         const int idx = threadIdx.x + i * T;
-        if (idx < nvec) amax = fmaxf(amax, absmax8(cache[i]));
+        if (idx < nvec) amax = fmaxf(amax, absmax8_h2(cache[i]));
     }
     for (int idx = threadIdx.x + CACHE * T; idx < nvec; idx += T)
-        amax = fmaxf(amax, absmax8(__ldg(row + idx)));
+        amax = fmaxf(amax, absmax8_h2(__ldg(row + idx)));
     amax = warp_max(amax);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
