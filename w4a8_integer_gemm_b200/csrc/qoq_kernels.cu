@@ -183,9 +183,10 @@ __device__ __forceinline__ float absmax8_h2(const uint4 &v)
 // (K <= 4096) take a small CTA (128 threads, few registers) so that the
 // quantizer of the next layer fits on an SM beside a running GEMM CTA: it
 // can then start, and trigger the launch of its own GEMM, before the
-// current GEMM ends.  Longer rows take 256 threads with 8 vectors each
-// (K <= 16384 in registers), so that every load of the row is in flight at
-// once: the quantizer of a large batch is on the step's critical path.
+// current GEMM ends.  Longer rows take 256 threads with 4 vectors each
+// (K <= 8192) or 8 (K <= 16384 in registers), so that every load of the
+// row is in flight at once: the quantizer of a large batch is on the
+// step's critical path.
 // With rowsum non-null it also writes rowsum[m] = sum_k X8[m][k] (INT32).
 template <int T, int CACHE>
 __global__ void __launch_bounds__(T, T == 128 ? 10 : CACHE <= 4 ? 5 : 4) act_quant_kernel(const uint16_t *__restrict__ X, int K,
