@@ -623,16 +623,16 @@ def run_ours(args, rank, world, local, dist):
 
 
 # ------------------------------------------------------------ CPU oracle --
-def oracle_sample(work, budget_s, indices=None):
+def oracle_sample(work, cpu_s, indices=None):
     """Time the oracle's act quant + INT32 GEMM + epilogue on the shapes of
     the workload (all, or those at `indices`), restricted to a channel
-    sample sized for `budget_s` CPU seconds in total; returns (TOPS, threads,
+    sample sized for `cpu_s` CPU seconds in total; returns (TOPS, threads,
     description)."""
     import oracle
 
     idx = list(range(len(work.shapes))) if indices is None else list(indices)
     n_sh = len(idx)
-    per_shape = budget_s / n_sh
+    per_shape = cpu_s / n_sh
     tot_ops = tot_s = 0.0
     descr = []
     for i in idx:
@@ -640,7 +640,7 @@ def oracle_sample(work, budget_s, indices=None):
         X, W = wl.make_case(work, i)
         Xn = X.numpy()
         rows = min(s.M, 256)
-        # calibrate on 128 channels, then size the sample to the budget
+        # calibrate on 128 channels, then size the sample to that time
         n_try = 128
         wq = oracle.quantize_weights(W[:n_try].numpy(), s.G)
         W8 = oracle.dequant_weights(wq["q"], wq["s_g"], wq["zs"], s.G)
@@ -663,7 +663,7 @@ def oracle_sample(work, budget_s, indices=None):
     return tot_ops / tot_s / 1e12, oracle.num_threads(), "; ".join(descr)
 
 
-def oracle_single_core(work, budget_s):
+def oracle_single_core(work, cpu_s):
     """The same oracle timing on one host core, for the workload's smallest
     shape (by operations)."""
     import oracle
@@ -672,7 +672,7 @@ def oracle_single_core(work, budget_s):
     before = oracle.num_threads()
     oracle.set_num_threads(1)
     try:
-        v, threads, descr = oracle_sample(work, budget_s, indices=[i])
+        v, threads, descr = oracle_sample(work, cpu_s, indices=[i])
     finally:
         oracle.set_num_threads(before)
     return {"value": round(v, 6), "unit": "TOPS", "cores": threads, "sample": descr}
@@ -685,14 +685,14 @@ def run_reference(args, rank, world, local, dist):
     oracle.build()
     work = select(args)
     steps = args.steps
-    budget = max(1.0, args.cpu_seconds / max(1, steps))
+    per_step_s = max(1.0, args.cpu_seconds / max(1, steps))
     vals = []
     descr = ""
     threads = oracle.num_threads()
     for _ in range(min(args.warmup, 1)):
-        oracle_sample(work, budget)
+        oracle_sample(work, per_step_s)
     for _ in range(steps):
-        v, threads, descr = oracle_sample(work, budget)
+        v, threads, descr = oracle_sample(work, per_step_s)
         vals.append(v)
     value = statistics.median(vals)
     return {
