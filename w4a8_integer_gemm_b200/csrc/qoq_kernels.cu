@@ -127,12 +127,13 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
 
 // quant_x(x, sx) = clamp(rint(fl(x / sx))) without a division for almost
 // every x.  With r = fl(1/sx), qa = fl(x * r) differs from fl(x / sx) by at
-// most |x/sx| * 3 * 2^-24 (two roundings of r and qa, one of the quotient),
-// under 2.3e-5 for every x of the row (|x| <= max|x| keeps |x/sx| below
-// 127.1).  So when qa is farther than 2^-12 from the nearest half-integer,
-// no half-integer lies between qa and fl(x / sx), and both round to the
-// same integer; and clamping first to [-128, 127] (whose ends are integers)
-// changes neither result.  The rounding itself: adding 1.5 * 2^23 to a
+// most |x/sx| * 3 * 2^-24 (two roundings of r and qa, one of the quotient):
+// under 2.3e-5 where |x/sx| < 128.5, the only quotients the clamp does not
+// decide, and under 2^-12 up to |x/sx| = 1365.  So when qa is farther than
+// 2^-12 from the nearest half-integer, no half-integer lies between qa and
+// fl(x / sx), and both round to the same integer; clamping first to
+// [-128, 127] (whose ends are integers) changes neither result, and beyond
+// |x/sx| = 1365 both sides clamp alike.  The rounding itself: adding 1.5 * 2^23 to a
 // float of magnitude below 2^22 leaves a float of unit spacing, so the sum
 // is rounded to an integer, ties to even as rint rounds, and that integer's
 // low byte (two's complement) is the low byte of the sum's bits.
