@@ -283,11 +283,14 @@ def load_traffic(workload_name: str, path: str = None):
     return t.get("captures", {})
 
 
-def regime_roofline(bound, shapes, ms, peaks, traffic):
+def regime_roofline(bound, shapes, ms, peaks, traffic, sm_mhz=None):
     """Roofline record of the GEMM over a chain of shapes of one regime
     (all HBM-bound or all tensor-bound), timed back to back: `ms` is the
     chain's time.  `traffic` comes from one ncu capture of a representative
-    shape of the regime, with that shape's algorithmic bytes beside it."""
+    shape of the regime, with that shape's algorithmic bytes beside it.
+    `sm_mhz`: the median SM clock seen under load (the maximum, 1965 MHz,
+    when no clock was sampled), for the MMA issue ceiling of the tensor
+    regime."""
     n = len(shapes)
     byt = sum(roofline.algorithmic_bytes(x.M, x.N, x.K, x.G) for x in shapes)
     ops = sum(roofline.ops(x.M, x.N, x.K) for x in shapes)
@@ -302,6 +305,9 @@ def regime_roofline(bound, shapes, ms, peaks, traffic):
               "unit": "TOPS", "frac": round(achieved / peaks["int8_tops"], 4), "traffic": None,
               "peak_source": peaks["source"] + " (2 x bf16 cuBLAS burst)",
               "frac_of_sustained_peak": round(achieved / peaks["int8_tops_sustained"], 4)}
+        ceil = roofline.mma_issue_ceiling_tops(float(sm_mhz) if sm_mhz else 1965.0)
+        rl["mma_issue_ceiling_tops"] = round(ceil, 1)
+        rl["frac_of_mma_issue_ceiling"] = round(achieved / ceil, 4)
     small = [x.name for x in shapes if x.M <= 8]
     kern = "w4a8_gemm_kernel" + (f" (w4a8_gemv_kernel for {', '.join(small)})" if small else "")
     rl.update({"kernel": kern, "launches": n, "chain_us": round(ms * 1e3, 2),
@@ -512,7 +518,7 @@ def run_ours(args, rank, world, local, dist):
     tot_ms = statistics.median(step_ms)
     ms_step, value = aggregate(tot_ops, tot_ms, world, dist)
     traffic = load_traffic(args.workload)
-    by_bound = {b: regime_roofline(b, [c["s"] for c in sub], chain_ms[b], peaks, traffic)
+    by_bound = {b: regime_roofline(b, [c["s"] for c in sub], chain_ms[b], peaks, traffic, clocks.get("sm_mhz"))
                 for b, sub in regimes.items()}
     # the dominant kernel's regime: where the GEMM spends most of the step
     dom = max(by_bound, key=lambda b: by_bound[b]["chain_us"])

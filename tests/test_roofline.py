@@ -26,3 +26,37 @@ def test_bytes_and_bound():
     assert roofline.bound(1, 14336, 4096, 128, 3.2e15, 6.5e12) == "hbm"
     assert roofline.bound(4096, 8192, 8192, 128, 3.2e15, 6.5e12) == "tensor"
     assert roofline.ops(2, 3, 5) == 60
+
+
+def test_mma_issue_ceiling():
+    # 148 SMs x 8192 INT8 MACs per clock x 2 ops at 1965 MHz
+    assert abs(roofline.mma_issue_ceiling_tops(1965.0) - 4764.8) < 0.1
+    assert abs(roofline.mma_issue_ceiling_tops(1000.0, sms=1) - 16.384) < 1e-9
+
+
+def test_regime_records_of_the_bench():
+    """The bench's roofline record for each regime, from made-up timings
+    (no GPU): the fields it reports and their arithmetic."""
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    if root not in sys.path:
+        sys.path.insert(0, root)
+    import bench
+    from w4a8_integer_gemm_b200 import workloads as wl
+    peaks = {"source": "measured", "hbm_gbs": 6543.4, "int8_tops": 3234.8, "int8_tops_sustained": 2745.4}
+    sweep = wl.WORKLOADS["sweep"].shapes
+    hbm = [s for s in sweep if s.M <= 128]
+    ten = [s for s in sweep if s.M >= 256]
+    traffic = {"sweep_M4096": {"dram_bytes": 352269824, "algorithmic_bytes": 135290880, "capture": "x",
+                               "tensor_pipe_pct": 67.2}}
+    r = bench.regime_roofline("tensor", ten, 0.9, peaks, traffic, 1965.0)
+    ops = sum(roofline.ops(s.M, s.N, s.K) for s in ten)
+    assert abs(r["achieved"] - ops / 0.9e-3 / 1e12) < 0.1
+    assert abs(r["frac"] - r["achieved"] / 3234.8) < 1e-4
+    assert abs(r["frac_of_mma_issue_ceiling"] - r["achieved"] / 4764.8) < 1e-4
+    assert r["traffic"] == 352269824 and r["ncu_tensor_pipe_pct"] == 67.2 and r["launches"] == 6
+    assert bench.regime_roofline("tensor", ten, 0.9, peaks, {}, None)["mma_issue_ceiling_tops"] == 4764.8
+    h = bench.regime_roofline("hbm", hbm, 0.12, peaks, {}, 1965.0)
+    byt = sum(roofline.algorithmic_bytes(s.M, s.N, s.K, s.G) for s in hbm)
+    assert abs(h["achieved"] - byt / 0.12e-3 / 1e9) < 0.1 and "frac_of_mma_issue_ceiling" not in h
+    assert "w4a8_gemv_kernel" in h["kernel"]

@@ -67,6 +67,20 @@ def crossover_m(fmt_a, fmt_b, bw_bytes: float, m_max: int = 1 << 16) -> int:
     return m_max
 
 
+# The INT8 MMA issue rate measured on this part: one tcgen05.mma kind::i8
+# of 128 x 256 x 32 per 128 SM cycles (one thread issuing back to back),
+# i.e. 8192 multiply-adds per clock per SM.  A second ceiling for the
+# tensor-bound GEMM beside the BF16-derived peak: it scales with the SM
+# clock the kernel actually ran at.
+MMA_I8_MACS_PER_CLK_PER_SM = 8192
+SMS = 148
+
+
+def mma_issue_ceiling_tops(sm_mhz: float, sms: int = SMS) -> float:
+    """INT8 ops/s (in TOPS) at the measured MMA issue rate and this SM clock."""
+    return sms * MMA_I8_MACS_PER_CLK_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+
+
 # ---------------------------------------------------------------- peaks ----
 # Nominal dense ratio INT8 : BF16 on B200 (4.5 : 2.25 PFLOP/s).
 INT8_PER_BF16 = 2.0
